@@ -1,0 +1,427 @@
+"""Benchmark of the B200 sparse top-k MoE FFN forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+A step is one whole forward (route, dispatch, grouped SwiGLU, shared expert,
+combine) over one batch of synthetic tokens. Default workload: the
+Qwen3-30B-A3B-shaped problem (T=4096, H=2048, E=128, top-8 softmax with
+renormalisation, I=768, bf16). With N > 1 (torchrun, one process per GPU)
+every rank runs its own batch with the same weights (weak scaling, no
+collective on the data path); the time is the max over ranks.
+
+Rank 0 prints one JSON line. ``value`` is tokens/s with inputs resident in
+HBM; ``e2e`` is the same metric through the public API from pinned host
+memory (host->device copy of x and device->host copy of out inside the timed
+region); ``roofline`` describes the dominant kernel (the grouped gate_up
+GEMM), timed with CUDA events on its stream inside the timed region;
+``cpu_baseline`` is the fp64 oracle timed on a bounded token sample on the
+host cores. ``--impl reference`` times that oracle as the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+DEFAULT_CONFIG = "qwen3_30b_a3b"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    """NVML sampling of SM clock and clock-event reasons on a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        rs = [name for bit, name in self.REASONS.items() if self.reasons & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": rs,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# workload accounting
+
+def active_experts(sel: torch.Tensor, E: int) -> int:
+    return int((torch.bincount(sel.reshape(-1), minlength=E) > 0).sum().item())
+
+
+def flops_and_bytes(cfg, n_active: int):
+    P = cfg.T * cfg.k
+    es = 4 if cfg.dtype == "f32" else 2
+    f_routed = 6.0 * cfg.H * cfg.I * P
+    f_shared = 6.0 * cfg.H * cfg.I_shared * cfg.T if cfg.shared != "none" else 0.0
+    f_router = 2.0 * cfg.T * cfg.H * cfg.E
+    # gate_up kernel alone: 4*H*I flops per pair; weights of active experts read
+    # once, x_perm read once, h written once.
+    gu_flops = 4.0 * cfg.H * cfg.I * P
+    gu_bytes = (n_active * 2 * cfg.I * cfg.H + P * cfg.H + P * cfg.I) * es
+    # whole forward, minimum: active weights once, x read, out written
+    w_bytes = n_active * 3 * cfg.I * cfg.H * es + cfg.E * cfg.H * es
+    if cfg.shared != "none":
+        w_bytes += 3 * cfg.I_shared * cfg.H * es
+    min_bytes = w_bytes + 2 * cfg.T * cfg.H * es
+    return {"active_flops": f_routed + f_shared, "router_flops": f_router, "gate_up_flops": gu_flops,
+            "gate_up_bytes": gu_bytes, "min_bytes": min_bytes, "weight_bytes": w_bytes}
+
+
+def launches_per_step(cfg) -> int:
+    # router logits + top-k; histogram + scan + permute; gate_up + down; shared
+    # gate_up + down; combine
+    return 2 + 3 + 2 + (2 if cfg.shared != "none" else 0) + 1
+
+
+def recorded_traffic(cfg_name: str):
+    """Per-launch DRAM traffic of the gate_up kernel from the committed ncu
+    summary, if the kernel source is unchanged since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"gate_up_{cfg_name}.md")
+    src = os.path.join(ROOT, "sparse_top_mixture_b200", "csrc", "gemm_tc.cu")
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"gemm_tc_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else None
+    except Exception:
+        return None
+
+
+class OracleTimer:
+    """Times the fp64 dense-masked oracle on a sample of tokens (each token
+    runs through every routed expert, as the oracle is defined)."""
+
+    def __init__(self, cfg, dev_inputs):
+        import numpy as np
+        self.np = np
+        self.cfg = cfg
+        f64 = workloads.to_numpy64
+        self.x = f64(dev_inputs["x"])
+        self.gw = f64(dev_inputs["gate_w"])
+        self.bias = f64(dev_inputs.get("bias"))
+        self.sg = f64(dev_inputs.get("shared_gate"))
+        self.sgu = f64(dev_inputs.get("shared_gate_up"))
+        self.sdn = f64(dev_inputs.get("shared_down"))
+        # expert weights converted once (input preparation, outside timing)
+        self.gu = [f64(dev_inputs["gate_up"][e]) for e in range(cfg.E)]
+        self.dn = [f64(dev_inputs["down"][e]) for e in range(cfg.E)]
+
+    def run(self, n_tokens: int, start: int = 0) -> float:
+        import oracle
+        c = self.cfg
+        rows = (start + self.np.arange(n_tokens)) % c.T
+        t0 = time.perf_counter()
+        oracle.moe_forward(self.x[rows], self.gw, self.gu, self.dn, k=c.k, score=c.score,
+                           renormalize=c.renormalize, bias=self.bias, bias_mode=c.bias_mode, shared=c.shared,
+                           shared_gate_up=self.sgu, shared_down=self.sdn, shared_gate=self.sg)
+        return time.perf_counter() - t0
+
+    def calibrate(self, target_s: float, max_tokens: int) -> int:
+        n = 4
+        t = self.run(n)
+        while t < target_s / 4 and n < max_tokens:
+            n = min(max_tokens, n * 4)
+            t = self.run(n)
+        per = t / n
+        return int(max(1, min(max_tokens, target_s / max(per, 1e-9))))
+
+
+def cpu_baseline(cfg, dev_inputs, target_s: float = 12.0):
+    ot = OracleTimer(cfg, dev_inputs)
+    n = ot.calibrate(target_s, cfg.T)
+    t = ot.run(n)
+    return {"value": n / t, "unit": "tokens/s", "cores": _blas_threads() or os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} of the {cfg.T} tokens of {cfg.name}, fp64 dense-masked (all {cfg.E} experts per token), "
+                      f"{t:.1f} s"}
+
+
+# ----------------------------------------------------------------------------
+
+def init_dist(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+    return rank, local, world
+
+
+def dist_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def make_inputs(cfg, rank: int):
+    r = workloads.router_inputs(cfg, rank=rank)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in r.items()}
+    dev.update(workloads.expert_weights(cfg, "cuda"))
+    return r, dev
+
+
+def run_reference(args, cfg, rank, world):
+    """Reference arm: the fp64 oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    torch.manual_seed(0)
+    r = workloads.router_inputs(cfg)
+    w = workloads.expert_weights(cfg, "cuda" if torch.cuda.is_available() else "cpu")
+    ot = OracleTimer(cfg, dict(r, **w))
+    n = ot.calibrate(max(1.0, 60.0 / max(1, args.steps + args.warmup)), cfg.T)
+    for i in range(args.warmup):
+        ot.run(n, start=i * n)
+    total = 0.0
+    for i in range(args.steps):
+        total += ot.run(n, start=(args.warmup + i) * n)
+    value = n * args.steps / total
+    line = {"impl": "reference", "metric": metric_name(), "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle",
+                             "cores": _blas_threads() or os.cpu_count(),
+                             "sample": f"{n} tokens per step of {cfg.name}, fp64 dense-masked"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def metric_name() -> str:
+    return "MoE FFN tokens/s and active-expert TFLOP/s (fraction of bf16/HBM roofline)"
+
+
+def config_dict(cfg) -> dict:
+    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+            "I_shared": cfg.I_shared, "score": cfg.score, "bias_mode": cfg.bias_mode,
+            "renormalize": cfg.renormalize, "shared": cfg.shared, "seed": cfg.seed}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(workloads.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = workloads.CONFIGS[args.config]
+    rank, local, world = init_dist(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+        if world > 1:
+            barrier(world)
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import sparse_top_mixture_b200 as stm
+
+    r_cpu, dev = make_inputs(cfg, rank)
+    p = stm.Problem.from_config(cfg)
+    moe = stm.SparseMoE(p, dev)
+    dt = p.torch_dtype
+    x = dev["x"]
+    out = torch.empty(cfg.T, cfg.H, dtype=dt, device="cuda")
+    rw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    sel = torch.empty(cfg.T, cfg.k, dtype=torch.int64, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        moe.forward(x, out, rw, sel)
+    torch.cuda.synchronize()
+    if moe.read_device_error() != 0:
+        raise RuntimeError("device error flag set during warm-up")
+    n_active = active_experts(sel, cfg.E)
+    fb = flops_and_bytes(cfg, n_active)
+
+    nst = len(stm.STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    for row in evs:  # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            moe.forward_profiled(x, out, rw, sel, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = dist_max(t_start.elapsed_time(t_end), world)
+    stage_ms = {}
+    for si, name in enumerate(stm.STAGES):
+        stage_ms[name] = sum(evs[i][si].elapsed_time(evs[i][si + 1]) for i in range(args.steps)) / args.steps
+    if moe.read_device_error() != 0:
+        raise RuntimeError("device error flag set during the timed region")
+
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_s = world * cfg.T * args.steps / (elapsed_ms / 1e3)
+    active_tflops = world * fb["active_flops"] * args.steps / (elapsed_ms / 1e3) / 1e12
+
+    # e2e: pinned host x in, host out back, through the public API
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 50))
+    x_host = r_cpu["x"].pin_memory()
+    out_host = torch.empty(cfg.T, cfg.H, dtype=dt).pin_memory()
+    x_dev2 = torch.empty_like(x)
+    for _ in range(2):
+        moe.forward_from_host(x_host, out_host, x_dev2, out, rw, sel)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        moe.forward_from_host(x_host, out_host, x_dev2, out, rw, sel)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1), world)
+    e2e_tps = world * cfg.T * e2e_steps / (e2e_ms / 1e3)
+
+    pk = peaks()
+    gu_ms = stage_ms["gate_up"]
+    t_tensor = fb["gate_up_flops"] / (pk["bf16_tflops_sustained"] * 1e12)
+    t_hbm = fb["gate_up_bytes"] / (pk["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        achieved = fb["gate_up_flops"] / (gu_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+    else:
+        achieved = fb["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(cfg.name)
+    roof["kernel"] = "tc_grouped_gemm_kernel<gate_up>"
+    roof["peak_source"] = pk["source"] + (" sustained bf16" if roof["bound"] == "tensor" else " copy bandwidth")
+    roof["algorithmic"] = {"flops": fb["gate_up_flops"], "bytes": fb["gate_up_bytes"], "ms": gu_ms}
+
+    whole_roof_s = max((fb["active_flops"] + fb["router_flops"]) / (pk["bf16_tflops_sustained"] * 1e12),
+                       fb["min_bytes"] / (pk["hbm_gbs"] * 1e9))
+
+    line = {
+        "metric": metric_name(), "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; weights ~N(0,1/fan_in))",
+        "config": dict(config_dict(cfg), parallelism=f"replicas x{world} (independent batches)",
+                       l2=f"inputs larger than L2: {fb['weight_bytes'] / 1e9:.2f} GB of weights read per step, "
+                          f"no flush"),
+        "active_expert_tflops": active_tflops,
+        "forward_roofline_frac": whole_roof_s / (ms_per_step / 1e3),
+        "active_experts": n_active,
+        "stage_ms": stage_ms,
+        "roofline": roof,
+        "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * x.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": e2e_steps},
+        "gpu_launches": launches_per_step(cfg) * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, dict(r_cpu, **{k: dev[k] for k in (
+            "gate_up", "down", "shared_gate_up", "shared_down")}))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(world)
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,228 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse top-k MoE FFN forward.
+ *
+ * The forward pass, step by step:
+ *   route    : logits = x . gate_w^T, scores (softmax / sigmoid / sqrtsoftplus),
+ *              top-k with an optional fp32 bias, optional renormalisation;
+ *   dispatch : per-expert histogram, exclusive scan to segment offsets, stable
+ *              permutation of token copies into contiguous per-expert segments;
+ *   grouped SwiGLU : h = silu(x W_g^T) * (x W_u^T) per routed segment, then
+ *              y = w * (h W_d^T), only over experts that received tokens;
+ *   shared expert  : the same MLP over all tokens, optionally sigmoid-gated;
+ *   combine  : out[t] = sum_j y[(t, j)] + shared[t], back in token order.
+ *
+ * Passages each call follows (page title, section):
+ *   "mstar.model.components.moe" -- Router contract (hidden_states [T,H] in;
+ *     routing_weights [T,k] and int64 selected_experts [T,k] out), TopKRouter
+ *     (softmax top-k, norm_topk_prob), SparseMoeBlock (fused layout
+ *     gate_up_proj [E,2I,H], down_proj [E,H,I]), SparseMoeBlockWithSharedExpert
+ *     (out = routed(x) + sigmoid(shared_gate(x)) * shared_expert(x)).
+ *   "Sparse MoE FFN for DFlash-family drafters" -- What's here: MoEGate
+ *     (sqrtsoftplus scores, fp32 aux-loss-free bias used for selection only),
+ *     GroupedExperts (stacked [E, out, in] weights), SparseMoE (one argsort into
+ *     contiguous per-expert segments, grouped GEMM with no host syncs, one
+ *     shared expert).
+ *   "feat: Phase 43 -- Sparse/Grouped MoE Dispatch" -- Summary and Neural
+ *     Network: only the assigned top-k experts are computed, tokens grouped per
+ *     expert (arg_sort, index_select, index_add); empty expert groups skipped.
+ *   "MoE: shared experts, parameterized V_TOPK routing, explicit stage
+ *     attribution" -- 1. (routing at any expert count, "topk must be
+ *     positive"), 3. Tests (ungated, sigmoid-gated and n_shared-fused shared
+ *     experts), 4. (shared width is the fused width n_shared * I).
+ *
+ * Conventions for every call:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *     stated otherwise. The library never allocates, frees or synchronises,
+ *     except moe_read_device_error, which synchronises the given stream.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously. Outputs are valid once the stream has
+ *     passed the call.
+ *   - Row-major, densely packed tensors. x, the weights, x_perm and out have
+ *     the problem dtype (fp32 or bf16). y_perm and shared_out are fp32 for
+ *     every problem dtype: the only roundings to bf16 on the path are the
+ *     SwiGLU activation h (an operand of the down GEMM) and the final output.
+ *     Biases, routing weights and the shared gate values are fp32.
+ *     selected_experts is int64; counts, offsets, sorted_pairs and pair_pos
+ *     are int32.
+ *   - Every pointer must be 16-byte aligned. H, I and I_shared must be
+ *     multiples of 8 (16-byte rows for the TMA engine).
+ *   - Arguments are validated on the host before any launch. On an error
+ *     status nothing is launched and no output is written.
+ *   - Bad data found on the device (an expert id outside [0, E) handed to
+ *     moe_dispatch) does not fault: the pair is skipped, a flag in the
+ *     workspace header is set, and moe_read_device_error reports it.
+ *   - The workspace (size from moe_workspace_size) is caller-owned device
+ *     memory. Zero its header once with moe_workspace_init. Calls on different
+ *     streams need distinct workspaces. There is no global mutable state.
+ *   - T == 0 is a valid no-op.
+ *   - Limits: 1 <= k <= E <= 256.
+ */
+#ifndef STM_MOE_H
+#define STM_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* the same type as cudaStream_t */
+typedef struct CUevent_st *moe_event_t;   /* the same type as cudaEvent_t  */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARGUMENT = 1,  /* bad size, pointer, alignment or enum    */
+  MOE_ERR_UNSUPPORTED = 2,       /* valid but not implemented combination  */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+  MOE_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed   */
+  MOE_ERR_DEVICE_FLAG = 5        /* a kernel flagged bad data or a timeout */
+} moe_status;
+
+typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1, MOE_SCORE_SQRTSOFTPLUS = 2 } moe_score;
+/* LOGIT: bias added to the router logits (enters the scores).
+ * SELECT: bias added to the scores for choosing the top-k only; the routing
+ * weights come from the unbiased scores (aux-loss-free balancing bias). */
+typedef enum { MOE_BIAS_NONE = 0, MOE_BIAS_LOGIT = 1, MOE_BIAS_SELECT = 2 } moe_bias_mode;
+typedef enum { MOE_SHARED_NONE = 0, MOE_SHARED_PLAIN = 1, MOE_SHARED_SIGMOID_GATED = 2 } moe_shared_kind;
+
+/* Device-side error bits reported by moe_read_device_error. */
+#define MOE_DEVERR_BAD_EXPERT_ID 1 /* selected_experts held an id outside [0,E) */
+#define MOE_DEVERR_WAIT_TIMEOUT 2  /* a pipeline wait gave up (never expected)   */
+
+typedef struct moe_problem {
+  int64_t T;        /* tokens                                               */
+  int64_t H;        /* hidden size                                          */
+  int64_t E;        /* routed experts                                       */
+  int64_t k;        /* experts per token (top-k)                            */
+  int64_t I;        /* routed expert intermediate size                      */
+  int64_t I_shared; /* shared expert intermediate size (fused width), or 0  */
+  int32_t dtype;    /* moe_dtype                                            */
+  int32_t score;    /* moe_score                                            */
+  int32_t bias_mode;   /* moe_bias_mode                                     */
+  int32_t renormalize; /* nonzero: routing weights divided by their sum     */
+  int32_t shared;      /* moe_shared_kind                                   */
+  int32_t reserved;    /* must be 0                                         */
+} moe_problem;
+
+typedef struct moe_weights {
+  const void *gate_w;         /* [E, H] router weight                            */
+  const float *bias;          /* [E] fp32, or NULL when bias_mode == NONE        */
+  const void *gate_up;        /* [E, 2I, H]: rows 0..I-1 gate, rows I..2I-1 up   */
+  const void *down;           /* [E, H, I]                                       */
+  const void *shared_gate_up; /* [2*I_shared, H] (gate rows first), or NULL      */
+  const void *shared_down;    /* [H, I_shared], or NULL                          */
+  const void *shared_gate;    /* [H] gate vector (SIGMOID_GATED only), or NULL   */
+} moe_weights;
+
+/* Stages timed by moe_forward_profiled, in launch order. */
+enum {
+  MOE_STAGE_ROUTE = 0,
+  MOE_STAGE_DISPATCH = 1,
+  MOE_STAGE_GATE_UP = 2,
+  MOE_STAGE_DOWN = 3,
+  MOE_STAGE_SHARED = 4,
+  MOE_STAGE_COMBINE = 5,
+  MOE_NUM_STAGES = 6
+};
+
+/* Bytes of workspace moe_forward needs for problem p (each of the other calls
+ * needs at most this much). Host only. */
+moe_status moe_workspace_size(const moe_problem *p, size_t *bytes);
+
+/* Zero the workspace header (error flags). Call once after allocating it. */
+moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router ("mstar.model.components.moe", Router contract and TopKRouter;
+ * "Sparse MoE FFN for DFlash-family drafters", MoEGate).
+ *   x [T,H], gate_w [E,H]; bias [E] fp32 or NULL (per p->bias_mode);
+ *   shared_gate [H] or NULL: when given, shared_gamma [T] (fp32) receives
+ *   sigmoid(x[t] . shared_gate).
+ *   routing_weights [T,k] fp32 and selected_experts [T,k] int64 are written;
+ *   slot j holds the (j+1)-th largest selection key, equal keys ordered by
+ *   ascending expert index. */
+moe_status moe_route(const moe_problem *p, const void *x, const void *gate_w, const float *bias,
+                     const void *shared_gate, float *routing_weights, int64_t *selected_experts,
+                     float *shared_gamma, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router selection only, from given fp32 logits [T,E] (bias applied per
+ * p->bias_mode). Lets tests compare selection bit-exactly on identical
+ * logits. */
+moe_status moe_topk_from_logits(const moe_problem *p, const float *logits, const float *bias,
+                                float *routing_weights, int64_t *selected_experts, moe_stream_t stream);
+
+/* Sorted-segment dispatch ("Sparse MoE FFN for DFlash-family drafters",
+ * SparseMoE; "feat: Phase 43", sparse_grouped_dispatch).
+ *   Pair q = t*k + j routes token t to expert selected_experts[q].
+ *   counts [E]: pairs per expert. offsets [E+1]: exclusive prefix sum,
+ *   offsets[E] = pairs dispatched. sorted_pairs [T*k]: pair at segment
+ *   position p, ascending q inside each segment (stable). pair_pos [T*k]:
+ *   inverse, -1 for a pair skipped because of a bad expert id.
+ *   x_perm [T*k, H]: x_perm[p] = x[sorted_pairs[p] / k]; x and x_perm may
+ *   both be NULL to compute the permutation only. */
+moe_status moe_dispatch(const moe_problem *p, const int64_t *selected_experts, const void *x,
+                        int32_t *counts, int32_t *offsets, int32_t *sorted_pairs, int32_t *pair_pos,
+                        void *x_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped SwiGLU over the routed segments ("mstar.model.components.moe",
+ * SparseMoeBlock fused layout; "Sparse MoE FFN for DFlash-family drafters",
+ * grouped GEMM with no host syncs).
+ *   For each expert e with offsets[e] < offsets[e+1] and each row p in that
+ *   segment: h = silu(x_perm[p] . gate^T) * (x_perm[p] . up^T) (h kept in
+ *   the workspace, rounded to the problem dtype), then
+ *   y_perm[p] = routing_weights[sorted_pairs[p]] * (h . down[e]^T), fp32
+ *   [T*k, H]. routing_weights and sorted_pairs may both be NULL (scale 1).
+ *   Experts with no rows are never read. The segment table stays on the
+ *   device; no host synchronisation. */
+moe_status moe_grouped_swiglu(const moe_problem *p, const void *x_perm, const int32_t *offsets,
+                              const void *gate_up, const void *down, const float *routing_weights,
+                              const int32_t *sorted_pairs, void *y_perm, void *ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/* Shared expert over all T tokens ("mstar.model.components.moe",
+ * SparseMoeBlockWithSharedExpert; "MoE: shared experts ...", 3. Tests).
+ *   shared_out [T,H] fp32 = gamma[t] * SwiGLU(x[t]) with gamma =
+ *   shared_gamma[t] when shared_gamma is not NULL, else 1. */
+moe_status moe_shared_expert(const moe_problem *p, const void *x, const void *shared_gate_up,
+                             const void *shared_down, const float *shared_gamma, void *shared_out,
+                             void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine back to token order ("feat: Phase 43", index_add scatter).
+ *   out[t] = round( sum_{j<k} y_perm[pair_pos[t*k+j]] + shared_out[t] ), with
+ *   fp32 y_perm [T*k,H] and shared_out [T,H], the sum in fp32 in slot order,
+ *   rounded once to the problem dtype; shared_out may be NULL; pairs with
+ *   pair_pos < 0 contribute nothing. */
+moe_status moe_combine(const moe_problem *p, const void *y_perm, const int32_t *pair_pos,
+                       const void *shared_out, void *out, moe_stream_t stream);
+
+/* Whole forward: route, dispatch, grouped SwiGLU, shared expert, combine.
+ *   x [T,H] -> out [T,H]; routing_weights [T,k] and selected_experts [T,k] are
+ *   also written (router contract). All intermediates live in ws. */
+moe_status moe_forward(const moe_problem *p, const moe_weights *w, const void *x, void *out,
+                       float *routing_weights, int64_t *selected_experts, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* moe_forward, recording stage_events[i] before stage i and
+ * stage_events[MOE_NUM_STAGES] after the last one (MOE_NUM_STAGES + 1
+ * caller-created events; a NULL entry is skipped). */
+moe_status moe_forward_profiled(const moe_problem *p, const moe_weights *w, const void *x, void *out,
+                                float *routing_weights, int64_t *selected_experts, void *ws,
+                                size_t ws_bytes, moe_stream_t stream, moe_event_t *stage_events);
+
+/* Which expert-GEMM implementation serves problem p: 1 = tcgen05/TMEM tensor
+ * core path (bf16), 0 = SIMT fp32 path. Host only. */
+moe_status moe_gemm_path(const moe_problem *p, int32_t *path);
+
+/* Synchronise `stream`, read the workspace error bits into *code (host
+ * pointer), clear them. Returns MOE_ERR_DEVICE_FLAG when any bit was set. */
+moe_status moe_read_device_error(void *ws, int32_t *code, moe_stream_t stream);
+
+/* Static description of a status code. */
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STM_MOE_H */

@@ -1,0 +1,369 @@
+// C ABI of the sparse top-k MoE FFN forward: argument validation, workspace
+// layout and the launch sequence. Declarations and per-call contracts are in
+// include/moe.h.
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+#define MOE_API extern "C" __attribute__((visibility("default")))
+
+namespace stm {
+namespace {
+
+// ---- workspace layout --------------------------------------------------------
+struct Layout {
+  size_t header, logits, gamma, local, counts, offsets, sorted_pairs, pair_pos, x_perm, h, y_perm, h_shared,
+      shared_out, total;
+  RouterSplit split;
+  int64_t Ecols;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+Layout make_layout(const moe_problem& p) {
+  Layout L;
+  const size_t es = p.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  const int64_t P = p.T * p.k;
+  L.Ecols = p.E + (p.shared == MOE_SHARED_SIGMOID_GATED ? 1 : 0);
+  L.split = router_split(std::max<int64_t>(p.T, 1), p.H, L.Ecols);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.header = take(sizeof(WsHeader));
+  // Router partial sums, for the routed columns alone or with the gate column.
+  size_t logit_bytes = 0;
+  for (int64_t ec = p.E; ec <= p.E + 1; ++ec) {
+    const RouterSplit sp = router_split(std::max<int64_t>(p.T, 1), p.H, ec);
+    logit_bytes = std::max(logit_bytes, (size_t)sp.splits * p.T * ec * 4);
+  }
+  L.logits = take(logit_bytes);
+  L.gamma = take((size_t)p.T * 4);
+  L.local = take((size_t)dispatch_num_blocks(p.T, p.k) * p.E * 4);
+  L.counts = take((size_t)p.E * 4);
+  L.offsets = take((size_t)(p.E + 1) * 4);
+  L.sorted_pairs = take((size_t)P * 4);
+  L.pair_pos = take((size_t)P * 4);
+  L.x_perm = take((size_t)P * p.H * es);
+  L.h = take((size_t)P * p.I * es);
+  L.y_perm = take((size_t)P * p.H * 4);  // fp32
+  const bool sh = p.shared != MOE_SHARED_NONE;
+  L.h_shared = take(sh ? (size_t)p.T * p.I_shared * es : 0);
+  L.shared_out = take(sh ? (size_t)p.T * p.H * 4 : 0);  // fp32
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ---- validation ---------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+
+moe_status validate_problem(const moe_problem* p) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->T < 0 || p->H <= 0 || p->I <= 0 || p->E < 1 || p->k < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->E > kMaxExperts || p->k > p->E) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->H % 8 != 0 || p->I % 8 != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->dtype != MOE_DTYPE_F32 && p->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->score < 0 || p->score > 2 || p->bias_mode < 0 || p->bias_mode > 2) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->shared < 0 || p->shared > 2 || p->reserved != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->shared != MOE_SHARED_NONE && (p->I_shared <= 0 || p->I_shared % 8 != 0)) return MOE_ERR_INVALID_ARGUMENT;
+  // 32-bit pair indices and TMA coordinates.
+  if (p->T * p->k >= (int64_t(1) << 31) || p->H >= (int64_t(1) << 31) || p->I >= (int64_t(1) << 31))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_problem& p, const void* ws, size_t ws_bytes, Layout* L) {
+  *L = make_layout(p);
+  if (!ok_ptr(ws)) return MOE_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < L->total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                         \
+  do {                                        \
+    const moe_status _st = (expr);            \
+    if (_st != MOE_OK) return _st;            \
+  } while (0)
+
+#define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
+
+// ---- stage implementations (arguments already validated) ----------------------
+moe_status do_route(const moe_problem& p, const Layout& L, const void* x, const void* gate_w, const float* bias,
+                    const void* shared_gate, float* weights, int64_t* selected, float* gamma, void* ws,
+                    cudaStream_t s) {
+  float* partial = at<float>(ws, L.logits);
+  const int64_t Ecols = shared_gate ? p.E + 1 : p.E;
+  const RouterSplit sp = router_split(std::max<int64_t>(p.T, 1), p.H, Ecols);
+  MOE_CUDA(launch_router_logits(p.dtype, x, gate_w, shared_gate, partial, p.T, p.H, p.E, Ecols, sp, s));
+  MOE_CUDA(launch_topk(partial, sp.splits, p.T, p.E, Ecols, p.k, p.score, p.bias_mode, p.renormalize ? 1 : 0,
+                       bias, weights, selected, shared_gate ? gamma : nullptr, s));
+  return MOE_OK;
+}
+
+moe_status do_dispatch(const moe_problem& p, const Layout& L, const int64_t* selected, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos, void* x_perm,
+                       void* ws, cudaStream_t s) {
+  MOE_CUDA(launch_dispatch(p.dtype, selected, x, p.T, p.H, p.E, p.k, at<int32_t>(ws, L.local), counts, offsets,
+                           sorted_pairs, pair_pos, x_perm, at<int32_t>(ws, L.header), s));
+  return MOE_OK;
+}
+
+moe_status do_grouped_gate_up(const moe_problem& p, const Layout& L, const void* x_perm, const int32_t* offsets,
+                              const void* gate_up, void* ws, cudaStream_t s) {
+  Segments sg{offsets, (int32_t)p.E, 0, p.T * p.k};
+  void* h = at<void>(ws, L.h);
+  if (p.dtype == MOE_DTYPE_F32)
+    MOE_CUDA(launch_simt_gate_up(sg, (const float*)x_perm, (const float*)gate_up, (float*)h, p.I, p.H,
+                                 at<int32_t>(ws, L.header), s));
+  else
+    MOE_CUDA(launch_tc_gate_up(sg, x_perm, gate_up, p.E, h, p.I, p.H, at<int32_t>(ws, L.header), s));
+  return MOE_OK;
+}
+
+moe_status do_grouped_down(const moe_problem& p, const Layout& L, const int32_t* offsets, const void* down,
+                           const float* weights, const int32_t* sorted_pairs, void* y_perm, void* ws,
+                           cudaStream_t s) {
+  Segments sg{offsets, (int32_t)p.E, 0, p.T * p.k};
+  const void* h = at<void>(ws, L.h);
+  if (p.dtype == MOE_DTYPE_F32)
+    MOE_CUDA(launch_simt_down(sg, (const float*)h, (const float*)down, (float*)y_perm, weights, sorted_pairs, p.H,
+                              p.I, at<int32_t>(ws, L.header), s));
+  else
+    MOE_CUDA(launch_tc_down(sg, h, down, p.E, y_perm, weights, sorted_pairs, p.H, p.I, at<int32_t>(ws, L.header),
+                            s));
+  return MOE_OK;
+}
+
+moe_status do_shared(const moe_problem& p, const Layout& L, const void* x, const void* sgu, const void* sdn,
+                     const float* gamma, void* shared_out, void* ws, cudaStream_t s) {
+  Segments sg{nullptr, 1, (int32_t)p.T, p.T};
+  void* hs = at<void>(ws, L.h_shared);
+  if (p.dtype == MOE_DTYPE_F32) {
+    int32_t* err = at<int32_t>(ws, L.header);
+    MOE_CUDA(launch_simt_gate_up(sg, (const float*)x, (const float*)sgu, (float*)hs, p.I_shared, p.H, err, s));
+    MOE_CUDA(launch_simt_down(sg, (const float*)hs, (const float*)sdn, (float*)shared_out, gamma, nullptr, p.H,
+                              p.I_shared, err, s));
+  } else {
+    int32_t* err = at<int32_t>(ws, L.header);
+    MOE_CUDA(launch_tc_gate_up(sg, x, sgu, 1, hs, p.I_shared, p.H, err, s));
+    MOE_CUDA(launch_tc_down(sg, hs, sdn, 1, shared_out, gamma, nullptr, p.H, p.I_shared, err, s));
+  }
+  return MOE_OK;
+}
+
+moe_status validate_weights(const moe_problem& p, const moe_weights* w) {
+  if (w == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ok_ptr(w->gate_w) || !ok_ptr(w->gate_up) || !ok_ptr(w->down)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((p.bias_mode != MOE_BIAS_NONE) != (w->bias != nullptr) || !ok_opt(w->bias)) return MOE_ERR_INVALID_ARGUMENT;
+  if (p.shared != MOE_SHARED_NONE) {
+    if (!ok_ptr(w->shared_gate_up) || !ok_ptr(w->shared_down)) return MOE_ERR_INVALID_ARGUMENT;
+  }
+  if ((p.shared == MOE_SHARED_SIGMOID_GATED) != (w->shared_gate != nullptr) || !ok_opt(w->shared_gate))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return MOE_OK;
+}
+
+moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* x, void* out, float* weights,
+                        int64_t* selected, void* ws, size_t ws_bytes, cudaStream_t s, cudaEvent_t* ev) {
+  MOE_TRY(validate_problem(p));
+  MOE_TRY(validate_weights(*p, w));
+  if (p->T == 0) return MOE_OK;
+  if (!ok_ptr(x) || !ok_ptr(out) || !ok_ptr(weights) || !ok_ptr(selected)) return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  auto mark = [&](int i) -> moe_status {
+    if (ev != nullptr && ev[i] != nullptr) return cuda_status(cudaEventRecord(ev[i], s));
+    return MOE_OK;
+  };
+  const bool gated = p->shared == MOE_SHARED_SIGMOID_GATED;
+  float* gamma = at<float>(ws, L.gamma);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* sorted_pairs = at<int32_t>(ws, L.sorted_pairs);
+  int32_t* pair_pos = at<int32_t>(ws, L.pair_pos);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  void* shared_out = p->shared != MOE_SHARED_NONE ? at<void>(ws, L.shared_out) : nullptr;
+
+  MOE_TRY(mark(MOE_STAGE_ROUTE));
+  MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, gated ? w->shared_gate : nullptr, weights, selected, gamma, ws,
+                   s));
+  MOE_TRY(mark(MOE_STAGE_DISPATCH));
+  MOE_TRY(do_dispatch(*p, L, selected, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws, s));
+  MOE_TRY(mark(MOE_STAGE_GATE_UP));
+  MOE_TRY(do_grouped_gate_up(*p, L, x_perm, offsets, w->gate_up, ws, s));
+  MOE_TRY(mark(MOE_STAGE_DOWN));
+  MOE_TRY(do_grouped_down(*p, L, offsets, w->down, weights, sorted_pairs, y_perm, ws, s));
+  MOE_TRY(mark(MOE_STAGE_SHARED));
+  if (shared_out != nullptr)
+    MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, gated ? gamma : nullptr, shared_out, ws, s));
+  MOE_TRY(mark(MOE_STAGE_COMBINE));
+  MOE_CUDA(launch_combine(p->dtype, (const float*)y_perm, pair_pos, (const float*)shared_out, out, p->T, p->H,
+                          p->k, s));
+  MOE_TRY(mark(MOE_NUM_STAGES));
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace stm
+
+using namespace stm;
+
+MOE_API moe_status moe_workspace_size(const moe_problem* p, size_t* bytes) {
+  MOE_TRY(validate_problem(p));
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  *bytes = make_layout(*p).total;
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ok_ptr(ws) || ws_bytes < sizeof(WsHeader)) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream));
+}
+
+MOE_API moe_status moe_route(const moe_problem* p, const void* x, const void* gate_w, const float* bias,
+                             const void* shared_gate, float* routing_weights, int64_t* selected_experts,
+                             float* shared_gamma, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->T == 0) return MOE_OK;
+  if (!ok_ptr(x) || !ok_ptr(gate_w) || !ok_ptr(routing_weights) || !ok_ptr(selected_experts))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if ((p->bias_mode != MOE_BIAS_NONE) != (bias != nullptr) || !ok_opt(bias)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((shared_gate != nullptr) != (shared_gamma != nullptr) || !ok_opt(shared_gate) || !ok_opt(shared_gamma))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (shared_gate != nullptr && p->shared != MOE_SHARED_SIGMOID_GATED) return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  return do_route(*p, L, x, gate_w, bias, shared_gate, routing_weights, selected_experts, shared_gamma, ws,
+                  (cudaStream_t)stream);
+}
+
+MOE_API moe_status moe_topk_from_logits(const moe_problem* p, const float* logits, const float* bias,
+                                        float* routing_weights, int64_t* selected_experts, moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->T == 0) return MOE_OK;
+  if (!ok_ptr(logits) || !ok_ptr(routing_weights) || !ok_ptr(selected_experts)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((p->bias_mode != MOE_BIAS_NONE) != (bias != nullptr) || !ok_opt(bias)) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_topk(logits, 1, p->T, p->E, p->E, p->k, p->score, p->bias_mode, p->renormalize ? 1 : 0,
+                                 bias, routing_weights, selected_experts, nullptr, (cudaStream_t)stream));
+}
+
+MOE_API moe_status moe_dispatch(const moe_problem* p, const int64_t* selected_experts, const void* x,
+                                int32_t* counts, int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
+                                void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (!ok_ptr(counts) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->T == 0) {
+    // Empty batch: every segment is empty.
+    MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)p->E * 4, (cudaStream_t)stream));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(p->E + 1) * 4, (cudaStream_t)stream));
+    return MOE_OK;
+  }
+  if (!ok_ptr(selected_experts) || !ok_ptr(sorted_pairs) || !ok_ptr(pair_pos)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((x == nullptr) != (x_perm == nullptr) || !ok_opt(x) || !ok_opt(x_perm)) return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  return do_dispatch(*p, L, selected_experts, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws,
+                     (cudaStream_t)stream);
+}
+
+MOE_API moe_status moe_grouped_swiglu(const moe_problem* p, const void* x_perm, const int32_t* offsets,
+                                      const void* gate_up, const void* down, const float* routing_weights,
+                                      const int32_t* sorted_pairs, void* y_perm, void* ws, size_t ws_bytes,
+                                      moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->T == 0) return MOE_OK;
+  if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(gate_up) || !ok_ptr(down) || !ok_ptr(y_perm))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if ((routing_weights == nullptr) != (sorted_pairs == nullptr) || !ok_opt(routing_weights) || !ok_opt(sorted_pairs))
+    return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  const cudaStream_t s = (cudaStream_t)stream;
+  MOE_TRY(do_grouped_gate_up(*p, L, x_perm, offsets, gate_up, ws, s));
+  return do_grouped_down(*p, L, offsets, down, routing_weights, sorted_pairs, y_perm, ws, s);
+}
+
+MOE_API moe_status moe_shared_expert(const moe_problem* p, const void* x, const void* shared_gate_up,
+                                     const void* shared_down, const float* shared_gamma, void* shared_out, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->shared == MOE_SHARED_NONE) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->T == 0) return MOE_OK;
+  if (!ok_ptr(x) || !ok_ptr(shared_gate_up) || !ok_ptr(shared_down) || !ok_ptr(shared_out) || !ok_opt(shared_gamma))
+    return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  return do_shared(*p, L, x, shared_gate_up, shared_down, shared_gamma, shared_out, ws, (cudaStream_t)stream);
+}
+
+MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* pair_pos,
+                               const void* shared_out, void* out, moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->T == 0) return MOE_OK;
+  if (!ok_ptr(y_perm) || !ok_ptr(pair_pos) || !ok_opt(shared_out) || !ok_ptr(out)) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_combine(p->dtype, (const float*)y_perm, pair_pos, (const float*)shared_out, out, p->T,
+                                    p->H, p->k, (cudaStream_t)stream));
+}
+
+MOE_API moe_status moe_forward(const moe_problem* p, const moe_weights* w, const void* x, void* out,
+                               float* routing_weights, int64_t* selected_experts, void* ws, size_t ws_bytes,
+                               moe_stream_t stream) {
+  return forward_impl(p, w, x, out, routing_weights, selected_experts, ws, ws_bytes, (cudaStream_t)stream, nullptr);
+}
+
+MOE_API moe_status moe_forward_profiled(const moe_problem* p, const moe_weights* w, const void* x, void* out,
+                                        float* routing_weights, int64_t* selected_experts, void* ws,
+                                        size_t ws_bytes, moe_stream_t stream, moe_event_t* stage_events) {
+  return forward_impl(p, w, x, out, routing_weights, selected_experts, ws, ws_bytes, (cudaStream_t)stream,
+                      reinterpret_cast<cudaEvent_t*>(stage_events));
+}
+
+MOE_API moe_status moe_gemm_path(const moe_problem* p, int32_t* path) {
+  MOE_TRY(validate_problem(p));
+  if (path == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  *path = p->dtype == MOE_DTYPE_BF16 ? 1 : 0;
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_read_device_error(void* ws, int32_t* code, moe_stream_t stream) {
+  if (!ok_ptr(ws) || code == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  const cudaStream_t s = (cudaStream_t)stream;
+  WsHeader h;
+  MOE_CUDA(cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaStreamSynchronize(s));
+  *code = h.error_bits;
+  if (h.error_bits != 0) {
+    MOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(WsHeader), s));
+    MOE_CUDA(cudaStreamSynchronize(s));
+    return MOE_ERR_DEVICE_FLAG;
+  }
+  return MOE_OK;
+}
+
+MOE_API const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported combination";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_FLAG: return "device-side error flag set";
+  }
+  return "unknown status";
+}

@@ -1,0 +1,104 @@
+"""The C-ABI library loads, exports every symbol include/moe.h declares, and
+its host-side validation behaves (no GPU: only calls that return before any
+CUDA work)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_top_mixture_b200 as stm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(moe_\w+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(stm.LIB_PATH):
+        stm.build_lib = __import__("sparse_top_mixture_b200.build", fromlist=["build"])
+        stm.build_lib.build()
+    return stm.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    syms = header_symbols()
+    assert len(syms) >= 13
+    for s in syms:
+        assert hasattr(L, s), f"{s} declared in include/ but not exported"
+    assert set(syms) == set(stm.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_status_strings(L):
+    assert L.moe_status_string(0) == b"ok"
+    assert b"workspace" in L.moe_status_string(3)
+    assert L.moe_status_string(99) == b"unknown status"
+
+
+def _p(**kw):
+    base = dict(T=64, H=256, E=8, k=2, I=128, dtype="bf16")
+    base.update(kw)
+    return stm.Problem(**base)
+
+
+def test_workspace_size_grows_with_problem(L):
+    a = stm.workspace_size(_p())
+    b = stm.workspace_size(_p(T=128))
+    c = stm.workspace_size(_p(shared="plain", I_shared=256))
+    assert 0 < a < b and a < c
+    # x_perm + h + y_perm dominate
+    assert a >= 64 * 2 * (256 + 128 + 256) * 2
+
+
+@pytest.mark.parametrize("bad", [
+    dict(k=0), dict(k=9), dict(E=0), dict(E=257, k=2), dict(H=250), dict(I=100), dict(T=-1),
+    dict(dtype="f32", shared="plain", I_shared=0), dict(shared="plain", I_shared=12),
+])
+def test_invalid_problems_rejected(L, bad):
+    with pytest.raises(stm.MoeError) as ei:
+        stm.workspace_size(_p(**bad))
+    assert ei.value.status == 1
+
+
+def test_gemm_path(L):
+    assert stm.gemm_path(_p()) == 1
+    assert stm.gemm_path(_p(dtype="f32")) == 0
+
+
+def test_calls_validate_before_launching(L):
+    p = _p().c()
+    # null / misaligned pointers are rejected on the host, before any CUDA call
+    st = L.moe_route(ctypes.byref(p), None, None, None, None, None, None, None, None, 0, None)
+    assert st == 1
+    # x given without x_perm
+    st = L.moe_dispatch(ctypes.byref(p), 16, 16, 16, 16, 16, 16, None, 16, 1 << 30, None)
+    assert st == 1
+    st = L.moe_combine(ctypes.byref(p), 8, 16, None, 16, None)
+    assert st == 1  # y_perm misaligned
+    # workspace too small
+    st = L.moe_grouped_swiglu(ctypes.byref(p), 16, 16, 16, 16, None, None, 16, 16, 1024, None)
+    assert st == 3
+    # bias mode without a bias
+    pb = _p(bias_mode="select").c()
+    st = L.moe_topk_from_logits(ctypes.byref(pb), 16, None, 16, 16, None)
+    assert st == 1
+
+
+def test_empty_batch_is_a_noop(L):
+    """T == 0 returns OK without launching anything (no GPU needed)."""
+    p = _p(T=0).c()
+    w = stm.moe_weights(16, None, 16, 16, None, None, None)
+    n = ctypes.c_size_t(0)
+    assert L.moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    st = L.moe_forward(ctypes.byref(p), ctypes.byref(w), 16, 16, 16, 16, 16, n.value, None)
+    assert st == 0

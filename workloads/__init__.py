@@ -139,11 +139,17 @@ def load_zipf_bias(E: int) -> torch.Tensor:
     return torch.tensor(d["bias_fp32"], dtype=torch.float32)
 
 
-def router_inputs(cfg: MoEConfig) -> Dict[str, Optional[torch.Tensor]]:
-    """x, gate_w, bias and shared gate vector, always drawn on the CPU."""
+def router_inputs(cfg: MoEConfig, rank: int = 0) -> Dict[str, Optional[torch.Tensor]]:
+    """x, gate_w, bias and shared gate vector, always drawn on the CPU.
+
+    ``rank`` selects an independent batch of hidden states (data-parallel
+    replicas share every weight); rank 0 is the problem's own batch."""
     dt = _torch_dtype(cfg)
     out: Dict[str, Optional[torch.Tensor]] = {}
-    out["x"] = _normal((cfg.T, cfg.H), 1.0, _gen(cfg, "x", "cpu"), "cpu", dt)
+    gx = _gen(cfg, "x", "cpu")
+    if rank:
+        gx.manual_seed(cfg.seed * 1000 + _TID["x"] + 100003 * rank)
+    out["x"] = _normal((cfg.T, cfg.H), 1.0, gx, "cpu", dt)
     out["gate_w"] = _normal((cfg.E, cfg.H), cfg.H ** -0.5, _gen(cfg, "gate_w", "cpu"), "cpu", dt)
     if cfg.bias_kind == "none":
         out["bias"] = None
