@@ -132,9 +132,9 @@ def flops_and_bytes(cfg, n_active: int):
 
 
 def launches_per_step(cfg) -> int:
-    # router logits + top-k; histogram + scan + permute; gate_up + down; shared
-    # gate_up + down; combine
-    return 2 + 3 + 2 + (2 if cfg.shared != "none" else 0) + 1
+    # router logits + top-k; histogram + scan + permute + gather; gate_up +
+    # down; shared gate_up + down; combine
+    return 2 + 4 + 2 + (2 if cfg.shared != "none" else 0) + 1
 
 
 def recorded_traffic(cfg_name: str):

@@ -18,8 +18,6 @@ namespace {
 struct Layout {
   size_t header, logits, gamma, local, counts, offsets, sorted_pairs, pair_pos, x_perm, h, y_perm, h_shared,
       shared_out, total;
-  RouterSplit split;
-  int64_t Ecols;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -28,8 +26,6 @@ Layout make_layout(const moe_problem& p) {
   Layout L;
   const size_t es = p.dtype == MOE_DTYPE_F32 ? 4 : 2;
   const int64_t P = p.T * p.k;
-  L.Ecols = p.E + (p.shared == MOE_SHARED_SIGMOID_GATED ? 1 : 0);
-  L.split = router_split(std::max<int64_t>(p.T, 1), p.H, L.Ecols);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -37,13 +33,7 @@ Layout make_layout(const moe_problem& p) {
     return at;
   };
   L.header = take(sizeof(WsHeader));
-  // Router partial sums, for the routed columns alone or with the gate column.
-  size_t logit_bytes = 0;
-  for (int64_t ec = p.E; ec <= p.E + 1; ++ec) {
-    const RouterSplit sp = router_split(std::max<int64_t>(p.T, 1), p.H, ec);
-    logit_bytes = std::max(logit_bytes, (size_t)sp.splits * p.T * ec * 4);
-  }
-  L.logits = take(logit_bytes);
+  L.logits = take(router_partial_bytes(p.dtype, p.T, p.H, p.E));
   L.gamma = take((size_t)p.T * 4);
   L.local = take((size_t)dispatch_num_blocks(p.T, p.k) * p.E * 4);
   L.counts = take((size_t)p.E * 4);
@@ -106,12 +96,9 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 moe_status do_route(const moe_problem& p, const Layout& L, const void* x, const void* gate_w, const float* bias,
                     const void* shared_gate, float* weights, int64_t* selected, float* gamma, void* ws,
                     cudaStream_t s) {
-  float* partial = at<float>(ws, L.logits);
-  const int64_t Ecols = shared_gate ? p.E + 1 : p.E;
-  const RouterSplit sp = router_split(std::max<int64_t>(p.T, 1), p.H, Ecols);
-  MOE_CUDA(launch_router_logits(p.dtype, x, gate_w, shared_gate, partial, p.T, p.H, p.E, Ecols, sp, s));
-  MOE_CUDA(launch_topk(partial, sp.splits, p.T, p.E, Ecols, p.k, p.score, p.bias_mode, p.renormalize ? 1 : 0,
-                       bias, weights, selected, shared_gate ? gamma : nullptr, s));
+  MOE_CUDA(launch_route(p.dtype, x, gate_w, shared_gate, bias, p.T, p.H, p.E, p.k, p.score, p.bias_mode,
+                        p.renormalize ? 1 : 0, at<float>(ws, L.logits), weights, selected, gamma,
+                        at<int32_t>(ws, L.header), s));
   return MOE_OK;
 }
 
@@ -259,8 +246,9 @@ MOE_API moe_status moe_topk_from_logits(const moe_problem* p, const float* logit
   if (p->T == 0) return MOE_OK;
   if (!ok_ptr(logits) || !ok_ptr(routing_weights) || !ok_ptr(selected_experts)) return MOE_ERR_INVALID_ARGUMENT;
   if ((p->bias_mode != MOE_BIAS_NONE) != (bias != nullptr) || !ok_opt(bias)) return MOE_ERR_INVALID_ARGUMENT;
-  return cuda_status(launch_topk(logits, 1, p->T, p->E, p->E, p->k, p->score, p->bias_mode, p->renormalize ? 1 : 0,
-                                 bias, routing_weights, selected_experts, nullptr, (cudaStream_t)stream));
+  return cuda_status(launch_topk(logits, 1, p->E, p->T, p->E, p->k, p->score, p->bias_mode, p->renormalize ? 1 : 0,
+                                 bias, routing_weights, selected_experts, nullptr, nullptr, p->H, p->dtype, nullptr,
+                                 (cudaStream_t)stream));
 }
 
 MOE_API moe_status moe_dispatch(const moe_problem* p, const int64_t* selected_experts, const void* x,
@@ -337,7 +325,13 @@ MOE_API moe_status moe_forward_profiled(const moe_problem* p, const moe_weights*
 MOE_API moe_status moe_gemm_path(const moe_problem* p, int32_t* path) {
   MOE_TRY(validate_problem(p));
   if (path == nullptr) return MOE_ERR_INVALID_ARGUMENT;
-  *path = p->dtype == MOE_DTYPE_BF16 ? 1 : 0;
+  if (p->dtype != MOE_DTYPE_BF16) {
+    *path = 0;
+  } else {
+    Segments sg{nullptr, (int32_t)p->E, 0, p->T * p->k};
+    sg.offsets = reinterpret_cast<const int32_t*>(16);  // any non-null: routed segments
+    *path = tc_gemm_variant(sg);
+  }
   return MOE_OK;
 }
 

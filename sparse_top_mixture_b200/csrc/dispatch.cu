@@ -12,9 +12,12 @@
 //   2. one block turns the [blocks x E] counts into segment offsets and the
 //      base position of every (block, expert) run;
 //   3. each block ranks its pairs inside each expert run in pair order (warp
-//      match + prefix counts across warps), writes the permutation and its
-//      inverse, then copies each token row once into its k destinations with
-//      16-byte vector loads and stores.
+//      match + prefix counts across warps) and writes the permutation and its
+//      inverse;
+//   4. the gather reads each token row once and writes it to its k segment
+//      slots with 16-byte vector loads and stores; its work units are
+//      (token, 4 KB column chunk) so that a 16-token decode batch still spreads
+//      over many SMs.
 // Every block handles whole tokens and at most 256 pairs, so the ranking is a
 // single pass. Counts are order-independent and positions are a pure function
 // of the pair order: the result is deterministic.
@@ -45,45 +48,86 @@ __global__ void __launch_bounds__(DTHREADS) hist_kernel(const int64_t* __restric
 }
 
 // One block: counts, offsets, and (in place) per-(block, expert) base positions.
-__global__ void __launch_bounds__(DTHREADS) scan_kernel(int32_t* __restrict__ local, int nblk, int E,
-                                                        int32_t* __restrict__ counts,
-                                                        int32_t* __restrict__ offsets) {
-  __shared__ int s[DTHREADS];
-  const int e = threadIdx.x;
-  int run = 0;
-  if (e < E) {
-    for (int b = 0; b < nblk; ++b) {
-      const int v = local[(int64_t)b * E + e];
-      local[(int64_t)b * E + e] = run;
-      run += v;
+// Each expert's column of the [blocks x E] count matrix is split among `tpe`
+// threads of one warp (tpe = 4..32), which read their ranges with independent
+// loads, combine through a segmented warp scan, and write the running bases.
+constexpr int SCAN_THREADS = 1024;
+
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict__ local, int nblk, int E,
+                                                            int tpe, int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+  __shared__ int tot[kMaxExperts];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int e = tid / tpe, part = tid % tpe;
+  const bool active = e < E;
+  const int chunk = (nblk + tpe - 1) / tpe;
+  const int b0 = min(nblk, part * chunk), b1 = min(nblk, b0 + chunk);
+  int sum = 0;
+  if (active) {
+    for (int b = b0; b < b1; b += 8) {
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? local[(int64_t)(b + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += v[i];
     }
   }
-  s[e] = (e < E) ? run : 0;
+  // segmented inclusive scan over the tpe parts of one expert (same warp)
+  int incl = sum;
+  for (int o = 1; o < tpe; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (part >= o) incl += v;
+  }
+  if (active && part == tpe - 1) tot[e] = incl;
   __syncthreads();
-  for (int o = 1; o < DTHREADS; o <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = (e >= o) ? s[e - o] : 0;
-    __syncthreads();
-    s[e] += v;
-    __syncthreads();
+  if (tid < 32) {  // exclusive scan of the expert totals, 8 per lane
+    int c[8], loc = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      c[i] = ee < E ? tot[ee] : 0;
+      loc += c[i];
+    }
+    int inc = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (tid >= o) inc += v;
+    }
+    int run = inc - loc;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      if (ee < E) {
+        counts[ee] = c[i];
+        offsets[ee] = run;
+        tot[ee] = run;
+      }
+      run += c[i];
+    }
+    if (tid == 31) offsets[E] = inc;
   }
-  const int excl = s[e] - ((e < E) ? run : 0);
-  if (e < E) {
-    counts[e] = run;
-    offsets[e] = excl;
-    for (int b = 0; b < nblk; ++b) local[(int64_t)b * E + e] += excl;
+  __syncthreads();
+  if (!active) return;
+  int run = tot[e] + incl - sum;
+  for (int b = b0; b < b1; b += 8) {
+    int v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? local[(int64_t)(b + i) * E + e] : 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (b + i < b1) local[(int64_t)(b + i) * E + e] = run;
+      run += v[i];
+    }
   }
-  if (e == DTHREADS - 1) offsets[E] = s[e];
 }
 
-template <typename T>
 __global__ void __launch_bounds__(DTHREADS) permute_kernel(const int64_t* __restrict__ sel, int64_t P, int k,
                                                            int E, int tok_per_blk,
                                                            const int32_t* __restrict__ bases,
                                                            int32_t* __restrict__ sorted_pairs,
-                                                           int32_t* __restrict__ pair_pos, const T* __restrict__ x,
-                                                           T* __restrict__ x_perm, int H) {
+                                                           int32_t* __restrict__ pair_pos) {
   __shared__ int wcnt[DTHREADS / 32][kMaxExperts];
-  __shared__ int pos_s[DTHREADS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < (DTHREADS / 32) * kMaxExperts; i += DTHREADS) (&wcnt[0][0])[i] = 0;
   __syncthreads();
@@ -117,20 +161,35 @@ __global__ void __launch_bounds__(DTHREADS) permute_kernel(const int64_t* __rest
     sorted_pairs[pos] = (int32_t)q;
   }
   if (active) pair_pos[q] = pos;
-  pos_s[tid] = pos;
-  __syncthreads();
+}
 
-  if (x_perm == nullptr) return;
+// x_perm[pair_pos[t*k + j]] = x[t] for every token t and slot j.
+constexpr int GCHUNK = 256;  // 16-byte vectors per work unit
+
+template <typename T>
+__global__ void __launch_bounds__(DTHREADS) gather_kernel(const T* __restrict__ x, const int32_t* __restrict__ pair_pos,
+                                                          T* __restrict__ x_perm, int64_t Tn, int H, int k) {
   constexpr int V = Elem<T>::kPerVec;
   const int nvec = H / V;
-  const int ntok = (int)((q1 - q0) / k);
-  const int64_t t0 = q0 / k;
-  for (int tt = warp; tt < ntok; tt += DTHREADS / 32) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + (t0 + tt) * (int64_t)H);
-    for (int v = lane; v < nvec; v += 32) {
+  const int nchunk = (nvec + GCHUNK - 1) / GCHUNK;
+  const int64_t units = Tn * nchunk;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * DTHREADS + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * DTHREADS) >> 5;
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t t = u / nchunk;
+    const int c0 = (int)(u - t * nchunk) * GCHUNK;
+    const int c1 = min(nvec, c0 + GCHUNK);
+    int pos[8];
+    const int kk = min(k, 8);
+    for (int j = 0; j < kk; ++j) pos[j] = pair_pos[t * k + j];
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * (int64_t)H);
+    for (int v = c0 + lane; v < c1; v += 32) {
       const uint4 val = src[v];
-      for (int j = 0; j < k; ++j) {
-        const int p = pos_s[tt * k + j];
+      for (int j = 0; j < kk; ++j)
+        if (pos[j] >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)pos[j] * H)[v] = val;
+      for (int j = 8; j < k; ++j) {
+        const int p = pair_pos[t * k + j];
         if (p >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)p * H)[v] = val;
       }
     }
@@ -191,14 +250,21 @@ cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, i
   const int nblk = (int)dispatch_num_blocks(T, k);
   const int64_t P = T * k;
   hist_kernel<<<nblk, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, err);
-  scan_kernel<<<1, DTHREADS, 0, s>>>(local, nblk, (int)E, counts, offsets);
-  if (dtype == 0)
-    permute_kernel<float><<<nblk, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos,
-                                                    (const float*)x, (float*)x_perm, (int)H);
-  else
-    permute_kernel<__nv_bfloat16><<<nblk, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, sorted_pairs,
-                                                            pair_pos, (const __nv_bfloat16*)x,
-                                                            (__nv_bfloat16*)x_perm, (int)H);
+  int ep = 1;
+  while (ep < E) ep <<= 1;
+  const int tpe = std::min(32, SCAN_THREADS / ep);
+  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(local, nblk, (int)E, tpe, counts, offsets);
+  permute_kernel<<<nblk, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos);
+  if (x_perm != nullptr) {
+    const int V = dtype == 0 ? 4 : 8;
+    const int64_t units = T * ceil_div(H / V, GCHUNK);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, DTHREADS / 32), 148 * 16));
+    if (dtype == 0)
+      gather_kernel<float><<<grid, DTHREADS, 0, s>>>((const float*)x, pair_pos, (float*)x_perm, T, (int)H, (int)k);
+    else
+      gather_kernel<__nv_bfloat16><<<grid, DTHREADS, 0, s>>>((const __nv_bfloat16*)x, pair_pos,
+                                                             (__nv_bfloat16*)x_perm, T, (int)H, (int)k);
+  }
   return cudaGetLastError();
 }
 

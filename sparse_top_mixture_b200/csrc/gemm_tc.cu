@@ -40,10 +40,14 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tiles.cuh"
+#include "tc_ptx.cuh"
+#include "tc_epilogue.cuh"
 
 namespace stm {
 
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BK = 64;          // 64 bf16 = 128 bytes = one swizzle row
@@ -55,9 +59,8 @@ constexpr int B_BYTES = UMMA_N * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * UMMA_N;
 constexpr int NTHREADS = 192;
-constexpr long long kWaitLimitCycles = 2000000000LL;
 
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
 
 struct Args {
   const int32_t* offsets;
@@ -65,7 +68,10 @@ struct Args {
   int32_t single_rows;
   int32_t N;        // output columns
   int32_t n_tiles;  // column tiles per row tile
-  int32_t k_tiles;
+  int32_t k_tiles;  // BK-deep k-steps over the whole K
+  int32_t k_splits; // independent partial sums along K (LOGITS only; else 1)
+  int32_t kps;      // k-steps per split
+  int64_t ldo;      // output row pitch in elements
   void* out;  // gate_up: bf16 h; down: fp32 y
   const float* row_scale;
   const int32_t* scale_idx;
@@ -87,168 +93,29 @@ struct __align__(8) Ctl {
 
 constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctl);
 
-// ---- PTX wrappers --------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for the phase of `bar` with the given parity to complete.
-// Gives up when another role has aborted (unless draining) or after about a
-// second of SM clocks, in which case it records the error and aborts.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, Ctl* ctl, int32_t* err, int site,
-                                            bool draining) {
-  const long long start = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (!draining && *reinterpret_cast<volatile int*>(&ctl->abort)) return false;
-      if (clock64() - start > kWaitLimitCycles) {
-        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
-        if (err) {
-          atomicOr(err, 2);
-          atomicExch(err + 1, site);
-        }
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, int32_t* err, int site,
-                                          bool draining = false) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, ctl, err, site, draining);
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
-      "%6}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive on `bar` once every previously issued tcgen05.mma of this thread is done.
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row core groups 1024 bytes apart (tcgen05 descriptor format:
-// start>>4 in bits 0-13, LBO>>4 in 16-29, SBO>>4 in 32-45, version 1 in
-// 46-47, layout type 2 = SWIZZLE_128B in 61-63).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)1 << 16;
-  d |= (uint64_t)(1024 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9 and 10-12 = 1), both K-major, N>>3 in bits 17-22, M>>4 in 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(UMMA_N >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t kIdesc128 = make_idesc(128, UMMA_N);
+// M=64 tail tiles: the accumulator then occupies TMEM lanes 0-15 of each
+// 32-lane sub-partition (tile row r -> lane (r % 16) + 32 * (r / 16)).
+constexpr uint32_t kIdesc64 = make_idesc(64, UMMA_N);
 
 struct TileCoord {
-  int e, row0, row_end, n_idx;
+  int e, row0, row_end, n_idx, kt0, kt1, split;
+  bool m64;  // at most 64 rows of the segment left: M=64 MMA
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const Ctl* ctl, int Eseg, int n_tiles, int tile) {
+// Tile index -> (row tile, column tile, k split); the split varies fastest.
+__device__ __forceinline__ TileCoord decode_tile(const Ctl* ctl, int Eseg, const Args& a, int tile) {
   TileCoord c;
-  const int mt = tile / n_tiles;
-  c.n_idx = tile - mt * n_tiles;
+  c.split = tile % a.k_splits;
+  const int rest = tile / a.k_splits;
+  const int mt = rest / a.n_tiles;
+  c.n_idx = rest - mt * a.n_tiles;
+  c.kt0 = c.split * a.kps;
+  c.kt1 = min(a.k_tiles, c.kt0 + a.kps);
   c.e = find_segment(ctl->pre, Eseg, mt);
   c.row0 = ctl->off[c.e] + (mt - ctl->pre[c.e]) * BM;
   c.row_end = ctl->off[c.e + 1];
+  c.m64 = c.row_end - c.row0 <= 64;
   return c;
 }
 
@@ -283,7 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  const int total_tiles = ctl->pre[Eseg] * args.n_tiles;
+  const int total_tiles = ctl->pre[Eseg] * args.n_tiles * args.k_splits;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -293,16 +160,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t issued = 0, last_parity = 0;  // per stage: ever issued, parity of the last issue
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileCoord tc = decode_tile(ctl, Eseg, args.n_tiles, tile);
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
-          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, ctl, args.err, 1)) { ok = false; break; }
+        const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
+        for (int kt = tc.kt0; kt < tc.kt1; ++kt) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, args.err, 1)) { ok = false; break; }
           uint8_t* sa = base + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
           const int k0 = kt * BK;
           tma_load_2d(sa, &tmA, &ctl->full[stage], k0, tc.row0);
           if (MODE == MODE_GATE_UP) {
-            const int n0 = tc.n_idx * 128;
+            const int n0 = tc.n_idx * 128;  // gate rows, then the matching up rows
             tma_load_4d(sb, &tmB, &ctl->full[stage], k0, n0, 0, tc.e);
             tma_load_4d(sb + B_BYTES / 2, &tmB, &ctl->full[stage], k0, n0, 1, tc.e);
           } else {
@@ -315,7 +182,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // Drain: every copy this thread issued has landed before the CTA may exit.
       for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (last_parity >> s) & 1u, ctl, args.err, 6, true);
+        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (last_parity >> s) & 1u, &ctl->abort, args.err, 6, true);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -326,11 +193,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, ctl, args.err, 2)) break;
+        const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
+        if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
-          if (!mbar_wait(&ctl->full[stage], phase, ctl, args.err, 3)) { ok = false; break; }
+        const uint32_t idesc = tc.m64 ? kIdesc64 : kIdesc128;
+        for (int kt = tc.kt0; kt < tc.kt1; ++kt) {
+          if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, args.err, 3)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(base + stage * STAGE_BYTES);
           const uint64_t adesc = sw128_desc(sa);
@@ -338,8 +207,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
             // advance K by 16 bf16 = 32 bytes inside the swizzled 128-byte row
-            umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), kIdesc,
-                      (kt > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+                      (kt > tc.kt0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -351,68 +220,53 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // Drain: all MMAs issued here are complete before TMEM is freed.
       umma_commit(&ctl->drain);
-      mbar_wait(&ctl->drain, 0, ctl, args.err, 7, true);
+      mbar_wait(&ctl->drain, 0, &ctl->abort, args.err, 7, true);
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int r = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord tc = decode_tile(ctl, Eseg, args.n_tiles, tile);
-      if (!mbar_wait(&ctl->tfull[acc], acc_phase, ctl, args.err, 4)) break;
+      const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
+      if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, args.err, 4)) break;
       tc_fence_after();
+      const int r = tc.m64 ? quarter * 16 + lane : quarter * 32 + lane;
       const int row = tc.row0 + r;
-      const bool valid = row < tc.row_end;
+      const bool valid = row < tc.row_end && (!tc.m64 || lane < 16);
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * UMMA_N);
       if (MODE == MODE_GATE_UP) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tbase + c * 32, g);
-          tmem_ld32(tbase + 128 + c * 32, u);
-          tmem_ld_wait();
-          const int col0 = tc.n_idx * 128 + c * 32;
-          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row * args.N;
-          if (valid) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col0 + v * 8 < args.N) {
-                float hv[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                  hv[q] = silu_f32(__uint_as_float(g[v * 8 + q])) * __uint_as_float(u[v * 8 + q]);
-                uint4 o;
-                o.x = pack_bf16x2(hv[0], hv[1]);
-                o.y = pack_bf16x2(hv[2], hv[3]);
-                o.z = pack_bf16x2(hv[4], hv[5]);
-                o.w = pack_bf16x2(hv[6], hv[7]);
-                *reinterpret_cast<uint4*>(orow + col0 + v * 8) = o;
-              }
-            }
-          }
-        }
-      } else {
+        epilogue_swiglu(tbase, valid, reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row * args.ldo,
+                        tc.n_idx * 128, args.N);
+      } else if (MODE == MODE_DOWN) {
         float sc = 1.f;
         if (valid && args.row_scale != nullptr) sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
+        epilogue_scale_f32(tbase, valid, sc, reinterpret_cast<float*>(args.out) + (int64_t)row * args.ldo,
+                           tc.n_idx * UMMA_N, args.N);
+      } else {
+        // router logits: fp32 partial sum of this k split; the row pitch is a
+        // multiple of 4 floats, columns past N are not written.
+        float* orow = reinterpret_cast<float*>(args.out) + (int64_t)tc.split * args.rows_total * args.ldo +
+                      (int64_t)row * args.ldo;
 #pragma unroll 1
         for (int c = 0; c < UMMA_N / 32; ++c) {
+          const int col0 = tc.n_idx * UMMA_N + c * 32;
+          if (col0 >= args.N) break;  // warp-uniform
           uint32_t d[32];
           tmem_ld32(tbase + c * 32, d);
           tmem_ld_wait();
-          const int col0 = tc.n_idx * UMMA_N + c * 32;
-          float* orow = reinterpret_cast<float*>(args.out) + (int64_t)row * args.N;
           if (valid) {
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
-              if (col0 + v * 4 < args.N) {
-                float4 o;
-                o.x = sc * __uint_as_float(d[v * 4 + 0]);
-                o.y = sc * __uint_as_float(d[v * 4 + 1]);
-                o.z = sc * __uint_as_float(d[v * 4 + 2]);
-                o.w = sc * __uint_as_float(d[v * 4 + 3]);
-                *reinterpret_cast<float4*>(orow + col0 + v * 4) = o;
+              const int cv = col0 + v * 4;
+              if (cv + 3 < args.N) {
+                *reinterpret_cast<float4*>(orow + cv) =
+                    make_float4(__uint_as_float(d[v * 4 + 0]), __uint_as_float(d[v * 4 + 1]),
+                                __uint_as_float(d[v * 4 + 2]), __uint_as_float(d[v * 4 + 3]));
+              } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (cv + q < args.N) orow[cv + q] = __uint_as_float(d[v * 4 + q]);
               }
             }
           }
@@ -434,10 +288,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+template <int MODE>
+cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, int64_t N, int64_t K,
+                      void* out, int64_t ldo, const float* row_scale, const int32_t* scale_idx, int32_t* err,
+                      cudaStream_t s, int k_splits = 1) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(tc_grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  Args a;
+  a.offsets = sg.offsets;
+  a.E = sg.E;
+  a.single_rows = sg.single_rows;
+  a.N = (int32_t)N;
+  a.n_tiles = (int32_t)ceil_div(N, MODE == MODE_GATE_UP ? 128 : UMMA_N);
+  a.k_tiles = (int32_t)ceil_div(K, BK);
+  a.k_splits = std::max(1, k_splits);
+  a.kps = (int32_t)ceil_div(a.k_tiles, a.k_splits);
+  a.ldo = ldo;
+  a.out = out;
+  a.row_scale = row_scale;
+  a.scale_idx = scale_idx;
+  a.err = err;
+  a.rows_total = sg.rows_total;
+  const int64_t nseg = sg.offsets ? sg.E : 1;
+  const int64_t max_tiles = (sg.rows_total / BM + nseg) * a.n_tiles * a.k_splits;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
+  tc_grouped_gemm_kernel<MODE><<<grid, NTHREADS, kSmemBytes, s>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 // ---- host side -----------------------------------------------------------
 
+namespace {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
+}  // namespace
 
 bool get_encode() {
   std::call_once(g_encode_once, [] {
@@ -451,8 +342,8 @@ bool get_encode() {
   return g_encode != nullptr;
 }
 
-bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
-              const uint32_t* box) {
+bool make_tensor_map_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box) {
   const uint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUresult r =
       g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), dims, strides_bytes,
@@ -468,36 +359,12 @@ int num_sms() {
   return n;
 }
 
-template <int MODE>
-cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, int64_t N, int64_t K,
-                      void* out, const float* row_scale, const int32_t* scale_idx, int32_t* err, cudaStream_t s) {
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(tc_grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  Args a;
-  a.offsets = sg.offsets;
-  a.E = sg.E;
-  a.single_rows = sg.single_rows;
-  a.N = (int32_t)N;
-  a.n_tiles = (int32_t)ceil_div(N, MODE == MODE_GATE_UP ? 128 : UMMA_N);
-  a.k_tiles = (int32_t)ceil_div(K, BK);
-  a.out = out;
-  a.row_scale = row_scale;
-  a.scale_idx = scale_idx;
-  a.err = err;
-  a.rows_total = sg.rows_total;
+int tc_gemm_variant(const Segments& sg) {
+  // Pair tiles are 256 rows: with segments of a few hundred rows their tail
+  // padding costs more than the halved operand traffic saves.
   const int64_t nseg = sg.offsets ? sg.E : 1;
-  const int64_t max_tiles = (sg.rows_total / BM + nseg) * a.n_tiles;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
-  tc_grouped_gemm_kernel<MODE><<<grid, NTHREADS, kSmemBytes, s>>>(tmA, tmB, a);
-  return cudaGetLastError();
+  return sg.rows_total >= 384 * nseg ? 2 : 1;
 }
-
-}  // namespace
 
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                               int64_t I, int64_t H, int32_t* err, cudaStream_t s) {
@@ -507,16 +374,17 @@ cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_g
     const uint64_t dims[2] = {(uint64_t)H, (uint64_t)sg.rows_total};
     const uint64_t strides[1] = {(uint64_t)H * 2};
     const uint32_t box[2] = {BK, BM};
-    if (!make_map(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
+  if (tc_gemm_variant(sg) == 2) return launch_tc2_gate_up(sg, tmA, w_gate_up, E_w, h, I, H, err, num_sms(), s);
   {
     // gate_up [E][2][I][H]: dim0 = H, dim1 = I (row within a half), dim2 = half, dim3 = expert
     const uint64_t dims[4] = {(uint64_t)H, (uint64_t)I, 2, (uint64_t)E_w};
     const uint64_t strides[3] = {(uint64_t)H * 2, (uint64_t)I * H * 2, (uint64_t)2 * I * H * 2};
     const uint32_t box[4] = {BK, 128, 1, 1};
-    if (!make_map(&tmB, w_gate_up, 4, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&tmB, w_gate_up, 4, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  return launch_tc<MODE_GATE_UP>(sg, tmA, tmB, I, H, h, nullptr, nullptr, err, s);
+  return launch_tc<MODE_GATE_UP>(sg, tmA, tmB, I, H, h, I, nullptr, nullptr, err, s);
 }
 
 cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down, int64_t E_w, void* y,
@@ -528,16 +396,47 @@ cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down
     const uint64_t dims[2] = {(uint64_t)I, (uint64_t)sg.rows_total};
     const uint64_t strides[1] = {(uint64_t)I * 2};
     const uint32_t box[2] = {BK, BM};
-    if (!make_map(&tmA, h, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&tmA, h, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
+  if (tc_gemm_variant(sg) == 2)
+    return launch_tc2_down(sg, tmA, w_down, E_w, y, row_scale, scale_idx, H, I, err, num_sms(), s);
   {
     // down [E][H][I]: dim0 = I, dim1 = H, dim2 = expert
     const uint64_t dims[3] = {(uint64_t)I, (uint64_t)H, (uint64_t)E_w};
     const uint64_t strides[2] = {(uint64_t)I * 2, (uint64_t)H * I * 2};
     const uint32_t box[3] = {BK, UMMA_N, 1};
-    if (!make_map(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  return launch_tc<MODE_DOWN>(sg, tmA, tmB, H, I, y, row_scale, scale_idx, err, s);
+  return launch_tc<MODE_DOWN>(sg, tmA, tmB, H, I, y, H, row_scale, scale_idx, err, s);
+}
+
+int tc_router_splits(int64_t T, int64_t H, int64_t E) {
+  const int64_t k_tiles = ceil_div(H, BK);
+  const int64_t tiles_mn = ceil_div(T, BM) * ceil_div(E, UMMA_N);
+  // At most 16 partials: the top-k kernel adds them serially per logit.
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>({k_tiles, (int64_t)16, 148 / std::max<int64_t>(1, tiles_mn)}));
+  const int64_t kps = ceil_div(k_tiles, splits);
+  return (int)ceil_div(k_tiles, kps);  // every split gets at least one k-step
+}
+
+cudaError_t launch_tc_logits(const void* x, const void* gate_w, int64_t T, int64_t H, int64_t E, float* partial,
+                             int64_t ldo, int splits, int32_t* err, cudaStream_t s) {
+  if (!get_encode()) return cudaErrorNotSupported;
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[2] = {(uint64_t)H, (uint64_t)T};
+    const uint64_t strides[1] = {(uint64_t)H * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!make_tensor_map_bf16(&tmA, x, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)H, (uint64_t)E, 1};
+    const uint64_t strides[2] = {(uint64_t)H * 2, (uint64_t)E * H * 2};
+    const uint32_t box[3] = {BK, UMMA_N, 1};
+    if (!make_tensor_map_bf16(&tmB, gate_w, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  Segments sg{nullptr, 1, (int32_t)T, T};
+  return launch_tc<MODE_LOGITS>(sg, tmA, tmB, E, H, partial, ldo, nullptr, nullptr, err, s, splits);
 }
 
 }  // namespace stm

@@ -1,0 +1,310 @@
+// bf16 grouped SwiGLU GEMMs on CTA pairs (tcgen05.mma.cta_group::2).
+//
+// Same computation as the one-CTA kernel in gemm_tc.cu (gate_up with the
+// SwiGLU epilogue, down with the routing-weight epilogue, over the device
+// segment table; "mstar.model.components.moe", SparseMoeBlock fused layout;
+// "Sparse MoE FFN for DFlash-family drafters", grouped GEMM with no host
+// syncs), but each tile is 256 rows x 256 accumulator columns computed by two
+// CTAs on two SMs of a cluster:
+//   - each CTA loads its own 128 rows of A and its own half of B (128 of the
+//     256 B rows: for gate_up the leader loads the gate rows n0..n0+127 and
+//     the peer the matching up rows), so a k-step moves 32 KB per CTA instead
+//     of 48 KB for the same MMA work per SM and the stage ring is 6 deep;
+//   - both CTAs' TMA loads complete on the leader's full barrier; the leader
+//     posts the pair's transaction bytes and issues the M=256 MMA, whose
+//     commits arrive on the empty / accumulator barriers of both CTAs;
+//   - each CTA's epilogue drains its own TMEM rows and arrives on the
+//     leader's accumulator-empty barrier.
+// No TMA multicast is used: every CTA fetches its own tiles.
+//
+// Used when segments average at least 384 rows. A row tile is 256 rows of one
+// segment; the peer skips its A load when the segment has no rows in its
+// half (its accumulator rows are then discarded).
+// All waits are bounded as in the one-CTA kernel; a cluster barrier before
+// TMEM is freed guarantees no remote arrive or MMA still targets a CTA that
+// is about to exit.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_epilogue.cuh"
+#include "tc_ptx.cuh"
+#include "tiles.cuh"
+
+namespace stm {
+
+namespace {
+
+using namespace tc;
+
+constexpr int BM2 = 256;         // rows per pair tile
+constexpr int HALF = 128;        // rows of A (and of B) per CTA
+constexpr int BK = 64;
+constexpr int UMMA_N = 256;
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = HALF * BK * 2;
+constexpr int B_BYTES = HALF * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * UMMA_N;
+constexpr int NTHREADS = 192;
+constexpr uint32_t kIdesc256 = make_idesc(256, UMMA_N);
+
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
+
+struct Args2 {
+  const int32_t* offsets;
+  int32_t E;
+  int32_t single_rows;
+  int32_t N;
+  int32_t n_tiles;
+  int32_t k_tiles;
+  int64_t ldo;
+  void* out;
+  const float* row_scale;
+  const int32_t* scale_idx;
+  int32_t* err;
+  int64_t rows_total;
+};
+
+struct __align__(8) Ctl2 {
+  uint64_t full[STAGES];   // leader only: both CTAs' bytes of a stage landed
+  uint64_t empty[STAGES];  // both: the pair MMA finished reading a stage
+  uint64_t tfull[2];       // both: accumulator ready
+  uint64_t tempty[2];      // leader only: both CTAs' epilogues drained it
+  uint64_t drain;          // both: every pair MMA complete
+  uint32_t tmem_base;
+  int abort;
+  int off[kMaxExperts + 1];
+  int pre[kMaxExperts + 1];
+};
+
+constexpr size_t kSmemBytes2 = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctl2);
+
+struct Tile2 {
+  int e, row0, row_end, n_idx;
+  bool peer_rows;  // the peer's 128 rows hold any row of the segment
+};
+
+__device__ __forceinline__ Tile2 decode_tile2(const Ctl2* ctl, int Eseg, int n_tiles, int tile) {
+  Tile2 t;
+  const int mt = tile / n_tiles;
+  t.n_idx = tile - mt * n_tiles;
+  t.e = find_segment(ctl->pre, Eseg, mt);
+  t.row0 = ctl->off[t.e] + (mt - ctl->pre[t.e]) * BM2;
+  t.row_end = ctl->off[t.e + 1];
+  t.peer_rows = t.row0 + HALF < t.row_end;
+  return t;
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    tc2_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            const Args2 args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl2* ctl = reinterpret_cast<Ctl2*>(base + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int Eseg = args.offsets ? args.E : 1;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&ctl->tfull[a], 1);
+      mbar_init(&ctl->tempty[a], 8);  // one arrive per epilogue warp, 4 warps x 2 CTAs
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2)
+    warp_build_tile_table(args.offsets, args.E, args.single_rows, BM2, ctl->off, ctl->pre, args.rows_total,
+                          args.err);
+  if (warp == 1) tmem_alloc2(&ctl->tmem_base, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int total_tiles = ctl->pre[Eseg] * args.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_parity = 0;
+      for (int tile = pair; tile < total_tiles; tile += npairs) {
+        const Tile2 tc = decode_tile2(ctl, Eseg, args.n_tiles, tile);
+        bool ok = true;
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, args.err, 11)) { ok = false; break; }
+          uint8_t* sa = base + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          const uint32_t full_leader = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+          if (leader)
+            mbar_arrive_expect_tx(&ctl->full[stage],
+                                  (uint32_t)(2 * B_BYTES + A_BYTES + (tc.peer_rows ? A_BYTES : 0)));
+          const int k0 = kt * BK;
+          if (leader || tc.peer_rows) tma2_load_2d(sa, &tmA, full_leader, k0, tc.row0 + (int)rank * HALF);
+          if (MODE == MODE_GATE_UP) {
+            // leader: gate rows n0..n0+127; peer: the matching up rows
+            tma2_load_4d(sb, &tmB, full_leader, k0, tc.n_idx * 128, (int)rank, tc.e);
+          } else {
+            tma2_load_3d(sb, &tmB, full_leader, k0, tc.n_idx * UMMA_N + (int)rank * HALF, tc.e);
+          }
+          if (leader) {
+            issued |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      // Drain (leader): the full barriers count both CTAs' bytes, so every
+      // copy of the pair has landed once they complete.
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1u) mbar_wait(&ctl->full[s], (last_parity >> s) & 1u, &ctl->abort, args.err, 16, true);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+        if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 12)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, args.err, 13)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(base + stage * STAGE_BYTES);
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), kIdesc256,
+                       (kt > 0 || kk > 0) ? 1u : 0u);
+          umma2_commit_mc(&ctl->empty[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma2_commit_mc(&ctl->tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      umma2_commit_mc(&ctl->drain, 0x3);
+      mbar_wait(&ctl->drain, 0, &ctl->abort, args.err, 17, true);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    const int quarter = warp & 3;
+    const int r = (int)rank * HALF + quarter * 32 + lane;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total_tiles; tile += npairs) {
+      const Tile2 tc = decode_tile2(ctl, Eseg, args.n_tiles, tile);
+      if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, args.err, 14)) break;
+      tc_fence_after();
+      const int row = tc.row0 + r;
+      const bool valid = row < tc.row_end;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * UMMA_N);
+      if (MODE == MODE_GATE_UP) {
+        epilogue_swiglu(tbase, valid, reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row * args.ldo,
+                        tc.n_idx * 128, args.N);
+      } else {
+        float sc = 1.f;
+        if (valid && args.row_scale != nullptr) sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
+        epilogue_scale_f32(tbase, valid, sc, reinterpret_cast<float*>(args.out) + (int64_t)row * args.ldo,
+                           tc.n_idx * UMMA_N, args.N);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no remote arrive or pair MMA still targets either CTA
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc2(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int MODE>
+cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, int64_t N, int64_t K,
+                       void* out, int64_t ldo, const float* row_scale, const int32_t* scale_idx, int32_t* err,
+                       int num_sms, cudaStream_t s) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(tc2_grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes2);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  Args2 a;
+  a.offsets = sg.offsets;
+  a.E = sg.E;
+  a.single_rows = sg.single_rows;
+  a.N = (int32_t)N;
+  a.n_tiles = (int32_t)ceil_div(N, MODE == MODE_GATE_UP ? 128 : UMMA_N);
+  a.k_tiles = (int32_t)ceil_div(K, BK);
+  a.ldo = ldo;
+  a.out = out;
+  a.row_scale = row_scale;
+  a.scale_idx = scale_idx;
+  a.err = err;
+  a.rows_total = sg.rows_total;
+  const int64_t nseg = sg.offsets ? sg.E : 1;
+  const int64_t max_tiles = (sg.rows_total / BM2 + nseg) * a.n_tiles;
+  const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms / 2, max_tiles));
+  tc2_grouped_gemm_kernel<MODE><<<2 * pairs, NTHREADS, kSmemBytes2, s>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc2_gate_up(const Segments& sg, const CUtensorMap& tmA, const void* w_gate_up, int64_t E_w,
+                               void* h, int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s) {
+  CUtensorMap tmB;
+  // gate_up [E][2][I][H], one half (128 rows of gate or of up) per CTA
+  const uint64_t dims[4] = {(uint64_t)H, (uint64_t)I, 2, (uint64_t)E_w};
+  const uint64_t strides[3] = {(uint64_t)H * 2, (uint64_t)I * H * 2, (uint64_t)2 * I * H * 2};
+  const uint32_t box[4] = {BK, HALF, 1, 1};
+  if (!make_tensor_map_bf16(&tmB, w_gate_up, 4, dims, strides, box)) return cudaErrorInvalidValue;
+  return launch_tc2<MODE_GATE_UP>(sg, tmA, tmB, I, H, h, I, nullptr, nullptr, err, num_sms, s);
+}
+
+cudaError_t launch_tc2_down(const Segments& sg, const CUtensorMap& tmA, const void* w_down, int64_t E_w, void* y,
+                            const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
+                            int num_sms, cudaStream_t s) {
+  CUtensorMap tmB;
+  // down [E][H][I], 128 of the tile's 256 output rows per CTA
+  const uint64_t dims[3] = {(uint64_t)I, (uint64_t)H, (uint64_t)E_w};
+  const uint64_t strides[2] = {(uint64_t)I * 2, (uint64_t)H * I * 2};
+  const uint32_t box[3] = {BK, HALF, 1};
+  if (!make_tensor_map_bf16(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  return launch_tc2<MODE_DOWN>(sg, tmA, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+}
+
+}  // namespace stm

@@ -1,6 +1,7 @@
 // Internal launch wrappers (host side). Not part of the public C ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -9,18 +10,26 @@
 namespace stm {
 
 // ---- router -----------------------------------------------------------
-struct RouterSplit {
-  int splits;       // partial sums along H
-  int k_per_split;  // H elements per partial
+// Logits are computed as `splits` fp32 partial sums along H, each [T, ldo]
+// (row pitch ldo >= E); the top-k kernel adds them in split order.
+struct RouterPlan {
+  bool tensor_cores;  // bf16: tcgen05 GEMM; fp32: SIMT GEMM
+  int splits;
+  int k_per_split;    // SIMT only: H elements per split
+  int64_t ldo;
 };
-RouterSplit router_split(int64_t T, int64_t H, int64_t Ecols);
+RouterPlan router_plan(int dtype, int64_t T, int64_t H, int64_t E);
+size_t router_partial_bytes(int dtype, int64_t T, int64_t H, int64_t E);
 
-cudaError_t launch_router_logits(int dtype, const void* x, const void* gate_w, const void* extra_row,
-                                 float* partial, int64_t T, int64_t H, int64_t E, int64_t Ecols,
-                                 const RouterSplit& sp, cudaStream_t s);
-cudaError_t launch_topk(const float* partial, int splits, int64_t T, int64_t E, int64_t Ecols, int64_t k,
-                        int score, int bias_mode, int renorm, const float* bias, float* weights,
-                        int64_t* selected, float* gamma, cudaStream_t s);
+// logits partials, then scores / top-k / weights (+ shared gate when
+// shared_gate != nullptr: gamma[t] = sigmoid(x[t] . shared_gate)).
+cudaError_t launch_route(int dtype, const void* x, const void* gate_w, const void* shared_gate, const float* bias,
+                         int64_t T, int64_t H, int64_t E, int64_t k, int score, int bias_mode, int renorm,
+                         float* partial, float* weights, int64_t* selected, float* gamma, int32_t* err,
+                         cudaStream_t s);
+cudaError_t launch_topk(const float* partial, int splits, int64_t ldo, int64_t T, int64_t E, int64_t k, int score,
+                        int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
+                        const void* x, const void* shared_gate, int64_t H, int dtype, float* gamma, cudaStream_t s);
 
 // ---- dispatch ---------------------------------------------------------
 int64_t dispatch_tokens_per_block(int64_t k);
@@ -52,8 +61,23 @@ cudaError_t launch_simt_down(const Segments& sg, const float* h, const float* w_
                              cudaStream_t s);
 
 // tcgen05 / TMEM bf16 grouped GEMMs: h is bf16, y is fp32.
+// Variant: 1 = one CTA per 128-row tile; 2 = CTA pairs (cta_group::2) per
+// 256-row tile, used when segments average at least 128 rows.
+int tc_gemm_variant(const Segments& sg);
+bool get_encode();
+bool make_tensor_map_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box);
+int num_sms();
+cudaError_t launch_tc2_gate_up(const Segments& sg, const CUtensorMap& tmA, const void* w_gate_up, int64_t E_w,
+                               void* h, int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s);
+cudaError_t launch_tc2_down(const Segments& sg, const CUtensorMap& tmA, const void* w_down, int64_t E_w, void* y,
+                            const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
+                            int num_sms, cudaStream_t s);
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                               int64_t I, int64_t H, int32_t* err, cudaStream_t s);
+int tc_router_splits(int64_t T, int64_t H, int64_t E);
+cudaError_t launch_tc_logits(const void* x, const void* gate_w, int64_t T, int64_t H, int64_t E, float* partial,
+                             int64_t ldo, int splits, int32_t* err, cudaStream_t s);
 cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down, int64_t E_w, void* y,
                            const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                            cudaStream_t s);

@@ -4,14 +4,15 @@
 // top-k with optional renormalisation, int64 indices) and "Sparse MoE FFN for
 // DFlash-family drafters" (What's here, MoEGate: sqrtsoftplus scores and an
 // fp32 aux-loss-free bias that only ranks experts). The shared-expert gate of
-// SparseMoeBlockWithSharedExpert (sigmoid(shared_gate(x))) is one more output
-// column of the same GEMM.
+// SparseMoeBlockWithSharedExpert, sigmoid(shared_gate(x)), is a per-token dot
+// product computed by the top-k kernel.
 //
-// The logits GEMM is small (2*T*H*E flops) and is computed in fp32 on the
-// SIMT pipes, split along H into a few deterministic partial sums when there
-// are too few token/expert tiles to fill the GPU (the 16-token decode batch).
-// The top-k kernel adds the partials in a fixed order, so routing is
-// bit-reproducible run to run.
+// Logits: for bf16 problems the tcgen05 GEMM (fp32 accumulate) computes x .
+// gate_w^T; it reads x once, so the router costs about one pass over the
+// hidden states. fp32 problems use the SIMT tile below. Both split the H
+// reduction into a few partial sums when there are too few token/expert tiles
+// to fill the GPU (the 16-token decode batch), and the top-k kernel adds the
+// partials in a fixed order, so routing is bit-reproducible run to run.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,9 +25,8 @@ constexpr int RBM = 64, RBN = 64, RBK = 32, RTHREADS = 256;
 template <typename T>
 __global__ void __launch_bounds__(RTHREADS) router_logits_kernel(const T* __restrict__ x,
                                                                  const T* __restrict__ gate_w,
-                                                                 const T* __restrict__ extra_row,
                                                                  float* __restrict__ partial, int Tn, int H,
-                                                                 int E, int Ecols, int k_per_split) {
+                                                                 int E, int ldo, int k_per_split) {
   __shared__ float As[RBK][RBM + 4];
   __shared__ float Bs[RBK][RBN + 4];
   constexpr int V = Elem<T>::kPerVec;
@@ -62,13 +62,11 @@ __global__ void __launch_bounds__(RTHREADS) router_logits_kernel(const T* __rest
 #pragma unroll
         for (int q = 0; q < V; ++q) As[c + q][r] = f[q];
       }
-      // B: expert rows (row E is the shared-gate vector when present)
+      // B: expert rows
       {
         const int col = n0 + r;
-        const T* src = nullptr;
-        if (col < E) src = gate_w + (int64_t)col * H;
-        else if (col < Ecols) src = extra_row;
-        if (src != nullptr && kk < ke) {
+        if (col < E && kk < ke) {
+          const T* src = gate_w + (int64_t)col * H;
           const uint4 v = *reinterpret_cast<const uint4*>(src + kk);
           if constexpr (V == 8) unpack16_bf16(v, f); else unpack16(v, f, nullptr);
         } else {
@@ -94,7 +92,7 @@ __global__ void __launch_bounds__(RTHREADS) router_logits_kernel(const T* __rest
     }
     __syncthreads();
   }
-  float* dst = partial + (int64_t)blockIdx.z * Tn * Ecols;
+  float* dst = partial + (int64_t)blockIdx.z * Tn * ldo;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int row = m0 + ty + 16 * i;
@@ -102,7 +100,7 @@ __global__ void __launch_bounds__(RTHREADS) router_logits_kernel(const T* __rest
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int col = n0 + tx + 16 * j;
-      if (col < Ecols) dst[(int64_t)row * Ecols + col] = acc[i][j];
+      if (col < E) dst[(int64_t)row * ldo + col] = acc[i][j];
     }
   }
 }
@@ -114,12 +112,15 @@ __device__ __forceinline__ bool ranks_before(float ka, int ea, float kb, int eb)
 
 constexpr int TOPK_WARPS = 8;
 
+template <typename TX>
 __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ partial, int splits,
-                                                                int Tn, int E, int Ecols, int k, int score,
+                                                                int64_t ldo, int Tn, int E, int k, int score,
                                                                 int bias_mode, int renorm,
                                                                 const float* __restrict__ bias,
                                                                 float* __restrict__ weights,
                                                                 int64_t* __restrict__ selected,
+                                                                const TX* __restrict__ x,
+                                                                const TX* __restrict__ shared_gate, int H,
                                                                 float* __restrict__ gamma) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * TOPK_WARPS + (threadIdx.x >> 5);
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
     float l = -INFINITY;
     if (e < E) {
       l = 0.f;
-      for (int s = 0; s < splits; ++s) l += partial[((int64_t)s * Tn + t) * Ecols + e];
+      for (int s = 0; s < splits; ++s) l += partial[((int64_t)s * Tn + t) * ldo + e];
       if (bias_mode == 1) l += bias[e];
     }
     logit[i] = l;
@@ -172,11 +173,12 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
     key[i] = (bias_mode == 2 && e < E) ? sc[i] + bias[e] : logit[i];
   }
 
+  // Slot j's expert and raw weight go to shared memory; the renormalising
+  // sum runs in slot order (identical in every lane).
+  __shared__ float s_w[TOPK_WARPS][kMaxExperts];
+  __shared__ int s_e[TOPK_WARPS][kMaxExperts];
+  const int wid = threadIdx.x >> 5;
   uint32_t taken = 0;
-  int sel_r[8];
-  float w_r[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) { sel_r[i] = 0; w_r[i] = 0.f; }
   float tot = 0.f;
   for (int j = 0; j < k; ++j) {
     float bk = -INFINITY, bs = 0.f;
@@ -196,66 +198,105 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
       if (ranks_before(ok, oe, bk, be)) { bk = ok; be = oe; bs = os; }
     }
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q == (j >> 5) && lane == (j & 31)) { sel_r[q] = be; w_r[q] = bs; }
+    if (lane == 0) {
+      s_w[wid][j] = bs;
+      s_e[wid][j] = be;
+    }
     tot += bs;
   }
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int j = lane + 32 * q;
-    if (j < k) {
-      float w = w_r[q];
-      if (renorm) w = tot > 0.f ? w / tot : 0.f;
-      weights[(int64_t)t * k + j] = w;
-      selected[(int64_t)t * k + j] = (int64_t)sel_r[q];
-    }
+  __syncwarp();
+  for (int j = lane; j < k; j += 32) {
+    float w = s_w[wid][j];
+    if (renorm) w = tot > 0.f ? w / tot : 0.f;
+    weights[(int64_t)t * k + j] = w;
+    selected[(int64_t)t * k + j] = (int64_t)s_e[wid][j];
   }
-  if (gamma != nullptr && lane == 0) {
-    float lg = 0.f;
-    for (int s = 0; s < splits; ++s) lg += partial[((int64_t)s * Tn + t) * Ecols + E];
-    gamma[t] = 1.0f / (1.0f + expf(-lg));
+  if (gamma != nullptr) {
+    // gamma[t] = sigmoid(x[t] . shared_gate): fp32 dot product, lanes over
+    // 16-byte vectors, butterfly sum (same result in every lane).
+    constexpr int V = Elem<TX>::kPerVec;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
+    const uint4* gr = reinterpret_cast<const uint4*>(shared_gate);
+    float acc = 0.f;
+    for (int v = lane; v < H / V; v += 32) {
+      float a[8], b[8];
+      if constexpr (V == 8) {
+        unpack16_bf16(xr[v], a);
+        unpack16_bf16(gr[v], b);
+      } else {
+        unpack16(xr[v], a, nullptr);
+        unpack16(gr[v], b, nullptr);
+      }
+#pragma unroll
+      for (int q = 0; q < V; ++q) acc = fmaf(a[q], b[q], acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) gamma[t] = 1.0f / (1.0f + expf(-acc));
   }
 }
 
 }  // namespace
 
-RouterSplit router_split(int64_t T, int64_t H, int64_t Ecols) {
-  RouterSplit r;
-  const int64_t blocks_mn = ceil_div(T, RBM) * ceil_div(Ecols, RBN);
+RouterPlan router_plan(int dtype, int64_t T, int64_t H, int64_t E) {
+  RouterPlan r;
+  T = std::max<int64_t>(T, 1);
+  r.ldo = round_up(E, 4);
+  if (dtype == 1) {
+    r.tensor_cores = true;
+    r.splits = tc_router_splits(T, H, E);
+    r.k_per_split = 0;
+    return r;
+  }
+  r.tensor_cores = false;
+  const int64_t blocks_mn = ceil_div(T, RBM) * ceil_div(E, RBN);
   int64_t splits = 1;
   const int64_t target = 2 * 148;
   if (blocks_mn < target) splits = ceil_div(target, blocks_mn);
   splits = std::min<int64_t>(splits, std::max<int64_t>(1, ceil_div(H, 256)));
-  int64_t kps = round_up(ceil_div(H, splits), RBK);
-  splits = ceil_div(H, kps);
-  r.splits = (int)splits;
+  const int64_t kps = round_up(ceil_div(H, splits), RBK);
+  r.splits = (int)ceil_div(H, kps);
   r.k_per_split = (int)kps;
   return r;
 }
 
-cudaError_t launch_router_logits(int dtype, const void* x, const void* gate_w, const void* extra_row,
-                                 float* partial, int64_t T, int64_t H, int64_t E, int64_t Ecols,
-                                 const RouterSplit& sp, cudaStream_t s) {
-  dim3 grid((unsigned)ceil_div(T, RBM), (unsigned)ceil_div(Ecols, RBN), (unsigned)sp.splits);
+size_t router_partial_bytes(int dtype, int64_t T, int64_t H, int64_t E) {
+  const RouterPlan r = router_plan(dtype, T, H, E);
+  return (size_t)r.splits * (size_t)T * (size_t)r.ldo * 4;
+}
+
+cudaError_t launch_topk(const float* partial, int splits, int64_t ldo, int64_t T, int64_t E, int64_t k, int score,
+                        int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
+                        const void* x, const void* shared_gate, int64_t H, int dtype, float* gamma, cudaStream_t s) {
+  dim3 grid((unsigned)ceil_div(T, TOPK_WARPS));
   if (dtype == 0)
-    router_logits_kernel<float><<<grid, RTHREADS, 0, s>>>(
-        (const float*)x, (const float*)gate_w, (const float*)extra_row, partial, (int)T, (int)H, (int)E,
-        (int)Ecols, sp.k_per_split);
+    topk_kernel<float><<<grid, TOPK_WARPS * 32, 0, s>>>(partial, splits, ldo, (int)T, (int)E, (int)k, score,
+                                                        bias_mode, renorm, bias, weights, selected, (const float*)x,
+                                                        (const float*)shared_gate, (int)H, gamma);
   else
-    router_logits_kernel<__nv_bfloat16><<<grid, RTHREADS, 0, s>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)gate_w, (const __nv_bfloat16*)extra_row, partial,
-        (int)T, (int)H, (int)E, (int)Ecols, sp.k_per_split);
+    topk_kernel<__nv_bfloat16><<<grid, TOPK_WARPS * 32, 0, s>>>(
+        partial, splits, ldo, (int)T, (int)E, (int)k, score, bias_mode, renorm, bias, weights, selected,
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)shared_gate, (int)H, gamma);
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const float* partial, int splits, int64_t T, int64_t E, int64_t Ecols, int64_t k,
-                        int score, int bias_mode, int renorm, const float* bias, float* weights,
-                        int64_t* selected, float* gamma, cudaStream_t s) {
-  dim3 grid((unsigned)ceil_div(T, TOPK_WARPS));
-  topk_kernel<<<grid, TOPK_WARPS * 32, 0, s>>>(partial, splits, (int)T, (int)E, (int)Ecols, (int)k, score,
-                                                bias_mode, renorm, bias, weights, selected, gamma);
-  return cudaGetLastError();
+cudaError_t launch_route(int dtype, const void* x, const void* gate_w, const void* shared_gate, const float* bias,
+                         int64_t T, int64_t H, int64_t E, int64_t k, int score, int bias_mode, int renorm,
+                         float* partial, float* weights, int64_t* selected, float* gamma, int32_t* err,
+                         cudaStream_t s) {
+  const RouterPlan plan = router_plan(dtype, T, H, E);
+  cudaError_t e;
+  if (plan.tensor_cores) {
+    e = launch_tc_logits(x, gate_w, T, H, E, partial, plan.ldo, plan.splits, err, s);
+  } else {
+    dim3 grid((unsigned)ceil_div(T, RBM), (unsigned)ceil_div(E, RBN), (unsigned)plan.splits);
+    router_logits_kernel<float><<<grid, RTHREADS, 0, s>>>((const float*)x, (const float*)gate_w, partial, (int)T,
+                                                          (int)H, (int)E, (int)plan.ldo, plan.k_per_split);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return e;
+  return launch_topk(partial, plan.splits, plan.ldo, T, E, k, score, bias_mode, renorm, bias, weights, selected, x,
+                     shared_gate, H, dtype, shared_gate ? gamma : nullptr, s);
 }
 
 }  // namespace stm

@@ -35,6 +35,10 @@ EDGE = {
     "tiny_ragged_f32": CONFIGS["decode_weight_streaming"].replace(name="ragged32", T=29, H=24, E=6, k=3, I=40,
                                                                   I_shared=8, dtype="f32"),
     "many_tiles_one_expert": CONFIGS["qwen3_30b_a3b"].replace(name="skew", T=700, H=192, E=4, k=1, I=136),
+    # routed segments averaging >= 128 rows run on CTA pairs (256-row tiles)
+    "pairs_ragged": CONFIGS["qwen3_30b_a3b"].replace(name="pairs", T=1731, H=384, E=8, k=2, I=200),
+    "pairs_shared_skew": CONFIGS["deepseek_v2_lite_zipf"].replace(name="pairs_zipf", T=4200, H=256, I=136,
+                                                                  I_shared=272),
 }
 
 
@@ -76,6 +80,15 @@ def test_forward_edge_cases(name):
     cfg = EDGE[name]
     cpu, dev = _inputs(cfg)
     _forward_and_check(cfg, cpu, dev)
+
+
+def test_both_tensor_core_variants_are_exercised():
+    """The one-CTA (128-row tiles) and CTA-pair (256-row tiles) tcgen05
+    kernels are both reached by the parity cases above."""
+    paths = {name: stm.gemm_path(stm.Problem.from_config(cfg)) for name, cfg in {**SMALL, **EDGE}.items()}
+    assert paths["tiny_fp32"] == 0
+    assert paths["pairs_ragged"] == 2 and paths["pairs_shared_skew"] == 2
+    assert paths["qwen3_30b_a3b"] == 1 and paths["decode_weight_streaming"] == 1
 
 
 @pytest.mark.parametrize("name", list(SMALL))
