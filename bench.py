@@ -131,11 +131,6 @@ def flops_and_bytes(cfg, n_active: int):
             "gate_up_bytes": gu_bytes, "min_bytes": min_bytes, "weight_bytes": w_bytes}
 
 
-def launches_per_step(cfg) -> int:
-    # router logits + top-k; histogram + scan + permute + gather; gate_up +
-    # down; shared gate_up + down; combine
-    return 2 + 4 + 2 + (2 if cfg.shared != "none" else 0) + 1
-
 
 def recorded_traffic(cfg_name: str):
     """Per-launch DRAM traffic of the gate_up kernel from the committed ncu
@@ -343,7 +338,7 @@ def main():
     with ClockSampler(local) as clocks:
         t_start.record(stream)
         for i in range(args.steps):
-            moe.forward_profiled(x, out, rw, sel, evs[i])
+            moe.forward(x, out, rw, sel, events=evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -409,7 +404,7 @@ def main():
         "roofline": roof,
         "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": e2e_steps},
-        "gpu_launches": launches_per_step(cfg) * args.steps,
+        "gpu_launches": stm.launches_per_forward(p, two_streams=moe.aux is not None) * args.steps,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

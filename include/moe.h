@@ -116,7 +116,7 @@ typedef struct moe_weights {
   const void *shared_gate;    /* [H] gate vector (SIGMOID_GATED only), or NULL   */
 } moe_weights;
 
-/* Stages timed by moe_forward_profiled, in launch order. */
+/* Stages timed through moe_forward_ex's stage events, in launch order. */
 enum {
   MOE_STAGE_ROUTE = 0,
   MOE_STAGE_DISPATCH = 1,
@@ -203,16 +203,32 @@ moe_status moe_forward(const moe_problem *p, const moe_weights *w, const void *x
                        float *routing_weights, int64_t *selected_experts, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
 
-/* moe_forward, recording stage_events[i] before stage i and
- * stage_events[MOE_NUM_STAGES] after the last one (MOE_NUM_STAGES + 1
- * caller-created events; a NULL entry is skipped). */
-moe_status moe_forward_profiled(const moe_problem *p, const moe_weights *w, const void *x, void *out,
-                                float *routing_weights, int64_t *selected_experts, void *ws,
-                                size_t ws_bytes, moe_stream_t stream, moe_event_t *stage_events);
+/* moe_forward with two options:
+ *   aux_stream: when not NULL (and not `stream`), the problem has a shared
+ *     expert and that expert is small (its gate_up GEMM has at most 74
+ *     128x128 tiles, as for a decode batch), the shared expert runs on
+ *     aux_stream concurrently with the routed path on `stream`, and `stream`
+ *     waits for it before the combine (fork / join through two events the
+ *     call creates and releases); the sigmoid gate is then computed by its
+ *     own small kernel. Larger shared experts run on `stream`, because they
+ *     occupy every SM. All work is complete once `stream` has passed the call.
+ *   stage_events: NULL, or MOE_NUM_STAGES + 1 caller-created events recorded
+ *     on `stream` before each stage (MOE_STAGE_*) and after the last one; a
+ *     NULL entry is skipped. */
+moe_status moe_forward_ex(const moe_problem *p, const moe_weights *w, const void *x, void *out,
+                          float *routing_weights, int64_t *selected_experts, void *ws, size_t ws_bytes,
+                          moe_stream_t stream, moe_stream_t aux_stream, moe_event_t *stage_events);
 
-/* Which expert-GEMM implementation serves problem p: 1 = tcgen05/TMEM tensor
- * core path (bf16), 0 = SIMT fp32 path. Host only. */
+/* Which routed expert-GEMM implementation serves problem p: 0 = SIMT fp32;
+ * 1 = tcgen05/TMEM, one CTA per 128-row tile; 2 = tcgen05 CTA pairs
+ * (cta_group::2) per 256-row tile, chosen when segments average at least
+ * 384 rows. Host only. */
 moe_status moe_gemm_path(const moe_problem *p, int32_t *path);
+
+/* Number of kernel launches one forward of problem p makes (0 when T == 0):
+ * moe_forward when two_streams == 0, moe_forward_ex with an aux_stream
+ * otherwise. Host only. */
+moe_status moe_launches_per_forward(const moe_problem *p, int32_t two_streams, int32_t *n);
 
 /* Synchronise `stream`, read the workspace error bits into *code (host
  * pointer), clear them. Returns MOE_ERR_DEVICE_FLAG when any bit was set. */

@@ -65,9 +65,10 @@ SIGNATURES = {
     "moe_shared_expert": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
     "moe_forward": (ctypes.c_int, [_PP, ctypes.POINTER(moe_weights), _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "moe_forward_profiled": (ctypes.c_int, [_PP, ctypes.POINTER(moe_weights), _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
-                                            ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_forward_ex": (ctypes.c_int, [_PP, ctypes.POINTER(moe_weights), _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP,
+                                      ctypes.POINTER(ctypes.c_void_p)]),
     "moe_gemm_path": (ctypes.c_int, [_PP, _I32P]),
+    "moe_launches_per_forward": (ctypes.c_int, [_PP, ctypes.c_int32, _I32P]),
     "moe_read_device_error": (ctypes.c_int, [_VP, _I32P, _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -159,6 +160,12 @@ def new_workspace(p: Problem, device="cuda") -> torch.Tensor:
 def gemm_path(p: Problem) -> int:
     out = ctypes.c_int32(-1)
     _check(lib().moe_gemm_path(ctypes.byref(p.c()), ctypes.byref(out)))
+    return int(out.value)
+
+
+def launches_per_forward(p: Problem, two_streams: bool = False) -> int:
+    out = ctypes.c_int32(-1)
+    _check(lib().moe_launches_per_forward(ctypes.byref(p.c()), int(bool(two_streams)), ctypes.byref(out)))
     return int(out.value)
 
 
@@ -286,16 +293,20 @@ class SparseMoE:
 
     ``weights``: gate_w [E,H], gate_up [E,2I,H], down [E,H,I], optional bias
     [E] fp32, shared_gate_up [2I_s,H], shared_down [H,I_s], shared_gate [H].
+    ``overlap_shared``: run the shared expert on a second stream concurrently
+    with the routed path (the call still completes on the current stream).
     """
 
-    def __init__(self, p: Problem, weights: Dict[str, Optional[torch.Tensor]], device="cuda"):
+    def __init__(self, p: Problem, weights: Dict[str, Optional[torch.Tensor]], device="cuda",
+                 overlap_shared: bool = True):
         self.p = p
         self.w = weights
         self._cw = _weights_struct(p, weights)
         self.device = torch.device(device)
         self.ws = new_workspace(p, self.device)
+        self.aux = torch.cuda.Stream(self.device) if (overlap_shared and p.shared != "none") else None
 
-    def forward(self, x, out=None, routing_weights=None, selected_experts=None):
+    def _outputs(self, x, out, routing_weights, selected_experts):
         p = self.p
         _req(x, "x", (p.T, p.H), p.torch_dtype)
         out = torch.empty(p.T, p.H, dtype=p.torch_dtype, device=x.device) if out is None else out
@@ -303,22 +314,25 @@ class SparseMoE:
             else routing_weights
         sel = torch.empty(p.T, p.k, dtype=torch.int64, device=x.device) if selected_experts is None \
             else selected_experts
-        _check(lib().moe_forward(ctypes.byref(p.c()), ctypes.byref(self._cw), _ptr(x), _ptr(out), _ptr(rw), _ptr(sel),
-                                 self.ws.data_ptr(), self.ws.numel(), _stream(x.device)))
+        return out, rw, sel
+
+    def forward(self, x, out=None, routing_weights=None, selected_experts=None, events=None):
+        """out, routing_weights, selected_experts = moe(x). ``events``: optional
+        len(STAGES)+1 torch.cuda.Event recorded before each stage and after the
+        combine."""
+        p = self.p
+        out, rw, sel = self._outputs(x, out, routing_weights, selected_experts)
+        arr = None
+        if events is not None:
+            if len(events) != len(STAGES) + 1:
+                raise ValueError("need one event per stage plus one")
+            arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        aux = self.aux.cuda_stream if self.aux is not None else None
+        _check(lib().moe_forward_ex(ctypes.byref(p.c()), ctypes.byref(self._cw), _ptr(x), _ptr(out), _ptr(rw),
+                                    _ptr(sel), self.ws.data_ptr(), self.ws.numel(), _stream(x.device), aux, arr))
         return out, rw, sel
 
     __call__ = forward
-
-    def forward_profiled(self, x, out, routing_weights, selected_experts, events: Sequence[torch.cuda.Event]):
-        """Forward recording ``events[i]`` before stage i (see STAGES) and the
-        last event after the combine."""
-        p = self.p
-        if len(events) != len(STAGES) + 1:
-            raise ValueError("need one event per stage plus one")
-        arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
-        _check(lib().moe_forward_profiled(ctypes.byref(p.c()), ctypes.byref(self._cw), _ptr(x), _ptr(out),
-                                          _ptr(routing_weights), _ptr(selected_experts), self.ws.data_ptr(),
-                                          self.ws.numel(), _stream(x.device), arr))
 
     def forward_from_host(self, x_host: torch.Tensor, out_host: torch.Tensor, x_dev=None, out_dev=None,
                           rw=None, sel=None):

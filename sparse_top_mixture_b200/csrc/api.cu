@@ -165,8 +165,26 @@ moe_status validate_weights(const moe_problem& p, const moe_weights* w) {
   return MOE_OK;
 }
 
+// Whether moe_forward_ex runs the shared expert on its aux stream: its
+// gate_up GEMM must have at most half as many tiles as a B200 has SMs.
+bool shared_overlaps(const moe_problem& p) {
+  if (p.shared == MOE_SHARED_NONE) return false;
+  const int64_t tiles = ceil_div(p.T, 128) * ceil_div(p.I_shared, 128);
+  return tiles <= 74;
+}
+
+// RAII pair of fork / join events for the two-stream forward.
+struct EventPair {
+  cudaEvent_t fork = nullptr, join = nullptr;
+  ~EventPair() {
+    if (fork) cudaEventDestroy(fork);  // safe while pending: released on completion
+    if (join) cudaEventDestroy(join);
+  }
+};
+
 moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* x, void* out, float* weights,
-                        int64_t* selected, void* ws, size_t ws_bytes, cudaStream_t s, cudaEvent_t* ev) {
+                        int64_t* selected, void* ws, size_t ws_bytes, cudaStream_t s, cudaStream_t aux,
+                        cudaEvent_t* ev) {
   MOE_TRY(validate_problem(p));
   MOE_TRY(validate_weights(*p, w));
   if (p->T == 0) return MOE_OK;
@@ -177,7 +195,12 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
     if (ev != nullptr && ev[i] != nullptr) return cuda_status(cudaEventRecord(ev[i], s));
     return MOE_OK;
   };
+  const bool has_shared = p->shared != MOE_SHARED_NONE;
   const bool gated = p->shared == MOE_SHARED_SIGMOID_GATED;
+  // A second stream only pays when the shared expert is too small to fill
+  // the GPU (few row tiles, as in decode): a large shared GEMM would take
+  // every SM and stall the routed chain instead of overlapping it.
+  const bool two_streams = has_shared && aux != nullptr && aux != s && shared_overlaps(*p);
   float* gamma = at<float>(ws, L.gamma);
   int32_t* counts = at<int32_t>(ws, L.counts);
   int32_t* offsets = at<int32_t>(ws, L.offsets);
@@ -185,11 +208,24 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   int32_t* pair_pos = at<int32_t>(ws, L.pair_pos);
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
-  void* shared_out = p->shared != MOE_SHARED_NONE ? at<void>(ws, L.shared_out) : nullptr;
+  void* shared_out = has_shared ? at<void>(ws, L.shared_out) : nullptr;
+
+  EventPair evp;
+  if (two_streams) {
+    // The shared expert needs only x (and its own gate): run it on `aux`
+    // while the routed path runs on `s`; join before the combine.
+    MOE_CUDA(cudaEventCreateWithFlags(&evp.fork, cudaEventDisableTiming));
+    MOE_CUDA(cudaEventCreateWithFlags(&evp.join, cudaEventDisableTiming));
+    MOE_CUDA(cudaEventRecord(evp.fork, s));
+    MOE_CUDA(cudaStreamWaitEvent(aux, evp.fork, 0));
+    if (gated) MOE_CUDA(launch_shared_gate(p->dtype, x, w->shared_gate, p->T, p->H, gamma, aux));
+    MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, gated ? gamma : nullptr, shared_out, ws, aux));
+    MOE_CUDA(cudaEventRecord(evp.join, aux));
+  }
 
   MOE_TRY(mark(MOE_STAGE_ROUTE));
-  MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, gated ? w->shared_gate : nullptr, weights, selected, gamma, ws,
-                   s));
+  MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, (gated && !two_streams) ? w->shared_gate : nullptr, weights,
+                   selected, gamma, ws, s));
   MOE_TRY(mark(MOE_STAGE_DISPATCH));
   MOE_TRY(do_dispatch(*p, L, selected, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws, s));
   MOE_TRY(mark(MOE_STAGE_GATE_UP));
@@ -197,8 +233,9 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   MOE_TRY(mark(MOE_STAGE_DOWN));
   MOE_TRY(do_grouped_down(*p, L, offsets, w->down, weights, sorted_pairs, y_perm, ws, s));
   MOE_TRY(mark(MOE_STAGE_SHARED));
-  if (shared_out != nullptr)
+  if (has_shared && !two_streams)
     MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, gated ? gamma : nullptr, shared_out, ws, s));
+  if (two_streams) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
   MOE_TRY(mark(MOE_STAGE_COMBINE));
   MOE_CUDA(launch_combine(p->dtype, (const float*)y_perm, pair_pos, (const float*)shared_out, out, p->T, p->H,
                           p->k, s));
@@ -312,14 +349,15 @@ MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const i
 MOE_API moe_status moe_forward(const moe_problem* p, const moe_weights* w, const void* x, void* out,
                                float* routing_weights, int64_t* selected_experts, void* ws, size_t ws_bytes,
                                moe_stream_t stream) {
-  return forward_impl(p, w, x, out, routing_weights, selected_experts, ws, ws_bytes, (cudaStream_t)stream, nullptr);
+  return forward_impl(p, w, x, out, routing_weights, selected_experts, ws, ws_bytes, (cudaStream_t)stream, nullptr,
+                      nullptr);
 }
 
-MOE_API moe_status moe_forward_profiled(const moe_problem* p, const moe_weights* w, const void* x, void* out,
-                                        float* routing_weights, int64_t* selected_experts, void* ws,
-                                        size_t ws_bytes, moe_stream_t stream, moe_event_t* stage_events) {
+MOE_API moe_status moe_forward_ex(const moe_problem* p, const moe_weights* w, const void* x, void* out,
+                                  float* routing_weights, int64_t* selected_experts, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream, moe_stream_t aux_stream, moe_event_t* stage_events) {
   return forward_impl(p, w, x, out, routing_weights, selected_experts, ws, ws_bytes, (cudaStream_t)stream,
-                      reinterpret_cast<cudaEvent_t*>(stage_events));
+                      (cudaStream_t)aux_stream, reinterpret_cast<cudaEvent_t*>(stage_events));
 }
 
 MOE_API moe_status moe_gemm_path(const moe_problem* p, int32_t* path) {
@@ -332,6 +370,29 @@ MOE_API moe_status moe_gemm_path(const moe_problem* p, int32_t* path) {
     sg.offsets = reinterpret_cast<const int32_t*>(16);  // any non-null: routed segments
     *path = tc_gemm_variant(sg);
   }
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_launches_per_forward(const moe_problem* p, int32_t two_streams, int32_t* n) {
+  MOE_TRY(validate_problem(p));
+  if (n == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->T == 0) {
+    *n = 0;
+    return MOE_OK;
+  }
+  int count = 2 + 4 + 1;  // router logits + top-k; histogram, scan, permute, gather; combine
+  if (p->dtype == MOE_DTYPE_BF16) {
+    Segments routed{reinterpret_cast<const int32_t*>(16), (int32_t)p->E, 0, p->T * p->k};
+    count += 2 * tc_gemm_launches(routed);
+    if (p->shared != MOE_SHARED_NONE) {
+      Segments sh{nullptr, 1, (int32_t)p->T, p->T};
+      count += 2 * tc_gemm_launches(sh);
+    }
+  } else {
+    count += 2 + (p->shared != MOE_SHARED_NONE ? 2 : 0);
+  }
+  if (two_streams && p->shared == MOE_SHARED_SIGMOID_GATED && shared_overlaps(*p)) count += 1;  // gate kernel
+  *n = count;
   return MOE_OK;
 }
 

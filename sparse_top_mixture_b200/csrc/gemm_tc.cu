@@ -143,8 +143,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 2) warp_build_tile_table(args.offsets, args.E, args.single_rows, BM, ctl->off, ctl->pre, args.rows_total,
-                                        args.err);
+  if (warp == 2)
+    warp_build_tile_table(args.offsets, args.E, args.single_rows, BM, ctl->off, ctl->pre, args.rows_total, args.err);
   if (warp == 1) tmem_alloc(&ctl->tmem_base, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -358,6 +358,9 @@ int num_sms() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
   return n;
 }
+
+// Launches one grouped GEMM takes.
+int tc_gemm_launches(const Segments&) { return 1; }
 
 int tc_gemm_variant(const Segments& sg) {
   // Pair tiles are 256 rows: with segments of a few hundred rows their tail

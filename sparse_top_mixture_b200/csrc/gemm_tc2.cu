@@ -19,7 +19,9 @@
 //
 // Used when segments average at least 384 rows. A row tile is 256 rows of one
 // segment; the peer skips its A load when the segment has no rows in its
-// half (its accumulator rows are then discarded).
+// half (its accumulator rows are then discarded). Handing short tails to a
+// separate one-CTA launch was measured slower: by then the tail experts'
+// weights have left L2 and are streamed from HBM a second time.
 // All waits are bounded as in the one-CTA kernel; a cluster barrier before
 // TMEM is freed guarantees no remote arrive or MMA still targets a CTA that
 // is about to exit.

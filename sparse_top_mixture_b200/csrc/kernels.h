@@ -27,6 +27,10 @@ cudaError_t launch_route(int dtype, const void* x, const void* gate_w, const voi
                          int64_t T, int64_t H, int64_t E, int64_t k, int score, int bias_mode, int renorm,
                          float* partial, float* weights, int64_t* selected, float* gamma, int32_t* err,
                          cudaStream_t s);
+// gamma[t] = sigmoid(x[t] . g) on its own (used when the shared expert runs
+// on a second stream, independent of the router).
+cudaError_t launch_shared_gate(int dtype, const void* x, const void* g, int64_t T, int64_t H, float* gamma,
+                               cudaStream_t s);
 cudaError_t launch_topk(const float* partial, int splits, int64_t ldo, int64_t T, int64_t E, int64_t k, int score,
                         int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
                         const void* x, const void* shared_gate, int64_t H, int dtype, float* gamma, cudaStream_t s);
@@ -64,6 +68,7 @@ cudaError_t launch_simt_down(const Segments& sg, const float* h, const float* w_
 // Variant: 1 = one CTA per 128-row tile; 2 = CTA pairs (cta_group::2) per
 // 256-row tile, used when segments average at least 128 rows.
 int tc_gemm_variant(const Segments& sg);
+int tc_gemm_launches(const Segments& sg);
 bool get_encode();
 bool make_tensor_map_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
                           const uint64_t* strides_bytes, const uint32_t* box);

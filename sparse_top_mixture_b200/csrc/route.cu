@@ -236,7 +236,46 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
   }
 }
 
+// gamma[t] = sigmoid(x[t] . g), one warp per token.
+template <typename TX>
+__global__ void __launch_bounds__(256) shared_gate_kernel(const TX* __restrict__ x, const TX* __restrict__ g, int Tn,
+                                                          int H, float* __restrict__ gamma) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= Tn) return;
+  constexpr int V = Elem<TX>::kPerVec;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
+  const uint4* gr = reinterpret_cast<const uint4*>(g);
+  float acc = 0.f;
+  for (int v = lane; v < H / V; v += 32) {
+    float a[8], b[8];
+    if constexpr (V == 8) {
+      unpack16_bf16(xr[v], a);
+      unpack16_bf16(gr[v], b);
+    } else {
+      unpack16(xr[v], a, nullptr);
+      unpack16(gr[v], b, nullptr);
+    }
+#pragma unroll
+    for (int q = 0; q < V; ++q) acc = fmaf(a[q], b[q], acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) gamma[t] = 1.0f / (1.0f + expf(-acc));
+}
+
 }  // namespace
+
+cudaError_t launch_shared_gate(int dtype, const void* x, const void* g, int64_t T, int64_t H, float* gamma,
+                               cudaStream_t s) {
+  const dim3 grid((unsigned)ceil_div(T, 8));
+  if (dtype == 0)
+    shared_gate_kernel<float><<<grid, 256, 0, s>>>((const float*)x, (const float*)g, (int)T, (int)H, gamma);
+  else
+    shared_gate_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)g,
+                                                           (int)T, (int)H, gamma);
+  return cudaGetLastError();
+}
 
 RouterPlan router_plan(int dtype, int64_t T, int64_t H, int64_t E) {
   RouterPlan r;

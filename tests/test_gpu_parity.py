@@ -251,6 +251,22 @@ def test_repeat_runs_are_bit_identical():
     assert all(torch.equal(u, v) for u, v in zip(a, b))
 
 
+@pytest.mark.parametrize("name", ["deepseek_v2_lite_zipf", "decode_weight_streaming", "dsv4_flash_ablation"])
+def test_two_stream_forward_matches_one_stream(name):
+    """The shared expert on a second stream (and its gate from its own kernel)
+    gives the same bits as the single-stream forward."""
+    cfg = SMALL[name]
+    cpu, dev = _inputs(cfg)
+    p = stm.Problem.from_config(cfg)
+    a = stm.SparseMoE(p, dev, overlap_shared=True)
+    b = stm.SparseMoE(p, dev, overlap_shared=False)
+    assert a.aux is not None and b.aux is None
+    ra = [t.clone() for t in a(dev["x"])]
+    rb = b(dev["x"])
+    torch.cuda.synchronize()
+    assert all(torch.equal(u, v) for u, v in zip(ra, rb))
+
+
 def test_empty_batch():
     cfg = SMALL["qwen3_30b_a3b"].replace(T=0)
     cpu, dev = _inputs(cfg)
