@@ -165,6 +165,31 @@ moe_status moe_dispatch(const moe_problem *p, const int64_t *selected_experts, c
                         int32_t *counts, int32_t *offsets, int32_t *sorted_pairs, int32_t *pair_pos,
                         void *x_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Sorted-segment dispatch that allocates nothing. The pages have no
+ * counterpart to this call; it exists for callers that cannot give the
+ * library a workspace because they may not allocate device memory: code
+ * running while another thread captures a CUDA graph in global capture mode
+ * (where cudaMalloc is an error), plug-ins inside a host framework whose
+ * memory pool owns the GPU, and latency-critical paths that must not wait on
+ * an allocator.
+ *   Same arguments and results as moe_dispatch, minus the workspace: the
+ *   per-block count matrix the dispatch kernels pass to each other lives in
+ *   a static 1 MiB device array inside this library (every GPU that loads the
+ *   library holds it until the process exits). Problems needing more than
+ *   2^18 count entries, ceil(T / max(1, 256 / k)) * E, are rejected with
+ *   MOE_ERR_UNSUPPORTED before anything is launched.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture. Calls allocate and free nothing.
+ *   Every call reuses the same array: calls whose work overlaps on the GPU
+ *   (two streams, or two host threads) race and corrupt each other's
+ *   results; serialise them. Nothing carried over from an earlier call is
+ *   read. A pair with an expert id outside [0, E) is skipped (pair_pos -1)
+ *   as in moe_dispatch, but no error flag is recorded. */
+moe_status moe_dispatch_noalloc(const moe_problem *p, const int64_t *selected_experts, const void *x,
+                                int32_t *counts, int32_t *offsets, int32_t *sorted_pairs, int32_t *pair_pos,
+                                void *x_perm, moe_stream_t stream);
+
 /* Grouped SwiGLU over the routed segments ("mstar.model.components.moe",
  * SparseMoeBlock fused layout; "Sparse MoE FFN for DFlash-family drafters",
  * grouped GEMM with no host syncs).

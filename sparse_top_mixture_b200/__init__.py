@@ -61,6 +61,7 @@ SIGNATURES = {
     "moe_route": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_topk_from_logits": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
     "moe_dispatch": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_dispatch_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_grouped_swiglu": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_shared_expert": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP]),
@@ -222,6 +223,27 @@ def dispatch(p: Problem, selected, x=None, ws=None) -> Dict[str, torch.Tensor]:
     _check(lib().moe_dispatch(ctypes.byref(p.c()), _ptr(selected), _ptr(x), _ptr(r["counts"]), _ptr(r["offsets"]),
                               _ptr(r["sorted_pairs"]), _ptr(r["pair_pos"]), _ptr(r["x_perm"]), ws.data_ptr(),
                               ws.numel(), _stream(dev)))
+    return r
+
+
+def dispatch_noalloc(p: Problem, selected, x=None) -> Dict[str, torch.Tensor]:
+    """moe_dispatch without a workspace, for callers that may not allocate
+    device memory (the library keeps the dispatch's scratch in a fixed device
+    array; concurrent calls must be serialised). The result tensors here are
+    still allocated by PyTorch for convenience."""
+    _req(selected, "selected_experts", (p.T, p.k), torch.int64)
+    dev = selected.device
+    P = p.T * p.k
+    if x is not None:
+        _req(x, "x", (p.T, p.H), p.torch_dtype)
+    r = {"counts": torch.empty(p.E, dtype=torch.int32, device=dev),
+         "offsets": torch.empty(p.E + 1, dtype=torch.int32, device=dev),
+         "sorted_pairs": torch.empty(P, dtype=torch.int32, device=dev),
+         "pair_pos": torch.empty(P, dtype=torch.int32, device=dev),
+         "x_perm": torch.empty(P, p.H, dtype=p.torch_dtype, device=dev) if x is not None else None}
+    _check(lib().moe_dispatch_noalloc(ctypes.byref(p.c()), _ptr(selected), _ptr(x), _ptr(r["counts"]),
+                                      _ptr(r["offsets"]), _ptr(r["sorted_pairs"]), _ptr(r["pair_pos"]),
+                                      _ptr(r["x_perm"]), _stream(dev)))
     return r
 
 
