@@ -132,19 +132,28 @@ def flops_and_bytes(cfg, n_active: int):
 
 
 
+GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc2.cu", "tc_ptx.cuh", "tc_epilogue.cuh", "tiles.cuh", "common.cuh")
+
+
+def kernel_source_hash() -> str:
+    """sha256 over the sources of the grouped-GEMM kernels."""
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "sparse_top_mixture_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def recorded_traffic(cfg_name: str):
     """Per-launch DRAM traffic of the gate_up kernel from the committed ncu
-    summary, if the kernel source is unchanged since it was taken."""
+    summary, if the kernel sources are unchanged since it was taken."""
     path = os.path.join(ROOT, "profiles", f"gate_up_{cfg_name}.md")
-    src = os.path.join(ROOT, "sparse_top_mixture_b200", "csrc", "gemm_tc.cu")
-    if not (os.path.exists(path) and os.path.exists(src)):
+    if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"gemm_tc_sha256:\s*([0-9a-f]+)", text)
-    if not m or not h:
-        return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+    h = re.search(r"kernel_sources_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h or kernel_source_hash() != h.group(1):
         return None
     return float(m.group(1))
 
