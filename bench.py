@@ -237,12 +237,19 @@ def init_dist(n_gpus: int):
 
 
 def dist_max(v: float, world: int) -> float:
+    """Max of v over ranks (the job's time is the slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, elapsed_ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (elapsed_ms_max / 1e3)
 
 
 def barrier(world: int):
@@ -359,7 +366,7 @@ def main():
         raise RuntimeError("device error flag set during the timed region")
 
     ms_per_step = elapsed_ms / args.steps
-    tokens_per_s = world * cfg.T * args.steps / (elapsed_ms / 1e3)
+    tokens_per_s = job_throughput(world, cfg.T, args.steps, elapsed_ms)
     active_tflops = world * fb["active_flops"] * args.steps / (elapsed_ms / 1e3) / 1e12
 
     # e2e: pinned host x in, host out back, through the public API
@@ -378,7 +385,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = dist_max(e0.elapsed_time(e1), world)
-    e2e_tps = world * cfg.T * e2e_steps / (e2e_ms / 1e3)
+    e2e_tps = job_throughput(world, cfg.T, e2e_steps, e2e_ms)
 
     pk = peaks()
     gu_ms = stage_ms["gate_up"]
