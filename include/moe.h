@@ -244,10 +244,10 @@ moe_status moe_forward_ex(const moe_problem *p, const moe_weights *w, const void
                           float *routing_weights, int64_t *selected_experts, void *ws, size_t ws_bytes,
                           moe_stream_t stream, moe_stream_t aux_stream, moe_event_t *stage_events);
 
-/* Which routed expert-GEMM implementation serves problem p: 0 = SIMT fp32;
- * 1 = tcgen05/TMEM, one CTA per 128-row tile; 2 = tcgen05 CTA pairs
- * (cta_group::2) per 256-row tile, chosen when segments average at least
- * 384 rows. Host only. */
+/* Which implementation serves problem p's routed gate_up GEMM: 0 = SIMT
+ * fp32; 1 = tcgen05/TMEM, one CTA per 128-row tile; 2 = tcgen05 CTA pairs
+ * (cta_group::2) per 256-row tile, chosen when segments average at least 192
+ * rows (the down GEMM switches to pairs from 384 rows). Host only. */
 moe_status moe_gemm_path(const moe_problem *p, int32_t *path);
 
 /* Number of kernel launches one forward of problem p makes (0 when T == 0):

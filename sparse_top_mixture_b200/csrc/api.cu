@@ -368,7 +368,7 @@ MOE_API moe_status moe_gemm_path(const moe_problem* p, int32_t* path) {
   } else {
     Segments sg{nullptr, (int32_t)p->E, 0, p->T * p->k};
     sg.offsets = reinterpret_cast<const int32_t*>(16);  // any non-null: routed segments
-    *path = tc_gemm_variant(sg);
+    *path = tc_gemm_variant(sg, false);
   }
   return MOE_OK;
 }

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
                                                             int tpe, int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets) {
   __shared__ int tot[kMaxExperts];
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int e = tid / tpe, part = tid % tpe;
   const bool active = e < E;
   const int chunk = (nblk + tpe - 1) / tpe;

@@ -91,7 +91,8 @@ struct __align__(8) Ctl {
   int pre[kMaxExperts + 1];
 };
 
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctl);
+constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;  // epilogue staging, one block per warp
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl);
 
 constexpr uint32_t kIdesc128 = make_idesc(128, UMMA_N);
 // M=64 tail tiles: the accumulator then occupies TMEM lanes 0-15 of each
@@ -125,7 +126,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                            const Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES);
+  float* epi_stage = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + EPI_BYTES);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int Eseg = args.offsets ? args.E : 1;
@@ -231,18 +233,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
       if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, args.err, 4)) break;
       tc_fence_after();
-      const int r = tc.m64 ? quarter * 16 + lane : quarter * 32 + lane;
-      const int row = tc.row0 + r;
-      const bool valid = row < tc.row_end && (!tc.m64 || lane < 16);
+      // this warp's rows: 32 consecutive (16 for an M=64 tile), lane = row
+      const int rows_w = tc.m64 ? 16 : 32;
+      const int row_w0 = tc.row0 + quarter * rows_w;
+      const int nrows = max(0, min(rows_w, tc.row_end - row_w0));
+      const int row = row_w0 + lane;
+      const bool valid = lane < nrows;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * UMMA_N);
+      float* stage = epi_stage + (warp - 2) * kStageFloatsPerWarp;
       if (MODE == MODE_GATE_UP) {
-        epilogue_swiglu(tbase, valid, reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row * args.ldo,
-                        tc.n_idx * 128, args.N);
+        epilogue_swiglu(tbase, 0, 128, 4, reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row_w0 * args.ldo,
+                        args.ldo, nrows, tc.n_idx * 128, args.N, lane);
       } else if (MODE == MODE_DOWN) {
         float sc = 1.f;
         if (valid && args.row_scale != nullptr) sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
-        epilogue_scale_f32(tbase, valid, sc, reinterpret_cast<float*>(args.out) + (int64_t)row * args.ldo,
-                           tc.n_idx * UMMA_N, args.N);
+        epilogue_scale_f32(tbase, UMMA_N / 32, sc, stage,
+                           reinterpret_cast<float*>(args.out) + (int64_t)row_w0 * args.ldo, args.ldo, nrows,
+                           tc.n_idx * UMMA_N, args.N, lane);
       } else {
         // router logits: fp32 partial sum of this k split; the row pitch is a
         // multiple of 4 floats, columns past N are not written.
@@ -362,11 +369,12 @@ int num_sms() {
 // Launches one grouped GEMM takes.
 int tc_gemm_launches(const Segments&) { return 1; }
 
-int tc_gemm_variant(const Segments& sg) {
-  // Pair tiles are 256 rows: with segments of a few hundred rows their tail
-  // padding costs more than the halved operand traffic saves.
+int tc_gemm_variant(const Segments& sg, bool down) {
+  // CTA pairs halve the operand bytes per SM but work on 256-row tiles. The
+  // gate_up GEMM (long K) gains from segments of about 192 rows on; the down
+  // GEMM (K = I, fp32 output, epilogue-heavy) only from about 384.
   const int64_t nseg = sg.offsets ? sg.E : 1;
-  return sg.rows_total >= 384 * nseg ? 2 : 1;
+  return sg.rows_total >= (down ? 384 : 192) * nseg ? 2 : 1;
 }
 
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
@@ -379,7 +387,7 @@ cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_g
     const uint32_t box[2] = {BK, BM};
     if (!make_tensor_map_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  if (tc_gemm_variant(sg) == 2) return launch_tc2_gate_up(sg, tmA, w_gate_up, E_w, h, I, H, err, num_sms(), s);
+  if (tc_gemm_variant(sg, false) == 2) return launch_tc2_gate_up(sg, tmA, w_gate_up, E_w, h, I, H, err, num_sms(), s);
   {
     // gate_up [E][2][I][H]: dim0 = H, dim1 = I (row within a half), dim2 = half, dim3 = expert
     const uint64_t dims[4] = {(uint64_t)H, (uint64_t)I, 2, (uint64_t)E_w};
@@ -401,7 +409,7 @@ cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down
     const uint32_t box[2] = {BK, BM};
     if (!make_tensor_map_bf16(&tmA, h, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  if (tc_gemm_variant(sg) == 2)
+  if (tc_gemm_variant(sg, true) == 2)
     return launch_tc2_down(sg, tmA, w_down, E_w, y, row_scale, scale_idx, H, I, err, num_sms(), s);
   {
     // down [E][H][I]: dim0 = I, dim1 = H, dim2 = expert

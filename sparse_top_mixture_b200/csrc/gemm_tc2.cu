@@ -18,10 +18,14 @@
 // No TMA multicast is used: every CTA fetches its own tiles.
 //
 // Used when segments average at least 384 rows. A row tile is 256 rows of one
-// segment; the peer skips its A load when the segment has no rows in its
-// half (its accumulator rows are then discarded). Handing short tails to a
-// separate one-CTA launch was measured slower: by then the tail experts'
-// weights have left L2 and are streamed from HBM a second time.
+// segment. A tile with at most 128 rows left (a segment's tail) runs as an
+// M=128 pair MMA instead, 64 rows per CTA, at half the MMA cost; its
+// accumulator holds output columns 0..127 in TMEM lanes 0-63 and 128..255 in
+// lanes 64-127, so for gate_up each CTA loads [64 gate rows | the matching 64
+// up rows] to keep every gate column next to its up column. The peer skips
+// its A load when the segment has no rows in its part of the tile (those
+// accumulator rows are discarded). Handing tails to a separate launch was
+// measured slower: the tail experts' weights had left L2 by then.
 // All waits are bounded as in the one-CTA kernel; a cluster barrier before
 // TMEM is freed guarantees no remote arrive or MMA still targets a CTA that
 // is about to exit.
@@ -53,6 +57,7 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * UMMA_N;
 constexpr int NTHREADS = 192;
 constexpr uint32_t kIdesc256 = make_idesc(256, UMMA_N);
+constexpr uint32_t kIdesc128 = make_idesc(128, UMMA_N);  // pair tile tails: 64 rows per CTA
 
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 
@@ -83,11 +88,14 @@ struct __align__(8) Ctl2 {
   int pre[kMaxExperts + 1];
 };
 
-constexpr size_t kSmemBytes2 = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctl2);
+constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;  // epilogue staging, one block per warp
+constexpr size_t kSmemBytes2 = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl2);
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
-  bool peer_rows;  // the peer's 128 rows hold any row of the segment
+  bool tail;       // at most 128 rows left: M=128 pair MMA, 64 rows per CTA
+  int rows_cta;    // rows per CTA: 128, or 64 for a tail
+  bool peer_rows;  // the peer's rows hold any row of the segment
 };
 
 __device__ __forceinline__ Tile2 decode_tile2(const Ctl2* ctl, int Eseg, int n_tiles, int tile) {
@@ -97,17 +105,20 @@ __device__ __forceinline__ Tile2 decode_tile2(const Ctl2* ctl, int Eseg, int n_t
   t.e = find_segment(ctl->pre, Eseg, mt);
   t.row0 = ctl->off[t.e] + (mt - ctl->pre[t.e]) * BM2;
   t.row_end = ctl->off[t.e + 1];
-  t.peer_rows = t.row0 + HALF < t.row_end;
+  t.tail = t.row_end - t.row0 <= HALF;
+  t.rows_cta = t.tail ? HALF / 2 : HALF;
+  t.peer_rows = t.row0 + t.rows_cta < t.row_end;
   return t;
 }
 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc2_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const Args2 args) {
+                            const __grid_constant__ CUtensorMap tmB64, const Args2 args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctl2* ctl = reinterpret_cast<Ctl2*>(base + STAGES * STAGE_BYTES);
+  float* epi_stage = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
+  Ctl2* ctl = reinterpret_cast<Ctl2*>(base + STAGES * STAGE_BYTES + EPI_BYTES);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -158,10 +169,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mbar_arrive_expect_tx(&ctl->full[stage],
                                   (uint32_t)(2 * B_BYTES + A_BYTES + (tc.peer_rows ? A_BYTES : 0)));
           const int k0 = kt * BK;
-          if (leader || tc.peer_rows) tma2_load_2d(sa, &tmA, full_leader, k0, tc.row0 + (int)rank * HALF);
+          if (leader || tc.peer_rows) tma2_load_2d(sa, &tmA, full_leader, k0, tc.row0 + (int)rank * tc.rows_cta);
           if (MODE == MODE_GATE_UP) {
-            // leader: gate rows n0..n0+127; peer: the matching up rows
-            tma2_load_4d(sb, &tmB, full_leader, k0, tc.n_idx * 128, (int)rank, tc.e);
+            if (!tc.tail) {
+              // leader: gate rows n0..n0+127; peer: the matching up rows
+              tma2_load_4d(sb, &tmB, full_leader, k0, tc.n_idx * 128, (int)rank, tc.e);
+            } else {
+              // each CTA: 64 gate rows then the matching 64 up rows
+              const int n0 = tc.n_idx * 128 + (int)rank * 64;
+              tma2_load_4d(sb, &tmB64, full_leader, k0, n0, 0, tc.e);
+              tma2_load_4d(sb + B_BYTES / 2, &tmB64, full_leader, k0, n0, 1, tc.e);
+            }
           } else {
             tma2_load_3d(sb, &tmB, full_leader, k0, tc.n_idx * UMMA_N + (int)rank * HALF, tc.e);
           }
@@ -187,6 +205,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+        const Tile2 tc = decode_tile2(ctl, Eseg, args.n_tiles, tile);
+        const uint32_t idesc = tc.tail ? kIdesc128 : kIdesc256;
         if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 12)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
@@ -198,7 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           const uint64_t bdesc = sw128_desc(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), kIdesc256,
+            umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
                        (kt > 0 || kk > 0) ? 1u : 0u);
           umma2_commit_mc(&ctl->empty[stage], 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -214,7 +234,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   } else {
     // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
     const int quarter = warp & 3;
-    const int r = (int)rank * HALF + quarter * 32 + lane;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
     int acc = 0;
@@ -223,17 +242,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       const Tile2 tc = decode_tile2(ctl, Eseg, args.n_tiles, tile);
       if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, args.err, 14)) break;
       tc_fence_after();
-      const int row = tc.row0 + r;
-      const bool valid = row < tc.row_end;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * UMMA_N);
+      // This warp's 32 consecutive rows (lane = row). Full tile: rows
+      // rank*128 + quarter*32 of the 256. Tail (M=128 pair): TMEM lane L holds
+      // row L % 64 of this CTA's 64 and column half L / 64.
+      const int half = tc.tail ? (quarter >> 1) : 0;
+      const int row_w0 = tc.tail ? tc.row0 + (int)rank * (HALF / 2) + 32 * (quarter & 1)
+                                 : tc.row0 + (int)rank * HALF + quarter * 32;
+      const int nrows = max(0, min(32, tc.row_end - row_w0));
+      const int row = row_w0 + lane;
+      float* stage = epi_stage + (warp - 2) * kStageFloatsPerWarp;
       if (MODE == MODE_GATE_UP) {
-        epilogue_swiglu(tbase, valid, reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row * args.ldo,
-                        tc.n_idx * 128, args.N);
+        __nv_bfloat16* orow0 = reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row_w0 * args.ldo;
+        if (!tc.tail)
+          epilogue_swiglu(tbase, 0, 128, 4, orow0, args.ldo, nrows, tc.n_idx * 128, args.N, lane);
+        else
+          epilogue_swiglu(tbase, 0, 64, 2, orow0, args.ldo, nrows, tc.n_idx * 128 + half * 64, args.N, lane);
       } else {
         float sc = 1.f;
-        if (valid && args.row_scale != nullptr) sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
-        epilogue_scale_f32(tbase, valid, sc, reinterpret_cast<float*>(args.out) + (int64_t)row * args.ldo,
-                           tc.n_idx * UMMA_N, args.N);
+        if (lane < nrows && args.row_scale != nullptr)
+          sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
+        float* orow0 = reinterpret_cast<float*>(args.out) + (int64_t)row_w0 * args.ldo;
+        if (!tc.tail)
+          epilogue_scale_f32(tbase, 8, sc, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N, args.N, lane);
+        else
+          epilogue_scale_f32(tbase, 4, sc, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N + half * 128, args.N,
+                             lane);
       }
       tc_fence_before();
       __syncwarp();
@@ -254,7 +288,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 template <int MODE>
-cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, int64_t N, int64_t K,
+cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmB64,
+                       int64_t N, int64_t K,
                        void* out, int64_t ldo, const float* row_scale, const int32_t* scale_idx, int32_t* err,
                        int num_sms, cudaStream_t s) {
   static std::once_flag attr_once;
@@ -280,7 +315,7 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM2 + nseg) * a.n_tiles;
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms / 2, max_tiles));
-  tc2_grouped_gemm_kernel<MODE><<<2 * pairs, NTHREADS, kSmemBytes2, s>>>(tmA, tmB, a);
+  tc2_grouped_gemm_kernel<MODE><<<2 * pairs, NTHREADS, kSmemBytes2, s>>>(tmA, tmB, tmB64, a);
   return cudaGetLastError();
 }
 
@@ -288,13 +323,16 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
 
 cudaError_t launch_tc2_gate_up(const Segments& sg, const CUtensorMap& tmA, const void* w_gate_up, int64_t E_w,
                                void* h, int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s) {
-  CUtensorMap tmB;
-  // gate_up [E][2][I][H], one half (128 rows of gate or of up) per CTA
+  CUtensorMap tmB, tmB64;
+  // gate_up [E][2][I][H]: 128 rows of gate or of up per CTA (full tiles), or
+  // 64 gate + 64 up rows per CTA (tail tiles)
   const uint64_t dims[4] = {(uint64_t)H, (uint64_t)I, 2, (uint64_t)E_w};
   const uint64_t strides[3] = {(uint64_t)H * 2, (uint64_t)I * H * 2, (uint64_t)2 * I * H * 2};
   const uint32_t box[4] = {BK, HALF, 1, 1};
+  const uint32_t box64[4] = {BK, HALF / 2, 1, 1};
   if (!make_tensor_map_bf16(&tmB, w_gate_up, 4, dims, strides, box)) return cudaErrorInvalidValue;
-  return launch_tc2<MODE_GATE_UP>(sg, tmA, tmB, I, H, h, I, nullptr, nullptr, err, num_sms, s);
+  if (!make_tensor_map_bf16(&tmB64, w_gate_up, 4, dims, strides, box64)) return cudaErrorInvalidValue;
+  return launch_tc2<MODE_GATE_UP>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
 }
 
 cudaError_t launch_tc2_down(const Segments& sg, const CUtensorMap& tmA, const void* w_down, int64_t E_w, void* y,
@@ -306,7 +344,7 @@ cudaError_t launch_tc2_down(const Segments& sg, const CUtensorMap& tmA, const vo
   const uint64_t strides[2] = {(uint64_t)I * 2, (uint64_t)H * I * 2};
   const uint32_t box[3] = {BK, HALF, 1};
   if (!make_tensor_map_bf16(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
-  return launch_tc2<MODE_DOWN>(sg, tmA, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+  return launch_tc2<MODE_DOWN>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
 }
 
 }  // namespace stm

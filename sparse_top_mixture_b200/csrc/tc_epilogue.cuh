@@ -8,60 +8,87 @@
 namespace stm {
 namespace tc {
 
-// gate_up: accumulator columns j (gate) and 128 + j (up) of output column
-// col0 + j; h = silu(gate) * up rounded to bf16, 16-byte stores, columns
-// past N skipped (N is a multiple of 8).
-__device__ __forceinline__ void epilogue_swiglu(uint32_t tbase, bool valid, __nv_bfloat16* orow, int col0, int N) {
+// Each epilogue warp owns 32 consecutive output rows (one per lane, i.e. per
+// TMEM lane) and walks the accumulator 32 columns at a time. The fp32 down
+// output goes through a per-warp staging block in shared memory, so that a
+// warp store instruction writes whole 128-byte row segments instead of one
+// 16-byte piece of 32 different rows (half-filled 32-byte sectors doubled
+// the L2 write traffic of that GEMM).
+constexpr int kStageStride = 36;                        // floats per staged row (144 B, keeps 16-byte alignment)
+constexpr int kStageFloatsPerWarp = 32 * kStageStride;  // 4608 B per epilogue warp
+
+// Write this lane's 32 fp32 values (row `lane` of the warp block) to
+// out_row0[r * ldo + j] for rows r < nrows and columns j < ncols (ncols a
+// multiple of 4).
+__device__ __forceinline__ void store_block_f32(const float (&v)[32], float* stage, float* out_row0, int64_t ldo,
+                                                int nrows, int ncols, int lane) {
+  float4* srow = reinterpret_cast<float4*>(stage + lane * kStageStride);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) srow[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int c4 = lane & 7;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = it * 4 + (lane >> 3);
+    if (r < nrows && c4 * 4 < ncols)
+      *reinterpret_cast<float4*>(out_row0 + (int64_t)r * ldo + c4 * 4) =
+          reinterpret_cast<const float4*>(stage + r * kStageStride)[c4];
+  }
+  __syncwarp();
+}
+
+// gate_up: TMEM columns gcol + j (gate) and ucol + j (up) hold output column
+// col0 + j; h = silu(gate) * up rounded to bf16. `nchunks` chunks of 32.
+// Each lane stores its own row directly (the bf16 output is small; staging
+// it through shared memory was measured slower than the write traffic it
+// saves). out_row0: output row of lane 0; nrows: valid rows of the warp.
+__device__ __forceinline__ void epilogue_swiglu(uint32_t tbase, int gcol, int ucol, int nchunks,
+                                                __nv_bfloat16* out_row0, int64_t ldo, int nrows, int col0, int N,
+                                                int lane) {
+  __nv_bfloat16* orow = out_row0 + (int64_t)lane * ldo;
+  const bool valid = lane < nrows;
 #pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < nchunks; ++c) {
     uint32_t g[32], u[32];
-    tmem_ld32(tbase + c * 32, g);
-    tmem_ld32(tbase + 128 + c * 32, u);
+    tmem_ld32(tbase + gcol + c * 32, g);
+    tmem_ld32(tbase + ucol + c * 32, u);
     tmem_ld_wait();
     const int cb = col0 + c * 32;
-    if (valid) {
+    if (!valid) continue;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        if (cb + v * 8 < N) {
-          float hv[8];
+    for (int v = 0; v < 4; ++v) {
+      if (cb + v * 8 < N) {
+        float hv[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            hv[q] = silu_f32(__uint_as_float(g[v * 8 + q])) * __uint_as_float(u[v * 8 + q]);
-          uint4 o;
-          o.x = pack_bf16x2(hv[0], hv[1]);
-          o.y = pack_bf16x2(hv[2], hv[3]);
-          o.z = pack_bf16x2(hv[4], hv[5]);
-          o.w = pack_bf16x2(hv[6], hv[7]);
-          *reinterpret_cast<uint4*>(orow + cb + v * 8) = o;
-        }
+        for (int q = 0; q < 8; ++q)
+          hv[q] = silu_f32(__uint_as_float(g[v * 8 + q])) * __uint_as_float(u[v * 8 + q]);
+        uint4 o;
+        o.x = pack_bf16x2(hv[0], hv[1]);
+        o.y = pack_bf16x2(hv[2], hv[3]);
+        o.z = pack_bf16x2(hv[4], hv[5]);
+        o.w = pack_bf16x2(hv[6], hv[7]);
+        *reinterpret_cast<uint4*>(orow + cb + v * 8) = o;
       }
     }
   }
 }
 
-// down: y = sc * accumulator in fp32, 16-byte stores, columns past N skipped
-// (N is a multiple of 8).
-__device__ __forceinline__ void epilogue_scale_f32(uint32_t tbase, bool valid, float sc, float* orow, int col0,
-                                                   int N) {
+// down: y = sc * accumulator in fp32 for `nchunks` chunks of 32 columns
+// starting at TMEM column 0 and output column col0. sc is this lane's row scale.
+__device__ __forceinline__ void epilogue_scale_f32(uint32_t tbase, int nchunks, float sc, float* stage,
+                                                   float* out_row0, int64_t ldo, int nrows, int col0, int N,
+                                                   int lane) {
 #pragma unroll 1
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < nchunks; ++c) {
     uint32_t d[32];
     tmem_ld32(tbase + c * 32, d);
     tmem_ld_wait();
     const int cb = col0 + c * 32;
-    if (valid) {
+    if (cb >= N || nrows <= 0) continue;  // warp-uniform
+    float v[32];
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        if (cb + v * 4 < N) {
-          float4 o;
-          o.x = sc * __uint_as_float(d[v * 4 + 0]);
-          o.y = sc * __uint_as_float(d[v * 4 + 1]);
-          o.z = sc * __uint_as_float(d[v * 4 + 2]);
-          o.w = sc * __uint_as_float(d[v * 4 + 3]);
-          *reinterpret_cast<float4*>(orow + cb + v * 4) = o;
-        }
-      }
-    }
+    for (int q = 0; q < 32; ++q) v[q] = sc * __uint_as_float(d[q]);
+    store_block_f32(v, stage, out_row0 + cb, ldo, nrows, N - cb, lane);
   }
 }
 

@@ -71,10 +71,10 @@ def test_invalid_problems_rejected(L, bad):
 
 
 def test_gemm_path(L):
-    # 0 = SIMT fp32; 1 = tcgen05 one CTA per 128-row tile; 2 = CTA pairs
+    # 0 = SIMT fp32; 1 = tcgen05 one CTA per 128-row tile; 2 = CTA pairs (gate_up GEMM reported)
     assert stm.gemm_path(_p(dtype="f32")) == 0
     assert stm.gemm_path(_p()) == 1  # 64*2 pairs over 8 experts: 16 rows per expert
-    assert stm.gemm_path(_p(T=4096, E=128, k=8)) == 1  # 256 rows per expert
+    assert stm.gemm_path(_p(T=4096, E=128, k=8)) == 2  # 256 rows per expert: gate_up on pairs
     assert stm.gemm_path(_p(T=8192, E=64, k=6)) == 2  # 768 rows per expert
     assert stm.gemm_path(_p(T=16, E=256, k=8)) == 1
 

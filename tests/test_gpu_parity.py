@@ -37,6 +37,8 @@ EDGE = {
     "many_tiles_one_expert": CONFIGS["qwen3_30b_a3b"].replace(name="skew", T=700, H=192, E=4, k=1, I=136),
     # routed segments averaging >= 128 rows run on CTA pairs (256-row tiles)
     "pairs_ragged": CONFIGS["qwen3_30b_a3b"].replace(name="pairs", T=1731, H=384, E=8, k=2, I=200),
+    # ~575 rows per expert: two 256-row pair tiles plus a ~40..100-row tail (M=128 pair MMA)
+    "pairs_tails": CONFIGS["qwen3_30b_a3b"].replace(name="pairs_tails", T=2300, H=320, E=8, k=2, I=200),
     "pairs_shared_skew": CONFIGS["deepseek_v2_lite_zipf"].replace(name="pairs_zipf", T=4200, H=256, I=136,
                                                                   I_shared=272),
 }
@@ -87,7 +89,7 @@ def test_both_tensor_core_variants_are_exercised():
     kernels are both reached by the parity cases above."""
     paths = {name: stm.gemm_path(stm.Problem.from_config(cfg)) for name, cfg in {**SMALL, **EDGE}.items()}
     assert paths["tiny_fp32"] == 0
-    assert paths["pairs_ragged"] == 2 and paths["pairs_shared_skew"] == 2
+    assert paths["pairs_ragged"] == 2 and paths["pairs_shared_skew"] == 2 and paths["pairs_tails"] == 2
     assert paths["qwen3_30b_a3b"] == 1 and paths["decode_weight_streaming"] == 1
 
 
