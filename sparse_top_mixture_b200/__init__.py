@@ -369,3 +369,48 @@ class SparseMoE:
 
     def read_device_error(self) -> int:
         return read_device_error(self.ws)
+
+
+class HostPipeline:
+    """Forward passes over batches that live in pinned host memory, with the
+    copies of one batch overlapping the compute of its neighbours.
+
+    Slot i % depth owns a stream, a workspace and device buffers; batch i is
+    copied in, run and copied back on its slot's stream, so batch i+1's
+    host->device copy and batch i-1's device->host copy proceed while batch i
+    computes (the GPU's copy engines run beside the SMs). Each batch's own
+    three steps stay ordered on its stream.
+    """
+
+    def __init__(self, moe: SparseMoE, depth: int = 2):
+        p = moe.p
+        self.moe = moe
+        self.slots = []
+        for i in range(depth):
+            m = moe if i == 0 else SparseMoE(p, moe.w, moe.device, overlap_shared=moe.aux is not None)
+            self.slots.append({
+                "moe": m,
+                "stream": torch.cuda.Stream(moe.device),
+                "x": torch.empty(p.T, p.H, dtype=p.torch_dtype, device=moe.device),
+                "out": torch.empty(p.T, p.H, dtype=p.torch_dtype, device=moe.device),
+                "rw": torch.empty(p.T, p.k, dtype=torch.float32, device=moe.device),
+                "sel": torch.empty(p.T, p.k, dtype=torch.int64, device=moe.device),
+            })
+        self.i = 0
+
+    def submit(self, x_host: torch.Tensor, out_host: torch.Tensor) -> torch.cuda.Stream:
+        """Enqueue one batch (pinned host tensors [T,H]); returns its stream.
+        out_host is complete once that stream has passed this call."""
+        slot = self.slots[self.i % len(self.slots)]
+        self.i += 1
+        s = slot["stream"]
+        s.wait_stream(torch.cuda.current_stream(self.moe.device))
+        with torch.cuda.stream(s):
+            slot["x"].copy_(x_host, non_blocking=True)
+            slot["moe"].forward(slot["x"], slot["out"], slot["rw"], slot["sel"])
+            out_host.copy_(slot["out"], non_blocking=True)
+        return s
+
+    def synchronize(self) -> None:
+        for slot in self.slots:
+            slot["stream"].synchronize()

@@ -269,6 +269,26 @@ def test_two_stream_forward_matches_one_stream(name):
     assert all(torch.equal(u, v) for u, v in zip(ra, rb))
 
 
+def test_host_pipeline_matches_forward():
+    """Batches from pinned host memory through the double-buffered pipeline
+    equal direct device forwards, bit for bit."""
+    cfg = SMALL["dsv4_flash_ablation"]
+    cpu, dev = _inputs(cfg)
+    p = stm.Problem.from_config(cfg)
+    moe = stm.SparseMoE(p, dev)
+    g = torch.Generator().manual_seed(3)
+    xs = [(torch.randn(cfg.T, cfg.H, generator=g)).to(torch.bfloat16).pin_memory() for _ in range(5)]
+    outs = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    pipe = stm.HostPipeline(moe, depth=2)
+    for xh, oh in zip(xs, outs):
+        pipe.submit(xh, oh)
+    pipe.synchronize()
+    for xh, oh in zip(xs, outs):
+        ref, _, _ = moe(xh.cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(oh, ref.cpu())
+
+
 def test_empty_batch():
     cfg = SMALL["qwen3_30b_a3b"].replace(T=0)
     cpu, dev = _inputs(cfg)
