@@ -259,6 +259,16 @@ moe_status moe_launches_per_forward(const moe_problem *p, int32_t two_streams, i
  * pointer), clear them. Returns MOE_ERR_DEVICE_FLAG when any bit was set. */
 moe_status moe_read_device_error(void *ws, int32_t *code, moe_stream_t stream);
 
+/* Diagnostic of the bounded pipeline waits. Every mbarrier wait in the
+ * tensor-core GEMMs gives up after a fixed budget of SM clocks, records
+ * MOE_DEVERR_WAIT_TIMEOUT in the workspace header and lets the kernel return,
+ * so a stalled pipeline is reported rather than hanging the GPU. This call
+ * launches one thread that waits, through the same routine with a ~10 ms
+ * budget, on an mbarrier nothing arrives on; afterwards moe_read_device_error
+ * on `ws` reports MOE_DEVERR_WAIT_TIMEOUT and the context stays usable. The
+ * pages have no counterpart to this call. */
+moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status s);
 

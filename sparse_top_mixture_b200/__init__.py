@@ -71,6 +71,7 @@ SIGNATURES = {
     "moe_gemm_path": (ctypes.c_int, [_PP, _I32P]),
     "moe_launches_per_forward": (ctypes.c_int, [_PP, ctypes.c_int32, _I32P]),
     "moe_read_device_error": (ctypes.c_int, [_VP, _I32P, _VP]),
+    "moe_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -177,6 +178,13 @@ def read_device_error(ws: torch.Tensor) -> int:
     if st not in (0, 5):
         _check(st)
     return int(code.value)
+
+
+def selftest_wait_timeout(ws: torch.Tensor) -> int:
+    """Run the bounded-wait self-test on ws's device; returns the error bits
+    it left (MOE_DEVERR_WAIT_TIMEOUT expected). Synchronises."""
+    _check(lib().moe_selftest_wait_timeout(ws.data_ptr(), ws.numel(), _stream(ws.device)))
+    return read_device_error(ws)
 
 
 def route(p: Problem, x, gate_w, bias=None, shared_gate=None, ws=None):

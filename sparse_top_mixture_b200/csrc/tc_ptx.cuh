@@ -51,13 +51,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int* abort, int32_t* err, int site,
-                                            bool draining) {
+                                            bool draining, long long limit_cycles = kWaitLimitCycles) {
   const long long start = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (!draining && *reinterpret_cast<volatile int*>(abort)) return false;
-      if (clock64() - start > kWaitLimitCycles) {
+      if (clock64() - start > limit_cycles) {
         *reinterpret_cast<volatile int*>(abort) = 1;
         if (err) {
           atomicOr(err, 2);

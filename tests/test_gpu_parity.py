@@ -289,6 +289,19 @@ def test_host_pipeline_matches_forward():
         assert torch.equal(oh, ref.cpu())
 
 
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A pipeline wait that runs out (a barrier nothing arrives on) returns an
+    error status the host reads; the CUDA context then still runs a forward."""
+    cfg = SMALL["qwen3_30b_a3b"]
+    cpu, dev = _inputs(cfg)
+    moe = _moe(cfg, dev)
+    assert stm.selftest_wait_timeout(moe.ws) == stm.DEVERR_WAIT_TIMEOUT
+    assert moe.read_device_error() == 0  # reading cleared the flag
+    out, _, _ = moe(dev["x"])
+    torch.cuda.synchronize()
+    assert moe.read_device_error() == 0 and torch.isfinite(out.float()).all()
+
+
 def test_empty_batch():
     cfg = SMALL["qwen3_30b_a3b"].replace(T=0)
     cpu, dev = _inputs(cfg)
