@@ -105,17 +105,27 @@ __global__ void __launch_bounds__(RTHREADS) router_logits_kernel(const T* __rest
   }
 }
 
-// (key, index) order of the top-k: larger key first, lower index on ties.
-__device__ __forceinline__ bool ranks_before(float ka, int ea, float kb, int eb) {
-  return ka > kb || (ka == kb && ea < eb);
+// The top-k orders experts by (key descending, index ascending). A float key
+// maps to an unsigned integer with the same order (sign bit flipped for
+// non-negative values, all bits for negative ones; -0 joins +0 and NaN ranks
+// below every number), so one warp-wide integer max finds the best key and one
+// integer min over the lanes holding it finds the lowest index among equals.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 0u;
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 constexpr int TOPK_WARPS = 8;
 
-template <typename TX>
+// One warp per token; lane l owns experts [l*NS, l*NS + NS), NS = 1, 2, 4 or
+// 8 (E up to 32, 64, 128 or 256), so a lane reads its logits of one partial
+// with one or two 16-byte loads when rows are 16-byte aligned.
+template <typename TX, int NS>
 __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ partial, int splits,
-                                                                int64_t ldo, int Tn, int E, int k, int score,
-                                                                int bias_mode, int renorm,
+                                                                int64_t ldo, int vec4, int Tn, int E, int k,
+                                                                int score, int bias_mode, int renorm,
                                                                 const float* __restrict__ bias,
                                                                 float* __restrict__ weights,
                                                                 int64_t* __restrict__ selected,
@@ -125,41 +135,58 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * TOPK_WARPS + (threadIdx.x >> 5);
   if (t >= Tn) return;
+  const int e0 = lane * NS;
 
-  float logit[8], sc[8], key[8];
+  float logit[NS], sc[NS];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    float l = -INFINITY;
-    if (e < E) {
-      l = 0.f;
-      for (int s = 0; s < splits; ++s) l += partial[((int64_t)s * Tn + t) * ldo + e];
-      if (bias_mode == 1) l += bias[e];
+  for (int i = 0; i < NS; ++i) logit[i] = 0.f;
+  if (NS >= 4 && vec4 && e0 + NS <= E) {
+    for (int s = 0; s < splits; ++s) {
+      const float4* src = reinterpret_cast<const float4*>(partial + ((int64_t)s * Tn + t) * ldo + e0);
+#pragma unroll
+      for (int v = 0; v < NS / 4; ++v) {
+        const float4 q = src[v];
+        logit[4 * v] += q.x;
+        logit[4 * v + 1] += q.y;
+        logit[4 * v + 2] += q.z;
+        logit[4 * v + 3] += q.w;
+      }
     }
-    logit[i] = l;
+  } else {
+    for (int s = 0; s < splits; ++s) {
+      const float* src = partial + ((int64_t)s * Tn + t) * ldo;
+#pragma unroll
+      for (int i = 0; i < NS; ++i)
+        if (e0 + i < E) logit[i] += src[e0 + i];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    if (e0 + i >= E) logit[i] = -INFINITY;
+    else if (bias_mode == 1) logit[i] += bias[e0 + i];
   }
   if (score == 0) {  // softmax over all E experts
     float m = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, logit[i]);
+    for (int i = 0; i < NS; ++i) m = fmaxf(m, logit[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float z = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      sc[i] = (lane + 32 * i < E) ? expf(logit[i] - m) : 0.f;
+    for (int i = 0; i < NS; ++i) {
+      sc[i] = (e0 + i < E) ? expf(logit[i] - m) : 0.f;
       z += sc[i];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sc[i] = sc[i] / z;
+    for (int i = 0; i < NS; ++i) sc[i] = sc[i] / z;
   } else if (score == 1) {  // sigmoid
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sc[i] = 1.0f / (1.0f + expf(-logit[i]));
+    for (int i = 0; i < NS; ++i) sc[i] = 1.0f / (1.0f + expf(-logit[i]));
   } else {  // sqrtsoftplus: sqrt(log(1 + e^l)), stable form
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < NS; ++i) {
       const float l = logit[i];
       sc[i] = sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
     }
@@ -167,44 +194,44 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
   // Selection key. Without a selection bias every score function is
   // increasing in the logit, so ranking by the logit ranks by the score and
   // avoids ties introduced by rounding the scores.
+  uint32_t key[NS];
+  uint32_t live = 0;  // bit i: expert e0 + i exists and is not yet taken
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = (bias_mode == 2 && e < E) ? sc[i] + bias[e] : logit[i];
+  for (int i = 0; i < NS; ++i) {
+    const int e = e0 + i;
+    key[i] = order_key((bias_mode == 2 && e < E) ? sc[i] + bias[e] : logit[i]);
+    if (e < E) live |= 1u << i;
   }
 
-  // Slot j's expert and raw weight go to shared memory; the renormalising
-  // sum runs in slot order (identical in every lane).
+  // Slot j's expert and raw weight go to shared memory, written by the lane
+  // that owns the expert; the renormalising sum runs in slot order.
   __shared__ float s_w[TOPK_WARPS][kMaxExperts];
   __shared__ int s_e[TOPK_WARPS][kMaxExperts];
   const int wid = threadIdx.x >> 5;
-  uint32_t taken = 0;
-  float tot = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY, bs = 0.f;
-    int be = 0x7fffffff;
+    // This lane's best live expert: largest key, then lowest index.
+    uint32_t bk = 0;
+    int bi = -1;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && ranks_before(key[i], e, bk, be)) {
-        bk = key[i]; be = e; bs = sc[i];
-      }
-    }
+    for (int i = 0; i < NS; ++i)
+      if (((live >> i) & 1u) && (bi < 0 || key[i] > bk)) { bk = key[i]; bi = i; }
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
+    const int cand = (bi >= 0 && bk == wk) ? e0 + bi : 0x7fffffff;
+    const int we = (int)__reduce_min_sync(0xffffffffu, (uint32_t)cand);
+    if (we == cand) {  // the owning lane
+      float w = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-      if (ranks_before(ok, oe, bk, be)) { bk = ok; be = oe; bs = os; }
+      for (int i = 0; i < NS; ++i)
+        if (i == bi) w = sc[i];
+      live &= ~(1u << bi);
+      s_w[wid][j] = w;
+      s_e[wid][j] = we;
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == 0) {
-      s_w[wid][j] = bs;
-      s_e[wid][j] = be;
-    }
-    tot += bs;
   }
   __syncwarp();
+  float tot = 0.f;
+  if (renorm)
+    for (int j = 0; j < k; ++j) tot += s_w[wid][j];
   for (int j = lane; j < k; j += 32) {
     float w = s_w[wid][j];
     if (renorm) w = tot > 0.f ? w / tot : 0.f;
@@ -304,18 +331,50 @@ size_t router_partial_bytes(int dtype, int64_t T, int64_t H, int64_t E) {
   return (size_t)r.splits * (size_t)T * (size_t)r.ldo * 4;
 }
 
+namespace {
+
+template <typename TX, int NS>
+void launch_topk_ns(dim3 grid, const float* partial, int splits, int64_t ldo, int vec4, int64_t T, int64_t E,
+                    int64_t k, int score, int bias_mode, int renorm, const float* bias, float* weights,
+                    int64_t* selected, const void* x, const void* shared_gate, int64_t H, float* gamma,
+                    cudaStream_t s) {
+  topk_kernel<TX, NS><<<grid, TOPK_WARPS * 32, 0, s>>>(partial, splits, ldo, vec4, (int)T, (int)E, (int)k, score,
+                                                       bias_mode, renorm, bias, weights, selected,
+                                                       (const TX*)x, (const TX*)shared_gate, (int)H, gamma);
+}
+
+template <typename TX>
+void launch_topk_t(dim3 grid, const float* partial, int splits, int64_t ldo, int vec4, int64_t T, int64_t E,
+                   int64_t k, int score, int bias_mode, int renorm, const float* bias, float* weights,
+                   int64_t* selected, const void* x, const void* shared_gate, int64_t H, float* gamma,
+                   cudaStream_t s) {
+  if (E <= 32)
+    launch_topk_ns<TX, 1>(grid, partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
+                          selected, x, shared_gate, H, gamma, s);
+  else if (E <= 64)
+    launch_topk_ns<TX, 2>(grid, partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
+                          selected, x, shared_gate, H, gamma, s);
+  else if (E <= 128)
+    launch_topk_ns<TX, 4>(grid, partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
+                          selected, x, shared_gate, H, gamma, s);
+  else
+    launch_topk_ns<TX, 8>(grid, partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
+                          selected, x, shared_gate, H, gamma, s);
+}
+
+}  // namespace
+
 cudaError_t launch_topk(const float* partial, int splits, int64_t ldo, int64_t T, int64_t E, int64_t k, int score,
                         int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
                         const void* x, const void* shared_gate, int64_t H, int dtype, float* gamma, cudaStream_t s) {
-  dim3 grid((unsigned)ceil_div(T, TOPK_WARPS));
+  const dim3 grid((unsigned)ceil_div(T, TOPK_WARPS));
+  const int vec4 = (ldo % 4 == 0 && (reinterpret_cast<uintptr_t>(partial) & 15u) == 0) ? 1 : 0;
   if (dtype == 0)
-    topk_kernel<float><<<grid, TOPK_WARPS * 32, 0, s>>>(partial, splits, ldo, (int)T, (int)E, (int)k, score,
-                                                        bias_mode, renorm, bias, weights, selected, (const float*)x,
-                                                        (const float*)shared_gate, (int)H, gamma);
+    launch_topk_t<float>(grid, partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights, selected,
+                         x, shared_gate, H, gamma, s);
   else
-    topk_kernel<__nv_bfloat16><<<grid, TOPK_WARPS * 32, 0, s>>>(
-        partial, splits, ldo, (int)T, (int)E, (int)k, score, bias_mode, renorm, bias, weights, selected,
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)shared_gate, (int)H, gamma);
+    launch_topk_t<__nv_bfloat16>(grid, partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
+                                 selected, x, shared_gate, H, gamma, s);
   return cudaGetLastError();
 }
 
