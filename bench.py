@@ -310,6 +310,7 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(workloads.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-graph", action="store_true", help="launch each kernel from the host every step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -343,27 +344,43 @@ def main():
     n_active = active_experts(sel, cfg.E)
     fb = flops_and_bytes(cfg, n_active)
 
-    nst = len(stm.STAGES) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
-    for row in evs:  # torch creates the CUDA event on its first record
-        for e in row:
-            e.record(stream)
+    # The timed steps replay the forward as one CUDA graph (the same kernels on
+    # the same buffers as the eager call, launched as one graph).
+    graphed = None if args.no_graph else stm.GraphedForward(moe, x, out, rw, sel)
+    step = graphed.replay if graphed is not None else (lambda: moe.forward(x, out, rw, sel))
+    for _ in range(args.warmup):
+        step()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         t_start.record(stream)
         for i in range(args.steps):
-            moe.forward(x, out, rw, sel, events=evs[i])
+            step()
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = dist_max(t_start.elapsed_time(t_end), world)
-    stage_ms = {}
-    for si, name in enumerate(stm.STAGES):
-        stage_ms[name] = sum(evs[i][si].elapsed_time(evs[i][si + 1]) for i in range(args.steps)) / args.steps
     if moe.read_device_error() != 0:
         raise RuntimeError("device error flag set during the timed region")
+
+    # Per-stage device times from a separate eager pass with CUDA events
+    # recorded between the stages, the median over its steps (the roofline
+    # below uses the gate_up one).
+    stage_steps = args.steps
+    nst = len(stm.STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(stage_steps)]
+    for row in evs:  # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for i in range(stage_steps):
+        moe.forward(x, out, rw, sel, events=evs[i])
+    torch.cuda.synchronize()
+    stage_ms = {}
+    for si, name in enumerate(stm.STAGES):
+        stage_ms[name] = statistics.median(evs[i][si].elapsed_time(evs[i][si + 1]) for i in range(stage_steps))
+    eager_ms = statistics.median(evs[i][0].elapsed_time(evs[i][nst - 1]) for i in range(stage_steps))
 
     ms_per_step = elapsed_ms / args.steps
     tokens_per_s = job_throughput(world, cfg.T, args.steps, elapsed_ms)
@@ -405,7 +422,8 @@ def main():
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(cfg.name)
-    roof["kernel"] = "tc_grouped_gemm_kernel<gate_up>"
+    roof["kernel"] = {0: "simt_grouped_kernel<gate_up>", 1: "tc_grouped_gemm_kernel<gate_up>",
+                      2: "tc2_grouped_gemm_kernel<gate_up> (CTA pairs)"}[stm.gemm_path(p)]
     roof["peak_source"] = pk["source"] + (" sustained bf16" if roof["bound"] == "tensor" else " copy bandwidth")
     roof["algorithmic"] = {"flops": fb["gate_up_flops"], "bytes": fb["gate_up_bytes"], "ms": gu_ms}
 
@@ -423,6 +441,8 @@ def main():
         "forward_roofline_frac": whole_roof_s / (ms_per_step / 1e3),
         "active_experts": n_active,
         "stage_ms": stage_ms,
+        "launch": "cuda_graph" if graphed is not None else "eager",
+        "eager_ms_per_step": eager_ms,
         "roofline": roof,
         "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": e2e_steps,

@@ -90,6 +90,8 @@ typedef enum { MOE_SHARED_NONE = 0, MOE_SHARED_PLAIN = 1, MOE_SHARED_SIGMOID_GAT
 /* Device-side error bits reported by moe_read_device_error. */
 #define MOE_DEVERR_BAD_EXPERT_ID 1 /* selected_experts held an id outside [0,E) */
 #define MOE_DEVERR_WAIT_TIMEOUT 2  /* a pipeline wait gave up (never expected)   */
+#define MOE_DEVERR_SMEM_LAYOUT 4   /* a GEMM found its shared memory misaligned
+                                      and computed nothing (never expected)   */
 
 typedef struct moe_problem {
   int64_t T;        /* tokens                                               */

@@ -31,6 +31,7 @@ TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 STAGES = ("route", "dispatch", "gate_up", "down", "shared", "combine")
 DEVERR_BAD_EXPERT_ID = 1
 DEVERR_WAIT_TIMEOUT = 2
+DEVERR_SMEM_LAYOUT = 4
 
 
 class MoeError(RuntimeError):
@@ -379,6 +380,36 @@ class SparseMoE:
         return read_device_error(self.ws)
 
 
+class GraphedForward:
+    """One forward recorded as a CUDA graph on fixed device buffers.
+
+    Replaying it runs the same kernels on the same buffers as
+    ``moe.forward(x, out, routing_weights, selected_experts)``, with one graph
+    launch in place of one launch per kernel. Write the next batch into ``x``
+    (on the stream the replay is issued on) and call ``replay()``; results
+    land in ``out``, ``routing_weights`` and ``selected_experts``.
+    """
+
+    def __init__(self, moe: "SparseMoE", x, out=None, routing_weights=None, selected_experts=None):
+        self.moe = moe
+        self.x = x
+        self.out, self.rw, self.sel = moe._outputs(x, out, routing_weights, selected_experts)
+        # one eager call first: the library's one-time host setup (kernel
+        # attributes, driver entry points) then happens outside the capture
+        moe.forward(self.x, self.out, self.rw, self.sel)
+        torch.cuda.synchronize(moe.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
+            moe.forward(self.x, self.out, self.rw, self.sel)
+        torch.cuda.synchronize(moe.device)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out, self.rw, self.sel
+
+    __call__ = replay
+
+
 class HostPipeline:
     """Forward passes over batches that live in pinned host memory, with the
     copies of one batch overlapping the compute of its neighbours.
@@ -390,20 +421,23 @@ class HostPipeline:
     three steps stay ordered on its stream.
     """
 
-    def __init__(self, moe: SparseMoE, depth: int = 2):
+    def __init__(self, moe: SparseMoE, depth: int = 2, graphs: bool = True):
         p = moe.p
         self.moe = moe
         self.slots = []
         for i in range(depth):
             m = moe if i == 0 else SparseMoE(p, moe.w, moe.device, overlap_shared=moe.aux is not None)
-            self.slots.append({
+            slot = {
                 "moe": m,
                 "stream": torch.cuda.Stream(moe.device),
                 "x": torch.empty(p.T, p.H, dtype=p.torch_dtype, device=moe.device),
                 "out": torch.empty(p.T, p.H, dtype=p.torch_dtype, device=moe.device),
                 "rw": torch.empty(p.T, p.k, dtype=torch.float32, device=moe.device),
                 "sel": torch.empty(p.T, p.k, dtype=torch.int64, device=moe.device),
-            })
+            }
+            # each slot's forward as one graph launch on the slot's buffers
+            slot["graph"] = GraphedForward(m, slot["x"], slot["out"], slot["rw"], slot["sel"]) if graphs else None
+            self.slots.append(slot)
         self.i = 0
 
     def submit(self, x_host: torch.Tensor, out_host: torch.Tensor) -> torch.cuda.Stream:
@@ -415,7 +449,10 @@ class HostPipeline:
         s.wait_stream(torch.cuda.current_stream(self.moe.device))
         with torch.cuda.stream(s):
             slot["x"].copy_(x_host, non_blocking=True)
-            slot["moe"].forward(slot["x"], slot["out"], slot["rw"], slot["sel"])
+            if slot["graph"] is not None:
+                slot["graph"].replay()
+            else:
+                slot["moe"].forward(slot["x"], slot["out"], slot["rw"], slot["sel"])
             out_host.copy_(slot["out"], non_blocking=True)
         return s
 

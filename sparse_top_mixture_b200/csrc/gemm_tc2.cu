@@ -35,6 +35,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "moe.h"
 #include "tc_epilogue.cuh"
 #include "tc_ptx.cuh"
 #include "tiles.cuh"
@@ -88,8 +89,13 @@ struct __align__(8) Ctl2 {
   int pre[kMaxExperts + 1];
 };
 
-constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;  // epilogue staging, one block per warp
-constexpr size_t kSmemBytes2 = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl2);
+// Shared memory: the stage ring, the epilogue staging blocks (one per
+// epilogue warp; used by down), then Ctl2. The dynamic shared memory starts
+// 1024-byte aligned (the 128-byte swizzle repeats every 1024 bytes); the
+// kernel checks this and does nothing if it is not.
+constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;
+constexpr size_t kSmemBytes2 = (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl2);
+static_assert(kSmemBytes2 <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
@@ -115,8 +121,14 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc2_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmB64, const Args2 args) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The same shared-window offset in every CTA of the grid: all of them
+  // return here, or none.
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) raise_error(args.err, MOE_DEVERR_SMEM_LAYOUT);
+    return;
+  }
+  uint8_t* base = smem_raw;
   float* epi_stage = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   Ctl2* ctl = reinterpret_cast<Ctl2*>(base + STAGES * STAGE_BYTES + EPI_BYTES);
   const int warp = threadIdx.x >> 5;
@@ -271,7 +283,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+      // down releases at CTA scope (its staged fp32 stores need not be
+      // visible to the leader first); gate_up measured faster with a
+      // cluster-scope release after its direct bf16 stores.
+      if (lane == 0) {
+        if (MODE == MODE_DOWN) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+        else mbar_arrive_remote_release(acc ? tempty_leader1 : tempty_leader0);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

@@ -185,8 +185,17 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).
+// Arrive on an mbarrier of a CTA of the cluster (shared::cluster address),
+// releasing at CTA scope: after tcgen05.fence::before_thread_sync this orders
+// the thread's TMEM loads before the arrive, without waiting for its global
+// stores to become visible across the cluster.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// The same arrive releasing at cluster scope: the thread's earlier global
+// stores are visible across the cluster before the arrive is.
+__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 

@@ -289,6 +289,31 @@ def test_host_pipeline_matches_forward():
         assert torch.equal(oh, ref.cpu())
 
 
+@pytest.mark.parametrize("name,overlap", [("pairs_shared_skew", False), ("decode_weight_streaming", True),
+                                           ("pairs_tails", False)])
+def test_graph_replay_matches_eager_forward(name, overlap):
+    """A forward captured as a CUDA graph (with the shared expert on its
+    second stream where it overlaps) gives the eager forward's bits, and
+    replays pick up new contents of the captured input buffer."""
+    cfg = EDGE.get(name) or SMALL[name]
+    cpu, dev = _inputs(cfg)
+    p = stm.Problem.from_config(cfg)
+    moe = stm.SparseMoE(p, dev, overlap_shared=overlap)
+    assert (moe.aux is not None) == (overlap and p.shared != "none")
+    x = dev["x"].clone()
+    gf = stm.GraphedForward(moe, x)
+    ref = stm.SparseMoE(p, dev, overlap_shared=False)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for it in range(3):
+        if it:
+            x.copy_(torch.randn(x.shape, generator=g, device="cuda").to(x.dtype))
+        got = [t.clone() for t in gf.replay()]
+        want = ref(x)
+        torch.cuda.synchronize()
+        assert all(torch.equal(u, v) for u, v in zip(got, want))
+    assert moe.read_device_error() == 0
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A pipeline wait that runs out (a barrier nothing arrives on) returns an
     error status the host reads; the CUDA context then still runs a forward."""
