@@ -344,6 +344,25 @@ def main():
     n_active = active_experts(sel, cfg.E)
     fb = flops_and_bytes(cfg, n_active)
 
+    # Per-stage device times from an eager pass with CUDA events recorded
+    # between the stages, right after the warm-up: the median per stage (the
+    # roofline below uses the gate_up one).
+    stage_steps = args.steps
+    nst = len(stm.STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(stage_steps)]
+    for row in evs:  # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as stage_clocks:
+        for i in range(stage_steps):
+            moe.forward(x, out, rw, sel, events=evs[i])
+        torch.cuda.synchronize()
+    stage_ms = {}
+    for si, name in enumerate(stm.STAGES):
+        stage_ms[name] = statistics.median(evs[i][si].elapsed_time(evs[i][si + 1]) for i in range(stage_steps))
+    eager_ms = statistics.median(evs[i][0].elapsed_time(evs[i][nst - 1]) for i in range(stage_steps))
+
     # The timed steps replay the forward as one CUDA graph (the same kernels on
     # the same buffers as the eager call, launched as one graph).
     graphed = None if args.no_graph else stm.GraphedForward(moe, x, out, rw, sel)
@@ -363,24 +382,6 @@ def main():
     elapsed_ms = dist_max(t_start.elapsed_time(t_end), world)
     if moe.read_device_error() != 0:
         raise RuntimeError("device error flag set during the timed region")
-
-    # Per-stage device times from a separate eager pass with CUDA events
-    # recorded between the stages, the median over its steps (the roofline
-    # below uses the gate_up one).
-    stage_steps = args.steps
-    nst = len(stm.STAGES) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(stage_steps)]
-    for row in evs:  # torch creates the CUDA event on its first record
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    for i in range(stage_steps):
-        moe.forward(x, out, rw, sel, events=evs[i])
-    torch.cuda.synchronize()
-    stage_ms = {}
-    for si, name in enumerate(stm.STAGES):
-        stage_ms[name] = statistics.median(evs[i][si].elapsed_time(evs[i][si + 1]) for i in range(stage_steps))
-    eager_ms = statistics.median(evs[i][0].elapsed_time(evs[i][nst - 1]) for i in range(stage_steps))
 
     ms_per_step = elapsed_ms / args.steps
     tokens_per_s = job_throughput(world, cfg.T, args.steps, elapsed_ms)
@@ -409,6 +410,23 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = dist_max(e0.elapsed_time(e1), world)
     e2e_tps = job_throughput(world, cfg.T, e2e_steps, e2e_ms)
+
+    # The balancer's deferred bias update (stash this forward's counts, then
+    # one sign-controller step), timed on its own: two one-block launches.
+    bal_stash = torch.zeros(cfg.E, dtype=torch.int64, device="cuda")
+    bal_bias = torch.zeros(cfg.E, dtype=torch.float32, device="cuda")
+    counts = moe.forward_counts()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        stm.bias_stash(p, counts, bal_stash)
+        stm.bias_update(p, bal_stash, bal_bias, 1e-3)
+    b0.record(stream)
+    for _ in range(100):
+        stm.bias_stash(p, counts, bal_stash)
+        stm.bias_update(p, bal_stash, bal_bias, 1e-3)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    balance_us = b0.elapsed_time(b1) * 1e3 / 100
 
     pk = peaks()
     gu_ms = stage_ms["gate_up"]
@@ -442,7 +460,9 @@ def main():
         "active_experts": n_active,
         "stage_ms": stage_ms,
         "launch": "cuda_graph" if graphed is not None else "eager",
+        "bias_update_us": balance_us,
         "eager_ms_per_step": eager_ms,
+        "stage_clocks": stage_clocks.summary(),
         "roofline": roof,
         "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": e2e_steps,

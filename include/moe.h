@@ -271,6 +271,31 @@ moe_status moe_read_device_error(void *ws, int32_t *code, moe_stream_t stream);
  * pages have no counterpart to this call. */
 moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Aux-loss-free balancing: the deferred sign-controller update of the fp32
+ * selection bias ("Sparse MoE FFN for DFlash-family drafters", What's here:
+ * MoEGate's bias moves by a sign controller from all-reduced expert loads,
+ * never by gradients; a forward stashes its routing counts and the update is
+ * applied before the next forward; a second apply changes nothing).
+ *   moe_bias_stash: load_stash[e] += counts[e] for e < p->E. counts [E] int32
+ *     as written by moe_dispatch / the forward; load_stash [E] int64, device,
+ *     caller-owned, zeroed by the caller before first use.
+ *   moe_bias_update: with L = load_stash (already summed over data-parallel
+ *     ranks when there are several) and mean m = sum(L) / E, bias[e] += rate
+ *     when L[e] < m, bias[e] -= rate when L[e] > m, unchanged when L[e] == m
+ *     (one fp32 add; the comparison is exact, in integers); then load_stash is
+ *     zeroed. bias [E] fp32, device. rate must be finite.
+ * Only p->E is read from the problem. One 256-thread block each; async on
+ * `stream`; pointers must be aligned to their element size. */
+moe_status moe_bias_stash(const moe_problem *p, const int32_t *counts, int64_t *load_stash, moe_stream_t stream);
+moe_status moe_bias_update(const moe_problem *p, int64_t *load_stash, float *bias, float rate,
+                           moe_stream_t stream);
+
+/* Device address of the per-expert counts [E] (int32) that the last
+ * moe_forward / moe_forward_ex on `ws` wrote, for moe_bias_stash: it stays
+ * valid, and the counts unchanged, until the next call that uses ws. Host
+ * only; checks ws_bytes against the problem's workspace size. */
+moe_status moe_forward_counts(const moe_problem *p, const void *ws, size_t ws_bytes, const int32_t **counts);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status s);
 

@@ -73,6 +73,9 @@ SIGNATURES = {
     "moe_launches_per_forward": (ctypes.c_int, [_PP, ctypes.c_int32, _I32P]),
     "moe_read_device_error": (ctypes.c_int, [_VP, _I32P, _VP]),
     "moe_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, _VP]),
+    "moe_bias_stash": (ctypes.c_int, [_PP, _VP, _VP, _VP]),
+    "moe_bias_update": (ctypes.c_int, [_PP, _VP, _VP, ctypes.c_float, _VP]),
+    "moe_forward_counts": (ctypes.c_int, [_PP, _VP, _SZ, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -378,6 +381,70 @@ class SparseMoE:
 
     def read_device_error(self) -> int:
         return read_device_error(self.ws)
+
+    def forward_counts(self) -> torch.Tensor:
+        """Per-expert counts [E] int32 of the last forward (a view into the
+        workspace, overwritten by the next forward)."""
+        ptr = ctypes.c_void_p()
+        _check(lib().moe_forward_counts(ctypes.byref(self.p.c()), self.ws.data_ptr(), self.ws.numel(),
+                                        ctypes.byref(ptr)))
+        off = ptr.value - self.ws.data_ptr()
+        return self.ws[off:off + 4 * self.p.E].view(torch.int32)
+
+
+def bias_stash(p: Problem, counts: torch.Tensor, load_stash: torch.Tensor) -> None:
+    """load_stash [E] int64 += counts [E] int32 (async on the current stream)."""
+    _req(counts, "counts", (p.E,), torch.int32)
+    _req(load_stash, "load_stash", (p.E,), torch.int64)
+    _check(lib().moe_bias_stash(ctypes.byref(p.c()), _ptr(counts), _ptr(load_stash), _stream(counts.device)))
+
+
+def bias_update(p: Problem, load_stash: torch.Tensor, bias: torch.Tensor, rate: float) -> None:
+    """Sign-controller step on bias [E] fp32 in place from load_stash [E]
+    int64 (then zeroed); async on the current stream."""
+    _req(load_stash, "load_stash", (p.E,), torch.int64)
+    _req(bias, "bias", (p.E,), torch.float32)
+    _check(lib().moe_bias_update(ctypes.byref(p.c()), _ptr(load_stash), _ptr(bias), float(rate),
+                                 _stream(bias.device)))
+
+
+def allreduce_loads(load_stash: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum the stashed loads over the ranks of `group` in place (no-op
+    without torch.distributed or with one rank)."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(load_stash, op=dist.ReduceOp.SUM, group=group)
+    return load_stash
+
+
+class BiasBalancer:
+    """Deferred aux-loss-free balancing of a SparseMoE's selection bias
+    ("Sparse MoE FFN for DFlash-family drafters", MoEGate and the deferred
+    balance updates): ``stash()`` after a forward adds that forward's
+    per-expert counts; ``update()`` before the next forward sums the stash
+    over the data-parallel ``group`` and moves the fp32 bias (the SparseMoE's
+    own ``bias`` tensor, in place) by ``rate`` toward balance, then clears the
+    stash, so a second ``update()`` changes nothing."""
+
+    def __init__(self, moe: "SparseMoE", rate: float, group=None):
+        if moe.p.bias_mode == "none" or moe.w.get("bias") is None:
+            raise ValueError("the problem has no selection / logit bias to balance")
+        self.moe = moe
+        self.rate = float(rate)
+        self.group = group
+        self.bias = moe.w["bias"]
+        self.load_stash = torch.zeros(moe.p.E, dtype=torch.int64, device=moe.device)
+
+    def forward_counts(self) -> torch.Tensor:
+        """View of the per-expert counts the last forward wrote (int32 [E])."""
+        return self.moe.forward_counts()
+
+    def stash(self, counts: Optional[torch.Tensor] = None) -> None:
+        bias_stash(self.moe.p, self.forward_counts() if counts is None else counts, self.load_stash)
+
+    def update(self) -> None:
+        allreduce_loads(self.load_stash, self.group)
+        bias_update(self.moe.p, self.load_stash, self.bias, self.rate)
 
 
 class GraphedForward:

@@ -396,6 +396,15 @@ MOE_API moe_status moe_launches_per_forward(const moe_problem* p, int32_t two_st
   return MOE_OK;
 }
 
+MOE_API moe_status moe_forward_counts(const moe_problem* p, const void* ws, size_t ws_bytes, const int32_t** counts) {
+  MOE_TRY(validate_problem(p));
+  if (counts == nullptr) return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  *counts = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + L.counts);
+  return MOE_OK;
+}
+
 MOE_API moe_status moe_read_device_error(void* ws, int32_t* code, moe_stream_t stream) {
   if (!ok_ptr(ws) || code == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   const cudaStream_t s = (cudaStream_t)stream;
