@@ -485,10 +485,12 @@ class HostPipeline:
     copied in, run and copied back on its slot's stream, so batch i+1's
     host->device copy and batch i-1's device->host copy proceed while batch i
     computes (the GPU's copy engines run beside the SMs). Each batch's own
-    three steps stay ordered on its stream.
+    three steps stay ordered on its stream. With depth 3 a slot's next input
+    copy never waits on its previous output copy while the compute engine is
+    busy, so the copies stay off the forward's critical path.
     """
 
-    def __init__(self, moe: SparseMoE, depth: int = 2, graphs: bool = True):
+    def __init__(self, moe: SparseMoE, depth: int = 3, graphs: bool = True):
         p = moe.p
         self.moe = moe
         self.slots = []
