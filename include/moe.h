@@ -249,7 +249,7 @@ moe_status moe_forward_ex(const moe_problem *p, const moe_weights *w, const void
 /* Which implementation serves problem p's routed gate_up GEMM: 0 = SIMT
  * fp32; 1 = tcgen05/TMEM, one CTA per 128-row tile; 2 = tcgen05 CTA pairs
  * (cta_group::2) per 256-row tile, chosen when segments average at least 192
- * rows (the down GEMM switches to pairs from 384 rows). Host only. */
+ * rows (the same threshold for the down GEMM). Host only. */
 moe_status moe_gemm_path(const moe_problem *p, int32_t *path);
 
 /* Number of kernel launches one forward of problem p makes (0 when T == 0):

@@ -369,12 +369,12 @@ int num_sms() {
 // Launches one grouped GEMM takes.
 int tc_gemm_launches(const Segments&) { return 1; }
 
-int tc_gemm_variant(const Segments& sg, bool down) {
-  // CTA pairs halve the operand bytes per SM but work on 256-row tiles. The
-  // gate_up GEMM (long K) gains from segments of about 192 rows on; the down
-  // GEMM (K = I, fp32 output, epilogue-heavy) only from about 384.
+int tc_gemm_variant(const Segments& sg, bool) {
+  // CTA pairs halve the operand bytes per SM (and the TMA loads in flight
+  // per unit of MMA work) but work on 256-row tiles: both GEMMs gain from
+  // segments of about 192 rows on.
   const int64_t nseg = sg.offsets ? sg.E : 1;
-  return sg.rows_total >= (down ? 384 : 192) * nseg ? 2 : 1;
+  return sg.rows_total >= 192 * nseg ? 2 : 1;
 }
 
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,

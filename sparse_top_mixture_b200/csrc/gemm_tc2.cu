@@ -17,7 +17,7 @@
 //     leader's accumulator-empty barrier.
 // No TMA multicast is used: every CTA fetches its own tiles.
 //
-// Used when segments average at least 384 rows. A row tile is 256 rows of one
+// Used when segments average at least 192 rows. A row tile is 256 rows of one
 // segment. A tile with at most 128 rows left (a segment's tail) runs as an
 // M=128 pair MMA instead, 64 rows per CTA, at half the MMA cost; its
 // accumulator holds output columns 0..127 in TMEM lanes 0-63 and 128..255 in

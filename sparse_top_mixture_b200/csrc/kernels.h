@@ -66,7 +66,7 @@ cudaError_t launch_simt_down(const Segments& sg, const float* h, const float* w_
 
 // tcgen05 / TMEM bf16 grouped GEMMs: h is bf16, y is fp32.
 // Variant: 1 = one CTA per 128-row tile; 2 = CTA pairs (cta_group::2) per
-// 256-row tile, for segments averaging at least 192 (gate_up) or 384 (down) rows.
+// 256-row tile, for segments averaging at least 192 rows.
 int tc_gemm_variant(const Segments& sg, bool down);
 int tc_gemm_launches(const Segments& sg);
 bool get_encode();
