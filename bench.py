@@ -344,25 +344,6 @@ def main():
     n_active = active_experts(sel, cfg.E)
     fb = flops_and_bytes(cfg, n_active)
 
-    # Per-stage device times from an eager pass with CUDA events recorded
-    # between the stages, right after the warm-up: the median per stage (the
-    # roofline below uses the gate_up one).
-    stage_steps = args.steps
-    nst = len(stm.STAGES) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(stage_steps)]
-    for row in evs:  # torch creates the CUDA event on its first record
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as stage_clocks:
-        for i in range(stage_steps):
-            moe.forward(x, out, rw, sel, events=evs[i])
-        torch.cuda.synchronize()
-    stage_ms = {}
-    for si, name in enumerate(stm.STAGES):
-        stage_ms[name] = statistics.median(evs[i][si].elapsed_time(evs[i][si + 1]) for i in range(stage_steps))
-    eager_ms = statistics.median(evs[i][0].elapsed_time(evs[i][nst - 1]) for i in range(stage_steps))
-
     # The timed steps replay the forward as one CUDA graph (the same kernels on
     # the same buffers as the eager call, launched as one graph).
     graphed = None if args.no_graph else stm.GraphedForward(moe, x, out, rw, sel)
@@ -383,13 +364,36 @@ def main():
     if moe.read_device_error() != 0:
         raise RuntimeError("device error flag set during the timed region")
 
+    # Per-stage device times: the same forward with CUDA events between the
+    # stages (recorded inside the graph when graphs are used), one step at a
+    # time, the median per stage over the steps (the roofline below uses the
+    # gate_up one).
+    nst = len(stm.STAGES) + 1
+    sev = [torch.cuda.Event(enable_timing=True) for _ in range(nst)]
+    for e in sev:  # torch creates the CUDA event on its first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    staged = None if args.no_graph else stm.GraphedForward(moe, x, out, rw, sel, events=sev)
+    stage_steps = min(args.steps, 100)
+    samples = []
+    with ClockSampler(local) as stage_clocks:
+        for i in range(stage_steps):
+            if staged is not None:
+                staged.replay()
+            else:
+                moe.forward(x, out, rw, sel, events=sev)
+            torch.cuda.synchronize()
+            samples.append([sev[si].elapsed_time(sev[si + 1]) for si in range(nst - 1)])
+    stage_ms = {name: statistics.median(row[si] for row in samples) for si, name in enumerate(stm.STAGES)}
+    staged_ms = statistics.median(sum(row) for row in samples)
+
     ms_per_step = elapsed_ms / args.steps
     tokens_per_s = job_throughput(world, cfg.T, args.steps, elapsed_ms)
     active_tflops = world * fb["active_flops"] * args.steps / (elapsed_ms / 1e3) / 1e12
 
     # e2e: pinned host x in, host out back, through the public API. Batches go
-    # through a double-buffered HostPipeline: every step still copies its own
-    # input in and its result out inside the timed region, overlapped with the
+    # through a three-slot HostPipeline: every step still copies its own input
+    # in and its result out inside the timed region, overlapped with the
     # neighbouring steps' compute.
     e2e_steps = args.e2e_steps or max(4, min(args.steps, 50))
     x_host = [r_cpu["x"].pin_memory(), r_cpu["x"].clone().pin_memory(), r_cpu["x"].clone().pin_memory()]
@@ -461,7 +465,7 @@ def main():
         "stage_ms": stage_ms,
         "launch": "cuda_graph" if graphed is not None else "eager",
         "bias_update_us": balance_us,
-        "eager_ms_per_step": eager_ms,
+        "stage_pass_ms_per_step": staged_ms,
         "stage_clocks": stage_clocks.summary(),
         "roofline": roof,
         "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * x.element_size(),

@@ -241,7 +241,9 @@ moe_status moe_forward(const moe_problem *p, const moe_weights *w, const void *x
  *     occupy every SM. All work is complete once `stream` has passed the call.
  *   stage_events: NULL, or MOE_NUM_STAGES + 1 caller-created events recorded
  *     on `stream` before each stage (MOE_STAGE_*) and after the last one; a
- *     NULL entry is skipped. */
+ *     NULL entry is skipped. While `stream` is being captured into a CUDA
+ *     graph they are recorded as event record nodes (cudaEventRecordExternal),
+ *     so every replay of the graph records them. */
 moe_status moe_forward_ex(const moe_problem *p, const moe_weights *w, const void *x, void *out,
                           float *routing_weights, int64_t *selected_experts, void *ws, size_t ws_bytes,
                           moe_stream_t stream, moe_stream_t aux_stream, moe_event_t *stage_events);

@@ -457,17 +457,19 @@ class GraphedForward:
     land in ``out``, ``routing_weights`` and ``selected_experts``.
     """
 
-    def __init__(self, moe: "SparseMoE", x, out=None, routing_weights=None, selected_experts=None):
+    def __init__(self, moe: "SparseMoE", x, out=None, routing_weights=None, selected_experts=None, events=None):
+        """``events``: optional len(STAGES)+1 timing events recorded between
+        the stages at every replay (as in ``SparseMoE.forward``)."""
         self.moe = moe
         self.x = x
         self.out, self.rw, self.sel = moe._outputs(x, out, routing_weights, selected_experts)
         # one eager call first: the library's one-time host setup (kernel
         # attributes, driver entry points) then happens outside the capture
-        moe.forward(self.x, self.out, self.rw, self.sel)
+        moe.forward(self.x, self.out, self.rw, self.sel, events=events)
         torch.cuda.synchronize(moe.device)
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
-            moe.forward(self.x, self.out, self.rw, self.sel)
+            moe.forward(self.x, self.out, self.rw, self.sel, events=events)
         torch.cuda.synchronize(moe.device)
 
     def replay(self):

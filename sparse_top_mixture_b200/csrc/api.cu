@@ -191,9 +191,15 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   if (!ok_ptr(x) || !ok_ptr(out) || !ok_ptr(weights) || !ok_ptr(selected)) return MOE_ERR_INVALID_ARGUMENT;
   Layout L;
   MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  // While `s` is being captured into a CUDA graph the events become event
+  // record nodes of the graph (recorded at every replay).
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (ev != nullptr) MOE_CUDA(cudaStreamIsCapturing(s, &capture));
   auto mark = [&](int i) -> moe_status {
-    if (ev != nullptr && ev[i] != nullptr) return cuda_status(cudaEventRecord(ev[i], s));
-    return MOE_OK;
+    if (ev == nullptr || ev[i] == nullptr) return MOE_OK;
+    if (capture == cudaStreamCaptureStatusActive)
+      return cuda_status(cudaEventRecordWithFlags(ev[i], s, cudaEventRecordExternal));
+    return cuda_status(cudaEventRecord(ev[i], s));
   };
   const bool has_shared = p->shared != MOE_SHARED_NONE;
   const bool gated = p->shared == MOE_SHARED_SIGMOID_GATED;

@@ -314,6 +314,26 @@ def test_graph_replay_matches_eager_forward(name, overlap):
     assert moe.read_device_error() == 0
 
 
+def test_graph_replay_records_stage_events():
+    """Stage events passed at capture become event record nodes: every
+    replay records them, in stage order, and the output is unchanged."""
+    cfg = EDGE["pairs_tails"]
+    cpu, dev = _inputs(cfg)
+    p = stm.Problem.from_config(cfg)
+    moe = stm.SparseMoE(p, dev)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stm.STAGES) + 1)]
+    for e in evs:
+        e.record()
+    gf = stm.GraphedForward(moe, dev["x"].clone(), events=evs)
+    ref = stm.SparseMoE(p, dev, overlap_shared=False)(dev["x"])[0]
+    for _ in range(2):
+        out = gf.replay()[0]
+        torch.cuda.synchronize()
+        times = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(stm.STAGES))]
+        assert all(t >= 0 for t in times) and times[stm.STAGES.index("gate_up")] > 0
+        assert torch.equal(out, ref)
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A pipeline wait that runs out (a barrier nothing arrives on) returns an
     error status the host reads; the CUDA context then still runs a forward."""
