@@ -142,6 +142,44 @@ def test_staged_calls_match_forward(name):
         gc.assert_within_bound(sh.cpu().double().numpy(), s_ref, s_bnd, "shared")
 
 
+@pytest.mark.parametrize("counts", [
+    [1, 64, 65, 127, 128, 129, 255, 256, 257, 300, 383, 384, 385, 512, 600, 641],
+    [300, 290, 257, 310, 384, 260, 270, 280],
+])
+def test_segment_sizes_around_pair_tile_edges(counts):
+    """Segments whose sizes sit on every edge of the CTA-pair tiling (pieces
+    of at most 128 rows that run as M=128 pair tiles, full and partial
+    256-row tiles): every y row of the grouped SwiGLU matches the fp64
+    per-segment reference within the arithmetic bound. Routing is planted,
+    so the sizes are exact."""
+    E, H, I = len(counts), 256, 192
+    T = sum(counts)
+    g = torch.Generator().manual_seed(len(counts))
+    ids = torch.cat([torch.full((c,), e, dtype=torch.int64) for e, c in enumerate(counts)])
+    sel = ids[torch.randperm(T, generator=g)].reshape(T, 1)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    gu = (torch.randn(E, 2 * I, H, generator=g) / H ** 0.5).to(torch.bfloat16)
+    dn = (torch.randn(E, H, I, generator=g) / I ** 0.5).to(torch.bfloat16)
+    rw = torch.rand(T, 1, generator=g) + 0.5
+    p = stm.Problem(T=T, H=H, E=E, k=1, I=I, dtype="bf16")
+    assert stm.gemm_path(p) == 2
+    ws = stm.new_workspace(p)
+    d = stm.dispatch(p, sel.cuda(), x.cuda(), ws=ws)
+    y = stm.grouped_swiglu(p, d["x_perm"], d["offsets"], gu.cuda(), dn.cuda(), rw.cuda(), d["sorted_pairs"], ws=ws)
+    torch.cuda.synchronize()
+    assert stm.read_device_error(ws) == 0
+    dd = gc.assert_dispatch_exact(d, sel.numpy(), E)
+    assert dd["counts"].tolist() == counts
+    xn, w = gc.np64(x), rw.double().numpy().reshape(-1)
+    y_ref = np.zeros((T, H))
+    y_bnd = np.zeros((T, H))
+    for e in range(E):
+        a, b = dd["offsets"][e], dd["offsets"][e + 1]
+        q = dd["sorted_pairs"][a:b]
+        y_ref[a:b], y_bnd[a:b] = gc.swiglu_with_bound(xn[q], gc.np64(gu[e]), gc.np64(dn[e]), w[q], "bf16")
+    gc.assert_within_bound(y.cpu().double().numpy(), y_ref, y_bnd, "y_perm")
+
+
 def test_topk_from_identical_logits_is_bit_exact():
     """On identical fp32 logits (with planted exact ties) the CUDA selection
     equals the oracle's, for every score function without a selection bias."""
