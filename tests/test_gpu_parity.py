@@ -218,8 +218,10 @@ def test_topk_selection_bias_within_tie_margin():
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (5, 3, 2), (257, 8, 2), (1000, 128, 8), (300, 64, 6), (64, 256, 256),
-                                   (4096, 128, 8)])
+                                   (4096, 128, 8), (8192, 256, 8)])
 def test_dispatch_bit_exact(T, E, k):
+    """Counting-sort dispatch equals the oracle's stable argsort bit for bit,
+    from one token up to a 256-block x 256-expert count matrix."""
     g = torch.Generator().manual_seed(T * 31 + E)
     sel = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int64)
     x = (torch.randn(T, 16, generator=g)).to(torch.bfloat16)
