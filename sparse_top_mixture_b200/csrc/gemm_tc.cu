@@ -299,12 +299,10 @@ template <int MODE>
 cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, int64_t N, int64_t K,
                       void* out, int64_t ldo, const float* row_scale, const int32_t* scale_idx, int32_t* err,
                       cudaStream_t s, int k_splits = 1) {
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(tc_grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemBytes);
-  });
+  static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance (MODE)
+  static cudaError_t attr_status[kSmemAttrDevices];
+  const void* kernel = reinterpret_cast<const void*>(tc_grouped_gemm_kernel<MODE>);
+  const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)kSmemBytes, attr_once, attr_status);
   if (attr_err != cudaSuccess) return attr_err;
   Args a;
   a.offsets = sg.offsets;

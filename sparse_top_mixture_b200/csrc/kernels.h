@@ -6,8 +6,22 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <mutex>
 
 namespace stm {
+
+// Raise a kernel's dynamic shared memory limit to `bytes` once per device
+// (the attribute belongs to the kernel's module in each device context).
+// Each kernel passes its own flag and status arrays of kSmemAttrDevices.
+constexpr int kSmemAttrDevices = 64;
+inline cudaError_t set_max_dynamic_smem_once(const void* kernel, int bytes, std::once_flag* once, cudaError_t* err) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSmemAttrDevices) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    err[dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+  return err[dev];
+}
 
 // ---- router -----------------------------------------------------------
 // Logits are computed as `splits` fp32 partial sums along H, each [T, ldo]
