@@ -443,6 +443,8 @@ def main():
         achieved = fb["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    if roof["bound"] == "hbm":  # also against the nominal 8 TB/s of HBM3e
+        roof["frac_of_nominal_8000gbs"] = roof["achieved"] / 8000.0
     roof["traffic"] = recorded_traffic(cfg.name)
     roof["kernel"] = {0: "simt_grouped_kernel<gate_up>", 1: "tc_grouped_gemm_kernel<gate_up>",
                       2: "tc2_grouped_gemm_kernel<gate_up> (CTA pairs)"}[stm.gemm_path(p)]
