@@ -325,6 +325,9 @@ def main():
         return
 
     import sparse_top_mixture_b200 as stm
+    if not os.path.exists(stm.LIB_PATH):  # the CUDA library is built in-tree
+        from sparse_top_mixture_b200 import build
+        build.build()
 
     r_cpu, dev = make_inputs(cfg, rank)
     p = stm.Problem.from_config(cfg)

@@ -8,6 +8,13 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    # The CUDA library is built in-tree; build it once if this checkout has none.
+    if not os.path.exists(os.path.join(ROOT, "sparse_top_mixture_b200", "libstm_moe.so")):
+        from sparse_top_mixture_b200 import build
+        build.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: takes more than a few seconds")
