@@ -89,13 +89,19 @@ struct __align__(8) Ctl2 {
   int pre[kMaxExperts + 1];
 };
 
-// Shared memory: the stage ring, the epilogue staging blocks (one per
-// epilogue warp; used by down), then Ctl2. The dynamic shared memory starts
-// 1024-byte aligned (the 128-byte swizzle repeats every 1024 bytes); the
-// kernel checks this and does nothing if it is not.
+// Shared memory: the stage ring (its base 1024-byte aligned: the 128-byte
+// swizzle repeats every 1024 bytes), the epilogue staging blocks (one per
+// epilogue warp; used by down), then Ctl2. down declares the dynamic shared
+// memory 1024-byte aligned and checks it (doing nothing if it is not);
+// gate_up requests 1 KB more and rounds its base up. Each variant measured
+// 3-9% faster for its GEMM than the other layout (the same code otherwise).
 constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;
-constexpr size_t kSmemBytes2 = (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl2);
-static_assert(kSmemBytes2 <= 232448, "dynamic shared memory above the 227 KB per-block limit");
+template <int MODE>
+constexpr size_t smem_bytes2() {
+  return (MODE == MODE_GATE_UP ? 1024 : 0) + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl2);
+}
+static_assert(smem_bytes2<MODE_GATE_UP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
+static_assert(smem_bytes2<MODE_DOWN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
@@ -121,14 +127,20 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc2_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmB64, const Args2 args) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // The same shared-window offset in every CTA of the grid: all of them
-  // return here, or none.
-  if ((smem_u32(smem_raw) & 1023u) != 0) {
-    if (threadIdx.x == 0) raise_error(args.err, MOE_DEVERR_SMEM_LAYOUT);
-    return;
+  uint8_t* base;
+  if constexpr (MODE == MODE_GATE_UP) {
+    extern __shared__ uint8_t smem_gu[];
+    base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_gu) + 1023) & ~uintptr_t(1023));
+  } else {
+    extern __shared__ __align__(1024) uint8_t smem_dn[];
+    // The same shared-window offset in every CTA of the grid: all of them
+    // return here, or none.
+    if ((smem_u32(smem_dn) & 1023u) != 0) {
+      if (threadIdx.x == 0) raise_error(args.err, MOE_DEVERR_SMEM_LAYOUT);
+      return;
+    }
+    base = smem_dn;
   }
-  uint8_t* base = smem_raw;
   float* epi_stage = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   Ctl2* ctl = reinterpret_cast<Ctl2*>(base + STAGES * STAGE_BYTES + EPI_BYTES);
   const int warp = threadIdx.x >> 5;
@@ -313,7 +325,7 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance (MODE)
   static cudaError_t attr_status[kSmemAttrDevices];
   const void* kernel = reinterpret_cast<const void*>(tc2_grouped_gemm_kernel<MODE>);
-  const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)kSmemBytes2, attr_once, attr_status);
+  const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)smem_bytes2<MODE>(), attr_once, attr_status);
   if (attr_err != cudaSuccess) return attr_err;
   Args2 a;
   a.offsets = sg.offsets;
@@ -331,7 +343,7 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM2 + nseg) * a.n_tiles;
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms / 2, max_tiles));
-  tc2_grouped_gemm_kernel<MODE><<<2 * pairs, NTHREADS, kSmemBytes2, s>>>(tmA, tmB, tmB64, a);
+  tc2_grouped_gemm_kernel<MODE><<<2 * pairs, NTHREADS, smem_bytes2<MODE>(), s>>>(tmA, tmB, tmB64, a);
   return cudaGetLastError();
 }
 
