@@ -33,7 +33,8 @@
  * Conventions for every call:
  *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
  *     stated otherwise. The library never allocates, frees or synchronises,
- *     except moe_read_device_error, which synchronises the given stream.
+ *     except moe_read_device_error / moe_check_device_error, which
+ *     synchronise the given stream.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and runs asynchronously. Outputs are valid once the stream has
  *     passed the call.
@@ -262,6 +263,9 @@ moe_status moe_launches_per_forward(const moe_problem *p, int32_t two_streams, i
 /* Synchronise `stream`, read the workspace error bits into *code (host
  * pointer), clear them. Returns MOE_ERR_DEVICE_FLAG when any bit was set. */
 moe_status moe_read_device_error(void *ws, int32_t *code, moe_stream_t stream);
+
+/* The same call with the stream before the result pointer. */
+moe_status moe_check_device_error(void *ws, moe_stream_t stream, int32_t *code);
 
 /* Diagnostic of the bounded pipeline waits. Every mbarrier wait in the
  * tensor-core GEMMs gives up after a fixed budget of SM clocks, records

@@ -72,6 +72,7 @@ SIGNATURES = {
     "moe_gemm_path": (ctypes.c_int, [_PP, _I32P]),
     "moe_launches_per_forward": (ctypes.c_int, [_PP, ctypes.c_int32, _I32P]),
     "moe_read_device_error": (ctypes.c_int, [_VP, _I32P, _VP]),
+    "moe_check_device_error": (ctypes.c_int, [_VP, _VP, _I32P]),
     "moe_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, _VP]),
     "moe_bias_stash": (ctypes.c_int, [_PP, _VP, _VP, _VP]),
     "moe_bias_update": (ctypes.c_int, [_PP, _VP, _VP, ctypes.c_float, _VP]),

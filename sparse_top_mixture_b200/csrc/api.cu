@@ -426,6 +426,10 @@ MOE_API moe_status moe_read_device_error(void* ws, int32_t* code, moe_stream_t s
   return MOE_OK;
 }
 
+MOE_API moe_status moe_check_device_error(void* ws, moe_stream_t stream, int32_t* code) {
+  return moe_read_device_error(ws, code, stream);
+}
+
 MOE_API const char* moe_status_string(moe_status s) {
   switch (s) {
     case MOE_OK: return "ok";
