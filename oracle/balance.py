@@ -15,7 +15,7 @@ balance-update semantics):
   bias once (the second apply finds nothing stashed);
 * the step size is a configured update rate.
 
-Readings taken where the page is silent (listed in the design doc):
+Readings taken where the page is silent:
 
 * loads L[e] = routing counts stashed since the last update, summed over
   data-parallel ranks; the target is their mean m = sum(L) / E;

@@ -35,7 +35,7 @@ What it computes, and where each step is defined:
   SparseMoeBlockWithSharedExpert; "MoE: shared experts, parameterized V_TOPK
   routing, explicit stage attribution", 3. Tests, the three variants).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 softmax is over all E experts before top-k; equal keys go to the lower expert
 index; the gate half of gate_up comes first; the shared gate is a bias-free
 vector [H]; the routed scaling factor is 1; a zero renormalisation sum gives
