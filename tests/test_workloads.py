@@ -3,6 +3,7 @@
 import json
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -65,3 +66,15 @@ def test_oracle_rows_are_independent():
     part = oracle.moe_forward(a["x"][rows], a["gate_w"], a["gate_up"], a["down"], skip_unrouted=True, **kw)
     assert np.array_equal(part["selected_experts"], full["selected_experts"][rows])
     assert np.abs(part["out"] - full["out"][rows]).max() <= 1e-13 * np.abs(full["out"]).max()
+
+
+def test_decode_shared_gate_is_not_saturated():
+    """The sigmoid shared-expert gate of the decode problem must stay away from
+    saturation (|x . g| < 15 on every token, and spread out), so that a gate
+    that is dropped or applied twice changes the output visibly."""
+    cfg = workloads.CONFIGS["decode_weight_streaming"]
+    r = workloads.router_inputs(cfg)
+    z = r["x"].double() @ r["shared_gate"].double()
+    assert z.abs().max().item() < 15
+    gamma = torch.sigmoid(z)
+    assert gamma.std().item() > 0.05 and (gamma - 0.5).abs().max().item() > 0.1
