@@ -302,6 +302,41 @@ moe_status moe_bias_update(const moe_problem *p, int64_t *load_stash, float *bia
  * only; checks ws_bytes against the problem's workspace size. */
 moe_status moe_forward_counts(const moe_problem *p, const void *ws, size_t ws_bytes, const int32_t **counts);
 
+/* Gradient outputs of moe_backward. All fp32, device, caller-owned, 16-byte
+ * aligned, fully overwritten (never accumulated into). */
+typedef struct moe_grads {
+  float *dx;               /* [T, H]                                          */
+  float *d_gate_w;         /* [E, H]                                          */
+  float *d_bias;           /* [E] when bias_mode == LOGIT, else NULL          */
+  float *d_gate_up;        /* [E, 2I, H]                                      */
+  float *d_down;           /* [E, H, I]                                       */
+  float *d_shared_gate_up; /* [2*I_shared, H] with a shared expert, else NULL */
+  float *d_shared_down;    /* [H, I_shared] with a shared expert, else NULL   */
+  float *d_shared_gate;    /* [H] when SIGMOID_GATED, else NULL               */
+} moe_grads;
+
+/* Backward of the whole forward ("Sparse MoE FFN for DFlash-family
+ * drafters", What's here: the backward pass through the grouped GEMM; Tests:
+ * grad parity against a per-expert loop). Gradients of sum(dout * out) for
+ * out = moe_forward(x) with the expert choice held at selected_experts:
+ * top-k selection is piecewise constant, so no gradient flows through the
+ * choice, and none reaches a SELECT bias (it only ranks experts; the
+ * balancer moves it). A LOGIT bias gets sum over tokens of dlogits.
+ *   x [T,H], dout [T,H], weights as for moe_forward, selected_experts [T,k]
+ *   int64 (normally the forward's). Routing weights, the per-expert
+ *   activations and outputs are recomputed from x; nothing from the forward
+ *   is needed besides the choice.
+ *   fp32 problems only (MOE_ERR_UNSUPPORTED for bf16). Each gradient element
+ *   is one thread's fixed-order fp32 sum (no atomics): results are
+ *   deterministic. A pair with an expert id outside [0, E) contributes
+ *   nothing and sets MOE_DEVERR_BAD_EXPERT_ID in the workspace header.
+ *   Workspace: moe_backward_workspace_size bytes (its header as for
+ *   moe_forward, zeroed by moe_workspace_init). Async on `stream`. */
+moe_status moe_backward_workspace_size(const moe_problem *p, size_t *bytes);
+moe_status moe_backward(const moe_problem *p, const moe_weights *w, const void *x, const void *dout,
+                        const int64_t *selected_experts, moe_grads *g, void *ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
 /* Static description of a status code. */
 const char *moe_status_string(moe_status s);
 

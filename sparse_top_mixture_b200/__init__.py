@@ -53,6 +53,12 @@ class moe_weights(ctypes.Structure):
                 ("shared_gate", ctypes.c_void_p)]
 
 
+class moe_grads(ctypes.Structure):
+    _fields_ = [("dx", ctypes.c_void_p), ("d_gate_w", ctypes.c_void_p), ("d_bias", ctypes.c_void_p),
+                ("d_gate_up", ctypes.c_void_p), ("d_down", ctypes.c_void_p), ("d_shared_gate_up", ctypes.c_void_p),
+                ("d_shared_down", ctypes.c_void_p), ("d_shared_gate", ctypes.c_void_p)]
+
+
 # name -> (restype, argtypes)
 _VP, _I32P, _SZ = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_size_t
 _PP = ctypes.POINTER(moe_problem)
@@ -77,6 +83,9 @@ SIGNATURES = {
     "moe_bias_stash": (ctypes.c_int, [_PP, _VP, _VP, _VP]),
     "moe_bias_update": (ctypes.c_int, [_PP, _VP, _VP, ctypes.c_float, _VP]),
     "moe_forward_counts": (ctypes.c_int, [_PP, _VP, _SZ, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_backward_workspace_size": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_backward": (ctypes.c_int, [_PP, ctypes.POINTER(moe_weights), _VP, _VP, _VP, ctypes.POINTER(moe_grads), _VP,
+                                    _SZ, _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -321,6 +330,41 @@ def _weights_struct(p: Problem, w: Dict[str, Optional[torch.Tensor]]) -> moe_wei
                        g("shared_gate_up") if p.shared != "none" else None,
                        g("shared_down") if p.shared != "none" else None,
                        g("shared_gate") if p.shared == "sigmoid_gated" else None)
+
+
+def backward_workspace_size(p: Problem) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().moe_backward_workspace_size(ctypes.byref(p.c()), ctypes.byref(n)))
+    return n.value
+
+
+def backward(p: Problem, weights: Dict[str, Optional[torch.Tensor]], x, dout, selected, ws=None
+             ) -> Dict[str, Optional[torch.Tensor]]:
+    """Gradients of sum(dout * out) for the fp32 forward with the expert choice
+    held at ``selected`` [T,k] int64: dx, d_gate_w, d_bias (logit bias only),
+    d_gate_up, d_down and, with a shared expert, d_shared_gate_up,
+    d_shared_down and d_shared_gate (gated only). Async on the current stream."""
+    if p.dtype != "f32":
+        raise MoeError(2, "moe_backward supports fp32 problems only")
+    cw = _weights_struct(p, weights)
+    _req(x, "x", (p.T, p.H), torch.float32)
+    _req(dout, "dout", (p.T, p.H), torch.float32)
+    _req(selected, "selected", (p.T, p.k), torch.int64)
+    dev = x.device
+    z = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)  # noqa: E731
+    g = {"dx": z(p.T, p.H), "d_gate_w": z(p.E, p.H), "d_bias": z(p.E) if p.bias_mode == "logit" else None,
+         "d_gate_up": z(p.E, 2 * p.I, p.H), "d_down": z(p.E, p.H, p.I), "d_shared_gate_up": None,
+         "d_shared_down": None, "d_shared_gate": None}
+    if p.shared != "none":
+        g["d_shared_gate_up"], g["d_shared_down"] = z(2 * p.I_shared, p.H), z(p.H, p.I_shared)
+    if p.shared == "sigmoid_gated":
+        g["d_shared_gate"] = z(p.H)
+    if ws is None:
+        ws = torch.zeros(backward_workspace_size(p), dtype=torch.uint8, device=dev)
+    cg = moe_grads(*[_ptr(g[f]) for f, _ in moe_grads._fields_])
+    _check(lib().moe_backward(ctypes.byref(p.c()), ctypes.byref(cw), _ptr(x), _ptr(dout), _ptr(selected),
+                              ctypes.byref(cg), ws.data_ptr(), ws.numel(), _stream(dev)))
+    return g
 
 
 class SparseMoE:

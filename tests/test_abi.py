@@ -119,3 +119,29 @@ def test_empty_batch_is_a_noop(L):
     assert L.moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
     st = L.moe_forward(ctypes.byref(p), ctypes.byref(w), 16, 16, 16, 16, 16, n.value, None)
     assert st == 0
+
+
+def test_backward_validates_before_launching(L):
+    """moe_backward rejects bad arguments on the host (no GPU needed)."""
+    w = stm.moe_weights(16, None, 16, 16, None, None, None)
+    g = stm.moe_grads(16, 16, None, 16, 16, None, None, None)
+    n = ctypes.c_size_t(0)
+    p32 = _p(dtype="f32").c()
+    assert L.moe_backward_workspace_size(ctypes.byref(p32), ctypes.byref(n)) == 0
+    assert n.value >= 256
+    # bf16 problems are not supported
+    pb = _p(dtype="bf16").c()
+    assert L.moe_backward(ctypes.byref(pb), ctypes.byref(w), 16, 16, 16, ctypes.byref(g), 16, n.value, None) == 2
+    # misaligned dout
+    assert L.moe_backward(ctypes.byref(p32), ctypes.byref(w), 16, 8, 16, ctypes.byref(g), 16, n.value, None) == 1
+    # logit bias without a d_bias output
+    pl = _p(dtype="f32", bias_mode="logit").c()
+    wl = stm.moe_weights(16, 16, 16, 16, None, None, None)
+    assert L.moe_backward(ctypes.byref(pl), ctypes.byref(wl), 16, 16, 16, ctypes.byref(g), 16, 1 << 40, None) == 1
+    # workspace too small
+    assert L.moe_backward(ctypes.byref(p32), ctypes.byref(w), 16, 16, 16, ctypes.byref(g), 16, 16, None) == 3
+    # gated shared expert without its gate gradient
+    pg = _p(dtype="f32", shared="sigmoid_gated", I_shared=64).c()
+    wg = stm.moe_weights(16, None, 16, 16, 16, 16, 16)
+    gg = stm.moe_grads(16, 16, None, 16, 16, 16, 16, None)
+    assert L.moe_backward(ctypes.byref(pg), ctypes.byref(wg), 16, 16, 16, ctypes.byref(gg), 16, 1 << 40, None) == 1
