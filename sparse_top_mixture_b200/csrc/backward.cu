@@ -1,4 +1,4 @@
-// Backward pass of the sparse top-k MoE FFN for fp32 problems (SIMT).
+// Backward pass of the sparse top-k MoE FFN for fp32 problems (SIMT tiles).
 //
 // Gradients of sum(dout * out) for the forward of moe_forward with the expert
 // choice held fixed (top-k selection is piecewise constant in its keys, so no
@@ -6,19 +6,27 @@
 // bias: "Sparse MoE FFN for DFlash-family drafters", What's here, MoEGate,
 // whose bias is moved by a sign controller and never by gradients; the same
 // page's tests check grouped-GEMM gradients against a per-expert loop). The
-// chain rule of the forward, written out:
-//   expert e on token t: g = x Wg^T, u = x Wu^T, h = silu(g) u, y = h Wd^T,
-//   out_t += w y;  dy = w dout;  dWd += dy^T h;  dh = dy Wd;
+// chain rule of the forward, written out for expert e on token t:
+//   g = x Wg^T, u = x Wu^T, h = silu(g) u, y = h Wd^T, out_t += w y;
+//   dhu = dout Wd (unscaled);  dh = w dhu;  dWd += (w dout)^T h;
 //   dg = dh u silu'(g), du = dh silu(g);  dWgu += [dg du]^T x;
-//   dx += dg Wg + du Wu;  dw = dout . y;
+//   dx += dg Wg + du Wu;  dw = dout . y = h . dhu;
 //   renormalised weights w_j = s_j / sum s: ds_i = (dw_i - sum_j dw_j w_j) / sum s;
 //   scores S = f(L): softmax dL = S (dS - sum dS S), sigmoid dL = dS S (1 - S),
 //   sqrtsoftplus dL = dS sig(L) / (2 S);  dgate_w = dL^T x, dx += dL gate_w,
 //   a logit bias gets sum_t dL;  shared expert: out += gamma Y_s(x), with
-//   gamma = sig(x . g) when gated: dz = (dout . Y_s) gamma (1 - gamma).
-// Every output element is computed by one thread looping over its reduction
-// in a fixed order (no atomics): the result is deterministic. This is the
-// reference-grade path for fp32 problems; bf16 problems are not supported.
+//   gamma = sig(x . g) when gated: dz = (h_s . dhu_s) gamma (1 - gamma).
+//
+// Layout of the work: the routed rows are sorted into per-expert segments by
+// the forward's dispatch kernels. Data gradients are grouped GEMMs over those
+// rows (one 128-row tile never crosses a segment, as in the forward); weight
+// gradients are per-expert GEMMs whose reduction walks the expert's segment
+// rows; dx is put back in token order by the forward's combine kernel. The
+// router and shared expert use the same two GEMM kernels over one all-token
+// segment. Every GEMM is 128x128 output tiles, 8-deep k slices
+// double-buffered in shared memory, 8x8 fp32 outputs per thread; every output
+// element is one thread's fixed-order sum (no atomics), so results are
+// deterministic. bf16 problems are not supported.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -26,13 +34,16 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "moe.h"
+#include "tiles.cuh"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
 
 namespace stm {
 namespace {
 
-constexpr int BT = 256;
+constexpr int BT = 256;                    // threads of every backward kernel
+constexpr int TM = 128, TN = 128, TK = 8;  // GEMM tile
+constexpr int TP = TM + 4;                 // padded shared row (keeps float4 alignment)
 
 __device__ __forceinline__ float sig_f(float a) { return 1.0f / (1.0f + expf(-a)); }
 __device__ __forceinline__ float silu_grad_f(float g) {
@@ -40,23 +51,276 @@ __device__ __forceinline__ float silu_grad_f(float g) {
   return s * (1.0f + g * (1.0f - s));
 }
 
-// Router forward for one token per block: logits, scores, and the routing
-// weights of its k selected experts (slot order), as in the forward.
-__global__ void __launch_bounds__(BT) bw_router_fwd(const float* __restrict__ x, const float* __restrict__ gw,
-                                                   const float* __restrict__ bias, int bias_mode, int score,
-                                                   int renorm, const int64_t* __restrict__ sel, int H, int E, int k,
-                                                   float* __restrict__ L, float* __restrict__ S,
-                                                   float* __restrict__ w) {
+// 8 x 8 outputs per thread from one TK-deep slice of the A [TK][TM] and
+// B [TK][TN] shared tiles. Thread (tx, ty) owns rows ty*4+{0..3}, 64+ty*4+{0..3}
+// and columns tx*4+{0..3}, 64+tx*4+{0..3}.
+__device__ __forceinline__ void mma_slice(const float (*As)[TP], const float (*Bs)[TP], int tx, int ty,
+                                          float (&acc)[8][8]) {
+#pragma unroll
+  for (int kk = 0; kk < TK; ++kk) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
+__device__ __forceinline__ int out_idx(int t, int i) { return i < 4 ? t * 4 + i : 64 + t * 4 + (i - 4); }
+
+// ---- grouped row GEMM ---------------------------------------------------------
+// C[r, n] = sum_k A[amap(r), k] * B_e[n, k]   (B_NT: B_e is [N, K])
+//        or sum_k A[amap(r), k] * B_e[k, n]   (otherwise: B_e is [K, N])
+// over rows r of each segment e (or one segment of single_rows rows).
+enum { EPI_STORE = 0, EPI_ADD = 1, EPI_DGU = 2 };
+
+struct RowGemm {
+  const float* A;
+  const int32_t* amap;  // row r reads A row amap[r] (NULL: row r)
+  int64_t lda;
+  const float* B;
+  int64_t b_stride;  // elements between experts' B
+  int N, K;
+  const int32_t* offsets;  // [E+1] segment table, or NULL for one segment
+  int E, single_rows;
+  int64_t rows_total;
+  float* C;  // EPI_STORE / EPI_ADD: C[r * ldc + n]
+  int64_t ldc;
+  const float* dz;    // EPI_ADD: optional C += dz[r] * gvec[n]
+  const float* gvec;
+  const float* GU;     // EPI_DGU (N == I): [g | u] rows [*, 2I]
+  const float* scale;  // EPI_DGU: dh = scale[r] * acc
+  float* DGU;          // EPI_DGU: [dg | du] rows [*, 2I]
+  float* DHU;          // EPI_DGU: acc rows [*, I]
+  int32_t* err;
+};
+
+template <bool B_NT, int EPI>
+__global__ void __launch_bounds__(BT) bw_row_gemm(RowGemm a) {
+  __shared__ int off[kMaxExperts + 1], pre[kMaxExperts + 1];
+  __shared__ __align__(16) float As[2][TK][TP];
+  __shared__ __align__(16) float Bs[2][TK][TP];
+  const int tid = threadIdx.x;
+  if (tid < 32) warp_build_tile_table(a.offsets, a.E, a.single_rows, TM, off, pre, a.rows_total, a.err);
+  __syncthreads();
+  const int nseg = a.offsets ? a.E : 1;
+  const int mt = blockIdx.x;
+  if (mt >= pre[nseg]) return;
+  const int e = find_segment(pre, nseg, mt);
+  const int row0 = off[e] + (mt - pre[e]) * TM, row_end = off[e + 1];
+  const int n0 = blockIdx.y * TN;
+  const int N = a.N, K = a.K;
+  const float* Be = a.B + (int64_t)e * a.b_stride;
+
+  // A loads: 8 consecutive k of rows (tid >> 3) + 32p.
+  const int ac = tid & 7;
+  const float* arow[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int r = row0 + (tid >> 3) + 32 * p;
+    arow[p] = r < row_end ? a.A + (int64_t)(a.amap ? a.amap[r] : r) * a.lda : nullptr;
+  }
+  float ra[4], rb[4];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int kk = k0 + ac;
+      ra[p] = (arow[p] != nullptr && kk < K) ? arow[p][kk] : 0.f;
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      if (B_NT) {
+        const int n = n0 + (tid >> 3) + 32 * p, kk = k0 + ac;
+        rb[p] = (n < N && kk < K) ? Be[(int64_t)n * K + kk] : 0.f;
+      } else {
+        const int n = n0 + (tid & 127), kk = k0 + (tid >> 7) + 2 * p;
+        rb[p] = (n < N && kk < K) ? Be[(int64_t)kk * N + n] : 0.f;
+      }
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      As[buf][ac][(tid >> 3) + 32 * p] = ra[p];
+      if (B_NT) Bs[buf][ac][(tid >> 3) + 32 * p] = rb[p];
+      else Bs[buf][(tid >> 7) + 2 * p][tid & 127] = rb[p];
+    }
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int tx = tid & 15, ty = tid >> 4;
+  load(0);
+  store(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < K; k0 += TK) {
+    const bool more = k0 + TK < K;
+    if (more) load(k0 + TK);
+    mma_slice(As[buf], Bs[buf], tx, ty, acc);
+    if (more) store(buf ^ 1);
+    __syncthreads();
+    buf ^= 1;
+  }
+
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = row0 + out_idx(ty, i);
+    if (r >= row_end) continue;
+    const float sc = EPI == EPI_DGU ? a.scale[r] : 1.f;
+    const float dzr = (EPI == EPI_ADD && a.dz != nullptr) ? a.dz[r] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + out_idx(tx, j);
+      if (n >= N) continue;
+      const float v = acc[i][j];
+      if (EPI == EPI_STORE) {
+        a.C[r * a.ldc + n] = v;
+      } else if (EPI == EPI_ADD) {
+        float add = v;
+        if (a.dz != nullptr) add = fmaf(dzr, a.gvec[n], add);
+        a.C[r * a.ldc + n] += add;
+      } else {
+        const float* gu = a.GU + (int64_t)r * 2 * N;
+        const float g = gu[n], u = gu[N + n];
+        const float dh = sc * v;
+        a.DGU[(int64_t)r * 2 * N + n] = dh * u * silu_grad_f(g);
+        a.DGU[(int64_t)r * 2 * N + N + n] = dh * silu_f32(g);
+        a.DHU[(int64_t)r * N + n] = v;
+      }
+    }
+  }
+}
+
+// ---- per-segment weight-gradient GEMM -------------------------------------------
+// C_e[i, j] = sum over rows r of segment e of Aop(r, i) * Bop(r, j), with
+//   Aop(r, i) = A[amap(r) * lda + i] * (ascale ? ascale[r] : 1)
+//   Bop(r, j) = B[bmap(r) * ldb + j], or (B_SWIGLU) silu(GU[r, j]) * GU[r, N + j]
+// C_e is [M, N] at C + e * M * N. Segments without rows write zeros.
+struct WGemm {
+  const float* A;
+  const int32_t* amap;
+  const float* ascale;
+  int64_t lda;
+  int M;
+  const float* B;  // B_SWIGLU: the [g | u] rows [*, 2N]
+  const int32_t* bmap;
+  int64_t ldb;
+  int N;
+  const int32_t* offsets;  // [E+1], or NULL for one segment of single_rows rows
+  int single_rows;
+  int64_t rows_total;
+  float* C;
+  int32_t* err;
+};
+
+template <bool B_SWIGLU>
+__global__ void __launch_bounds__(BT) bw_wgrad_gemm(WGemm a) {
+  __shared__ __align__(16) float As[2][TK][TP];
+  __shared__ __align__(16) float Bs[2][TK][TP];
+  const int tid = threadIdx.x;
+  const int e = blockIdx.y;
+  int r0 = a.offsets ? a.offsets[e] : 0, r1 = a.offsets ? a.offsets[e + 1] : a.single_rows;
+  if (r0 < 0 || r1 < r0 || (int64_t)r1 > a.rows_total) {  // malformed table: no rows are read
+    if (tid == 0) raise_error(a.err, MOE_DEVERR_BAD_EXPERT_ID);
+    r0 = r1 = 0;
+  }
+  const int M = a.M, N = a.N;
+  const int mtiles = (M + TM - 1) / TM;
+  const int m0 = (blockIdx.x % mtiles) * TM, n0 = (blockIdx.x / mtiles) * TN;
+  const int li = tid & 127, lc = tid >> 7;  // loads: column li of slice rows lc + 2p
+
+  float ra[4], rb[4];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int r = r0 + k0 + lc + 2 * p;
+      const bool rv = r < r1;
+      const int i = m0 + li, j = n0 + li;
+      float av = 0.f, bv = 0.f;
+      if (rv && i < M) {
+        av = a.A[(int64_t)(a.amap ? a.amap[r] : r) * a.lda + i];
+        if (a.ascale) av *= a.ascale[r];
+      }
+      if (rv && j < N) {
+        if (B_SWIGLU) {
+          const float* gu = a.B + (int64_t)r * 2 * N;
+          bv = silu_f32(gu[j]) * gu[N + j];
+        } else {
+          bv = a.B[(int64_t)(a.bmap ? a.bmap[r] : r) * a.ldb + j];
+        }
+      }
+      ra[p] = av;
+      rb[p] = bv;
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      As[buf][lc + 2 * p][li] = ra[p];
+      Bs[buf][lc + 2 * p][li] = rb[p];
+    }
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int K = r1 - r0;
+  if (K > 0) {
+    load(0);
+    store(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < K; k0 += TK) {
+      const bool more = k0 + TK < K;
+      if (more) load(k0 + TK);
+      mma_slice(As[buf], Bs[buf], tx, ty, acc);
+      if (more) store(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+  float* Ce = a.C + (int64_t)e * M * N;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + out_idx(ty, i);
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + out_idx(tx, j);
+      if (n < N) Ce[(int64_t)m * N + n] = acc[i][j];
+    }
+  }
+}
+
+// ---- router and small per-row kernels ---------------------------------------------
+
+// One token per block: logits L (+ logit bias, in place), scores S and the
+// routing weights w of its k chosen experts (slot order), as in the forward.
+__global__ void __launch_bounds__(BT) bw_scores(float* __restrict__ L, const float* __restrict__ bias, int bias_mode,
+                                              int score, int renorm, const int64_t* __restrict__ sel, int E, int k,
+                                              float* __restrict__ S, float* __restrict__ w) {
   __shared__ float red[BT];
   __shared__ float s_sc[kMaxExperts];
   const int t = blockIdx.x, e = threadIdx.x;
   float l = -INFINITY;
   if (e < E) {
-    float acc = 0.f;
-    for (int h = 0; h < H; ++h) acc = fmaf(x[(int64_t)t * H + h], gw[(int64_t)e * H + h], acc);
-    if (bias_mode == MOE_BIAS_LOGIT) acc += bias[e];
-    l = acc;
-    L[(int64_t)t * E + e] = l;
+    l = L[(int64_t)t * E + e];
+    if (bias_mode == MOE_BIAS_LOGIT) {
+      l += bias[e];
+      L[(int64_t)t * E + e] = l;
+    }
   }
   float sc = 0.f;
   if (score == MOE_SCORE_SOFTMAX) {
@@ -101,166 +365,38 @@ __global__ void __launch_bounds__(BT) bw_router_fwd(const float* __restrict__ x,
   }
 }
 
-// gu[r][j] = x[token(r)] . Wgu[e(r)][j], r over rows of a segment-sorted or
-// token-ordered row set (tok/ex give each row's token and expert).
-__global__ void __launch_bounds__(BT) bw_gate_up(const float* __restrict__ x, const float* __restrict__ wgu,
-                                               const int32_t* __restrict__ tok, const int32_t* __restrict__ ex,
-                                               int64_t R, int H, int I2, float* __restrict__ gu) {
-  const int64_t n = R * I2;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t r = i / I2;
-    const int j = (int)(i - r * I2);
-    const int e = ex ? ex[r] : 0;
-    const int t = tok ? tok[r] : (int)r;
-    if (e < 0) { gu[i] = 0.f; continue; }
-    const float* xr = x + (int64_t)t * H;
-    const float* wr = wgu + ((int64_t)e * I2 + j) * H;
-    float acc = 0.f;
-    for (int h = 0; h < H; ++h) acc = fmaf(xr[h], wr[h], acc);
-    gu[i] = acc;
-  }
-}
-
-// y[r][n] = (silu(g) u)[r] . Wd[e(r)][n]   (unscaled expert output)
-__global__ void __launch_bounds__(BT) bw_down_fwd(const float* __restrict__ gu, const float* __restrict__ wd,
-                                                const int32_t* __restrict__ ex, int64_t R, int H, int I,
-                                                float* __restrict__ y) {
-  const int64_t n = R * H;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t r = i / H;
-    const int c = (int)(i - r * H);
-    const int e = ex ? ex[r] : 0;
-    if (e < 0) { y[i] = 0.f; continue; }
-    const float* g = gu + r * 2 * I;
-    const float* wr = wd + ((int64_t)e * H + c) * I;
-    float acc = 0.f;
-    for (int m = 0; m < I; ++m) acc = fmaf(silu_f32(g[m]) * g[I + m], wr[m], acc);
-    y[i] = acc;
-  }
-}
-
-// dgu[r] = [dh u silu'(g) | dh silu(g)] with dh = scale(r) * (dout[token(r)] . Wd[e(r)][:, m])
-__global__ void __launch_bounds__(BT) bw_dgu(const float* __restrict__ dout, const float* __restrict__ gu,
-                                           const float* __restrict__ wd, const int32_t* __restrict__ tok,
-                                           const int32_t* __restrict__ ex, const float* __restrict__ scale,
-                                           int64_t R, int H, int I, float* __restrict__ dgu) {
-  const int64_t n = R * I;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t r = i / I;
-    const int m = (int)(i - r * I);
-    const int e = ex ? ex[r] : 0;
-    float* d = dgu + r * 2 * I;
-    if (e < 0) { d[m] = 0.f; d[I + m] = 0.f; continue; }
-    const int t = tok ? tok[r] : (int)r;
-    const float* dr = dout + (int64_t)t * H;
-    const float* wcol = wd + (int64_t)e * H * I + m;
-    float acc = 0.f;
-    for (int c = 0; c < H; ++c) acc = fmaf(dr[c], wcol[(int64_t)c * I], acc);
-    const float dh = scale[r] * acc;
-    const float g = gu[r * 2 * I + m], u = gu[r * 2 * I + I + m];
-    d[m] = dh * u * silu_grad_f(g);
-    d[I + m] = dh * silu_f32(g);
-  }
-}
-
-// Routed dx[t][h] = sum_j dgu[row(t,j)] . Wgu[e_j][:, h]  (written, not added)
-__global__ void __launch_bounds__(BT) bw_dx_routed(const float* __restrict__ dgu, const float* __restrict__ wgu,
-                                                 const int64_t* __restrict__ sel, const int32_t* __restrict__ pair_pos,
-                                                 int T, int H, int E, int k, int I2, float* __restrict__ dx) {
-  const int64_t n = (int64_t)T * H;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t t = i / H;
-    const int h = (int)(i - t * H);
-    float acc = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int64_t e = sel[t * k + j];
-      const int p = pair_pos[t * k + j];
-      if (e < 0 || e >= E || p < 0) continue;
-      const float* d = dgu + (int64_t)p * I2;
-      const float* wc = wgu + (int64_t)e * I2 * H + h;
-      for (int m = 0; m < I2; ++m) acc = fmaf(d[m], wc[(int64_t)m * H], acc);
-    }
-    dx[i] = acc;
-  }
-}
-
-// dWd[e][n][m] = sum over e's rows r of scale(r) dout[token(r)][n] h[r][m]
-__global__ void __launch_bounds__(BT) bw_dwd(const float* __restrict__ dout, const float* __restrict__ gu,
-                                           const int32_t* __restrict__ tok, const float* __restrict__ scale,
-                                           const int32_t* __restrict__ offsets, int nseg, int64_t rows_single,
-                                           int H, int I, float* __restrict__ dwd) {
-  const int64_t n = (int64_t)nseg * H * I;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t e = i / ((int64_t)H * I);
-    const int64_t rem = i - e * H * I;
-    const int c = (int)(rem / I), m = (int)(rem - (int64_t)c * I);
-    const int64_t r0 = offsets ? offsets[e] : 0, r1 = offsets ? offsets[e + 1] : rows_single;
-    float acc = 0.f;
-    for (int64_t r = r0; r < r1; ++r) {
-      const int t = tok ? tok[r] : (int)r;
-      const float* g = gu + r * 2 * I;
-      acc = fmaf(scale[r] * dout[(int64_t)t * H + c], silu_f32(g[m]) * g[I + m], acc);
-    }
-    dwd[i] = acc;
-  }
-}
-
-// dWgu[e][m][h] = sum over e's rows r of dgu[r][m] x[token(r)][h]
-__global__ void __launch_bounds__(BT) bw_dwgu(const float* __restrict__ dgu, const float* __restrict__ x,
-                                            const int32_t* __restrict__ tok, const int32_t* __restrict__ offsets,
-                                            int nseg, int64_t rows_single, int H, int I2,
-                                            float* __restrict__ dwgu) {
-  const int64_t n = (int64_t)nseg * I2 * H;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t e = i / ((int64_t)I2 * H);
-    const int64_t rem = i - e * I2 * H;
-    const int m = (int)(rem / H), h = (int)(rem - (int64_t)m * H);
-    const int64_t r0 = offsets ? offsets[e] : 0, r1 = offsets ? offsets[e + 1] : rows_single;
-    float acc = 0.f;
-    for (int64_t r = r0; r < r1; ++r) {
-      const int t = tok ? tok[r] : (int)r;
-      acc = fmaf(dgu[r * I2 + m], x[(int64_t)t * H + h], acc);
-    }
-    dwgu[i] = acc;
-  }
-}
-
-// Per sorted row: token, expert and routing weight of its pair.
-// Rows at or past offsets[E] (pairs skipped for a bad expert id) get expert -1.
+// Per sorted row p < offsets[E]: its token and routing weight.
 __global__ void __launch_bounds__(BT) bw_rows(const int32_t* __restrict__ sorted_pairs,
-                                            const int32_t* __restrict__ offsets, const int64_t* __restrict__ sel,
-                                            const float* __restrict__ w, int64_t P, int E, int k,
-                                            int32_t* __restrict__ tok, int32_t* __restrict__ ex,
-                                            float* __restrict__ scale) {
+                                            const int32_t* __restrict__ offsets, const float* __restrict__ w,
+                                            int E, int k, int32_t* __restrict__ tok, float* __restrict__ scale) {
   const int64_t used = offsets[E];
-  for (int64_t p = blockIdx.x * (int64_t)BT + threadIdx.x; p < P; p += (int64_t)gridDim.x * BT) {
-    if (p >= used) {
-      tok[p] = 0;
-      ex[p] = -1;
-      scale[p] = 0.f;
-      continue;
-    }
+  for (int64_t p = blockIdx.x * (int64_t)BT + threadIdx.x; p < used; p += (int64_t)gridDim.x * BT) {
     const int q = sorted_pairs[p];
-    const int64_t e = sel[q];
     tok[p] = q / k;
-    ex[p] = (e >= 0 && e < E) ? (int)e : -1;
     scale[p] = w[q];
   }
 }
 
-// dw[q] = dout[token(q)] . y[pair_pos[q]]
-__global__ void __launch_bounds__(BT) bw_dw(const float* __restrict__ dout, const float* __restrict__ y,
-                                          const int32_t* __restrict__ pair_pos, int64_t P, int H, int k,
-                                          float* __restrict__ dw) {
-  for (int64_t q = blockIdx.x * (int64_t)BT + threadIdx.x; q < P; q += (int64_t)gridDim.x * BT) {
-    const int p = pair_pos[q];
+// One warp per output q: out[q] = sum_m silu(g) u dhu over row p = map(q)
+// (0 when p < 0), times gamma (1 - gamma) when gamma is given.
+__global__ void __launch_bounds__(BT) bw_rowdot(const float* __restrict__ GU, const float* __restrict__ DHU, int I,
+                                              const int32_t* __restrict__ map, int64_t R,
+                                              const float* __restrict__ gamma, float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t q = (blockIdx.x * (int64_t)BT + threadIdx.x) >> 5; q < R; q += ((int64_t)gridDim.x * BT) >> 5) {
+    const int64_t p = map ? map[q] : q;
     float acc = 0.f;
     if (p >= 0) {
-      const float* d = dout + (q / k) * H;
-      const float* yr = y + (int64_t)p * H;
-      for (int c = 0; c < H; ++c) acc = fmaf(d[c], yr[c], acc);
+      const float* gu = GU + p * 2 * I;
+      const float* d = DHU + p * I;
+      for (int m = lane; m < I; m += 32) acc = fmaf(silu_f32(gu[m]) * gu[I + m], d[m], acc);
     }
-    dw[q] = acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      if (gamma) acc *= gamma[q] * (1.f - gamma[q]);
+      out[q] = acc;
+    }
   }
 }
 
@@ -308,72 +444,13 @@ __global__ void __launch_bounds__(BT) bw_router_bwd(const float* __restrict__ L,
   if (e < E) dL[(int64_t)t * E + e] = dl;
 }
 
-// dgate_w[e][h] = sum_t dL[t][e] x[t][h]; d_bias[e] = sum_t dL[t][e]
-__global__ void __launch_bounds__(BT) bw_dgate(const float* __restrict__ dL, const float* __restrict__ x, int T,
-                                             int H, int E, float* __restrict__ dgw, float* __restrict__ dbias) {
-  const int64_t n = (int64_t)E * H;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t e = i / H;
-    const int h = (int)(i - e * H);
-    float acc = 0.f, sb = 0.f;
-    for (int t = 0; t < T; ++t) {
-      const float d = dL[(int64_t)t * E + e];
-      acc = fmaf(d, x[(int64_t)t * H + h], acc);
-      sb += d;
-    }
-    dgw[i] = acc;
-    if (dbias && h == 0) dbias[e] = sb;
-  }
-}
-
-// dx[t][h] += sum_e dL[t][e] gate_w[e][h]  (+ dz[t] g[h] for a gated shared expert)
-__global__ void __launch_bounds__(BT) bw_dx_router(const float* __restrict__ dL, const float* __restrict__ gw,
-                                                 const float* __restrict__ dz, const float* __restrict__ g, int T,
-                                                 int H, int E, float* __restrict__ dx) {
-  const int64_t n = (int64_t)T * H;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t t = i / H;
-    const int h = (int)(i - t * H);
+// out[c] = sum_t v[t * ldv + c] for c < C (fixed order over t)
+__global__ void __launch_bounds__(BT) bw_colsum(const float* __restrict__ v, int64_t ldv, int T, int C,
+                                              float* __restrict__ out) {
+  for (int c = blockIdx.x * BT + threadIdx.x; c < C; c += gridDim.x * BT) {
     float acc = 0.f;
-    for (int e = 0; e < E; ++e) acc = fmaf(dL[t * E + e], gw[(int64_t)e * H + h], acc);
-    if (dz) acc = fmaf(dz[t], g[h], acc);
-    dx[i] += acc;
-  }
-}
-
-// Shared expert gate: gamma[t] (1 plain, sig(x.g) gated) and dz[t]
-// = (dout[t] . Y_s[t]) gamma (1 - gamma) (gated only).
-__global__ void __launch_bounds__(BT) bw_shared_gate(const float* __restrict__ x, const float* __restrict__ g,
-                                                   const float* __restrict__ dout, const float* __restrict__ ys,
-                                                   int T, int H, int gated, float* __restrict__ gamma,
-                                                   float* __restrict__ dz) {
-  for (int t = blockIdx.x * BT + threadIdx.x; t < T; t += gridDim.x * BT) {
-    float gm = 1.f, d = 0.f;
-    if (gated) {
-      float z = 0.f, dy = 0.f;
-      for (int h = 0; h < H; ++h) {
-        z = fmaf(x[(int64_t)t * H + h], g[h], z);
-        dy = fmaf(dout[(int64_t)t * H + h], ys[(int64_t)t * H + h], dy);
-      }
-      gm = sig_f(z);
-      d = dy * gm * (1.f - gm);
-    }
-    gamma[t] = gm;
-    dz[t] = d;
-  }
-}
-
-// Shared expert dx: dx[t][h] += dgu_s[t] . Wsgu[:, h]
-__global__ void __launch_bounds__(BT) bw_dx_shared(const float* __restrict__ dgus, const float* __restrict__ wsgu,
-                                                 int T, int H, int I2, float* __restrict__ dx) {
-  const int64_t n = (int64_t)T * H;
-  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
-    const int64_t t = i / H;
-    const int h = (int)(i - t * H);
-    const float* d = dgus + t * I2;
-    float acc = 0.f;
-    for (int m = 0; m < I2; ++m) acc = fmaf(d[m], wsgu[(int64_t)m * H + h], acc);
-    dx[i] += acc;
+    for (int t = 0; t < T; ++t) acc += v[(int64_t)t * ldv + c];
+    out[c] = acc;
   }
 }
 
@@ -387,11 +464,43 @@ __global__ void __launch_bounds__(BT) bw_dgvec(const float* __restrict__ dz, con
   }
 }
 
+// gamma[t] = sig(x[t] . g) when g is given, else 1. One warp per token.
+__global__ void __launch_bounds__(BT) bw_gamma(const float* __restrict__ x, const float* __restrict__ g, int T, int H,
+                                             float* __restrict__ gamma) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t t = (blockIdx.x * (int64_t)BT + threadIdx.x) >> 5; t < T; t += ((int64_t)gridDim.x * BT) >> 5) {
+    if (g == nullptr) {
+      if (lane == 0) gamma[t] = 1.f;
+      continue;
+    }
+    float acc = 0.f;
+    for (int h = lane; h < H; h += 32) acc = fmaf(x[t * H + h], g[h], acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) gamma[t] = sig_f(acc);
+  }
+}
+
 unsigned grid_for(int64_t n) { return (unsigned)std::max<int64_t>(1, std::min<int64_t>(ceil_div(n, BT), 148 * 32)); }
 
+template <bool B_NT, int EPI>
+cudaError_t run_rows(const RowGemm& a, cudaStream_t s) {
+  const int64_t nseg = a.offsets ? a.E : 1;
+  const dim3 grid((unsigned)(a.rows_total / TM + nseg), (unsigned)ceil_div(a.N, TN));
+  bw_row_gemm<B_NT, EPI><<<grid, BT, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <bool B_SWIGLU>
+cudaError_t run_wgrad(const WGemm& a, int nseg, cudaStream_t s) {
+  const dim3 grid((unsigned)(ceil_div(a.M, TM) * ceil_div(a.N, TN)), (unsigned)nseg);
+  bw_wgrad_gemm<B_SWIGLU><<<grid, BT, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 struct BwLayout {
-  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, ex, scale, w, dw, L, S, dL, gu, y, dgu, gus,
-      ys, dgus, gamma, dz, total;
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, gu, dgu, dhu, dxr,
+      extra, gus, dgus, dhus, gamma, dz, total;
 };
 
 size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -412,7 +521,6 @@ BwLayout bw_layout(const moe_problem& p) {
   b.sorted_pairs = take((size_t)P * 4);
   b.pair_pos = take((size_t)P * 4);
   b.tok = take((size_t)P * 4);
-  b.ex = take((size_t)P * 4);
   b.scale = take((size_t)P * 4);
   b.w = take((size_t)P * 4);
   b.dw = take((size_t)P * 4);
@@ -420,12 +528,15 @@ BwLayout bw_layout(const moe_problem& p) {
   b.S = take((size_t)p.T * p.E * 4);
   b.dL = take((size_t)p.T * p.E * 4);
   b.gu = take((size_t)P * 2 * p.I * 4);
-  b.y = take((size_t)P * p.H * 4);
   b.dgu = take((size_t)P * 2 * p.I * 4);
+  b.dhu = take((size_t)P * p.I * 4);
+  b.dxr = take((size_t)P * p.H * 4);
+  b.extra = take((size_t)p.T * p.H * 4);
   const bool sh = p.shared != MOE_SHARED_NONE;
-  b.gus = take(sh ? (size_t)p.T * 2 * p.I_shared * 4 : 0);
-  b.ys = take(sh ? (size_t)p.T * p.H * 4 : 0);
-  b.dgus = take(sh ? (size_t)p.T * 2 * p.I_shared * 4 : 0);
+  const size_t Is = sh ? (size_t)p.I_shared : 0;
+  b.gus = take((size_t)p.T * 2 * Is * 4);
+  b.dgus = take((size_t)p.T * 2 * Is * 4);
+  b.dhus = take((size_t)p.T * Is * 4);
   b.gamma = take(sh ? (size_t)p.T * 4 : 0);
   b.dz = take(sh ? (size_t)p.T * 4 : 0);
   b.total = off;
@@ -441,6 +552,45 @@ bool ok16(const void* q) { return q != nullptr && (reinterpret_cast<uintptr_t>(q
 // NULL or 4-byte aligned
 bool ok4(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0; }
 
+RowGemm row_gemm(const float* A, const int32_t* amap, int64_t lda, const float* B, int64_t b_stride, int N, int K,
+                 const int32_t* offsets, int E, int single_rows, int64_t rows_total, int32_t* err) {
+  RowGemm a{};
+  a.A = A;
+  a.amap = amap;
+  a.lda = lda;
+  a.B = B;
+  a.b_stride = b_stride;
+  a.N = N;
+  a.K = K;
+  a.offsets = offsets;
+  a.E = E;
+  a.single_rows = single_rows;
+  a.rows_total = rows_total;
+  a.err = err;
+  return a;
+}
+
+WGemm wgrad(const float* A, const int32_t* amap, const float* ascale, int64_t lda, int M, const float* B,
+            const int32_t* bmap, int64_t ldb, int N, const int32_t* offsets, int single_rows, int64_t rows_total,
+            float* C, int32_t* err) {
+  WGemm a{};
+  a.A = A;
+  a.amap = amap;
+  a.ascale = ascale;
+  a.lda = lda;
+  a.M = M;
+  a.B = B;
+  a.bmap = bmap;
+  a.ldb = ldb;
+  a.N = N;
+  a.offsets = offsets;
+  a.single_rows = single_rows;
+  a.rows_total = rows_total;
+  a.C = C;
+  a.err = err;
+  return a;
+}
+
 }  // namespace
 }  // namespace stm
 
@@ -455,6 +605,11 @@ MOE_API moe_status moe_backward_workspace_size(const moe_problem* p, size_t* byt
   return MOE_OK;
 }
 
+#define BW_CUDA(...)                                       \
+  do {                                                     \
+    if ((__VA_ARGS__) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
 MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, const void* x_, const void* dout_,
                                 const int64_t* selected, moe_grads* g, void* ws, size_t ws_bytes,
                                 moe_stream_t stream) {
@@ -465,8 +620,9 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   if (w == nullptr || g == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   const bool sh = p->shared != MOE_SHARED_NONE, gated = p->shared == MOE_SHARED_SIGMOID_GATED;
   const bool has_tokens = p->T > 0;  // per-token arrays and the workspace may be NULL without tokens
-  if ((has_tokens && (!ok16(x_) || !ok16(dout_) || !ok16(selected) || !ok16(g->dx) || !ok16(ws))) || !ok16(w->gate_w) ||
-      !ok16(w->gate_up) || !ok16(w->down) || !ok16(g->d_gate_w) || !ok16(g->d_gate_up) || !ok16(g->d_down))
+  if ((has_tokens && (!ok16(x_) || !ok16(dout_) || !ok16(selected) || !ok16(g->dx) || !ok16(ws))) ||
+      !ok16(w->gate_w) || !ok16(w->gate_up) || !ok16(w->down) || !ok16(g->d_gate_w) || !ok16(g->d_gate_up) ||
+      !ok16(g->d_down))
     return MOE_ERR_INVALID_ARGUMENT;
   if ((p->bias_mode != MOE_BIAS_NONE) != (w->bias != nullptr) || !ok4(w->bias)) return MOE_ERR_INVALID_ARGUMENT;
   if ((p->bias_mode == MOE_BIAS_LOGIT) != (g->d_bias != nullptr) || !ok4(g->d_bias))
@@ -479,16 +635,16 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
     return MOE_ERR_INVALID_ARGUMENT;
   if (has_tokens && ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (p->T == 0) {  // no tokens: every weight gradient is zero
+  if (!has_tokens) {  // no tokens: every weight gradient is zero
     const size_t f = sizeof(float);
-    cudaError_t e = cudaMemsetAsync(g->d_gate_w, 0, (size_t)(p->E * p->H) * f, s);
-    if (e == cudaSuccess && g->d_bias) e = cudaMemsetAsync(g->d_bias, 0, (size_t)p->E * f, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(g->d_gate_up, 0, (size_t)(p->E * 2 * p->I * p->H) * f, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(g->d_down, 0, (size_t)(p->E * p->H * p->I) * f, s);
-    if (e == cudaSuccess && sh) e = cudaMemsetAsync(g->d_shared_gate_up, 0, (size_t)(2 * p->I_shared * p->H) * f, s);
-    if (e == cudaSuccess && sh) e = cudaMemsetAsync(g->d_shared_down, 0, (size_t)(p->H * p->I_shared) * f, s);
-    if (e == cudaSuccess && gated) e = cudaMemsetAsync(g->d_shared_gate, 0, (size_t)p->H * f, s);
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    BW_CUDA(cudaMemsetAsync(g->d_gate_w, 0, (size_t)(p->E * p->H) * f, s));
+    if (g->d_bias) BW_CUDA(cudaMemsetAsync(g->d_bias, 0, (size_t)p->E * f, s));
+    BW_CUDA(cudaMemsetAsync(g->d_gate_up, 0, (size_t)(p->E * 2 * p->I * p->H) * f, s));
+    BW_CUDA(cudaMemsetAsync(g->d_down, 0, (size_t)(p->E * p->H * p->I) * f, s));
+    if (sh) BW_CUDA(cudaMemsetAsync(g->d_shared_gate_up, 0, (size_t)(2 * p->I_shared * p->H) * f, s));
+    if (sh) BW_CUDA(cudaMemsetAsync(g->d_shared_down, 0, (size_t)(p->H * p->I_shared) * f, s));
+    if (gated) BW_CUDA(cudaMemsetAsync(g->d_shared_gate, 0, (size_t)p->H * f, s));
+    return MOE_OK;
   }
   const BwLayout b = bw_layout(*p);
   const int T = (int)p->T, H = (int)p->H, E = (int)p->E, k = (int)p->k, I = (int)p->I, Is = (int)p->I_shared;
@@ -503,7 +659,6 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   int32_t* sorted_pairs = at<int32_t>(ws, b.sorted_pairs);
   int32_t* pair_pos = at<int32_t>(ws, b.pair_pos);
   int32_t* tok = at<int32_t>(ws, b.tok);
-  int32_t* ex = at<int32_t>(ws, b.ex);
   float* scale = at<float>(ws, b.scale);
   float* wts = at<float>(ws, b.w);
   float* dw = at<float>(ws, b.dw);
@@ -511,51 +666,117 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   float* S = at<float>(ws, b.S);
   float* dL = at<float>(ws, b.dL);
   float* gu = at<float>(ws, b.gu);
-  float* y = at<float>(ws, b.y);
   float* dgu = at<float>(ws, b.dgu);
-  auto chk = [](cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; };
+  float* dhu = at<float>(ws, b.dhu);
+  float* dxr = at<float>(ws, b.dxr);
+  float* extra = at<float>(ws, b.extra);
 
-  // routing weights of the given choice, and its sorted segments
-  bw_router_fwd<<<T, BT, 0, s>>>(x, gw, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, H, E, k,
-                                 L, S, wts);
-  if (launch_dispatch(MOE_DTYPE_F32, selected, nullptr, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
-                      at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, nullptr, err, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, selected, wts, P, E, k, tok, ex, scale);
-  // routed experts, rows in segment order
-  bw_gate_up<<<grid_for(P * 2 * I), BT, 0, s>>>(x, wgu, tok, ex, P, H, 2 * I, gu);
-  bw_down_fwd<<<grid_for(P * H), BT, 0, s>>>(gu, wd, ex, P, H, I, y);
-  bw_dw<<<grid_for(P), BT, 0, s>>>(dout, y, pair_pos, P, H, k, dw);
-  bw_dgu<<<grid_for(P * I), BT, 0, s>>>(dout, gu, wd, tok, ex, scale, P, H, I, dgu);
-  bw_dx_routed<<<grid_for((int64_t)T * H), BT, 0, s>>>(dgu, wgu, selected, pair_pos, T, H, E, k, 2 * I, g->dx);
-  bw_dwd<<<grid_for((int64_t)E * H * I), BT, 0, s>>>(dout, gu, tok, scale, offsets, E, 0, H, I, g->d_down);
-  bw_dwgu<<<grid_for((int64_t)E * 2 * I * H), BT, 0, s>>>(dgu, x, tok, offsets, E, 0, H, 2 * I, g->d_gate_up);
-  // router
+  // Router: logits, scores and the routing weights of the given choice.
+  BW_CUDA(run_rows<true, EPI_STORE>(
+      [&] {
+        RowGemm a = row_gemm(x, nullptr, H, gw, 0, E, H, nullptr, 1, T, T, err);
+        a.C = L;
+        a.ldc = E;
+        return a;
+      }(),
+      s));
+  bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
+  // Sorted segments of the choice, each row's token and weight.
+  BW_CUDA(launch_dispatch(MOE_DTYPE_F32, selected, nullptr, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
+                          at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, nullptr, err, s));
+  bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, wts, E, k, tok, scale);
+  // Routed experts: recompute [g | u]; dhu and [dg | du]; dx rows; dw.
+  BW_CUDA(run_rows<true, EPI_STORE>(
+      [&] {
+        RowGemm a = row_gemm(x, tok, H, wgu, (int64_t)2 * I * H, 2 * I, H, offsets, E, 0, P, err);
+        a.C = gu;
+        a.ldc = 2 * I;
+        return a;
+      }(),
+      s));
+  BW_CUDA(run_rows<false, EPI_DGU>(
+      [&] {
+        RowGemm a = row_gemm(dout, tok, H, wd, (int64_t)H * I, I, H, offsets, E, 0, P, err);
+        a.GU = gu;
+        a.scale = scale;
+        a.DGU = dgu;
+        a.DHU = dhu;
+        return a;
+      }(),
+      s));
+  BW_CUDA(run_rows<false, EPI_STORE>(
+      [&] {
+        RowGemm a = row_gemm(dgu, nullptr, 2 * I, wgu, (int64_t)2 * I * H, H, 2 * I, offsets, E, 0, P, err);
+        a.C = dxr;
+        a.ldc = H;
+        return a;
+      }(),
+      s));
+  bw_rowdot<<<grid_for(P * 32), BT, 0, s>>>(gu, dhu, I, pair_pos, P, nullptr, dw);
+  // Routed weight gradients: dWd_e = (w dout)^T h, dWgu_e = [dg du]^T x.
+  BW_CUDA(run_wgrad<true>(wgrad(dout, tok, scale, H, H, gu, nullptr, 0, I, offsets, 0, P, g->d_down, err), E, s));
+  BW_CUDA(run_wgrad<false>(wgrad(dgu, nullptr, nullptr, 2 * I, 2 * I, x, tok, H, H, offsets, 0, P, g->d_gate_up, err),
+                           E, s));
+  // Router backward: dL, dgate_w = dL^T x, d_bias = sum_t dL.
   bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL);
-  bw_dgate<<<grid_for((int64_t)E * H), BT, 0, s>>>(dL, x, T, H, E, g->d_gate_w, g->d_bias);
+  BW_CUDA(run_wgrad<false>(wgrad(dL, nullptr, nullptr, E, E, x, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1,
+                           s));
+  if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
+  // Shared expert over all tokens, scaled by gamma; its dx goes to `extra`.
   float* dz = nullptr;
+  const float* gvec = static_cast<const float*>(w->shared_gate);
   if (sh) {
     const float* wsgu = static_cast<const float*>(w->shared_gate_up);
     const float* wsd = static_cast<const float*>(w->shared_down);
     float* gus = at<float>(ws, b.gus);
-    float* ys = at<float>(ws, b.ys);
     float* dgus = at<float>(ws, b.dgus);
+    float* dhus = at<float>(ws, b.dhus);
     float* gamma = at<float>(ws, b.gamma);
     dz = at<float>(ws, b.dz);
-    bw_gate_up<<<grid_for((int64_t)T * 2 * Is), BT, 0, s>>>(x, wsgu, nullptr, nullptr, T, H, 2 * Is, gus);
-    bw_down_fwd<<<grid_for((int64_t)T * H), BT, 0, s>>>(gus, wsd, nullptr, T, H, Is, ys);
-    bw_shared_gate<<<grid_for(T), BT, 0, s>>>(x, static_cast<const float*>(w->shared_gate), dout, ys, T, H,
-                                              gated ? 1 : 0, gamma, dz);
-    bw_dgu<<<grid_for((int64_t)T * Is), BT, 0, s>>>(dout, gus, wsd, nullptr, nullptr, gamma, T, H, Is, dgus);
-    bw_dx_shared<<<grid_for((int64_t)T * H), BT, 0, s>>>(dgus, wsgu, T, H, 2 * Is, g->dx);
-    bw_dwd<<<grid_for((int64_t)H * Is), BT, 0, s>>>(dout, gus, nullptr, gamma, nullptr, 1, T, H, Is,
-                                                   g->d_shared_down);
-    bw_dwgu<<<grid_for((int64_t)2 * Is * H), BT, 0, s>>>(dgus, x, nullptr, nullptr, 1, T, H, 2 * Is,
-                                                        g->d_shared_gate_up);
+    bw_gamma<<<grid_for((int64_t)T * 32), BT, 0, s>>>(x, gated ? gvec : nullptr, T, H, gamma);
+    BW_CUDA(run_rows<true, EPI_STORE>(
+        [&] {
+          RowGemm a = row_gemm(x, nullptr, H, wsgu, 0, 2 * Is, H, nullptr, 1, T, T, err);
+          a.C = gus;
+          a.ldc = 2 * Is;
+          return a;
+        }(),
+        s));
+    BW_CUDA(run_rows<false, EPI_DGU>(
+        [&] {
+          RowGemm a = row_gemm(dout, nullptr, H, wsd, 0, Is, H, nullptr, 1, T, T, err);
+          a.GU = gus;
+          a.scale = gamma;
+          a.DGU = dgus;
+          a.DHU = dhus;
+          return a;
+        }(),
+        s));
+    BW_CUDA(run_rows<false, EPI_STORE>(
+        [&] {
+          RowGemm a = row_gemm(dgus, nullptr, 2 * Is, wsgu, 0, H, 2 * Is, nullptr, 1, T, T, err);
+          a.C = extra;
+          a.ldc = H;
+          return a;
+        }(),
+        s));
+    if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(gus, dhus, Is, nullptr, T, gamma, dz);
+    BW_CUDA(run_wgrad<true>(wgrad(dout, nullptr, gamma, H, H, gus, nullptr, 0, Is, nullptr, T, T,
+                                  g->d_shared_down, err),
+                            1, s));
+    BW_CUDA(run_wgrad<false>(wgrad(dgus, nullptr, nullptr, 2 * Is, 2 * Is, x, nullptr, H, H, nullptr, T, T,
+                                   g->d_shared_gate_up, err),
+                             1, s));
     if (gated) bw_dgvec<<<grid_for(H), BT, 0, s>>>(dz, x, T, H, g->d_shared_gate);
   }
-  bw_dx_router<<<grid_for((int64_t)T * H), BT, 0, s>>>(dL, gw, gated ? dz : nullptr,
-                                                      gated ? static_cast<const float*>(w->shared_gate) : nullptr,
-                                                      T, H, E, g->dx);
-  return chk(cudaGetLastError());
+  // Router (and shared gate) dx into `extra`, then dx = sum of each token's rows + extra.
+  RowGemm rd = row_gemm(dL, nullptr, E, gw, 0, H, E, nullptr, 1, T, T, err);
+  rd.C = extra;
+  rd.ldc = H;
+  rd.dz = gated ? dz : nullptr;
+  rd.gvec = gated ? gvec : nullptr;
+  if (sh) BW_CUDA(run_rows<false, EPI_ADD>(rd, s));
+  else BW_CUDA(run_rows<false, EPI_STORE>(rd, s));
+  BW_CUDA(launch_combine(MOE_DTYPE_F32, dxr, pair_pos, extra, g->dx, p->T, p->H, p->k, s));
+  return MOE_OK;
 }
