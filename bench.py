@@ -221,6 +221,57 @@ def cpu_baseline(cfg, dev_inputs, target_s: float = 12.0):
 
 # ----------------------------------------------------------------------------
 
+FP32_LANES_PER_SM = 128  # FFMA lanes per Blackwell SM (4 sub-partitions x 32)
+NUM_SMS = 148
+
+
+def backward_flops(cfg) -> float:
+    """Algorithmic FLOPs of one backward (moe_backward): per routed pair the
+    recomputed [g | u] (4HI), dhu = dout Wd (2HI), dx rows (4HI) and the two
+    weight gradients (2HI + 4HI); the router's logits, dgate_w and dx (2EH
+    each per token); the shared expert like one routed pair per token."""
+    P = cfg.T * cfg.k
+    return 16.0 * P * cfg.H * cfg.I + 6.0 * cfg.T * cfg.E * cfg.H + 16.0 * cfg.T * cfg.H * cfg.I_shared
+
+
+def measure_backward(cfg, local: int, steps: int = 5) -> dict:
+    """The fp32 backward on the bench workload's shapes, timed with CUDA events
+    on the current stream, against the FFMA peak at the sampled SM clock."""
+    import sparse_top_mixture_b200 as stm
+    cfg32 = cfg.replace(dtype="f32")
+    inp = workloads.generate(cfg32, "cuda")
+    p = stm.Problem.from_config(cfg32)
+    moe = stm.SparseMoE(p, inp)
+    out, _, sel = moe(inp["x"])
+    dout = torch.randn(out.shape, generator=torch.Generator("cuda").manual_seed(7), device="cuda")
+    ws = torch.zeros(stm.backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        stm.backward(p, inp, inp["x"], dout, sel, ws=ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        a.record(stream)
+        for _ in range(steps):
+            stm.backward(p, inp, inp["x"], dout, sel, ws=ws)
+        b.record(stream)
+        torch.cuda.synchronize()
+    if stm.read_device_error(ws) != 0:
+        raise RuntimeError("device error flag set during the backward")
+    ms = a.elapsed_time(b) / steps
+    fl = backward_flops(cfg32)
+    c = clk.summary()
+    mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965
+    peak = NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    achieved = fl / (ms / 1e3) / 1e12
+    return {"workload": f"{cfg.name} shapes in fp32 (T={cfg.T}, H={cfg.H}, E={cfg.E}, k={cfg.k}, I={cfg.I}, "
+                        f"I_shared={cfg.I_shared})",
+            "ms": ms, "steps": steps, "flops": fl, "bound": "alu", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)",
+            "clocks": c}
+
+
 def init_dist(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -311,6 +362,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-graph", action="store_true", help="launch each kernel from the host every step")
+    ap.add_argument("--no-backward", action="store_true", help="skip the fp32 backward measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -479,6 +531,8 @@ def main():
         "gpu_launches": stm.launches_per_forward(p, two_streams=moe.aux is not None) * args.steps,
         "clocks": clocks.summary(),
     }
+    if world == 1 and not args.no_backward:
+        line["backward"] = measure_backward(cfg, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, dict(r_cpu, **{k: dev[k] for k in (
             "gate_up", "down", "shared_gate_up", "shared_down")}))

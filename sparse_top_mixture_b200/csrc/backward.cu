@@ -97,11 +97,12 @@ struct RowGemm {
   const float* scale;  // EPI_DGU: dh = scale[r] * acc
   float* DGU;          // EPI_DGU: [dg | du] rows [*, 2I]
   float* DHU;          // EPI_DGU: acc rows [*, I]
+  float* Hact;         // EPI_DGU: h = silu(g) u rows [*, I]
   int32_t* err;
 };
 
 template <bool B_NT, int EPI>
-__global__ void __launch_bounds__(BT) bw_row_gemm(RowGemm a) {
+__global__ void __launch_bounds__(BT, 2) bw_row_gemm(RowGemm a) {
   __shared__ int off[kMaxExperts + 1], pre[kMaxExperts + 1];
   __shared__ __align__(16) float As[2][TK][TP];
   __shared__ __align__(16) float Bs[2][TK][TP];
@@ -195,6 +196,7 @@ __global__ void __launch_bounds__(BT) bw_row_gemm(RowGemm a) {
         a.DGU[(int64_t)r * 2 * N + n] = dh * u * silu_grad_f(g);
         a.DGU[(int64_t)r * 2 * N + N + n] = dh * silu_f32(g);
         a.DHU[(int64_t)r * N + n] = v;
+        a.Hact[(int64_t)r * N + n] = silu_f32(g) * u;
       }
     }
   }
@@ -203,32 +205,35 @@ __global__ void __launch_bounds__(BT) bw_row_gemm(RowGemm a) {
 // ---- per-segment weight-gradient GEMM -------------------------------------------
 // C_e[i, j] = sum over rows r of segment e of Aop(r, i) * Bop(r, j), with
 //   Aop(r, i) = A[amap(r) * lda + i] * (ascale ? ascale[r] : 1)
-//   Bop(r, j) = B[bmap(r) * ldb + j], or (B_SWIGLU) silu(GU[r, j]) * GU[r, N + j]
-// C_e is [M, N] at C + e * M * N. Segments without rows write zeros.
+//   Bop(r, j) = B[bmap(r) * ldb + j]
+// C_e is [M, N] at C + e * M * N. Segments without rows write zeros. Without
+// a segment table, segment e is rows [e * chunk, min((e + 1) * chunk,
+// single_rows)): a split of one long reduction into partial sums that
+// bw_sum_parts adds up in order.
 struct WGemm {
   const float* A;
   const int32_t* amap;
   const float* ascale;
   int64_t lda;
   int M;
-  const float* B;  // B_SWIGLU: the [g | u] rows [*, 2N]
+  const float* B;
   const int32_t* bmap;
   int64_t ldb;
   int N;
-  const int32_t* offsets;  // [E+1], or NULL for one segment of single_rows rows
-  int single_rows;
+  const int32_t* offsets;  // [E+1], or NULL: chunks of single_rows rows
+  int single_rows, chunk;
   int64_t rows_total;
   float* C;
   int32_t* err;
 };
 
-template <bool B_SWIGLU>
-__global__ void __launch_bounds__(BT) bw_wgrad_gemm(WGemm a) {
+__global__ void __launch_bounds__(BT, 2) bw_wgrad_gemm(WGemm a) {
   __shared__ __align__(16) float As[2][TK][TP];
   __shared__ __align__(16) float Bs[2][TK][TP];
   const int tid = threadIdx.x;
   const int e = blockIdx.y;
-  int r0 = a.offsets ? a.offsets[e] : 0, r1 = a.offsets ? a.offsets[e + 1] : a.single_rows;
+  int r0 = a.offsets ? a.offsets[e] : e * a.chunk;
+  int r1 = a.offsets ? a.offsets[e + 1] : min(a.single_rows, r0 + a.chunk);
   if (r0 < 0 || r1 < r0 || (int64_t)r1 > a.rows_total) {  // malformed table: no rows are read
     if (tid == 0) raise_error(a.err, MOE_DEVERR_BAD_EXPERT_ID);
     r0 = r1 = 0;
@@ -250,14 +255,7 @@ __global__ void __launch_bounds__(BT) bw_wgrad_gemm(WGemm a) {
         av = a.A[(int64_t)(a.amap ? a.amap[r] : r) * a.lda + i];
         if (a.ascale) av *= a.ascale[r];
       }
-      if (rv && j < N) {
-        if (B_SWIGLU) {
-          const float* gu = a.B + (int64_t)r * 2 * N;
-          bv = silu_f32(gu[j]) * gu[N + j];
-        } else {
-          bv = a.B[(int64_t)(a.bmap ? a.bmap[r] : r) * a.ldb + j];
-        }
-      }
+      if (rv && j < N) bv = a.B[(int64_t)(a.bmap ? a.bmap[r] : r) * a.ldb + j];
       ra[p] = av;
       rb[p] = bv;
     }
@@ -377,9 +375,9 @@ __global__ void __launch_bounds__(BT) bw_rows(const int32_t* __restrict__ sorted
   }
 }
 
-// One warp per output q: out[q] = sum_m silu(g) u dhu over row p = map(q)
-// (0 when p < 0), times gamma (1 - gamma) when gamma is given.
-__global__ void __launch_bounds__(BT) bw_rowdot(const float* __restrict__ GU, const float* __restrict__ DHU, int I,
+// One warp per output q: out[q] = sum_m h dhu over row p = map(q) (0 when
+// p < 0), times gamma (1 - gamma) when gamma is given.
+__global__ void __launch_bounds__(BT) bw_rowdot(const float* __restrict__ Hact, const float* __restrict__ DHU, int I,
                                               const int32_t* __restrict__ map, int64_t R,
                                               const float* __restrict__ gamma, float* __restrict__ out) {
   const int lane = threadIdx.x & 31;
@@ -387,9 +385,9 @@ __global__ void __launch_bounds__(BT) bw_rowdot(const float* __restrict__ GU, co
     const int64_t p = map ? map[q] : q;
     float acc = 0.f;
     if (p >= 0) {
-      const float* gu = GU + p * 2 * I;
+      const float* h = Hact + p * I;
       const float* d = DHU + p * I;
-      for (int m = lane; m < I; m += 32) acc = fmaf(silu_f32(gu[m]) * gu[I + m], d[m], acc);
+      for (int m = lane; m < I; m += 32) acc = fmaf(h[m], d[m], acc);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -444,6 +442,16 @@ __global__ void __launch_bounds__(BT) bw_router_bwd(const float* __restrict__ L,
   if (e < E) dL[(int64_t)t * E + e] = dl;
 }
 
+// out[i] = sum_{s < S} part[s * n + i], in order of s
+__global__ void __launch_bounds__(BT) bw_sum_parts(const float* __restrict__ part, int S, int64_t n,
+                                                 float* __restrict__ out) {
+  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
+    float acc = 0.f;
+    for (int q = 0; q < S; ++q) acc += part[q * n + i];
+    out[i] = acc;
+  }
+}
+
 // out[c] = sum_t v[t * ldv + c] for c < C (fixed order over t)
 __global__ void __launch_bounds__(BT) bw_colsum(const float* __restrict__ v, int64_t ldv, int T, int C,
                                               float* __restrict__ out) {
@@ -491,16 +499,26 @@ cudaError_t run_rows(const RowGemm& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <bool B_SWIGLU>
 cudaError_t run_wgrad(const WGemm& a, int nseg, cudaStream_t s) {
   const dim3 grid((unsigned)(ceil_div(a.M, TM) * ceil_div(a.N, TN)), (unsigned)nseg);
-  bw_wgrad_gemm<B_SWIGLU><<<grid, BT, 0, s>>>(a);
+  bw_wgrad_gemm<<<grid, BT, 0, s>>>(a);
   return cudaGetLastError();
 }
 
+// Row chunks of the router's dgate_w = dL^T x: its [E, H] output has few
+// tiles, so its T-long reduction is split until about two blocks per SM are
+// busy (at least 64 rows a chunk, at most 32 chunks).
+int router_chunks(const moe_problem& p) {
+  const int64_t tiles = ceil_div(p.E, TM) * ceil_div(p.H, TN);
+  int64_t S = std::min<int64_t>({ceil_div(2 * 148, tiles), ceil_div(p.T, 64), 32});
+  S = std::max<int64_t>(S, 1);
+  const int64_t chunk = ceil_div(p.T, S);
+  return (int)ceil_div(p.T, std::max<int64_t>(chunk, 1));
+}
+
 struct BwLayout {
-  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, gu, dgu, dhu, dxr,
-      extra, gus, dgus, dhus, gamma, dz, total;
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, parts, gu, dgu, dhu,
+      hact, dxr, extra, gus, dgus, dhus, hacts, gamma, dz, total;
 };
 
 size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -527,9 +545,12 @@ BwLayout bw_layout(const moe_problem& p) {
   b.L = take((size_t)p.T * p.E * 4);
   b.S = take((size_t)p.T * p.E * 4);
   b.dL = take((size_t)p.T * p.E * 4);
+  const int S = router_chunks(p);
+  b.parts = take(S > 1 ? (size_t)S * p.E * p.H * 4 : 0);
   b.gu = take((size_t)P * 2 * p.I * 4);
   b.dgu = take((size_t)P * 2 * p.I * 4);
   b.dhu = take((size_t)P * p.I * 4);
+  b.hact = take((size_t)P * p.I * 4);
   b.dxr = take((size_t)P * p.H * 4);
   b.extra = take((size_t)p.T * p.H * 4);
   const bool sh = p.shared != MOE_SHARED_NONE;
@@ -537,6 +558,7 @@ BwLayout bw_layout(const moe_problem& p) {
   b.gus = take((size_t)p.T * 2 * Is * 4);
   b.dgus = take((size_t)p.T * 2 * Is * 4);
   b.dhus = take((size_t)p.T * Is * 4);
+  b.hacts = take((size_t)p.T * Is * 4);
   b.gamma = take(sh ? (size_t)p.T * 4 : 0);
   b.dz = take(sh ? (size_t)p.T * 4 : 0);
   b.total = off;
@@ -572,7 +594,7 @@ RowGemm row_gemm(const float* A, const int32_t* amap, int64_t lda, const float* 
 
 WGemm wgrad(const float* A, const int32_t* amap, const float* ascale, int64_t lda, int M, const float* B,
             const int32_t* bmap, int64_t ldb, int N, const int32_t* offsets, int single_rows, int64_t rows_total,
-            float* C, int32_t* err) {
+            float* C, int32_t* err, int chunk = 0) {
   WGemm a{};
   a.A = A;
   a.amap = amap;
@@ -585,6 +607,7 @@ WGemm wgrad(const float* A, const int32_t* amap, const float* ascale, int64_t ld
   a.N = N;
   a.offsets = offsets;
   a.single_rows = single_rows;
+  a.chunk = chunk > 0 ? chunk : single_rows;
   a.rows_total = rows_total;
   a.C = C;
   a.err = err;
@@ -668,6 +691,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   float* gu = at<float>(ws, b.gu);
   float* dgu = at<float>(ws, b.dgu);
   float* dhu = at<float>(ws, b.dhu);
+  float* hact = at<float>(ws, b.hact);
   float* dxr = at<float>(ws, b.dxr);
   float* extra = at<float>(ws, b.extra);
 
@@ -701,6 +725,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
         a.scale = scale;
         a.DGU = dgu;
         a.DHU = dhu;
+        a.Hact = hact;
         return a;
       }(),
       s));
@@ -712,15 +737,23 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
         return a;
       }(),
       s));
-  bw_rowdot<<<grid_for(P * 32), BT, 0, s>>>(gu, dhu, I, pair_pos, P, nullptr, dw);
+  bw_rowdot<<<grid_for(P * 32), BT, 0, s>>>(hact, dhu, I, pair_pos, P, nullptr, dw);
   // Routed weight gradients: dWd_e = (w dout)^T h, dWgu_e = [dg du]^T x.
-  BW_CUDA(run_wgrad<true>(wgrad(dout, tok, scale, H, H, gu, nullptr, 0, I, offsets, 0, P, g->d_down, err), E, s));
-  BW_CUDA(run_wgrad<false>(wgrad(dgu, nullptr, nullptr, 2 * I, 2 * I, x, tok, H, H, offsets, 0, P, g->d_gate_up, err),
-                           E, s));
-  // Router backward: dL, dgate_w = dL^T x, d_bias = sum_t dL.
+  BW_CUDA(run_wgrad(wgrad(dout, tok, scale, H, H, hact, nullptr, I, I, offsets, 0, P, g->d_down, err), E, s));
+  BW_CUDA(run_wgrad(wgrad(dgu, nullptr, nullptr, 2 * I, 2 * I, x, tok, H, H, offsets, 0, P, g->d_gate_up, err), E,
+                    s));
+  // Router backward: dL, dgate_w = dL^T x (in row chunks summed in order), d_bias = sum_t dL.
   bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL);
-  BW_CUDA(run_wgrad<false>(wgrad(dL, nullptr, nullptr, E, E, x, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1,
-                           s));
+  const int nchunk = router_chunks(*p);
+  if (nchunk == 1) {
+    BW_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1, s));
+  } else {
+    float* parts = at<float>(ws, b.parts);
+    const int chunk = (int)ceil_div(T, nchunk);
+    BW_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x, nullptr, H, H, nullptr, T, T, parts, err, chunk), nchunk,
+                      s));
+    bw_sum_parts<<<grid_for((int64_t)E * H), BT, 0, s>>>(parts, nchunk, (int64_t)E * H, g->d_gate_w);
+  }
   if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
   // Shared expert over all tokens, scaled by gamma; its dx goes to `extra`.
   float* dz = nullptr;
@@ -731,6 +764,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
     float* gus = at<float>(ws, b.gus);
     float* dgus = at<float>(ws, b.dgus);
     float* dhus = at<float>(ws, b.dhus);
+    float* hacts = at<float>(ws, b.hacts);
     float* gamma = at<float>(ws, b.gamma);
     dz = at<float>(ws, b.dz);
     bw_gamma<<<grid_for((int64_t)T * 32), BT, 0, s>>>(x, gated ? gvec : nullptr, T, H, gamma);
@@ -749,6 +783,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
           a.scale = gamma;
           a.DGU = dgus;
           a.DHU = dhus;
+          a.Hact = hacts;
           return a;
         }(),
         s));
@@ -760,13 +795,13 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
           return a;
         }(),
         s));
-    if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(gus, dhus, Is, nullptr, T, gamma, dz);
-    BW_CUDA(run_wgrad<true>(wgrad(dout, nullptr, gamma, H, H, gus, nullptr, 0, Is, nullptr, T, T,
-                                  g->d_shared_down, err),
-                            1, s));
-    BW_CUDA(run_wgrad<false>(wgrad(dgus, nullptr, nullptr, 2 * Is, 2 * Is, x, nullptr, H, H, nullptr, T, T,
-                                   g->d_shared_gate_up, err),
-                             1, s));
+    if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(hacts, dhus, Is, nullptr, T, gamma, dz);
+    BW_CUDA(run_wgrad(wgrad(dout, nullptr, gamma, H, H, hacts, nullptr, Is, Is, nullptr, T, T, g->d_shared_down,
+                            err),
+                      1, s));
+    BW_CUDA(run_wgrad(wgrad(dgus, nullptr, nullptr, 2 * Is, 2 * Is, x, nullptr, H, H, nullptr, T, T,
+                            g->d_shared_gate_up, err),
+                      1, s));
     if (gated) bw_dgvec<<<grid_for(H), BT, 0, s>>>(dz, x, T, H, g->d_shared_gate);
   }
   // Router (and shared gate) dx into `extra`, then dx = sum of each token's rows + extra.
