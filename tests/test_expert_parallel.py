@@ -1,0 +1,189 @@
+"""Expert parallelism's host orchestration (sparse_top_mixture_b200/expert_parallel.py)
+with gloo ranks on the CPU.
+
+The split arithmetic is checked by brute force. The whole exchange (counts,
+rows and weights out, the receiver's regrouping by local expert, rows back,
+the combine) runs on 2 and 4 gloo ranks with the library's stage calls
+replaced, inside each test process only, by CPU stand-ins with the same
+contracts built from the oracle; each rank's output must equal the oracle's
+one-process forward of its own tokens with all experts. A planted mistake in
+the receiver's layout must break that equality."""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from sparse_top_mixture_b200 import expert_parallel as ep
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+# ---- split arithmetic ---------------------------------------------------------
+
+def test_send_splits_sum_each_ranks_experts():
+    counts = [3, 0, 5, 1, 0, 0, 7, 2]
+    assert ep.send_splits(counts, 1) == [18]
+    assert ep.send_splits(counts, 2) == [9, 9]
+    assert ep.send_splits(counts, 4) == [3, 6, 0, 9]
+    assert ep.send_splits(counts, 8) == counts
+    with pytest.raises(ValueError):
+        ep.send_splits(counts, 3)
+
+
+def test_receive_layout_brute_force():
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        G, El = rng.integers(1, 5), rng.integers(1, 5)
+        rc = rng.integers(0, 4, size=(G, El))
+        splits, ids = ep.receive_layout(rc)
+        want = [e for s in range(G) for e in range(El) for _ in range(rc[s, e])]
+        assert ids.tolist() == want
+        assert splits == [int(v) for v in rc.sum(axis=1)]
+
+
+# ---- CPU stand-ins with the stage calls' contracts ----------------------------
+
+def _install_cpu_stages():
+    """Replace the stage calls the orchestration makes with CPU versions of
+    the same contracts (fp32 in and out, fp64 inside), built from the oracle."""
+    import oracle
+
+    def f64(t):
+        return None if t is None else t.detach().to(torch.float64).numpy()
+
+    def route(p, x, gate_w, bias=None, shared_gate=None):
+        r = oracle.route(f64(x), f64(gate_w), p.k, p.score, f64(bias), p.bias_mode, p.renormalize)
+        gam = None
+        if shared_gate is not None:
+            gam = torch.from_numpy(oracle.shared_gate_values(f64(x), f64(shared_gate), p.shared)).float()
+        return (torch.from_numpy(r["routing_weights"]).float(), torch.from_numpy(r["selected_experts"]), gam)
+
+    def dispatch(p, selected, x=None):
+        d = oracle.dispatch(selected.numpy(), p.E)
+        return {"counts": torch.from_numpy(d["counts"]).int(), "offsets": torch.from_numpy(d["offsets"]).int(),
+                "sorted_pairs": torch.from_numpy(d["sorted_pairs"]).int(),
+                "pair_pos": torch.from_numpy(d["pair_pos"]).int(),
+                "x_perm": None if x is None else x[torch.from_numpy(d["sorted_pairs"] // p.k)]}
+
+    def grouped_swiglu(p, x_perm, offsets, gate_up, down, routing_weights=None, sorted_pairs=None):
+        xp, off = f64(x_perm), offsets.numpy()
+        w = f64(routing_weights).reshape(-1)
+        y = np.zeros((p.T * p.k, p.H))
+        for e in range(p.E):
+            a, b = off[e], off[e + 1]
+            if b > a:
+                rows = oracle.swiglu_mlp(xp[a:b], f64(gate_up[e]), f64(down[e]))
+                y[a:b] = w[sorted_pairs[a:b].numpy()][:, None] * rows
+        return torch.from_numpy(y).float()
+
+    def shared_expert(p, x, shared_gate_up, shared_down, gamma=None):
+        s = oracle.swiglu_mlp(f64(x), f64(shared_gate_up), f64(shared_down))
+        if gamma is not None:
+            s = f64(gamma)[:, None] * s
+        return torch.from_numpy(s).float()
+
+    def combine(p, y_perm, pair_pos, shared_out=None):
+        y, pp = f64(y_perm), pair_pos.numpy().reshape(p.T, p.k)
+        out = np.zeros((p.T, p.H))
+        for j in range(p.k):
+            ok = pp[:, j] >= 0
+            out[ok] += y[pp[ok, j]]
+        if shared_out is not None:
+            out += f64(shared_out)
+        return torch.from_numpy(out).float()
+
+    for name, fn in dict(route=route, dispatch=dispatch, grouped_swiglu=grouped_swiglu,
+                         shared_expert=shared_expert, combine=combine).items():
+        setattr(ep, name, fn)
+
+
+CASES = {
+    "softmax_plain": dict(T=13, H=16, E=8, k=2, I=8, I_shared=8, score="softmax", bias_mode="logit",
+                          renormalize=False, shared="plain", bias_kind="uniform0.1"),
+    "sigmoid_gated": dict(T=17, H=24, E=8, k=3, I=16, I_shared=8, score="sigmoid", bias_mode="none",
+                          renormalize=True, shared="sigmoid_gated"),
+    "sqrtsoftplus_select": dict(T=9, H=16, E=8, k=4, I=8, I_shared=0, score="sqrtsoftplus", bias_mode="select",
+                                renormalize=True, shared="none", bias_kind="uniform0.1"),
+}
+
+
+def _worker(rank, world, port, case, planted, q):
+    import dataclasses
+
+    import torch.distributed as dist
+
+    import oracle
+    import sparse_top_mixture_b200 as stm
+    import workloads
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        _install_cpu_stages()
+        if planted:  # receiver layout in expert-major order instead of arrival order
+            right = ep.receive_layout
+
+            def wrong(rc):
+                splits, ids = right(rc)
+                return splits, np.sort(ids, kind="stable")
+            ep.receive_layout = wrong
+        cfg = workloads.CONFIGS["tiny_fp32"].replace(name="ep", **CASES[case])
+        full = workloads.generate(cfg, "cpu")
+        mine = workloads.router_inputs(cfg, rank=rank)  # this rank's own batch
+        El = cfg.E // world
+        w = dict(full, gate_up=full["gate_up"][rank * El:(rank + 1) * El].contiguous(),
+                 down=full["down"][rank * El:(rank + 1) * El].contiguous())
+        p = dataclasses.replace(stm.Problem.from_config(cfg))
+        layer = ep.ExpertParallelMoE(p, w)
+        out, rw, sel = layer(mine["x"])
+        n = workloads.to_numpy64
+        ref = oracle.moe_forward(n(mine["x"]), n(full["gate_w"]), n(full["gate_up"]), n(full["down"]), k=cfg.k,
+                                 score=cfg.score, renormalize=cfg.renormalize, bias=n(full.get("bias")),
+                                 bias_mode=cfg.bias_mode, shared=cfg.shared,
+                                 shared_gate_up=n(full.get("shared_gate_up")),
+                                 shared_down=n(full.get("shared_down")), shared_gate=n(full.get("shared_gate")))
+        got = out.double().numpy()
+        rel = float(np.linalg.norm(got - ref["out"]) / np.linalg.norm(ref["out"]))
+        same = bool(np.array_equal(sel.numpy(), ref["selected_experts"]))
+        q.put((rank, rel, same, None))
+    except Exception as exc:  # reported to the parent, which fails the test
+        q.put((rank, None, None, repr(exc)))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, case, planted=False):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, case, planted, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = sorted(q.get(timeout=180) for _ in procs)
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    for rank, rel, same, err in res:
+        assert err is None, f"rank {rank}: {err}"
+    return res
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("case", list(CASES))
+def test_expert_parallel_matches_one_process_oracle(world, case):
+    for rank, rel, same, _ in _run(world, case):
+        assert same, f"rank {rank}: selection differs"
+        assert rel <= 1e-6, f"rank {rank}: rel L2 {rel:.3e}"
+
+
+def test_planted_receive_layout_mistake_is_caught():
+    res = _run(2, "sigmoid_gated", planted=True)
+    assert max(rel for _, rel, _, _ in res) > 1e-3
