@@ -14,7 +14,6 @@ import socket
 
 import numpy as np
 import pytest
-import torch
 import torch.multiprocessing as mp
 
 from sparse_top_mixture_b200 import expert_parallel as ep
@@ -49,62 +48,6 @@ def test_receive_layout_brute_force():
         assert splits == [int(v) for v in rc.sum(axis=1)]
 
 
-# ---- CPU stand-ins with the stage calls' contracts ----------------------------
-
-def _install_cpu_stages():
-    """Replace the stage calls the orchestration makes with CPU versions of
-    the same contracts (fp32 in and out, fp64 inside), built from the oracle."""
-    import oracle
-
-    def f64(t):
-        return None if t is None else t.detach().to(torch.float64).numpy()
-
-    def route(p, x, gate_w, bias=None, shared_gate=None):
-        r = oracle.route(f64(x), f64(gate_w), p.k, p.score, f64(bias), p.bias_mode, p.renormalize)
-        gam = None
-        if shared_gate is not None:
-            gam = torch.from_numpy(oracle.shared_gate_values(f64(x), f64(shared_gate), p.shared)).float()
-        return (torch.from_numpy(r["routing_weights"]).float(), torch.from_numpy(r["selected_experts"]), gam)
-
-    def dispatch(p, selected, x=None):
-        d = oracle.dispatch(selected.numpy(), p.E)
-        return {"counts": torch.from_numpy(d["counts"]).int(), "offsets": torch.from_numpy(d["offsets"]).int(),
-                "sorted_pairs": torch.from_numpy(d["sorted_pairs"]).int(),
-                "pair_pos": torch.from_numpy(d["pair_pos"]).int(),
-                "x_perm": None if x is None else x[torch.from_numpy(d["sorted_pairs"] // p.k)]}
-
-    def grouped_swiglu(p, x_perm, offsets, gate_up, down, routing_weights=None, sorted_pairs=None):
-        xp, off = f64(x_perm), offsets.numpy()
-        w = f64(routing_weights).reshape(-1)
-        y = np.zeros((p.T * p.k, p.H))
-        for e in range(p.E):
-            a, b = off[e], off[e + 1]
-            if b > a:
-                rows = oracle.swiglu_mlp(xp[a:b], f64(gate_up[e]), f64(down[e]))
-                y[a:b] = w[sorted_pairs[a:b].numpy()][:, None] * rows
-        return torch.from_numpy(y).float()
-
-    def shared_expert(p, x, shared_gate_up, shared_down, gamma=None):
-        s = oracle.swiglu_mlp(f64(x), f64(shared_gate_up), f64(shared_down))
-        if gamma is not None:
-            s = f64(gamma)[:, None] * s
-        return torch.from_numpy(s).float()
-
-    def combine(p, y_perm, pair_pos, shared_out=None):
-        y, pp = f64(y_perm), pair_pos.numpy().reshape(p.T, p.k)
-        out = np.zeros((p.T, p.H))
-        for j in range(p.k):
-            ok = pp[:, j] >= 0
-            out[ok] += y[pp[ok, j]]
-        if shared_out is not None:
-            out += f64(shared_out)
-        return torch.from_numpy(out).float()
-
-    for name, fn in dict(route=route, dispatch=dispatch, grouped_swiglu=grouped_swiglu,
-                         shared_expert=shared_expert, combine=combine).items():
-        setattr(ep, name, fn)
-
-
 CASES = {
     "softmax_plain": dict(T=13, H=16, E=8, k=2, I=8, I_shared=8, score="softmax", bias_mode="logit",
                           renormalize=False, shared="plain", bias_kind="uniform0.1"),
@@ -116,18 +59,17 @@ CASES = {
 
 
 def _worker(rank, world, port, case, planted, q):
-    import dataclasses
-
     import torch.distributed as dist
 
     import oracle
     import sparse_top_mixture_b200 as stm
+    import stage_standins
     import workloads
 
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        _install_cpu_stages()
+        stage_standins.install(ep)
         if planted:  # receiver layout in expert-major order instead of arrival order
             right = ep.receive_layout
 
@@ -141,7 +83,7 @@ def _worker(rank, world, port, case, planted, q):
         El = cfg.E // world
         w = dict(full, gate_up=full["gate_up"][rank * El:(rank + 1) * El].contiguous(),
                  down=full["down"][rank * El:(rank + 1) * El].contiguous())
-        p = dataclasses.replace(stm.Problem.from_config(cfg))
+        p = stm.Problem.from_config(cfg)
         layer = ep.ExpertParallelMoE(p, w)
         out, rw, sel = layer(mine["x"])
         n = workloads.to_numpy64
