@@ -40,7 +40,7 @@ from typing import Dict, List, Optional, Sequence, Tuple
 import numpy as np
 import torch
 
-from . import Problem, combine, dispatch, grouped_swiglu, route, shared_expert
+from . import Problem, combine, dispatch, grouped_swiglu, new_workspace, route, shared_expert, workspace_size
 
 
 def send_splits(counts: Sequence[int], world: int) -> List[int]:
@@ -61,6 +61,25 @@ def receive_layout(recv_counts: np.ndarray) -> Tuple[List[int], np.ndarray]:
     local = np.arange(rc.shape[1], dtype=np.int64)
     ids = np.concatenate([np.repeat(local, row) for row in rc]) if rc.size else np.zeros(0, np.int64)
     return splits, ids.astype(np.int64)
+
+
+class WorkspacePool:
+    """Library workspaces kept across calls: one per problem kind (the
+    problem with T set aside), replaced by a larger one only when a call
+    needs more bytes than the kept one has."""
+
+    def __init__(self, device):
+        self.device = device
+        self._kept: Dict[Problem, Tuple[int, torch.Tensor]] = {}
+
+    def get(self, p: Problem) -> torch.Tensor:
+        key = dataclasses.replace(p, T=0)
+        need = workspace_size(p)
+        kept = self._kept.get(key)
+        if kept is None or kept[0] < need:
+            kept = (need, new_workspace(p, self.device))
+            self._kept[key] = kept
+        return kept[1]
 
 
 class ExpertParallelMoE:
@@ -86,6 +105,7 @@ class ExpertParallelMoE:
         gu, dn = weights["gate_up"], weights["down"]
         if tuple(gu.shape) != (self.E_local, 2 * p.I, p.H) or tuple(dn.shape) != (self.E_local, p.H, p.I):
             raise ValueError(f"local expert weights must be [{self.E_local}, 2I, H] and [{self.E_local}, H, I]")
+        self.pool = WorkspacePool(gu.device)
 
     def _a2a(self, out: torch.Tensor, inp: torch.Tensor, out_splits, in_splits) -> None:
         import torch.distributed as dist
@@ -97,8 +117,9 @@ class ExpertParallelMoE:
         p, w = self.p, self.w
         dev = x.device
         gate = w.get("shared_gate") if p.shared == "sigmoid_gated" else None
-        rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate)
-        d = dispatch(p, sel, x)
+        ws = self.pool.get(p)
+        rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate, ws=ws)
+        d = dispatch(p, sel, x, ws=ws)
 
         # counts to the experts' owners; one host read sizes the row exchange
         counts = d["counts"].to(torch.int64)
@@ -122,7 +143,7 @@ class ExpertParallelMoE:
         self._a2a(y_perm[:n_send], y_recv, sends, recvs)
         shared = None
         if p.shared != "none":
-            shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma)
+            shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma, ws=ws)
         return combine(p, y_perm, d["pair_pos"], shared), rw, sel
 
     __call__ = forward
@@ -136,7 +157,8 @@ class ExpertParallelMoE:
             return torch.zeros(0, p.H, dtype=torch.float32, device=x_recv.device)
         pr = dataclasses.replace(p, T=n, E=self.E_local, k=1, I_shared=0, bias_mode="none", shared="none")
         ids = torch.from_numpy(local_ids).to(x_recv.device).view(n, 1)
-        d = dispatch(pr, ids, x_recv)
+        ws = self.pool.get(pr)
+        d = dispatch(pr, ids, x_recv, ws=ws)
         y = grouped_swiglu(pr, d["x_perm"], d["offsets"], self.w["gate_up"], self.w["down"], w_recv.view(n, 1),
-                           d["sorted_pairs"])
+                           d["sorted_pairs"], ws=ws)
         return combine(dataclasses.replace(pr, dtype="f32"), y, d["pair_pos"], None)

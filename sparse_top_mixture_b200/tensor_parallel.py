@@ -29,7 +29,7 @@ from typing import Dict, Optional
 
 import torch
 
-from . import Problem, combine, dispatch, grouped_swiglu, route, shared_expert
+from . import Problem, combine, dispatch, grouped_swiglu, new_workspace, route, shared_expert
 
 
 def shard_expert_weights(weights: Dict[str, Optional[torch.Tensor]], rank: int, world: int
@@ -74,6 +74,7 @@ class TensorParallelMoE:
             raise ValueError(f"I={p.I} / I_shared={p.I_shared} do not split over {self.world} ranks")
         self.local = dataclasses.replace(p, I=p.I // self.world,
                                          I_shared=p.I_shared // self.world if p.shared != "none" else 0)
+        self.ws = new_workspace(p, weights["gate_up"].device)  # the full problem's: the largest of the calls
 
     def forward(self, x: torch.Tensor):
         """out [T,H] (problem dtype), routing_weights [T,k] fp32, selected_experts [T,k] int64."""
@@ -81,12 +82,13 @@ class TensorParallelMoE:
 
         p, pl, w = self.p, self.local, self.w
         gate = w.get("shared_gate") if p.shared == "sigmoid_gated" else None
-        rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate)
-        d = dispatch(p, sel, x)
-        y = grouped_swiglu(pl, d["x_perm"], d["offsets"], w["gate_up"], w["down"], rw, d["sorted_pairs"])
+        ws = self.ws
+        rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate, ws=ws)
+        d = dispatch(p, sel, x, ws=ws)
+        y = grouped_swiglu(pl, d["x_perm"], d["offsets"], w["gate_up"], w["down"], rw, d["sorted_pairs"], ws=ws)
         shared = None
         if p.shared != "none":
-            shared = shared_expert(pl, x, w["shared_gate_up"], w["shared_down"], gamma)
+            shared = shared_expert(pl, x, w["shared_gate_up"], w["shared_down"], gamma, ws=ws)
         part = combine(dataclasses.replace(pl, dtype="f32"), y, d["pair_pos"], shared)  # fp32 [T, H]
         dist.all_reduce(part, group=self.group)
         # round the fp32 sum once: a one-slot combine of the rows in order
