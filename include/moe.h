@@ -326,8 +326,9 @@ typedef struct moe_grads {
  *   int64 (normally the forward's). Routing weights, the per-expert
  *   activations and outputs are recomputed from x; nothing from the forward
  *   is needed besides the choice.
- *   fp32 problems only (MOE_ERR_UNSUPPORTED for bf16). Each gradient element
- *   is one thread's fixed-order fp32 sum (no atomics): results are
+ *   fp32 problems only (MOE_ERR_UNSUPPORTED for bf16). Every gradient
+ *   element is an fp32 sum in a fixed order (no atomics; the router weight
+ *   gradient adds row-chunk partial sums in chunk order): results are
  *   deterministic. A pair with an expert id outside [0, E) contributes
  *   nothing and sets MOE_DEVERR_BAD_EXPERT_ID in the workspace header.
  *   Workspace: moe_backward_workspace_size bytes (its header as for

@@ -25,8 +25,9 @@
 // router and shared expert use the same two GEMM kernels over one all-token
 // segment. Every GEMM is 128x128 output tiles, 8-deep k slices
 // double-buffered in shared memory, 8x8 fp32 outputs per thread; every output
-// element is one thread's fixed-order sum (no atomics), so results are
-// deterministic. bf16 problems are not supported.
+// element is one thread's fixed-order sum (dgate_w: row-chunk partials added
+// in chunk order), with no atomics, so results are deterministic. bf16
+// problems are not supported.
 #include <cuda_runtime.h>
 
 #include <algorithm>
