@@ -1,5 +1,6 @@
 /*
- * moe.h -- C ABI of the B200 (sm_100a) sparse top-k MoE FFN forward.
+ * moe.h -- C ABI of the B200 (sm_100a) sparse top-k MoE FFN: the forward
+ * pass, the aux-loss-free balancer's bias update, and an fp32 backward pass.
  *
  * The forward pass, step by step:
  *   route    : logits = x . gate_w^T, scores (softmax / sigmoid / sqrtsoftplus),
@@ -130,8 +131,9 @@ enum {
   MOE_NUM_STAGES = 6
 };
 
-/* Bytes of workspace moe_forward needs for problem p (each of the other calls
- * needs at most this much). Host only. */
+/* Bytes of workspace moe_forward needs for problem p (each of the other
+ * forward calls needs at most this much; moe_backward has its own size,
+ * moe_backward_workspace_size). Host only. */
 moe_status moe_workspace_size(const moe_problem *p, size_t *bytes);
 
 /* Zero the workspace header (error flags). Call once after allocating it. */
