@@ -195,7 +195,13 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   // record nodes of the graph (recorded at every replay).
   cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
   if (ev != nullptr) MOE_CUDA(cudaStreamIsCapturing(s, &capture));
+  static const char* const kStageNames[MOE_NUM_STAGES] = {"route", "dispatch", "gate_up",
+                                                          "down",  "shared",   "combine"};
+  NvtxRange range("moe_forward");
+  NvtxStages stage;
   auto mark = [&](int i) -> moe_status {
+    if (i < MOE_NUM_STAGES) stage.next(kStageNames[i]);
+    else stage.close();
     if (ev == nullptr || ev[i] == nullptr) return MOE_OK;
     if (capture == cudaStreamCaptureStatusActive)
       return cuda_status(cudaEventRecordWithFlags(ev[i], s, cudaEventRecordExternal));

@@ -670,6 +670,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
     if (gated) BW_CUDA(cudaMemsetAsync(g->d_shared_gate, 0, (size_t)p->H * f, s));
     return MOE_OK;
   }
+  NvtxRange range("moe_backward");
   const BwLayout b = bw_layout(*p);
   const int T = (int)p->T, H = (int)p->H, E = (int)p->E, k = (int)p->k, I = (int)p->I, Is = (int)p->I_shared;
   const int64_t P = p->T * p->k;

@@ -5,10 +5,42 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <mutex>
 
 namespace stm {
+
+// Host-side NVTX ranges naming the launch sequence (a profiler can select
+// "moe_forward/" or "moe_backward/" launches). Header-only NVTX: without an
+// attached tool each call is a no-op. A range is closed on every return path.
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// Consecutive stages inside one range: next() closes the previous stage's
+// range and opens the next one; the last one closes with the object.
+class NvtxStages {
+ public:
+  void next(const char* name) {
+    close();
+    nvtxRangePushA(name);
+    open_ = true;
+  }
+  void close() {
+    if (open_) nvtxRangePop();
+    open_ = false;
+  }
+  ~NvtxStages() { close(); }
+
+ private:
+  bool open_ = false;
+};
 
 // Raise a kernel's dynamic shared memory limit to `bytes` once per device
 // (the attribute belongs to the kernel's module in each device context).
