@@ -338,12 +338,14 @@ def backward_workspace_size(p: Problem) -> int:
     return n.value
 
 
-def backward(p: Problem, weights: Dict[str, Optional[torch.Tensor]], x, dout, selected, ws=None
+def backward(p: Problem, weights: Dict[str, Optional[torch.Tensor]], x, dout, selected, ws=None, out=None
              ) -> Dict[str, Optional[torch.Tensor]]:
     """Gradients of sum(dout * out) for the fp32 forward with the expert choice
     held at ``selected`` [T,k] int64: dx, d_gate_w, d_bias (logit bias only),
     d_gate_up, d_down and, with a shared expert, d_shared_gate_up,
-    d_shared_down and d_shared_gate (gated only). Async on the current stream."""
+    d_shared_down and d_shared_gate (gated only). ``out``: optional dict of
+    preallocated fp32 tensors for any of them (written, never accumulated
+    into). Async on the current stream."""
     if p.dtype != "f32":
         raise MoeError(2, "moe_backward supports fp32 problems only")
     cw = _weights_struct(p, weights)
@@ -351,14 +353,21 @@ def backward(p: Problem, weights: Dict[str, Optional[torch.Tensor]], x, dout, se
     _req(dout, "dout", (p.T, p.H), torch.float32)
     _req(selected, "selected", (p.T, p.k), torch.int64)
     dev = x.device
-    z = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)  # noqa: E731
-    g = {"dx": z(p.T, p.H), "d_gate_w": z(p.E, p.H), "d_bias": z(p.E) if p.bias_mode == "logit" else None,
-         "d_gate_up": z(p.E, 2 * p.I, p.H), "d_down": z(p.E, p.H, p.I), "d_shared_gate_up": None,
-         "d_shared_down": None, "d_shared_gate": None}
-    if p.shared != "none":
-        g["d_shared_gate_up"], g["d_shared_down"] = z(2 * p.I_shared, p.H), z(p.H, p.I_shared)
-    if p.shared == "sigmoid_gated":
-        g["d_shared_gate"] = z(p.H)
+    sh, gated = p.shared != "none", p.shared == "sigmoid_gated"
+    shapes = {"dx": (p.T, p.H), "d_gate_w": (p.E, p.H), "d_bias": (p.E,) if p.bias_mode == "logit" else None,
+              "d_gate_up": (p.E, 2 * p.I, p.H), "d_down": (p.E, p.H, p.I),
+              "d_shared_gate_up": (2 * p.I_shared, p.H) if sh else None,
+              "d_shared_down": (p.H, p.I_shared) if sh else None, "d_shared_gate": (p.H,) if gated else None}
+    g: Dict[str, Optional[torch.Tensor]] = {}
+    for key, shape in shapes.items():
+        t = None if (out is None or shape is None) else out.get(key)
+        if shape is None:
+            g[key] = None
+        elif t is None:
+            g[key] = torch.empty(*shape, dtype=torch.float32, device=dev)
+        else:
+            _req(t, key, shape, torch.float32)
+            g[key] = t
     if ws is None:
         ws = torch.zeros(backward_workspace_size(p), dtype=torch.uint8, device=dev)
     cg = moe_grads(*[_ptr(g[f]) for f, _ in moe_grads._fields_])

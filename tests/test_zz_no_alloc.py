@@ -9,8 +9,9 @@ moe_dispatch on the same inputs -- bit for bit, as for all index work --
 on two calls in a row with different inputs, so that anything left in the
 shared array by the first call would show up in the second.
 
-This file is collected last so that a run stopping at the first failure has
-already run every other test.
+This file is collected after the parity tests (only the guard-band checks
+come later) so that a run stopping at the first failure has already run
+them.
 """
 
 import pytest
