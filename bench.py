@@ -267,7 +267,7 @@ def measure_backward(cfg, local: int, steps: int = 5) -> dict:
     return {"workload": f"{cfg.name} shapes in fp32 (T={cfg.T}, H={cfg.H}, E={cfg.E}, k={cfg.k}, I={cfg.I}, "
                         f"I_shared={cfg.I_shared})",
             "ms": ms, "steps": steps, "flops": fl, "bound": "alu", "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s", "frac": achieved / peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
             "peak_source": f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)",
             "clocks": c}
 
