@@ -14,6 +14,7 @@ import socket
 
 import numpy as np
 import pytest
+import torch
 import torch.multiprocessing as mp
 
 from sparse_top_mixture_b200 import expert_parallel as ep
@@ -58,7 +59,7 @@ CASES = {
 }
 
 
-def _worker(rank, world, port, case, planted, q):
+def _worker(rank, world, port, case, planted, q, skew=False):
     import torch.distributed as dist
 
     import oracle
@@ -79,6 +80,8 @@ def _worker(rank, world, port, case, planted, q):
             ep.receive_layout = wrong
         cfg = workloads.CONFIGS["tiny_fp32"].replace(name="ep", **CASES[case])
         full = workloads.generate(cfg, "cpu")
+        if skew:  # a selection bias that sends every pair to rank 0's experts
+            full["bias"] = (torch.arange(cfg.E) < cfg.E // world).float() * 10.0
         mine = workloads.router_inputs(cfg, rank=rank)  # this rank's own batch
         El = cfg.E // world
         w = dict(full, gate_up=full["gate_up"][rank * El:(rank + 1) * El].contiguous(),
@@ -102,11 +105,11 @@ def _worker(rank, world, port, case, planted, q):
         dist.destroy_process_group()
 
 
-def _run(world, case, planted=False):
+def _run(world, case, planted=False, skew=False):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, case, planted, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, case, planted, q, skew)) for r in range(world)]
     for pr in procs:
         pr.start()
     res = sorted(q.get(timeout=180) for _ in procs)
@@ -129,3 +132,11 @@ def test_expert_parallel_matches_one_process_oracle(world, case):
 def test_planted_receive_layout_mistake_is_caught():
     res = _run(2, "sigmoid_gated", planted=True)
     assert max(rel for _, rel, _, _ in res) > 1e-3
+
+
+def test_ranks_that_receive_no_rows():
+    """A selection bias sends every pair to rank 0's experts: the other ranks
+    receive nothing, send everything, and still finish their own tokens."""
+    for rank, rel, same, _ in _run(2, "sqrtsoftplus_select", skew=True):
+        assert same, f"rank {rank}: selection differs"
+        assert rel <= 1e-6, f"rank {rank}: rel L2 {rel:.3e}"
