@@ -234,9 +234,44 @@ def backward_flops(cfg) -> float:
     return 16.0 * P * cfg.H * cfg.I + 6.0 * cfg.T * cfg.E * cfg.H + 16.0 * cfg.T * cfg.H * cfg.I_shared
 
 
-def measure_backward(cfg, local: int, steps: int = 5) -> dict:
+def backward_cpu_baseline(cfg32, inp, dout, target_s: float = 8.0) -> dict:
+    """The fp64 backward oracle, as it stands, on the first n tokens of the
+    fp32 workload (its own top-k choice), n sized so that one call takes about
+    ``target_s``. Each call also builds the oracle's gradient of every expert
+    weight, a fixed cost that dominates small samples; n is sized from two
+    short runs that separate it from the per-token cost."""
+    import numpy as np
+
+    import oracle.backward as ob
+    f64 = workloads.to_numpy64
+    x, do = f64(inp["x"]), f64(dout)
+    gw, bias = f64(inp["gate_w"]), f64(inp.get("bias"))
+    gu = [f64(inp["gate_up"][e]) for e in range(cfg32.E)]
+    dn = [f64(inp["down"][e]) for e in range(cfg32.E)]
+    sgu, sdn, sg = f64(inp.get("shared_gate_up")), f64(inp.get("shared_down")), f64(inp.get("shared_gate"))
+
+    def run(n: int) -> float:
+        t0 = time.perf_counter()
+        ob.moe_backward(x[:n], gw, gu, dn, do[:n], k=cfg32.k, score=cfg32.score, renormalize=cfg32.renormalize,
+                        bias=bias, bias_mode=cfg32.bias_mode, shared=cfg32.shared, shared_gate_up=sgu,
+                        shared_down=sdn, shared_gate=sg)
+        return time.perf_counter() - t0
+
+    # t(n) = fixed + per_token * n, from two short runs; then one run of ~target_s
+    t_small, t_big = run(4), run(64)
+    per = max((t_big - t_small) / 60.0, 1e-9)
+    fixed = max(t_small - 4 * per, 0.0)
+    n = int(np.clip((target_s - fixed) / per, 4, cfg32.T))
+    t = run(n)
+    return {"value": n / t, "unit": "tokens/s", "cores": _blas_threads() or os.cpu_count(), "kind": "oracle",
+            "sample": f"backward of the first {n} of the {cfg32.T} tokens of {cfg32.name} in fp64 "
+                      f"(oracle.backward, its own top-k choice), {t:.1f} s"}
+
+
+def measure_backward(cfg, local: int, steps: int = 5, cpu: bool = False) -> dict:
     """The fp32 backward on the bench workload's shapes, timed with CUDA events
-    on the current stream, against the FFMA peak at the sampled SM clock."""
+    on the current stream, against the FFMA peak at the sampled SM clock;
+    with ``cpu``, the backward oracle timed on the host beside it."""
     import sparse_top_mixture_b200 as stm
     cfg32 = cfg.replace(dtype="f32")
     inp = workloads.generate(cfg32, "cuda")
@@ -264,12 +299,18 @@ def measure_backward(cfg, local: int, steps: int = 5) -> dict:
     mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965
     peak = NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
     achieved = fl / (ms / 1e3) / 1e12
-    return {"workload": f"{cfg.name} shapes in fp32 (T={cfg.T}, H={cfg.H}, E={cfg.E}, k={cfg.k}, I={cfg.I}, "
-                        f"I_shared={cfg.I_shared})",
-            "ms": ms, "steps": steps, "flops": fl, "bound": "alu", "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-            "peak_source": f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)",
-            "clocks": c}
+    res = {"workload": f"{cfg.name} shapes in fp32 (T={cfg.T}, H={cfg.H}, E={cfg.E}, k={cfg.k}, I={cfg.I}, "
+                       f"I_shared={cfg.I_shared})",
+           "ms": ms, "tokens_per_s": cfg.T / (ms / 1e3), "steps": steps, "flops": fl, "bound": "alu",
+           "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+           "peak_source": f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)",
+           "clocks": c}
+    if cpu:
+        try:
+            res["cpu_baseline"] = backward_cpu_baseline(cfg32, inp, dout)
+        except Exception as exc:  # the host baseline never costs the bench line
+            res["cpu_baseline"] = {"value": None, "error": repr(exc)[:200]}
+    return res
 
 
 def init_dist(n_gpus: int):
@@ -532,7 +573,7 @@ def main():
         "clocks": clocks.summary(),
     }
     if world == 1 and not args.no_backward:
-        line["backward"] = measure_backward(cfg, local)
+        line["backward"] = measure_backward(cfg, local, cpu=not args.no_cpu_baseline)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, dict(r_cpu, **{k: dev[k] for k in (
             "gate_up", "down", "shared_gate_up", "shared_down")}))
