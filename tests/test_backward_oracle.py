@@ -1,6 +1,7 @@
 """Pins of the backward oracle (oracle/backward.py) by central finite
-differences of the forward oracle, with the expert choice held fixed, and
-planted mistakes that those pins must catch. CPU only."""
+differences of the forward oracle, with the expert choice held fixed, by
+torch autograd of a plain per-expert loop in fp64, and planted mistakes that
+those pins must catch. CPU only."""
 
 from __future__ import annotations
 
@@ -8,6 +9,8 @@ import numpy as np
 import pytest
 
 import oracle.backward as ob
+import torch
+import torch_loop
 from oracle_pins import oracle_run, tiny_problem
 
 CASES = []
@@ -135,3 +138,24 @@ def test_planted_shared_gate_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(ob, "moe_backward", no_gate_grad)
     caught = [c for c in CASES if c[3] == "sigmoid_gated" and not finite_difference_pin(c)[0]]
     assert caught
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(str(v) for v in c))
+def test_backward_matches_autograd_of_a_per_expert_loop(case):
+    """torch autograd (fp64) of the per-expert loop, for the oracle's choice,
+    gives the oracle's gradients to rounding."""
+    score, bias_mode, renorm, shared = case
+    cfg, a = _problem(score, bias_mode, renorm, shared, 2)
+    dout = np.random.default_rng(7).normal(size=(cfg.T, cfg.H))
+    sel = oracle_run(cfg, a)["selected_experts"]
+    g = _backward(cfg, a, dout, sel)
+    leaves = {k: torch.from_numpy(v).requires_grad_(True) for k, v in a.items() if v is not None}
+    out = torch_loop.forward(cfg, leaves, torch.from_numpy(sel))
+    assert np.allclose(out.detach().numpy(), oracle_run(cfg, a, selected=sel)["out"], rtol=1e-12, atol=1e-12)
+    (out * torch.from_numpy(dout)).sum().backward()
+    for name, key in torch_loop.GRAD_OF.items():
+        if g.get(key) is None:  # no such parameter, or a selection bias: no gradient on either side
+            assert leaves.get(name) is None or leaves[name].grad is None, key
+            continue
+        auto = leaves[name].grad.numpy()
+        assert np.allclose(g[key], auto, rtol=1e-10, atol=1e-12), f"{case} {key}"
