@@ -234,6 +234,26 @@ def backward_flops(cfg) -> float:
     return 16.0 * P * cfg.H * cfg.I + 6.0 * cfg.T * cfg.E * cfg.H + 16.0 * cfg.T * cfg.H * cfg.I_shared
 
 
+def host_memory_available() -> float:
+    """Bytes this process may still allocate: the smaller of the host's
+    available memory and what its cgroup (v2 or v1) limit leaves."""
+    import psutil
+    avail = float(psutil.virtual_memory().available)
+    for limit_f, usage_f in (("/sys/fs/cgroup/memory.max", "/sys/fs/cgroup/memory.current"),
+                             ("/sys/fs/cgroup/memory/memory.limit_in_bytes",
+                              "/sys/fs/cgroup/memory/memory.usage_in_bytes")):
+        try:
+            with open(limit_f) as f:
+                lim = f.read().strip()
+            with open(usage_f) as f:
+                used = float(f.read().strip())
+        except OSError:
+            continue
+        if lim.isdigit():
+            avail = min(avail, float(lim) - used)
+    return avail
+
+
 def backward_cpu_baseline(cfg32, inp, dout, target_s: float = 8.0) -> dict:
     """The fp64 backward oracle, as it stands, on the first n tokens of the
     fp32 workload (its own top-k choice), n sized so that one call takes about
@@ -243,6 +263,12 @@ def backward_cpu_baseline(cfg32, inp, dout, target_s: float = 8.0) -> dict:
     import numpy as np
 
     import oracle.backward as ob
+    # fp64 weights, the oracle's per-expert weight gradients and their stacked copy
+    need = 3.0 * 8 * (cfg32.E * 3 * cfg32.I * cfg32.H + 3 * cfg32.I_shared * cfg32.H)
+    have = host_memory_available()
+    if have < 1.5 * need:
+        return {"value": None, "unit": "tokens/s", "kind": "oracle",
+                "skipped": f"needs ~{need / 1e9:.1f} GB of host memory, {have / 1e9:.1f} GB available"}
     f64 = workloads.to_numpy64
     x, do = f64(inp["x"]), f64(dout)
     gw, bias = f64(inp["gate_w"]), f64(inp.get("bias"))
