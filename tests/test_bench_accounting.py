@@ -1,0 +1,55 @@
+"""The bench's work accounting (CPU): the algorithmic FLOPs and bytes that
+the roofline figures divide by, recounted here contraction by contraction
+from the shapes, for every named problem."""
+
+import pytest
+
+import bench
+import workloads
+from workloads import CONFIGS
+
+
+def _gemm(m, n, k):
+    return 2.0 * m * n * k
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_backward_flops_count_every_contraction(name):
+    c = CONFIGS[name]
+    P = c.T * c.k
+    routed = (_gemm(P, 2 * c.I, c.H)     # recompute [g | u] = x W_gu^T
+              + _gemm(P, c.I, c.H)       # dhu = dout W_d
+              + _gemm(P, c.H, 2 * c.I)   # dx rows = [dg du] W_gu
+              + _gemm(c.H, c.I, P)       # dW_d = (w dout)^T h, summed over the experts' rows
+              + _gemm(2 * c.I, c.H, P))  # dW_gu = [dg du]^T x
+    router = _gemm(c.T, c.E, c.H) * 3    # logits, dgate_w = dL^T x, dx += dL gate_w
+    Is = c.I_shared
+    shared = (_gemm(c.T, 2 * Is, c.H) + _gemm(c.T, Is, c.H) + _gemm(c.T, c.H, 2 * Is) + _gemm(c.H, Is, c.T)
+              + _gemm(2 * Is, c.H, c.T))
+    assert bench.backward_flops(c) == pytest.approx(routed + router + shared, rel=1e-12)
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_forward_accounting(name):
+    c = CONFIGS[name]
+    P = c.T * c.k
+    es = 4 if c.dtype == "f32" else 2
+    active = min(c.E, P)
+    fb = bench.flops_and_bytes(c, active)
+    assert fb["gate_up_flops"] == _gemm(P, 2 * c.I, c.H)
+    assert fb["active_flops"] == pytest.approx(
+        _gemm(P, 2 * c.I, c.H) + _gemm(P, c.H, c.I) + (_gemm(c.T, 2 * c.I_shared, c.H) + _gemm(c.T, c.H, c.I_shared)),
+        rel=1e-12)
+    assert fb["router_flops"] == _gemm(c.T, c.E, c.H)
+    # gate_up kernel: the active experts' gate_up weights once, x_perm read once, h written once
+    assert fb["gate_up_bytes"] == (active * 2 * c.I * c.H + P * c.H + P * c.I) * es
+
+
+def test_host_memory_probe_is_positive():
+    assert bench.host_memory_available() > 0
+
+
+def test_job_throughput_is_whole_job():
+    # two ranks of 4096 tokens, 10 steps in 20 ms (the slower rank's time)
+    assert bench.job_throughput(2, 4096, 10, 20.0) == pytest.approx(2 * 4096 * 10 / 0.020)
+    assert workloads.CONFIGS["qwen3_30b_a3b"].P == 4096 * 8
