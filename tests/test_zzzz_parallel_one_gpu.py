@@ -28,7 +28,6 @@ def _free_port() -> int:
 def _child(name, port, q):
     import datetime
 
-    import numpy as np
     import torch
     import torch.distributed as dist
 
