@@ -3,7 +3,7 @@ with gloo ranks on the CPU.
 
 The split arithmetic is checked by brute force. The whole exchange (counts,
 rows and weights out, the receiver's regrouping by local expert, rows back,
-the combine) runs on 2 and 4 gloo ranks with the library's stage calls
+the combine) runs on 1, 2 and 4 gloo ranks with the library's stage calls
 replaced, inside each test process only, by CPU stand-ins with the same
 contracts built from the oracle; each rank's output must equal the oracle's
 one-process forward of its own tokens with all experts. A planted mistake in
@@ -121,7 +121,7 @@ def _run(world, case, planted=False, skew=False):
     return res
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world", [1, 2, 4])
 @pytest.mark.parametrize("case", list(CASES))
 def test_expert_parallel_matches_one_process_oracle(world, case):
     for rank, rel, same, _ in _run(world, case):

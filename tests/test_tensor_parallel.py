@@ -3,7 +3,7 @@ with gloo ranks on the CPU.
 
 The weight sharding is checked against the full weights directly. The whole
 layer (replicated routing, each rank's slice of every expert, the fp32
-all-reduce of the partial outputs, one rounding) runs on 2 and 4 gloo ranks
+all-reduce of the partial outputs, one rounding) runs on 1, 2 and 4 gloo ranks
 with the library's stage calls replaced, inside each test process only, by
 CPU stand-ins with the same contracts built from the oracle; every rank's
 output must equal the oracle's one-process forward with unsharded experts. A
@@ -108,7 +108,7 @@ def _run(world, case, planted=False):
     return res
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world", [1, 2, 4])
 @pytest.mark.parametrize("case", list(CASES))
 def test_tensor_parallel_matches_one_process_oracle(world, case):
     for rank, rel, same, _ in _run(world, case):
