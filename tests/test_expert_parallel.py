@@ -140,3 +140,53 @@ def test_ranks_that_receive_no_rows():
     for rank, rel, same, _ in _run(2, "sqrtsoftplus_select", skew=True):
         assert same, f"rank {rank}: selection differs"
         assert rel <= 1e-6, f"rank {rank}: rel L2 {rel:.3e}"
+
+
+def _leaving_worker(rank, world, port, q):
+    """Rank 1 leaves before the layer's first exchange; rank 0 must get an
+    error from its collective (peer gone, or the group's short timeout), not
+    wait forever."""
+    import datetime
+
+    import torch.distributed as dist
+
+    import sparse_top_mixture_b200 as stm
+    import stage_standins
+    import workloads
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    def report(msg):
+        q.put((rank, msg))
+        q.close()
+        q.join_thread()  # flushed before the process ends
+
+    if rank == 1:
+        report("left")
+        os._exit(0)  # leaves between steps: nothing of its own is in flight
+    try:
+        stage_standins.install(ep)
+        cfg = workloads.CONFIGS["tiny_fp32"].replace(name="ep", **CASES["softmax_plain"])
+        full = workloads.generate(cfg, "cpu")
+        El = cfg.E // world
+        w = dict(full, gate_up=full["gate_up"][:El].contiguous(), down=full["down"][:El].contiguous())
+        ep.ExpertParallelMoE(stm.Problem.from_config(cfg), w)(full["x"])
+        msg = "no error"
+    except Exception as exc:
+        msg = "error: " + type(exc).__name__
+    report(msg)
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_others_exchange_with_an_error():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, q)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for pr in procs:
+        pr.join(timeout=60)
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res[0]
