@@ -4,18 +4,22 @@
 
 A step is one whole forward (route, dispatch, grouped SwiGLU, shared expert,
 combine) over one batch of synthetic tokens. Default workload: the
-Qwen3-30B-A3B-shaped problem (T=4096, H=2048, E=128, top-8 softmax with
-renormalisation, I=768, bf16). With N > 1 (torchrun, one process per GPU)
+DSV4-Flash-ablation-shaped problem (T=8192, H=4096, 64 routed experts + 1
+shared, top-6 sqrtsoftplus with an fp32 selection bias, I=2048, bf16), the
+largest of the named problems. With N > 1 (torchrun, one process per GPU)
 every rank runs its own batch with the same weights (weak scaling, no
 collective on the data path); the time is the max over ranks.
 
 Rank 0 prints one JSON line. ``value`` is tokens/s with inputs resident in
 HBM; ``e2e`` is the same metric through the public API from pinned host
 memory (host->device copy of x and device->host copy of out inside the timed
-region); ``roofline`` describes the dominant kernel (the grouped gate_up
-GEMM), timed with CUDA events on its stream inside the timed region;
-``cpu_baseline`` is the fp64 oracle timed on a bounded token sample on the
-host cores. ``--impl reference`` times that oracle as the reference arm.
+region); ``roofline`` describes the dominant kernel (the routed gate_up
+GEMM), timed with CUDA events on its stream inside graph replays, against its
+algorithmic FLOPs and bytes (active expert weights read once, x read once);
+``forward_roofline`` does the same for the whole forward; ``per_config``
+repeats the measurement on every named problem; ``cpu_baseline`` is the fp64
+oracle timed on a bounded token sample on the host cores. ``--impl
+reference`` times that oracle as the reference arm.
 """
 
 from __future__ import annotations
@@ -25,7 +29,6 @@ import datetime
 import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -38,7 +41,7 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
-DEFAULT_CONFIG = "qwen3_30b_a3b"
+DEFAULT_CONFIG = "dsv4_flash_ablation"
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -106,33 +109,91 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------
-# workload accounting
+# workload accounting (algorithmic work only: the active experts' weights read
+# once, x read once, out written once; the implementation's own intermediates
+# x_perm, h and y rows are not counted)
 
 def active_experts(sel: torch.Tensor, E: int) -> int:
     return int((torch.bincount(sel.reshape(-1), minlength=E) > 0).sum().item())
 
 
 def flops_and_bytes(cfg, n_active: int):
+    """Algorithmic FLOPs and bytes of the whole forward and of its two grouped
+    GEMMs, for ``n_active`` experts that receive at least one row."""
     P = cfg.T * cfg.k
     es = 4 if cfg.dtype == "f32" else 2
     f_routed = 6.0 * cfg.H * cfg.I * P
     f_shared = 6.0 * cfg.H * cfg.I_shared * cfg.T if cfg.shared != "none" else 0.0
     f_router = 2.0 * cfg.T * cfg.H * cfg.E
-    # gate_up kernel alone: 4*H*I flops per pair; weights of active experts read
-    # once, x_perm read once, h written once.
+    x_bytes = cfg.T * cfg.H * es
+    # routed gate_up GEMM: 4*H*I flops per (token, expert) row; the active
+    # experts' gate_up weights read once and x read once
     gu_flops = 4.0 * cfg.H * cfg.I * P
-    gu_bytes = (n_active * 2 * cfg.I * cfg.H + P * cfg.H + P * cfg.I) * es
-    # whole forward, minimum: active weights once, x read, out written
+    gu_bytes = n_active * 2 * cfg.I * cfg.H * es + x_bytes
+    # routed down GEMM: 2*H*I flops per row; the active down weights once and
+    # the output written once
+    dn_flops = 2.0 * cfg.H * cfg.I * P
+    dn_bytes = n_active * cfg.I * cfg.H * es + x_bytes
+    # whole forward: active weights once (+ router and shared weights), x in, out back
     w_bytes = n_active * 3 * cfg.I * cfg.H * es + cfg.E * cfg.H * es
     if cfg.shared != "none":
         w_bytes += 3 * cfg.I_shared * cfg.H * es
-    min_bytes = w_bytes + 2 * cfg.T * cfg.H * es
+    min_bytes = w_bytes + 2 * x_bytes
     return {"active_flops": f_routed + f_shared, "router_flops": f_router, "gate_up_flops": gu_flops,
-            "gate_up_bytes": gu_bytes, "min_bytes": min_bytes, "weight_bytes": w_bytes}
+            "gate_up_bytes": gu_bytes, "down_flops": dn_flops, "down_bytes": dn_bytes, "min_bytes": min_bytes,
+            "weight_bytes": w_bytes}
 
+
+def total_weight_bytes(cfg) -> int:
+    """Bytes of every expert weight of the problem (all E routed + shared)."""
+    es = 4 if cfg.dtype == "f32" else 2
+    b = cfg.E * 3 * cfg.I * cfg.H * es + cfg.E * cfg.H * es
+    if cfg.shared != "none":
+        b += 3 * cfg.I_shared * cfg.H * es
+    return b
+
+
+FP32_LANES_PER_SM = 128  # FFMA lanes per Blackwell SM (4 sub-partitions x 32)
+NUM_SMS = 148
+
+
+def ffma_peak_tflops(mhz: float) -> float:
+    """fp32 FFMA peak from the unit counts at the given SM clock."""
+    return NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+
+
+def roofline_entry(flops: float, nbytes: float, ms: float, pk: dict, dtype: str, mhz: float = None) -> dict:
+    """Bound, achieved and fraction of one kernel (or of the whole forward)
+    from its algorithmic FLOPs and bytes and its measured time: the bound is
+    the larger of FLOPs / tensor peak (burst: the kernels are timed inside
+    sub-10-ms replays) and bytes / HBM copy bandwidth; bf16 contractions use
+    the measured bf16 peak, fp32 ones the FFMA peak from the unit counts."""
+    s = ms / 1e3
+    if dtype == "f32":
+        peak_t = ffma_peak_tflops(mhz or 1965.0)
+        t_src = f"148 SMs x 128 FFMA lanes x 2 flop x {mhz or 1965.0:.0f} MHz"
+    else:
+        peak_t = pk["bf16_tflops"]
+        t_src = pk["source"] + " bf16 (burst)"
+    t_tensor = flops / (peak_t * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        e = {"bound": "alu" if dtype == "f32" else "tensor", "achieved": flops / s / 1e12, "peak": peak_t,
+             "unit": "TFLOP/s", "peak_source": t_src}
+        if dtype != "f32":
+            e["frac_of_sustained"] = e["achieved"] / pk["bf16_tflops_sustained"]
+    else:
+        e = {"bound": "hbm", "achieved": nbytes / s / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+             "peak_source": pk["source"] + " copy bandwidth"}
+        e["frac_of_nominal_8000gbs"] = e["achieved"] / 8000.0
+    e["frac"] = e["achieved"] / e["peak"]
+    e["t_roof_ms"] = 1e3 * max(t_tensor, t_hbm)
+    e["algorithmic"] = {"flops": flops, "bytes": nbytes, "ms": ms}
+    return e
 
 
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc2.cu", "tc_ptx.cuh", "tc_epilogue.cuh", "tiles.cuh", "common.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def kernel_source_hash() -> str:
@@ -144,18 +205,19 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(cfg_name: str):
-    """Per-launch DRAM traffic of the gate_up kernel from the committed ncu
-    summary, if the kernel sources are unchanged since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"gate_up_{cfg_name}.md")
-    if not os.path.exists(path):
+def recorded_traffic(cfg_name: str, kernel: str = "gate_up"):
+    """Per-launch DRAM traffic (read + write bytes) of a grouped GEMM from the
+    ncu record in ``profiles/traffic.json``, if the kernel sources are
+    unchanged since it was taken; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
         return None
-    text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"kernel_sources_sha256:\s*([0-9a-f]+)", text)
-    if not m or not h or kernel_source_hash() != h.group(1):
-        return None
-    return float(m.group(1))
+    with open(TRAFFIC_FILE) as f:
+        entries = json.load(f).get("entries", [])
+    sha = kernel_source_hash()
+    for e in entries:
+        if e.get("config") == cfg_name and e.get("kernel") == kernel and e.get("kernel_sources_sha256") == sha:
+            return float(e["bytes_per_launch"])
+    return None
 
 
 # ----------------------------------------------------------------------------
@@ -211,6 +273,11 @@ class OracleTimer:
 
 
 def cpu_baseline(cfg, dev_inputs, target_s: float = 12.0):
+    need = 8.0 * total_weight_bytes(cfg) / (4 if cfg.dtype == "f32" else 2)
+    have = host_memory_available()
+    if have < 1.5 * need:
+        return {"value": None, "unit": "tokens/s", "kind": "oracle",
+                "skipped": f"fp64 weights need ~{need / 1e9:.1f} GB of host memory, {have / 1e9:.1f} GB available"}
     ot = OracleTimer(cfg, dev_inputs)
     n = ot.calibrate(target_s, cfg.T)
     t = ot.run(n)
@@ -220,10 +287,6 @@ def cpu_baseline(cfg, dev_inputs, target_s: float = 12.0):
 
 
 # ----------------------------------------------------------------------------
-
-FP32_LANES_PER_SM = 128  # FFMA lanes per Blackwell SM (4 sub-partitions x 32)
-NUM_SMS = 148
-
 
 def backward_flops(cfg) -> float:
     """Algorithmic FLOPs of one backward (moe_backward): per routed pair the
@@ -383,6 +446,25 @@ def make_inputs(cfg, rank: int):
     return r, dev
 
 
+def metric_name() -> str:
+    return "MoE FFN tokens/s and active-expert TFLOP/s (fraction of bf16/HBM roofline)"
+
+
+def l2_policy(cfg) -> str:
+    """How the timed steps keep L2 from serving the next step's inputs."""
+    wb = total_weight_bytes(cfg)
+    if wb > L2_BYTES:
+        return f"inputs larger than L2: {wb / 1e9:.2f} GB of expert weights > 126 MB L2, no flush"
+    return f"L2 flushed between timed steps ({FLUSH_BYTES >> 20} MB write); weights {wb / 1e6:.1f} MB"
+
+
+def config_dict(cfg) -> dict:
+    """The workload's name and shape (the same for both arms of the bench)."""
+    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+            "I_shared": cfg.I_shared, "score": cfg.score, "bias_mode": cfg.bias_mode,
+            "renormalize": cfg.renormalize, "shared": cfg.shared, "seed": cfg.seed, "l2": l2_policy(cfg)}
+
+
 def run_reference(args, cfg, rank, world):
     """Reference arm: the fp64 oracle on the host cores, rank 0 only."""
     if rank != 0:
@@ -391,6 +473,7 @@ def run_reference(args, cfg, rank, world):
     r = workloads.router_inputs(cfg)
     w = workloads.expert_weights(cfg, "cuda" if torch.cuda.is_available() else "cpu")
     ot = OracleTimer(cfg, dict(r, **w))
+    del w
     n = ot.calibrate(max(1.0, 60.0 / max(1, args.steps + args.warmup)), cfg.T)
     for i in range(args.warmup):
         ot.run(n, start=i * n)
@@ -409,14 +492,131 @@ def run_reference(args, cfg, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def metric_name() -> str:
-    return "MoE FFN tokens/s and active-expert TFLOP/s (fraction of bf16/HBM roofline)"
+FLUSH_BYTES = 256 << 20
 
 
-def config_dict(cfg) -> dict:
-    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
-            "I_shared": cfg.I_shared, "score": cfg.score, "bias_mode": cfg.bias_mode,
-            "renormalize": cfg.renormalize, "shared": cfg.shared, "seed": cfg.seed}
+class ForwardRun:
+    """One problem's inputs, module and graphs on this rank's GPU, and the
+    device-timed measurement of its forward."""
+
+    def __init__(self, cfg, rank: int, graph: bool = True):
+        import sparse_top_mixture_b200 as stm
+        self.stm = stm
+        self.cfg = cfg
+        self.r_cpu, self.dev = make_inputs(cfg, rank)
+        self.p = stm.Problem.from_config(cfg)
+        self.moe = stm.SparseMoE(self.p, self.dev)
+        dt = self.p.torch_dtype
+        self.x = self.dev["x"]
+        self.out = torch.empty(cfg.T, cfg.H, dtype=dt, device="cuda")
+        self.rw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+        self.sel = torch.empty(cfg.T, cfg.k, dtype=torch.int64, device="cuda")
+        self.use_graph = graph
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") \
+            if total_weight_bytes(cfg) <= L2_BYTES else None
+
+    def warm(self, warmup: int):
+        for _ in range(warmup):
+            self.moe.forward(self.x, self.out, self.rw, self.sel)
+        torch.cuda.synchronize()
+        if self.moe.read_device_error() != 0:
+            raise RuntimeError(f"{self.cfg.name}: device error flag set during warm-up")
+        self.n_active = active_experts(self.sel, self.cfg.E)
+        self.fb = flops_and_bytes(self.cfg, self.n_active)
+        # The timed steps replay the forward as one CUDA graph (the same kernels
+        # on the same buffers as the eager call, launched as one graph).
+        self.graphed = self.stm.GraphedForward(self.moe, self.x, self.out, self.rw, self.sel) \
+            if self.use_graph else None
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+
+    def step(self):
+        if self.graphed is not None:
+            self.graphed.replay()
+        else:
+            self.moe.forward(self.x, self.out, self.rw, self.sel)
+
+    def timed(self, steps: int, local: int, world: int):
+        """Device time of `steps` forwards (ms, max over ranks) and the clocks
+        sampled meanwhile. Problems whose weights fit in L2 flush it between
+        steps (outside the timed intervals)."""
+        stream = torch.cuda.current_stream()
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clocks:
+            if self.flush is None:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(steps):
+                    self.step()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ms = a.elapsed_time(b)
+            else:
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(steps)]
+                for a, b in ev:
+                    self.flush.zero_()
+                    a.record(stream)
+                    self.step()
+                    b.record(stream)
+                torch.cuda.synchronize()
+                ms = sum(a.elapsed_time(b) for a, b in ev)
+        barrier(world)
+        if self.moe.read_device_error() != 0:
+            raise RuntimeError(f"{self.cfg.name}: device error flag set during the timed region")
+        return dist_max(ms, world), clocks.summary()
+
+    def stages(self, steps: int, local: int):
+        """Median device time of each stage: the same forward with CUDA events
+        between the stages (recorded inside the graph at every replay), one
+        step at a time."""
+        stm = self.stm
+        stream = torch.cuda.current_stream()
+        nst = len(stm.STAGES) + 1
+        sev = [torch.cuda.Event(enable_timing=True) for _ in range(nst)]
+        for e in sev:  # torch creates the CUDA event on its first record
+            e.record(stream)
+        torch.cuda.synchronize()
+        staged = stm.GraphedForward(self.moe, self.x, self.out, self.rw, self.sel, events=sev) \
+            if self.use_graph else None
+        samples = []
+        with ClockSampler(local) as clk:
+            for _ in range(steps):
+                if self.flush is not None:
+                    self.flush.zero_()
+                if staged is not None:
+                    staged.replay()
+                else:
+                    self.moe.forward(self.x, self.out, self.rw, self.sel, events=sev)
+                torch.cuda.synchronize()
+                samples.append([sev[si].elapsed_time(sev[si + 1]) for si in range(nst - 1)])
+        stage_ms = {name: statistics.median(row[si] for row in samples) for si, name in enumerate(stm.STAGES)}
+        return stage_ms, statistics.median(sum(row) for row in samples), clk.summary()
+
+    def release(self):
+        for name in ("graphed", "moe", "dev", "x", "out", "rw", "sel", "flush"):
+            if hasattr(self, name):
+                delattr(self, name)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def forward_summary(cfg, fb, n_active, ms_per_step, stage_ms, clocks, pk, world: int = 1) -> dict:
+    """Throughput, the whole forward's roofline fraction and the dominant
+    kernel's (the routed gate_up GEMM) from algorithmic work and device times."""
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    whole = roofline_entry(fb["active_flops"] + fb["router_flops"], fb["min_bytes"], ms_per_step, pk, cfg.dtype, mhz)
+    gu = roofline_entry(fb["gate_up_flops"], fb["gate_up_bytes"], stage_ms["gate_up"], pk, cfg.dtype, mhz)
+    dn = roofline_entry(fb["down_flops"], fb["down_bytes"], stage_ms["down"], pk, cfg.dtype, mhz)
+    return {
+        "workload": cfg.name, "ms_per_step": ms_per_step, "tokens_per_s": world * cfg.T / (ms_per_step / 1e3),
+        "active_expert_tflops": world * fb["active_flops"] / (ms_per_step / 1e3) / 1e12,
+        "active_experts": n_active, "forward_roofline": whole,
+        "dominant_kernel": dict(gu, kernel="gate_up"), "down_kernel": dict(dn, kernel="down"),
+        "stage_ms": stage_ms, "clocks": clocks,
+    }
 
 
 def main():
@@ -430,10 +630,21 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-graph", action="store_true", help="launch each kernel from the host every step")
     ap.add_argument("--no-backward", action="store_true", help="skip the fp32 backward measurement")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per_config block (the other workloads)")
+    ap.add_argument("--per-config-steps", type=int, default=50)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="profiling only: override T (the line then names a reduced workload, not a bench line)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling only: override E (with --tokens, keeps rows per expert for smaller captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = workloads.CONFIGS[args.config]
+    if args.tokens is not None or args.experts is not None:
+        T, E = args.tokens or cfg.T, args.experts or cfg.E
+        cfg = cfg.replace(name=f"{cfg.name}@T{T}E{E}", T=T, E=E, bias_kind="none" if cfg.bias_kind == "zipf"
+                          else cfg.bias_kind, bias_mode="none" if cfg.bias_kind == "zipf" else cfg.bias_mode)
+        args.no_per_config = True
     rank, local, world = init_dist(args.gpus)
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
@@ -447,78 +658,27 @@ def main():
     if not os.path.exists(stm.LIB_PATH):  # the CUDA library is built in-tree
         from sparse_top_mixture_b200 import build
         build.build()
+    pk = peaks()
 
-    r_cpu, dev = make_inputs(cfg, rank)
-    p = stm.Problem.from_config(cfg)
-    moe = stm.SparseMoE(p, dev)
-    dt = p.torch_dtype
-    x = dev["x"]
-    out = torch.empty(cfg.T, cfg.H, dtype=dt, device="cuda")
-    rw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
-    sel = torch.empty(cfg.T, cfg.k, dtype=torch.int64, device="cuda")
-    stream = torch.cuda.current_stream()
-
-    for _ in range(args.warmup):
-        moe.forward(x, out, rw, sel)
-    torch.cuda.synchronize()
-    if moe.read_device_error() != 0:
-        raise RuntimeError("device error flag set during warm-up")
-    n_active = active_experts(sel, cfg.E)
-    fb = flops_and_bytes(cfg, n_active)
-
-    # The timed steps replay the forward as one CUDA graph (the same kernels on
-    # the same buffers as the eager call, launched as one graph).
-    graphed = None if args.no_graph else stm.GraphedForward(moe, x, out, rw, sel)
-    step = graphed.replay if graphed is not None else (lambda: moe.forward(x, out, rw, sel))
-    for _ in range(args.warmup):
-        step()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step()
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    elapsed_ms = dist_max(t_start.elapsed_time(t_end), world)
-    if moe.read_device_error() != 0:
-        raise RuntimeError("device error flag set during the timed region")
-
-    # Per-stage device times: the same forward with CUDA events between the
-    # stages (recorded inside the graph when graphs are used), one step at a
-    # time, the median per stage over the steps (the roofline below uses the
-    # gate_up one).
-    nst = len(stm.STAGES) + 1
-    sev = [torch.cuda.Event(enable_timing=True) for _ in range(nst)]
-    for e in sev:  # torch creates the CUDA event on its first record
-        e.record(stream)
-    torch.cuda.synchronize()
-    staged = None if args.no_graph else stm.GraphedForward(moe, x, out, rw, sel, events=sev)
+    run = ForwardRun(cfg, rank, graph=not args.no_graph)
+    run.warm(args.warmup)
+    elapsed_ms, clocks = run.timed(args.steps, local, world)
     stage_steps = min(args.steps, 100)
-    samples = []
-    with ClockSampler(local) as stage_clocks:
-        for i in range(stage_steps):
-            if staged is not None:
-                staged.replay()
-            else:
-                moe.forward(x, out, rw, sel, events=sev)
-            torch.cuda.synchronize()
-            samples.append([sev[si].elapsed_time(sev[si + 1]) for si in range(nst - 1)])
-    stage_ms = {name: statistics.median(row[si] for row in samples) for si, name in enumerate(stm.STAGES)}
-    staged_ms = statistics.median(sum(row) for row in samples)
-
+    stage_ms, staged_ms, stage_clocks = run.stages(stage_steps, local)
     ms_per_step = elapsed_ms / args.steps
+    fb, n_active = run.fb, run.n_active
+    summ = forward_summary(cfg, fb, n_active, ms_per_step, stage_ms, clocks, pk, world)
     tokens_per_s = job_throughput(world, cfg.T, args.steps, elapsed_ms)
-    active_tflops = world * fb["active_flops"] * args.steps / (elapsed_ms / 1e3) / 1e12
+    moe, p, x, out = run.moe, run.p, run.x, run.out
+    stream = torch.cuda.current_stream()
+    dt = p.torch_dtype
 
     # e2e: pinned host x in, host out back, through the public API. Batches go
     # through a three-slot HostPipeline: every step still copies its own input
     # in and its result out inside the timed region, overlapped with the
     # neighbouring steps' compute.
     e2e_steps = args.e2e_steps or max(4, min(args.steps, 50))
-    x_host = [r_cpu["x"].pin_memory(), r_cpu["x"].clone().pin_memory(), r_cpu["x"].clone().pin_memory()]
+    x_host = [run.r_cpu["x"].pin_memory(), run.r_cpu["x"].clone().pin_memory(), run.r_cpu["x"].clone().pin_memory()]
     out_host = [torch.empty(cfg.T, cfg.H, dtype=dt).pin_memory() for _ in range(3)]
     pipe = stm.HostPipeline(moe, depth=3)
     for i in range(4):
@@ -536,6 +696,7 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = dist_max(e0.elapsed_time(e1), world)
     e2e_tps = job_throughput(world, cfg.T, e2e_steps, e2e_ms)
+    del pipe
 
     # The balancer's deferred bias update (stash this forward's counts, then
     # one sign-controller step), timed on its own: two one-block launches.
@@ -554,55 +715,63 @@ def main():
     torch.cuda.synchronize()
     balance_us = b0.elapsed_time(b1) * 1e3 / 100
 
-    pk = peaks()
-    gu_ms = stage_ms["gate_up"]
-    t_tensor = fb["gate_up_flops"] / (pk["bf16_tflops_sustained"] * 1e12)
-    t_hbm = fb["gate_up_bytes"] / (pk["hbm_gbs"] * 1e9)
-    if t_tensor >= t_hbm:
-        achieved = fb["gate_up_flops"] / (gu_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s"}
-    else:
-        achieved = fb["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    if roof["bound"] == "hbm":  # also against the nominal 8 TB/s of HBM3e
-        roof["frac_of_nominal_8000gbs"] = roof["achieved"] / 8000.0
-    roof["traffic"] = recorded_traffic(cfg.name)
+    roof = dict(summ["dominant_kernel"])
+    roof["traffic"] = recorded_traffic(cfg.name, "gate_up")
     roof["kernel"] = {0: "simt_grouped_kernel<gate_up>", 1: "tc_grouped_gemm_kernel<gate_up>",
                       2: "tc2_grouped_gemm_kernel<gate_up> (CTA pairs)"}[stm.gemm_path(p)]
-    roof["peak_source"] = pk["source"] + (" sustained bf16" if roof["bound"] == "tensor" else " copy bandwidth")
-    roof["algorithmic"] = {"flops": fb["gate_up_flops"], "bytes": fb["gate_up_bytes"], "ms": gu_ms}
-
-    whole_roof_s = max((fb["active_flops"] + fb["router_flops"]) / (pk["bf16_tflops_sustained"] * 1e12),
-                       fb["min_bytes"] / (pk["hbm_gbs"] * 1e9))
+    if roof["traffic"] is not None:
+        roof["traffic_over_algorithmic"] = roof["traffic"] / roof["algorithmic"]["bytes"]
 
     line = {
         "metric": metric_name(), "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; weights ~N(0,1/fan_in))",
-        "config": dict(config_dict(cfg), parallelism=f"replicas x{world} (independent batches)",
-                       l2=f"inputs larger than L2: {fb['weight_bytes'] / 1e9:.2f} GB of weights read per step, "
-                          f"no flush"),
-        "active_expert_tflops": active_tflops,
-        "forward_roofline_frac": whole_roof_s / (ms_per_step / 1e3),
+        "config": config_dict(cfg),
+        "parallelism": f"replicas x{world} (independent batches, no collective on the data path)",
+        "active_expert_tflops": summ["active_expert_tflops"],
+        "forward_roofline_frac": summ["forward_roofline"]["frac"],
+        "forward_roofline": summ["forward_roofline"],
         "active_experts": n_active,
         "stage_ms": stage_ms,
-        "launch": "cuda_graph" if graphed is not None else "eager",
+        "launch": "cuda_graph" if run.graphed is not None else "eager",
         "bias_update_us": balance_us,
         "stage_pass_ms_per_step": staged_ms,
-        "stage_clocks": stage_clocks.summary(),
+        "stage_clocks": stage_clocks,
         "roofline": roof,
+        "down_kernel": summ["down_kernel"],
         "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": e2e_steps,
                 "how": "HostPipeline depth 3: per step H2D of x, forward (graph replay), D2H of out on the step's stream"},
         "gpu_launches": stm.launches_per_forward(p, two_streams=moe.aux is not None) * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clocks,
     }
-    if world == 1 and not args.no_backward:
-        line["backward"] = measure_backward(cfg, local, cpu=not args.no_cpu_baseline)
+    cpu_inputs = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, dict(r_cpu, **{k: dev[k] for k in (
-            "gate_up", "down", "shared_gate_up", "shared_down")}))
+        cpu_inputs = dict(run.r_cpu, **{k: run.dev[k] for k in ("gate_up", "down", "shared_gate_up", "shared_down")})
+    run.release()
+    del moe, x, out, counts
+
+    if world == 1 and not args.no_per_config:
+        # Every named workload, each measured the same way (graph replays,
+        # per-stage events) on this GPU, one after the other.
+        per = {}
+        for name in workloads.CONFIG_ORDER:
+            if name == cfg.name:
+                per[name] = dict(summ, steps=args.steps)
+                continue
+            c = workloads.CONFIGS[name]
+            r = ForwardRun(c, rank, graph=not args.no_graph)
+            r.warm(5)
+            ms, clk = r.timed(args.per_config_steps, local, world)
+            st, _, _ = r.stages(min(args.per_config_steps, 20), local)
+            per[name] = dict(forward_summary(c, r.fb, r.n_active, ms / args.per_config_steps, st, clk, pk),
+                             steps=args.per_config_steps, l2=l2_policy(c))
+            r.release()
+        line["per_config"] = per
+    if world == 1 and not args.no_backward:
+        line["backward"] = measure_backward(workloads.CONFIGS["qwen3_30b_a3b"], local, cpu=not args.no_cpu_baseline)
+    if cpu_inputs is not None:
+        line["cpu_baseline"] = cpu_baseline(cfg, cpu_inputs)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -179,14 +179,18 @@ moe_status moe_dispatch(const moe_problem *p, const int64_t *selected_experts, c
  * an allocator.
  *   Same arguments and results as moe_dispatch, minus the workspace: the
  *   per-block count matrix the dispatch kernels pass to each other lives in
- *   a static 1 MiB device array inside this library (every GPU that loads the
- *   library holds it until the process exits). Problems needing more than
+ *   a static 1 MiB device array inside this library, and the histogram's
+ *   completion ticket in a static 4-byte one (every GPU that loads the
+ *   library holds both until the process exits). Problems needing more than
  *   2^18 count entries, ceil(T / max(1, 256 / k)) * E, are rejected with
  *   MOE_ERR_UNSUPPORTED before anything is launched.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture. Calls allocate and free nothing.
- *   Every call reuses the same array: calls whose work overlaps on the GPU
+ *   `stream` must belong to the current device: the arrays used are the
+ *   current device's. The first call on a device looks up their device
+ *   addresses (with that device current; a failed lookup is retried by the
+ *   next call); make that first call before any stream capture. Calls
+ *   allocate and free nothing; each clears the ticket (an async memset on
+ *   `stream`) before its two kernels.
+ *   Every call reuses the same arrays: calls whose work overlaps on the GPU
  *   (two streams, or two host threads) race and corrupt each other's
  *   results; serialise them. Nothing carried over from an earlier call is
  *   read. A pair with an expert id outside [0, E) is skipped (pair_pos -1)
@@ -234,14 +238,19 @@ moe_status moe_forward(const moe_problem *p, const moe_weights *w, const void *x
                        moe_stream_t stream);
 
 /* moe_forward with two options:
- *   aux_stream: when not NULL (and not `stream`), the problem has a shared
- *     expert and that expert is small (its gate_up GEMM has at most 74
- *     128x128 tiles, as for a decode batch), the shared expert runs on
- *     aux_stream concurrently with the routed path on `stream`, and `stream`
- *     waits for it before the combine (fork / join through two events the
- *     call creates and releases); the sigmoid gate is then computed by its
- *     own small kernel. Larger shared experts run on `stream`, because they
- *     occupy every SM. All work is complete once `stream` has passed the call.
+ *   aux_stream: when not NULL (and not `stream`) and the problem has a shared
+ *     expert, that expert runs on aux_stream (fork / join through two events
+ *     the call creates and releases):
+ *     - a small shared expert (its gate_up GEMM has at most 74 128x128
+ *       tiles, as for a decode batch) runs beside the whole routed path and
+ *       `stream` waits for it before the combine; its sigmoid gate is then
+ *       computed by its own small kernel;
+ *     - a larger one occupies every SM while it runs, so it starts after the
+ *       route (whose top-k kernel computes the gate) and runs beside the
+ *       dispatch kernels only; `stream` waits for it before the routed gate_up
+ *       GEMM. The dispatch stage's event interval then ends when both are
+ *       done and the shared stage's interval is empty.
+ *     All work is complete once `stream` has passed the call.
  *   stage_events: NULL, or MOE_NUM_STAGES + 1 caller-created events recorded
  *     on `stream` before each stage (MOE_STAGE_*) and after the last one; a
  *     NULL entry is skipped. While `stream` is being captured into a CUDA

@@ -248,24 +248,36 @@ def dispatch(p: Problem, selected, x=None, ws=None) -> Dict[str, torch.Tensor]:
     return r
 
 
-def dispatch_noalloc(p: Problem, selected, x=None) -> Dict[str, torch.Tensor]:
+def dispatch_noalloc(p: Problem, selected, x=None, out: Optional[Dict[str, torch.Tensor]] = None
+                     ) -> Dict[str, torch.Tensor]:
     """moe_dispatch without a workspace, for callers that may not allocate
-    device memory (the library keeps the dispatch's scratch in a fixed device
-    array; concurrent calls must be serialised). The result tensors here are
-    still allocated by PyTorch for convenience."""
+    device memory (the library keeps the dispatch's scratch in fixed device
+    arrays; concurrent calls must be serialised). ``out``: optional dict of
+    preallocated results (counts, offsets, sorted_pairs, pair_pos and, with
+    ``x``, x_perm), so that the call itself allocates nothing; missing ones
+    are allocated by PyTorch here. Runs with selected's device current."""
     _req(selected, "selected_experts", (p.T, p.k), torch.int64)
     dev = selected.device
     P = p.T * p.k
     if x is not None:
         _req(x, "x", (p.T, p.H), p.torch_dtype)
-    r = {"counts": torch.empty(p.E, dtype=torch.int32, device=dev),
-         "offsets": torch.empty(p.E + 1, dtype=torch.int32, device=dev),
-         "sorted_pairs": torch.empty(P, dtype=torch.int32, device=dev),
-         "pair_pos": torch.empty(P, dtype=torch.int32, device=dev),
-         "x_perm": torch.empty(P, p.H, dtype=p.torch_dtype, device=dev) if x is not None else None}
-    _check(lib().moe_dispatch_noalloc(ctypes.byref(p.c()), _ptr(selected), _ptr(x), _ptr(r["counts"]),
-                                      _ptr(r["offsets"]), _ptr(r["sorted_pairs"]), _ptr(r["pair_pos"]),
-                                      _ptr(r["x_perm"]), _stream(dev)))
+    shapes = {"counts": ((p.E,), torch.int32), "offsets": ((p.E + 1,), torch.int32),
+              "sorted_pairs": ((P,), torch.int32), "pair_pos": ((P,), torch.int32),
+              "x_perm": ((P, p.H), p.torch_dtype)}
+    r: Dict[str, Optional[torch.Tensor]] = {}
+    for key, (shape, dt) in shapes.items():
+        t = None if out is None else out.get(key)
+        if key == "x_perm" and x is None:
+            r[key] = None
+        elif t is None:
+            r[key] = torch.empty(*shape, dtype=dt, device=dev)
+        else:
+            _req(t, key, shape, dt)
+            r[key] = t
+    with torch.cuda.device(dev):
+        _check(lib().moe_dispatch_noalloc(ctypes.byref(p.c()), _ptr(selected), _ptr(x), _ptr(r["counts"]),
+                                          _ptr(r["offsets"]), _ptr(r["sorted_pairs"]), _ptr(r["pair_pos"]),
+                                          _ptr(r["x_perm"]), _stream(dev)))
     return r
 
 

@@ -105,8 +105,9 @@ moe_status do_route(const moe_problem& p, const Layout& L, const void* x, const 
 moe_status do_dispatch(const moe_problem& p, const Layout& L, const int64_t* selected, const void* x,
                        int32_t* counts, int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos, void* x_perm,
                        void* ws, cudaStream_t s) {
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
   MOE_CUDA(launch_dispatch(p.dtype, selected, x, p.T, p.H, p.E, p.k, at<int32_t>(ws, L.local), counts, offsets,
-                           sorted_pairs, pair_pos, x_perm, at<int32_t>(ws, L.header), s));
+                           sorted_pairs, pair_pos, x_perm, &hdr->error_bits, &hdr->dispatch_ticket, s));
   return MOE_OK;
 }
 
@@ -209,10 +210,17 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   };
   const bool has_shared = p->shared != MOE_SHARED_NONE;
   const bool gated = p->shared == MOE_SHARED_SIGMOID_GATED;
-  // A second stream only pays when the shared expert is too small to fill
-  // the GPU (few row tiles, as in decode): a large shared GEMM would take
-  // every SM and stall the routed chain instead of overlapping it.
-  const bool two_streams = has_shared && aux != nullptr && aux != s && shared_overlaps(*p);
+  // Schedules with an aux stream:
+  //  - a small shared expert (too few row tiles to fill the GPU, as in
+  //    decode) runs on `aux` beside the whole routed path, joined before the
+  //    combine; its sigmoid gate comes from its own small kernel;
+  //  - a large one occupies every SM while it runs, so it cannot overlap the
+  //    routed GEMMs; it runs on `aux` after the route (whose top-k kernel
+  //    already computed the gate) beside the dispatch kernels, which fit next
+  //    to its persistent CTAs, and `s` waits for it before the routed gate_up.
+  const bool use_aux = has_shared && aux != nullptr && aux != s;
+  const bool small_shared = use_aux && shared_overlaps(*p);
+  const bool large_shared = use_aux && !small_shared;
   float* gamma = at<float>(ws, L.gamma);
   int32_t* counts = at<int32_t>(ws, L.counts);
   int32_t* offsets = at<int32_t>(ws, L.offsets);
@@ -223,11 +231,13 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   void* shared_out = has_shared ? at<void>(ws, L.shared_out) : nullptr;
 
   EventPair evp;
-  if (two_streams) {
-    // The shared expert needs only x (and its own gate): run it on `aux`
-    // while the routed path runs on `s`; join before the combine.
+  if (use_aux) {
     MOE_CUDA(cudaEventCreateWithFlags(&evp.fork, cudaEventDisableTiming));
     MOE_CUDA(cudaEventCreateWithFlags(&evp.join, cudaEventDisableTiming));
+  }
+  if (small_shared) {
+    // The shared expert needs only x (and its own gate): run it on `aux`
+    // while the routed path runs on `s`; join before the combine.
     MOE_CUDA(cudaEventRecord(evp.fork, s));
     MOE_CUDA(cudaStreamWaitEvent(aux, evp.fork, 0));
     if (gated) MOE_CUDA(launch_shared_gate(p->dtype, x, w->shared_gate, p->T, p->H, gamma, aux));
@@ -236,18 +246,28 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   }
 
   MOE_TRY(mark(MOE_STAGE_ROUTE));
-  MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, (gated && !two_streams) ? w->shared_gate : nullptr, weights,
+  MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, (gated && !small_shared) ? w->shared_gate : nullptr, weights,
                    selected, gamma, ws, s));
+  if (large_shared) {
+    MOE_CUDA(cudaEventRecord(evp.fork, s));
+    MOE_CUDA(cudaStreamWaitEvent(aux, evp.fork, 0));
+    MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, gated ? gamma : nullptr, shared_out, ws, aux));
+    MOE_CUDA(cudaEventRecord(evp.join, aux));
+  }
+  // With a large shared expert on `aux`, the dispatch stage's interval ends
+  // when both the dispatch and the shared expert are done, and the shared
+  // stage is empty.
   MOE_TRY(mark(MOE_STAGE_DISPATCH));
   MOE_TRY(do_dispatch(*p, L, selected, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws, s));
+  if (large_shared) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
   MOE_TRY(mark(MOE_STAGE_GATE_UP));
   MOE_TRY(do_grouped_gate_up(*p, L, x_perm, offsets, w->gate_up, ws, s));
   MOE_TRY(mark(MOE_STAGE_DOWN));
   MOE_TRY(do_grouped_down(*p, L, offsets, w->down, weights, sorted_pairs, y_perm, ws, s));
   MOE_TRY(mark(MOE_STAGE_SHARED));
-  if (has_shared && !two_streams)
+  if (has_shared && !use_aux)
     MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, gated ? gamma : nullptr, shared_out, ws, s));
-  if (two_streams) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
+  if (small_shared) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
   MOE_TRY(mark(MOE_STAGE_COMBINE));
   MOE_CUDA(launch_combine(p->dtype, (const float*)y_perm, pair_pos, (const float*)shared_out, out, p->T, p->H,
                           p->k, s));
@@ -392,7 +412,7 @@ MOE_API moe_status moe_launches_per_forward(const moe_problem* p, int32_t two_st
     *n = 0;
     return MOE_OK;
   }
-  int count = 2 + 4 + 1;  // router logits + top-k; histogram, scan, permute, gather; combine
+  int count = 2 + 2 + 1;  // router logits + top-k; histogram + scan, permute + gather; combine
   if (p->dtype == MOE_DTYPE_BF16) {
     Segments routed{reinterpret_cast<const int32_t*>(16), (int32_t)p->E, 0, p->T * p->k};
     count += 2 * tc_gemm_launches(routed);
@@ -403,7 +423,8 @@ MOE_API moe_status moe_launches_per_forward(const moe_problem* p, int32_t two_st
   } else {
     count += 2 + (p->shared != MOE_SHARED_NONE ? 2 : 0);
   }
-  if (two_streams && p->shared == MOE_SHARED_SIGMOID_GATED && shared_overlaps(*p)) count += 1;  // gate kernel
+  // the small shared expert's own gate kernel
+  if (two_streams && p->shared == MOE_SHARED_SIGMOID_GATED && shared_overlaps(*p)) count += 1;
   *n = count;
   return MOE_OK;
 }

@@ -709,7 +709,8 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
   // Sorted segments of the choice, each row's token and weight.
   BW_CUDA(launch_dispatch(MOE_DTYPE_F32, selected, nullptr, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
-                          at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, nullptr, err, s));
+                          at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, nullptr, err,
+                          &at<WsHeader>(ws, b.header)->dispatch_ticket, s));
   bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, wts, E, k, tok, scale);
   // Routed experts: recompute [g | u]; dhu and [dg | du]; dx rows; dw.
   BW_CUDA(run_rows<true, EPI_STORE>(

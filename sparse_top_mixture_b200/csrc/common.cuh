@@ -12,9 +12,11 @@ constexpr int kMaxExperts = 256;  // warp top-k keeps E/32 <= 8 keys per lane
 // Workspace header: the first 256 bytes of every workspace.
 struct WsHeader {
   int32_t error_bits;
-  int32_t wait_site;  // which pipeline wait gave up, when one did
-  int32_t pad[62];
+  int32_t wait_site;         // which pipeline wait gave up, when one did
+  uint32_t dispatch_ticket;  // CTAs of the running dispatch histogram that are done (0 between calls)
+  int32_t pad[61];
 };
+static_assert(sizeof(WsHeader) == 256, "the workspace header is 256 bytes");
 
 __host__ __device__ constexpr inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }

@@ -7,20 +7,22 @@
 // arg_sort grouping, then index_select of each expert's tokens).
 //
 // The argsort is done as a counting sort, which is stable by construction and
-// needs no comparison passes:
-//   1. each block counts the experts of its own pairs (block-local histogram);
-//   2. one block turns the [blocks x E] counts into segment offsets and the
-//      base position of every (block, expert) run;
-//   3. each block ranks its pairs inside each expert run in pair order (warp
-//      match + prefix counts across warps) and writes the permutation and its
-//      inverse;
-//   4. the gather reads each token row once and writes it to its k segment
-//      slots with 16-byte vector loads and stores; its work units are
-//      (token, 4 KB column chunk) so that a 16-token decode batch still spreads
-//      over many SMs.
-// Every block handles whole tokens and at most 256 pairs, so the ranking is a
-// single pass. Counts are order-independent and positions are a pure function
-// of the pair order: the result is deterministic.
+// needs no comparison passes. Two launches:
+//   1. hist_scan_kernel: each 256-pair dispatch block counts the experts of
+//      its own pairs (four dispatch blocks per 1024-thread CTA); the last CTA
+//      to finish (an atomic ticket, no waiting on other CTAs) turns the
+//      [blocks x E] counts into segment offsets and the base position of
+//      every (block, expert) run, and resets the ticket;
+//   2. permute_gather_kernel: each dispatch block ranks its pairs inside each
+//      expert run in pair order (warp match + prefix counts across warps),
+//      writes the permutation and its inverse, and copies its tokens' rows to
+//      their k segment slots with 16-byte vector loads and stores. Several
+//      CTAs share one dispatch block, each copying a slice of the columns (the
+//      ranking, a few hundred integer operations, is repeated by each), so
+//      that the copy spreads over the whole GPU even for a 16-token batch.
+// Every dispatch block handles whole tokens and at most 256 pairs, so the
+// ranking is a single pass. Counts are order-independent and positions are a
+// pure function of the pair order: the result is deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,35 +30,18 @@ namespace stm {
 
 namespace {
 
-constexpr int DTHREADS = 256;
+constexpr int DTHREADS = 256;     // pairs per dispatch block
+constexpr int HIST_SUB = 4;       // dispatch blocks per histogram CTA
+constexpr int SCAN_THREADS = DTHREADS * HIST_SUB;
 
-__global__ void __launch_bounds__(DTHREADS) hist_kernel(const int64_t* __restrict__ sel, int64_t P, int k, int E,
-                                                        int tok_per_blk, int32_t* __restrict__ local,
-                                                        int32_t* err) {
-  __shared__ int cnt[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += DTHREADS) cnt[e] = 0;
-  __syncthreads();
-  const int64_t q0 = (int64_t)blockIdx.x * tok_per_blk * k;
-  const int64_t q1 = min(P, q0 + (int64_t)tok_per_blk * k);
-  for (int64_t q = q0 + threadIdx.x; q < q1; q += DTHREADS) {
-    const int64_t e = sel[q];
-    if (e < 0 || e >= E) raise_error(err, 1);
-    else atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += DTHREADS) local[(int64_t)blockIdx.x * E + e] = cnt[e];
-}
-
-// One block: counts, offsets, and (in place) per-(block, expert) base positions.
-// Each expert's column of the [blocks x E] count matrix is split among `tpe`
+// Exclusive scan of the [nblk x E] per-block counts by one CTA of
+// SCAN_THREADS threads: counts, offsets, and (in place) the base position of
+// every (block, expert) run. Each expert's column is split among `tpe`
 // threads of one warp (tpe = 4..32), which read their ranges with independent
 // loads, combine through a segmented warp scan, and write the running bases.
-constexpr int SCAN_THREADS = 1024;
-
-__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict__ local, int nblk, int E,
-                                                            int tpe, int32_t* __restrict__ counts,
-                                                            int32_t* __restrict__ offsets) {
-  __shared__ int tot[kMaxExperts];
+// The counts were written by other CTAs of the same grid: read through L2.
+__device__ void block_scan_counts(int32_t* __restrict__ local, int nblk, int E, int tpe,
+                                  int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* tot) {
   const int tid = threadIdx.x;
   const int e = tid / tpe, part = tid % tpe;
   const bool active = e < E;
@@ -67,7 +52,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
     for (int b = b0; b < b1; b += 8) {
       int v[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? local[(int64_t)(b + i) * E + e] : 0;
+      for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) sum += v[i];
     }
@@ -113,7 +98,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
   for (int b = b0; b < b1; b += 8) {
     int v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? local[(int64_t)(b + i) * E + e] : 0;
+    for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (b + i < b1) local[(int64_t)(b + i) * E + e] = run;
@@ -122,12 +107,55 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int32_t* __restrict_
   }
 }
 
-__global__ void __launch_bounds__(DTHREADS) permute_kernel(const int64_t* __restrict__ sel, int64_t P, int k,
-                                                           int E, int tok_per_blk,
-                                                           const int32_t* __restrict__ bases,
-                                                           int32_t* __restrict__ sorted_pairs,
-                                                           int32_t* __restrict__ pair_pos) {
+__global__ void __launch_bounds__(SCAN_THREADS) hist_scan_kernel(const int64_t* __restrict__ sel, int64_t P, int k,
+                                                                 int E, int tok_per_blk, int nblk, int tpe,
+                                                                 int32_t* __restrict__ local,
+                                                                 int32_t* __restrict__ counts,
+                                                                 int32_t* __restrict__ offsets,
+                                                                 uint32_t* __restrict__ ticket, int32_t* err) {
+  __shared__ int cnt[HIST_SUB][kMaxExperts];
+  __shared__ int last;
+  const int sub = threadIdx.x / DTHREADS, t = threadIdx.x % DTHREADS;
+  for (int e = t; e < E; e += DTHREADS) cnt[sub][e] = 0;
+  __syncthreads();
+  const int b = blockIdx.x * HIST_SUB + sub;
+  if (b < nblk) {
+    const int64_t q0 = (int64_t)b * tok_per_blk * k;
+    const int64_t q1 = min(P, q0 + (int64_t)tok_per_blk * k);
+    for (int64_t q = q0 + t; q < q1; q += DTHREADS) {
+      const int64_t e = sel[q];
+      if (e < 0 || e >= E) raise_error(err, 1);
+      else atomicAdd(&cnt[sub][e], 1);
+    }
+  }
+  __syncthreads();
+  if (b < nblk)
+    for (int e = t; e < E; e += DTHREADS) local[(int64_t)b * E + e] = cnt[sub][e];
+  // Publish this CTA's counts, then take a ticket: the CTA that draws the
+  // last one sees every other CTA's counts and does the scan.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  block_scan_counts(local, nblk, E, tpe, counts, offsets, &cnt[0][0]);
+  if (threadIdx.x == 0) *ticket = 0u;  // ready for the next dispatch on this workspace
+}
+
+// Rank the block's pairs, write sorted_pairs / pair_pos (column slice 0
+// only), and copy column slice blockIdx.y of each token row to the slots of
+// its k pairs: x_perm[pair_pos[t*k + j]] = x[t].
+template <typename T>
+__global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t* __restrict__ sel, int64_t P, int k,
+                                                                  int E, int tok_per_blk,
+                                                                  const int32_t* __restrict__ bases,
+                                                                  int32_t* __restrict__ sorted_pairs,
+                                                                  int32_t* __restrict__ pair_pos,
+                                                                  const T* __restrict__ x, T* __restrict__ x_perm,
+                                                                  int64_t Tn, int H, int vec_per_slice) {
   __shared__ int wcnt[DTHREADS / 32][kMaxExperts];
+  __shared__ int s_pos[DTHREADS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < (DTHREADS / 32) * kMaxExperts; i += DTHREADS) (&wcnt[0][0])[i] = 0;
   __syncthreads();
@@ -156,42 +184,30 @@ __global__ void __launch_bounds__(DTHREADS) permute_kernel(const int64_t* __rest
   }
   __syncthreads();
   int pos = -1;
-  if (e >= 0) {
-    pos = wcnt[warp][e] + rank;
-    sorted_pairs[pos] = (int32_t)q;
+  if (e >= 0) pos = wcnt[warp][e] + rank;
+  s_pos[tid] = pos;
+  if (blockIdx.y == 0) {
+    if (e >= 0) sorted_pairs[pos] = (int32_t)q;
+    if (active) pair_pos[q] = pos;
   }
-  if (active) pair_pos[q] = pos;
-}
-
-// x_perm[pair_pos[t*k + j]] = x[t] for every token t and slot j.
-constexpr int GCHUNK = 256;  // 16-byte vectors per work unit
-
-template <typename T>
-__global__ void __launch_bounds__(DTHREADS) gather_kernel(const T* __restrict__ x, const int32_t* __restrict__ pair_pos,
-                                                          T* __restrict__ x_perm, int64_t Tn, int H, int k) {
+  if (x_perm == nullptr) return;
+  __syncthreads();
+  // Copy: work items (token of the block, 16-byte vector of this slice),
+  // consecutive threads on consecutive vectors of one row.
   constexpr int V = Elem<T>::kPerVec;
   const int nvec = H / V;
-  const int nchunk = (nvec + GCHUNK - 1) / GCHUNK;
-  const int64_t units = Tn * nchunk;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = ((int64_t)blockIdx.x * DTHREADS + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * DTHREADS) >> 5;
-  for (int64_t u = warp0; u < units; u += nwarps) {
-    const int64_t t = u / nchunk;
-    const int c0 = (int)(u - t * nchunk) * GCHUNK;
-    const int c1 = min(nvec, c0 + GCHUNK);
-    int pos[8];
-    const int kk = min(k, 8);
-    for (int j = 0; j < kk; ++j) pos[j] = pair_pos[t * k + j];
-    const uint4* src = reinterpret_cast<const uint4*>(x + t * (int64_t)H);
-    for (int v = c0 + lane; v < c1; v += 32) {
-      const uint4 val = src[v];
-      for (int j = 0; j < kk; ++j)
-        if (pos[j] >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)pos[j] * H)[v] = val;
-      for (int j = 8; j < k; ++j) {
-        const int p = pair_pos[t * k + j];
-        if (p >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)p * H)[v] = val;
-      }
+  const int v0 = blockIdx.y * vec_per_slice;
+  const int nv = min(nvec, v0 + vec_per_slice) - v0;
+  if (nv <= 0) return;
+  const int64_t t0 = (int64_t)blockIdx.x * tok_per_blk;
+  const int ntok = (int)min((int64_t)tok_per_blk, Tn - t0);
+  const int items = ntok * nv;
+  for (int it = tid; it < items; it += DTHREADS) {
+    const int i = it / nv, v = v0 + (it - i * nv);
+    const uint4 val = reinterpret_cast<const uint4*>(x + (t0 + i) * (int64_t)H)[v];
+    for (int j = 0; j < k; ++j) {
+      const int p = s_pos[i * k + j];
+      if (p >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)p * H)[v] = val;
     }
   }
 }
@@ -245,26 +261,32 @@ int64_t dispatch_num_blocks(int64_t T, int64_t k) { return ceil_div(T, dispatch_
 
 cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
                             int64_t k, int32_t* local, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
-                            int32_t* pair_pos, void* x_perm, int32_t* err, cudaStream_t s) {
+                            int32_t* pair_pos, void* x_perm, int32_t* err, uint32_t* ticket, cudaStream_t s) {
   const int tpb = (int)dispatch_tokens_per_block(k);
   const int nblk = (int)dispatch_num_blocks(T, k);
   const int64_t P = T * k;
-  hist_kernel<<<nblk, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, err);
   int ep = 1;
   while (ep < E) ep <<= 1;
   const int tpe = std::min(32, SCAN_THREADS / ep);
-  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(local, nblk, (int)E, tpe, counts, offsets);
-  permute_kernel<<<nblk, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos);
-  if (x_perm != nullptr) {
-    const int V = dtype == 0 ? 4 : 8;
-    const int64_t units = T * ceil_div(H / V, GCHUNK);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, DTHREADS / 32), 148 * 16));
-    if (dtype == 0)
-      gather_kernel<float><<<grid, DTHREADS, 0, s>>>((const float*)x, pair_pos, (float*)x_perm, T, (int)H, (int)k);
-    else
-      gather_kernel<__nv_bfloat16><<<grid, DTHREADS, 0, s>>>((const __nv_bfloat16*)x, pair_pos,
-                                                             (__nv_bfloat16*)x_perm, T, (int)H, (int)k);
-  }
+  hist_scan_kernel<<<(unsigned)ceil_div(nblk, HIST_SUB), SCAN_THREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, nblk,
+                                                                             tpe, local, counts, offsets, ticket, err);
+  // Column slices per dispatch block: enough CTAs for about eight per SM,
+  // each slice at least 32 vectors (512 bytes) of a row.
+  const int V = dtype == 0 ? 4 : 8;
+  const int64_t nvec = H / V;
+  int slices = 1;
+  if (x_perm != nullptr)
+    slices = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(148 * 8, nblk), nvec / 32));
+  const int vps = (int)ceil_div(nvec, slices);
+  slices = (int)ceil_div(nvec, vps);
+  const dim3 grid((unsigned)nblk, (unsigned)slices);
+  if (dtype == 0)
+    permute_gather_kernel<float><<<grid, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, sorted_pairs,
+                                                           pair_pos, (const float*)x, (float*)x_perm, T, (int)H, vps);
+  else
+    permute_gather_kernel<__nv_bfloat16><<<grid, DTHREADS, 0, s>>>(
+        selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos, (const __nv_bfloat16*)x,
+        (__nv_bfloat16*)x_perm, T, (int)H, vps);
   return cudaGetLastError();
 }
 

@@ -28,25 +28,33 @@ namespace {
 constexpr int64_t kStaticCountEntries = int64_t(1) << 18;
 
 static __device__ __align__(256) int32_t g_dispatch_counts[kStaticCountEntries];
+// The histogram's completion ticket (CTAs done so far; zero between calls).
+static __device__ __align__(256) uint32_t g_dispatch_ticket;
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_setup_once[kMaxDevices];
+std::mutex g_setup_mutex;
 int32_t* g_counts_addr[kMaxDevices] = {};
-cudaError_t g_setup_err[kMaxDevices] = {};
+uint32_t* g_ticket_addr[kMaxDevices] = {};
 
-// Device address of the static array on the current device. In host code
-// the array's name only stands in for it, so the address is looked up once
-// per device, with that device current.
-moe_status static_counts(int32_t** out) {
+// Device addresses of the static arrays on the current device. In host code
+// their names only stand in for them, so the addresses are looked up per
+// device, with that device current, and kept once a lookup has succeeded (a
+// failed lookup, e.g. one made while a graph is being captured, is retried by
+// the next call).
+moe_status static_scratch(int32_t** counts, uint32_t** ticket) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  std::call_once(g_setup_once[dev], [dev] {
-    void* addr = nullptr;
-    g_setup_err[dev] = cudaGetSymbolAddress(&addr, g_dispatch_counts);
-    g_counts_addr[dev] = static_cast<int32_t*>(addr);
-  });
-  if (g_setup_err[dev] != cudaSuccess || g_counts_addr[dev] == nullptr) return MOE_ERR_CUDA;
-  *out = g_counts_addr[dev];
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_counts_addr[dev] == nullptr || g_ticket_addr[dev] == nullptr) {
+    void* a = nullptr;
+    void* b = nullptr;
+    if (cudaGetSymbolAddress(&a, g_dispatch_counts) != cudaSuccess || a == nullptr) return MOE_ERR_CUDA;
+    if (cudaGetSymbolAddress(&b, g_dispatch_ticket) != cudaSuccess || b == nullptr) return MOE_ERR_CUDA;
+    g_counts_addr[dev] = static_cast<int32_t*>(a);
+    g_ticket_addr[dev] = static_cast<uint32_t*>(b);
+  }
+  *counts = g_counts_addr[dev];
+  *ticket = g_ticket_addr[dev];
   return MOE_OK;
 }
 
@@ -77,13 +85,17 @@ MOE_API moe_status moe_dispatch_noalloc(const moe_problem* p, const int64_t* sel
   if ((x == nullptr) != (x_perm == nullptr) || !aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARGUMENT;
   if (dispatch_num_blocks(p->T, p->k) * p->E > kStaticCountEntries) return MOE_ERR_UNSUPPORTED;
   int32_t* scratch = nullptr;
-  const moe_status ss = static_counts(&scratch);
+  uint32_t* ticket = nullptr;
+  const moe_status ss = static_scratch(&scratch, &ticket);
   if (ss != MOE_OK) return ss;
   // Every count entry the scan reads is written by the histogram first, so
-  // nothing carried over from an earlier call is read. The error flag is not
-  // kept: a pair with an expert id outside [0, E) is skipped (pair_pos -1)
-  // exactly as in moe_dispatch, without a flag to read back.
+  // nothing carried over from an earlier call is read; the ticket must start
+  // at zero (each dispatch leaves it there; it is cleared here as well). The
+  // error flag is not kept: a pair with an expert id outside [0, E) is
+  // skipped (pair_pos -1) exactly as in moe_dispatch, without a flag to read
+  // back.
+  if (cudaMemsetAsync(ticket, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   const cudaError_t e = launch_dispatch(p->dtype, selected_experts, x, p->T, p->H, p->E, p->k, scratch, counts,
-                                        offsets, sorted_pairs, pair_pos, x_perm, nullptr, s);
+                                        offsets, sorted_pairs, pair_pos, x_perm, nullptr, ticket, s);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -86,7 +86,7 @@ int64_t dispatch_tokens_per_block(int64_t k);
 int64_t dispatch_num_blocks(int64_t T, int64_t k);
 cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
                             int64_t k, int32_t* local, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
-                            int32_t* pair_pos, void* x_perm, int32_t* err, cudaStream_t s);
+                            int32_t* pair_pos, void* x_perm, int32_t* err, uint32_t* ticket, cudaStream_t s);
 
 // ---- combine ----------------------------------------------------------
 // y_perm [T*k, H] and shared_out [T, H] are fp32 for every problem dtype.

@@ -6,12 +6,26 @@ Tolerances:
 * routing weights and shared gate values (fp32): max-abs <= 1e-5;
 * indices, counts, offsets and permutations: bit-exact.
 
-Near ties. The CUDA router accumulates logits in fp32 (error ~1e-6 against
-the oracle's fp64). Where a token's k-th and (k+1)-th selection keys are
-closer than TAU * max(1, max|key|), more than one top-k set is correct. Such a
-token passes if the CUDA choice is one of the correct ones (every chosen key
->= every unchosen key - tau, slot order descending within tau); the reference
-output is then recomputed by the oracle from the CUDA choice.
+Near ties. The CUDA router accumulates logits in fp32 while the oracle works
+in fp64. Each bf16 x bf16 product is exact in fp32, so the logit error is the
+rounding of an H-term fp32 sum (plus at most 16 split partials added in
+order): every addition rounds by at most u = 2^-24 of the running sum, and
+those roundings are independent in sign, so the error behaves like a random
+walk of sqrt(H) steps of size u * |running sum|. With H <= 7168 and running
+sums of a few units (the logits here are ~N(0,1), |l| <= ~5), that is about
+85 * 6e-8 * 2 ~ 1e-5 at the very worst token of a batch and ~1e-6 typically;
+scores and keys add a few fp32 ulps, and adding a logit bias rounds once more
+at the key's own magnitude. Hence the tie margin of the survey's reading,
+TAU * max(1, |key|) with TAU = 1e-5, where |key| is the larger magnitude of
+the token's k-th and (k+1)-th oracle keys (the keys at the decision, not the
+token's largest key: a dead expert's -1e4 logit bias must not widen the
+margin). On a token whose oracle margin between those two keys is below it,
+more than one top-k set is correct: the CUDA choice passes if it is one of
+them (every chosen key >= every unchosen key - tau, slot order descending
+within tau), and the reference output is recomputed from the CUDA choice.
+Every test asserts how many tokens took this escape (EXPECTED_NEAR_TIES; 0
+unless listed), so a router that mis-ordered keys inside the margin would
+change the count and fail.
 """
 
 from __future__ import annotations
@@ -24,7 +38,18 @@ import torch
 import oracle
 import workloads
 
-TAU = 5e-5
+TAU = 1e-5
+
+# Tokens whose CUDA top-k differs from the oracle's inside the tie margin, at
+# the fixed seeds (problem name -> count). Every other problem: 0.
+# The Zipf-skewed problem at full size has 26 tokens whose oracle margin is
+# below 1e-5 (the smallest 1.1e-7); the CUDA router's fp32 logits order four
+# of them the other way.
+EXPECTED_NEAR_TIES = {"deepseek_v2_lite_zipf": 4}
+
+
+def expected_near_ties(name: str) -> int:
+    return EXPECTED_NEAR_TIES.get(name, 0)
 
 
 class LazyExperts:
@@ -72,6 +97,13 @@ def ranking_keys(cfg, r) -> np.ndarray:
     return r["keys"] if cfg.bias_mode == "select" else r["logits"]
 
 
+def tie_margin(K_t: np.ndarray, k: int) -> float:
+    """TAU * max(1, |k-th key|, |(k+1)-th key|) for one token's oracle keys."""
+    s = np.sort(K_t)[::-1]
+    mag = abs(float(s[k - 1])) if k >= len(s) else max(abs(float(s[k - 1])), abs(float(s[k])))
+    return TAU * max(1.0, mag)
+
+
 def check_selection(cfg, r, gpu_sel: np.ndarray) -> int:
     """Assert the CUDA top-k is exact except at near ties, where it must be a
     correct alternative. Returns the number of tokens that differ."""
@@ -83,7 +115,7 @@ def check_selection(cfg, r, gpu_sel: np.ndarray) -> int:
         g = gpu_sel[t]
         assert len(set(g.tolist())) == cfg.k, f"token {t}: repeated expert {g}"
         assert g.min() >= 0 and g.max() < cfg.E
-        tau = TAU * max(1.0, float(np.abs(K[t]).max()))
+        tau = tie_margin(K[t], cfg.k)
         chosen = K[t, g]
         mask = np.ones(cfg.E, bool)
         mask[g] = False

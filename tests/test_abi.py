@@ -80,15 +80,15 @@ def test_gemm_path(L):
 
 
 def test_launch_counts(L):
-    # route 2, dispatch 4, combine 1, plus the expert GEMMs
-    assert stm.launches_per_forward(_p()) == 7 + 2
-    assert stm.launches_per_forward(_p(T=8192, E=64, k=6)) == 7 + 2
-    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256)) == 7 + 2 + 2
-    assert stm.launches_per_forward(_p(dtype="f32", shared="plain", I_shared=256)) == 7 + 4
+    # route 2 (logits, top-k), dispatch 2 (histogram + scan, permute + gather), combine 1, plus the expert GEMMs
+    assert stm.launches_per_forward(_p()) == 5 + 2
+    assert stm.launches_per_forward(_p(T=8192, E=64, k=6)) == 5 + 2
+    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256)) == 5 + 2 + 2
+    assert stm.launches_per_forward(_p(dtype="f32", shared="plain", I_shared=256)) == 5 + 4
     assert stm.launches_per_forward(_p(T=0)) == 0
     gated = _p(shared="sigmoid_gated", I_shared=256)  # small shared expert: runs on the aux stream
     assert stm.launches_per_forward(gated, two_streams=True) == stm.launches_per_forward(gated) + 1
-    big = _p(T=8192, shared="sigmoid_gated", I_shared=2048)  # fills the GPU: stays on the main stream
+    big = _p(T=8192, shared="sigmoid_gated", I_shared=2048)  # fills the GPU: beside the dispatch, no gate kernel
     assert stm.launches_per_forward(big, two_streams=True) == stm.launches_per_forward(big)
 
 

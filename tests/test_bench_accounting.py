@@ -41,8 +41,14 @@ def test_forward_accounting(name):
         _gemm(P, 2 * c.I, c.H) + _gemm(P, c.H, c.I) + (_gemm(c.T, 2 * c.I_shared, c.H) + _gemm(c.T, c.H, c.I_shared)),
         rel=1e-12)
     assert fb["router_flops"] == _gemm(c.T, c.E, c.H)
-    # gate_up kernel: the active experts' gate_up weights once, x_perm read once, h written once
-    assert fb["gate_up_bytes"] == (active * 2 * c.I * c.H + P * c.H + P * c.I) * es
+    # gate_up kernel: the active experts' gate_up weights once and x read once (x_perm and h are the
+    # implementation's intermediates, not algorithmic traffic); down: its weights once and out written once
+    assert fb["gate_up_bytes"] == (active * 2 * c.I * c.H + c.T * c.H) * es
+    assert fb["down_flops"] == _gemm(P, c.H, c.I)
+    assert fb["down_bytes"] == (active * c.H * c.I + c.T * c.H) * es
+    # whole forward: every active weight once, the router and shared weights, x in and out back
+    shared_w = 3 * c.I_shared * c.H if c.shared != "none" else 0
+    assert fb["min_bytes"] == (active * 3 * c.I * c.H + c.E * c.H + shared_w + 2 * c.T * c.H) * es
 
 
 def test_host_memory_probe_is_positive():
@@ -76,3 +82,27 @@ def test_reference_arm_prints_one_contract_line():
     assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2 and line["warmup"] == 3
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["config"]["workload"] == "tiny_fp32"
+
+
+def test_roofline_entry_by_hand():
+    """The fraction is algorithmic work / time / peak, bounded by the larger of
+    the tensor and HBM times; a reader can redo it from the printed numbers."""
+    pk = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured"}
+    e = bench.roofline_entry(206.16e9, 822e6, 0.2171, pk, "bf16")
+    assert e["bound"] == "tensor"
+    assert e["achieved"] == pytest.approx(206.16e9 / 0.2171e-3 / 1e12)
+    assert e["frac"] == pytest.approx(206.16e9 / 0.2171e-3 / 1e12 / 1600.0)
+    assert e["t_roof_ms"] == pytest.approx(206.16e9 / 1600e12 * 1e3)
+    h = bench.roofline_entry(12.7e9, 9.08e9, 1.45, pk, "bf16")
+    assert h["bound"] == "hbm" and h["frac"] == pytest.approx(9.08e9 / 1.45e-3 / 1e9 / 6500.0)
+    f = bench.roofline_entry(1e12, 1e6, 100.0, pk, "f32", mhz=1965.0)
+    assert f["bound"] == "alu" and f["peak"] == pytest.approx(148 * 128 * 2 * 1965e6 / 1e12)
+
+
+def test_config_is_the_same_for_both_arms():
+    """The workload dict carries no arm-specific key: the reference arm's
+    config equals ours for every named problem."""
+    for c in CONFIGS.values():
+        d = bench.config_dict(c)
+        assert d == bench.config_dict(c) and "parallelism" not in d
+        assert d["workload"] == c.name and "l2" in d

@@ -41,6 +41,10 @@ EDGE = {
     "pairs_tails": CONFIGS["qwen3_30b_a3b"].replace(name="pairs_tails", T=2300, H=320, E=8, k=2, I=200),
     "pairs_shared_skew": CONFIGS["deepseek_v2_lite_zipf"].replace(name="pairs_zipf", T=4200, H=256, I=136,
                                                                   I_shared=272),
+    # a sigmoid-gated shared expert too large to overlap the routed GEMMs
+    # (8 x 16 row x column tiles): it runs beside the dispatch
+    "large_shared_gated": CONFIGS["decode_weight_streaming"].replace(name="large_gated", T=1000, H=512, E=32, k=4,
+                                                                     I=128, I_shared=2048),
 }
 
 
@@ -74,6 +78,7 @@ def test_forward_parity(name):
     cpu, dev = _inputs(cfg)
     moe, out, o, ntie, stats = _forward_and_check(cfg, cpu, dev)
     print(f"{name}: near-tie tokens {ntie}, {stats}")
+    assert ntie == gc.expected_near_ties(cfg.name), f"{cfg.name}: {ntie} tokens took the near-tie escape"
     assert stm.gemm_path(moe.p) == (1 if cfg.dtype == "bf16" else 0)
 
 
@@ -81,7 +86,8 @@ def test_forward_parity(name):
 def test_forward_edge_cases(name):
     cfg = EDGE[name]
     cpu, dev = _inputs(cfg)
-    _forward_and_check(cfg, cpu, dev)
+    _, _, _, ntie, _ = _forward_and_check(cfg, cpu, dev)
+    assert ntie == gc.expected_near_ties(cfg.name), f"{cfg.name}: {ntie} tokens took the near-tie escape"
 
 
 def test_both_tensor_core_variants_are_exercised():
@@ -116,7 +122,7 @@ def test_staged_calls_match_forward(name):
     # stage-level parity
     gsel = sel.cpu().numpy()
     r = gc.oracle_route(cfg, cpu)
-    gc.check_selection(cfg, r, gsel)
+    assert gc.check_selection(cfg, r, gsel) == gc.expected_near_ties(cfg.name)
     dd = gc.assert_dispatch_exact(d, gsel, cfg.E)
     xs = d["x_perm"].cpu()
     assert torch.equal(xs, cpu["x"][torch.from_numpy(dd["sorted_pairs"] // cfg.k)])
@@ -293,13 +299,18 @@ def test_repeat_runs_are_bit_identical():
     assert all(torch.equal(u, v) for u, v in zip(a, b))
 
 
-@pytest.mark.parametrize("name", ["deepseek_v2_lite_zipf", "decode_weight_streaming", "dsv4_flash_ablation"])
+@pytest.mark.parametrize("name", ["deepseek_v2_lite_zipf", "decode_weight_streaming", "dsv4_flash_ablation",
+                                  "pairs_shared_skew", "large_shared_gated"])
 def test_two_stream_forward_matches_one_stream(name):
-    """The shared expert on a second stream (and its gate from its own kernel)
-    gives the same bits as the single-stream forward."""
-    cfg = SMALL[name]
+    """The shared expert on a second stream gives the same bits as the
+    single-stream forward: a small one beside the whole routed path (its gate
+    from its own kernel), a large one (more row x column tiles than half the
+    SMs) beside the dispatch only, joined before the routed GEMMs."""
+    cfg = EDGE.get(name) or SMALL[name]
     cpu, dev = _inputs(cfg)
     p = stm.Problem.from_config(cfg)
+    large = (cfg.T + 127) // 128 * ((cfg.I_shared + 127) // 128) > 74
+    assert large == (name in ("pairs_shared_skew", "large_shared_gated"))
     a = stm.SparseMoE(p, dev, overlap_shared=True)
     b = stm.SparseMoE(p, dev, overlap_shared=False)
     assert a.aux is not None and b.aux is None
@@ -329,8 +340,8 @@ def test_host_pipeline_matches_forward():
         assert torch.equal(oh, ref.cpu())
 
 
-@pytest.mark.parametrize("name,overlap", [("pairs_shared_skew", False), ("decode_weight_streaming", True),
-                                           ("pairs_tails", False)])
+@pytest.mark.parametrize("name,overlap", [("pairs_shared_skew", False), ("pairs_shared_skew", True),
+                                           ("decode_weight_streaming", True), ("pairs_tails", False)])
 def test_graph_replay_matches_eager_forward(name, overlap):
     """A forward captured as a CUDA graph (with the shared expert on its
     second stream where it overlaps) gives the eager forward's bits, and
@@ -418,10 +429,16 @@ def test_full_size_sampled(name):
     # dispatch of the whole batch, bit-exact
     d = stm.dispatch(p, sel, None)
     gc.assert_dispatch_exact(d, gsel, cfg.E)
-    # sampled tokens through the oracle
+    assert ntie == gc.expected_near_ties(name), f"{name}: {ntie} tokens took the near-tie escape"
+    # sampled tokens through the oracle: every token of the small problems,
+    # 128 (the first, the last and 126 drawn) of the large ones
     rng = np.random.RandomState(5)
-    n = min(cfg.T, 12)
-    rows = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, n, replace=False)]))
+    if cfg.T <= 256:
+        rows = np.arange(cfg.T)
+    else:
+        pick = rng.choice(np.arange(1, cfg.T - 1), 126, replace=False)
+        rows = np.unique(np.concatenate([[0, cfg.T - 1], pick]))
+        assert rows.size == 128
     x_rows = gc.np64(r_cpu["x"])[rows]
     inp = dict(r_cpu, gate_up=dev["gate_up"], down=dev["down"], shared_gate_up=dev["shared_gate_up"],
                shared_down=dev["shared_down"])

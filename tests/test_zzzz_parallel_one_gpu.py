@@ -54,7 +54,8 @@ def _child(name, port, q):
             out, rw, sel = layer(dev["x"])
             torch.cuda.synchronize()
             gsel = sel.cpu().numpy()
-            gc.check_selection(cfg, r, gsel)
+            ntie = gc.check_selection(cfg, r, gsel)
+            assert ntie == gc.expected_near_ties(cfg.name), f"{name} {label}: {ntie} near-tie tokens"
             o = gc.oracle_forward(cfg, cpu, selected=gsel)
             stats = gc.assert_close(out.cpu().double().numpy(), o["out"], cfg.dtype, f"{name} {label}")
             res[label] = (stats["rel_l2"], float((out.float() - ref_out.float()).abs().max()))
