@@ -357,48 +357,60 @@ def backward_cpu_baseline(cfg32, inp, dout, target_s: float = 8.0) -> dict:
                       f"(oracle.backward, its own top-k choice), {t:.1f} s"}
 
 
-def measure_backward(cfg, local: int, steps: int = 5, cpu: bool = False) -> dict:
-    """The fp32 backward on the bench workload's shapes, timed with CUDA events
-    on the current stream, against the FFMA peak at the sampled SM clock;
-    with ``cpu``, the backward oracle timed on the host beside it."""
+def measure_backward(cfg, local: int, steps: int = 5, cpu: bool = False, dtype: str = "bf16") -> dict:
+    """The backward on the given workload's shapes in ``dtype`` (bf16: the
+    tensor-core path, against the measured bf16 peak; f32: the SIMT path,
+    against the FFMA peak at the sampled SM clock), timed with CUDA events on
+    the current stream; with ``cpu``, the backward oracle timed on the host
+    beside it on the same inputs, widened to fp64."""
     import sparse_top_mixture_b200 as stm
-    cfg32 = cfg.replace(dtype="f32")
-    inp = workloads.generate(cfg32, "cuda")
-    p = stm.Problem.from_config(cfg32)
+    c = cfg.replace(dtype=dtype)
+    inp = workloads.generate(c, "cuda")
+    p = stm.Problem.from_config(c)
     moe = stm.SparseMoE(p, inp)
     out, _, sel = moe(inp["x"])
-    dout = torch.randn(out.shape, generator=torch.Generator("cuda").manual_seed(7), device="cuda")
+    dout = torch.randn(out.shape, generator=torch.Generator("cuda").manual_seed(7), device="cuda").to(out.dtype)
     ws = torch.zeros(stm.backward_workspace_size(p), dtype=torch.uint8, device="cuda")
-    for _ in range(3):
-        stm.backward(p, inp, inp["x"], dout, sel, ws=ws)
+    grads = stm.backward(p, inp, inp["x"], dout, sel, ws=ws)
+    for _ in range(2):
+        stm.backward(p, inp, inp["x"], dout, sel, ws=ws, out=grads)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         a.record(stream)
         for _ in range(steps):
-            stm.backward(p, inp, inp["x"], dout, sel, ws=ws)
+            stm.backward(p, inp, inp["x"], dout, sel, ws=ws, out=grads)
         b.record(stream)
         torch.cuda.synchronize()
     if stm.read_device_error(ws) != 0:
         raise RuntimeError("device error flag set during the backward")
     ms = a.elapsed_time(b) / steps
-    fl = backward_flops(cfg32)
-    c = clk.summary()
-    mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965
-    peak = NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    fl = backward_flops(c)
+    ck = clk.summary()
+    mhz = ck["sm_mhz"] or ck["sm_max_mhz"] or 1965
+    if dtype == "f32":
+        peak = ffma_peak_tflops(mhz)
+        src = f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)"
+        bound = "alu"
+    else:
+        pk = peaks()
+        peak = pk["bf16_tflops"]
+        src = pk["source"] + " bf16 (burst)"
+        bound = "tensor"
     achieved = fl / (ms / 1e3) / 1e12
-    res = {"workload": f"{cfg.name} shapes in fp32 (T={cfg.T}, H={cfg.H}, E={cfg.E}, k={cfg.k}, I={cfg.I}, "
-                       f"I_shared={cfg.I_shared})",
-           "ms": ms, "tokens_per_s": cfg.T / (ms / 1e3), "steps": steps, "flops": fl, "bound": "alu",
+    res = {"workload": f"{cfg.name} shapes in {dtype} (T={c.T}, H={c.H}, E={c.E}, k={c.k}, I={c.I}, "
+                       f"I_shared={c.I_shared})",
+           "dtype": dtype, "ms": ms, "tokens_per_s": c.T / (ms / 1e3), "steps": steps, "flops": fl, "bound": bound,
            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-           "peak_source": f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)",
-           "clocks": c}
+           "peak_source": src, "clocks": ck}
     if cpu:
         try:
-            res["cpu_baseline"] = backward_cpu_baseline(cfg32, inp, dout)
+            res["cpu_baseline"] = backward_cpu_baseline(cfg.replace(dtype="f32"), inp, dout.float())
         except Exception as exc:  # the host baseline never costs the bench line
             res["cpu_baseline"] = {"value": None, "error": repr(exc)[:200]}
+    del moe, grads, ws, inp
+    torch.cuda.empty_cache()
     return res
 
 
@@ -769,7 +781,11 @@ def main():
             r.release()
         line["per_config"] = per
     if world == 1 and not args.no_backward:
-        line["backward"] = measure_backward(workloads.CONFIGS["qwen3_30b_a3b"], local, cpu=not args.no_cpu_baseline)
+        # the backward on the Qwen3-shaped problem: bf16 on the tensor cores
+        # (with the oracle's host baseline), and the fp32 SIMT path beside it
+        bw_cfg = workloads.CONFIGS["qwen3_30b_a3b"]
+        line["backward"] = measure_backward(bw_cfg, local, cpu=not args.no_cpu_baseline, dtype="bf16")
+        line["backward_f32"] = measure_backward(bw_cfg, local, dtype="f32")
     if cpu_inputs is not None:
         line["cpu_baseline"] = cpu_baseline(cfg, cpu_inputs)
     if rank == 0:

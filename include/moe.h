@@ -337,10 +337,13 @@ typedef struct moe_grads {
  *   int64 (normally the forward's). Routing weights, the per-expert
  *   activations and outputs are recomputed from x; nothing from the forward
  *   is needed besides the choice.
- *   fp32 problems only (MOE_ERR_UNSUPPORTED for bf16). Every gradient
- *   element is an fp32 sum in a fixed order (no atomics; the router weight
- *   gradient adds row-chunk partial sums in chunk order): results are
- *   deterministic. A pair with an expert id outside [0, E) contributes
+ *   fp32 problems run on SIMT kernels in fp32 throughout. bf16 problems
+ *   (x, dout and the weights bf16) run the expert GEMMs on the tensor cores
+ *   (bf16 operands, fp32 accumulation; [dg du], w*dout and h are rounded to
+ *   bf16 where they become operands) and the router in fp32; the gradients
+ *   are fp32 for both. Every gradient element is an fp32 sum in a fixed
+ *   order (no atomics; the router weight gradient adds row-chunk partial sums
+ *   in chunk order): results are deterministic. A pair with an expert id outside [0, E) contributes
  *   nothing and sets MOE_DEVERR_BAD_EXPERT_ID in the workspace header.
  *   Workspace: moe_backward_workspace_size bytes (its header as for
  *   moe_forward, zeroed by moe_workspace_init). Async on `stream`. */

@@ -352,17 +352,17 @@ def backward_workspace_size(p: Problem) -> int:
 
 def backward(p: Problem, weights: Dict[str, Optional[torch.Tensor]], x, dout, selected, ws=None, out=None
              ) -> Dict[str, Optional[torch.Tensor]]:
-    """Gradients of sum(dout * out) for the fp32 forward with the expert choice
+    """Gradients of sum(dout * out) for the forward with the expert choice
     held at ``selected`` [T,k] int64: dx, d_gate_w, d_bias (logit bias only),
     d_gate_up, d_down and, with a shared expert, d_shared_gate_up,
-    d_shared_down and d_shared_gate (gated only). ``out``: optional dict of
-    preallocated fp32 tensors for any of them (written, never accumulated
-    into). Async on the current stream."""
-    if p.dtype != "f32":
-        raise MoeError(2, "moe_backward supports fp32 problems only")
+    d_shared_down and d_shared_gate (gated only). x and dout are in the
+    problem's dtype (fp32: SIMT kernels; bf16: tensor-core GEMMs); every
+    gradient is fp32. ``out``: optional dict of preallocated fp32 tensors for
+    any of them (written, never accumulated into). Async on the current
+    stream."""
     cw = _weights_struct(p, weights)
-    _req(x, "x", (p.T, p.H), torch.float32)
-    _req(dout, "dout", (p.T, p.H), torch.float32)
+    _req(x, "x", (p.T, p.H), p.torch_dtype)
+    _req(dout, "dout", (p.T, p.H), p.torch_dtype)
     _req(selected, "selected", (p.T, p.k), torch.int64)
     dev = x.device
     sh, gated = p.shared != "none", p.shared == "sigmoid_gated"

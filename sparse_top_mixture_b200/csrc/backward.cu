@@ -615,6 +615,392 @@ WGemm wgrad(const float* A, const int32_t* amap, const float* ascale, int64_t ld
   return a;
 }
 
+
+// ---- bf16 problems: tensor-core backward ------------------------------------------
+// The same chain rule on the 5th-generation tensor cores. bf16 inputs (x,
+// dout, weights) stay bf16 as GEMM operands, products accumulate in fp32:
+//   [g | u] = x_perm Wgu^T (fp32), dhu = dout_perm Wd (fp32, via a transposed
+//   copy Wd^T [E,I,H]), then elementwise h = silu(g) u (fp32) and
+//   [dg | du] rounded to bf16 (the next GEMMs' operand), dx rows =
+//   [dg du] Wgu (fp32, via Wgu^T [E,H,2I]) -- all four on the forward's
+//   grouped kernels over the dispatch's segments; weight gradients on the
+//   weight-gradient mode of the one-CTA kernel, whose K loop walks an
+//   expert's rows: dWd = (w dout)^T h and dWgu = [dg du]^T x from K-major
+//   transposed copies [features][rows] in which every expert's rows are a
+//   run of columns zero-padded to a multiple of 64 (w dout and h rounded to
+//   bf16 there). The router (E logits per token) and the gate vector keep
+//   the fp32 SIMT code above, on fp32 copies of x and gate_w. Gradients are
+//   fp32. Still no atomics: results are deterministic.
+
+// out[i] = float(in[i])
+__global__ void __launch_bounds__(BT) bw16_to_f32(const __nv_bfloat16* __restrict__ in, int64_t n,
+                                                float* __restrict__ out) {
+  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT)
+    out[i] = __bfloat162float(in[i]);
+}
+
+// out[b][c][r] = in[b][r][c] for R x C slabs, 64 x 64 tiles through shared memory.
+__global__ void __launch_bounds__(BT) bw16_transpose(const __nv_bfloat16* __restrict__ in, int R, int C,
+                                                   __nv_bfloat16* __restrict__ out) {
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int64_t slab = (int64_t)blockIdx.z * R * C;
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
+  for (int i = ty; i < 64; i += 4) {
+    const int r = r0 + i, c = c0 + tx;
+    tile[i][tx] = (r < R && c < C) ? in[slab + (int64_t)r * C + c] : __float2bfloat16_rn(0.f);
+  }
+  __syncthreads();
+  for (int i = ty; i < 64; i += 4) {
+    const int c = c0 + i, r = r0 + tx;
+    if (c < C && r < R) out[slab + (int64_t)c * R + r] = tile[tx][i];
+  }
+}
+
+// Padded K offsets of the weight-gradient GEMMs: koff[e] = sum over e' < e of
+// round_up(count[e'], 64); also the one-segment ranges of the shared expert:
+// ranges = {0, T, 0, round_up(T, 64)}.
+__global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int32_t* __restrict__ koff,
+                          int32_t* __restrict__ ranges) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int run = 0;
+  for (int e = 0; e < E; ++e) {
+    koff[e] = run;
+    run += (offsets[e + 1] - offsets[e] + 63) / 64 * 64;
+  }
+  koff[E] = run;
+  ranges[0] = 0;
+  ranges[1] = T;
+  ranges[2] = 0;
+  ranges[3] = (T + 63) / 64 * 64;
+}
+
+// Transpose of row-major activations into the padded K-major layout:
+// out[c * ld + kk] for kk in [0, ld): inside expert e's run [koff[e],
+// koff[e] + count_e) it holds bf16(scale[r] * in[src(r) * ld_in + c]) with r =
+// off[e] + (kk - koff[e]) and src(r) = rowmap[r] (or r); everywhere else 0.
+// 64 x 64 tiles: a quarter-warp reads 64 consecutive columns of one source
+// row, a quarter-warp writes 64 consecutive kk of one output row.
+template <typename Tin>
+__global__ void __launch_bounds__(BT) bw16_transpose_pad(const Tin* __restrict__ in, int64_t ld_in,
+                                                       const int32_t* __restrict__ rowmap,
+                                                       const float* __restrict__ scale,
+                                                       const int32_t* __restrict__ off,
+                                                       const int32_t* __restrict__ koff, int E, int X,
+                                                       __nv_bfloat16* __restrict__ out, int64_t ld) {
+  __shared__ float tile[64][65];
+  __shared__ int s_off[kMaxExperts + 1], s_koff[kMaxExperts + 1];
+  __shared__ int s_src[64];
+  __shared__ float s_sc[64];
+  for (int e = threadIdx.x; e <= E; e += BT) {
+    s_off[e] = off[e];
+    s_koff[e] = koff[e];
+  }
+  __syncthreads();
+  const int64_t kk0 = (int64_t)blockIdx.y * 64;
+  const int c0 = blockIdx.x * 64;
+  if (threadIdx.x < 64) {
+    const int kk = (int)(kk0 + threadIdx.x);
+    int lo = 0, hi = E;  // expert with koff[lo] <= kk < koff[lo + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_koff[mid] <= kk) lo = mid;
+      else hi = mid;
+    }
+    const int j = kk - s_koff[lo];
+    int src = -1;
+    float sc = 0.f;
+    if (kk < s_koff[E] && j < s_off[lo + 1] - s_off[lo]) {
+      const int r = s_off[lo] + j;
+      src = rowmap ? rowmap[r] : r;
+      sc = scale ? scale[r] : 1.f;
+    }
+    s_src[threadIdx.x] = src;
+    s_sc[threadIdx.x] = sc;
+  }
+  __syncthreads();
+  const int q = threadIdx.x & 3, rr = threadIdx.x >> 2;  // 4 threads per row, 16 columns each
+  {
+    const int src = s_src[rr];
+    const float sc = s_sc[rr];
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int c = c0 + q * 16 + i;
+      float v = 0.f;
+      if (src >= 0 && c < X) {
+        if constexpr (sizeof(Tin) == 2) v = __bfloat162float(in[(int64_t)src * ld_in + c]);
+        else v = in[(int64_t)src * ld_in + c];
+        v *= sc;
+      }
+      tile[q * 16 + i][rr] = v;
+    }
+  }
+  __syncthreads();
+  const int c = c0 + rr;
+  if (c < X) {
+    __nv_bfloat16* orow = out + (int64_t)c * ld + kk0 + q * 16;
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(tile[rr][q * 16 + 2 * i], tile[rr][q * 16 + 2 * i + 1]);
+    reinterpret_cast<uint4*>(orow)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(orow)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// SwiGLU backward of one routed row block: for rows r < rows (rows = *nrows
+// when nrows is given) and i < I, with g, u from gu [*, 2I], dhu [*, I] and
+// the row's weight scale[r]: hact = silu(g) u (fp32); dgdu = bf16([dh u
+// silu'(g) | dh silu(g)]), dh = scale dhu.
+__global__ void __launch_bounds__(BT) bw16_swiglu(const float* __restrict__ gu, const float* __restrict__ dhu,
+                                                const float* __restrict__ scale, const int32_t* __restrict__ nrows,
+                                                int64_t rows, int I, float* __restrict__ hact,
+                                                __nv_bfloat16* __restrict__ dgdu) {
+  const int64_t R = nrows ? (int64_t)*nrows : rows;
+  const int64_t n = R * I;
+  for (int64_t idx = blockIdx.x * (int64_t)BT + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * BT) {
+    const int64_t r = idx / I;
+    const int i = (int)(idx - r * I);
+    const float g = gu[r * 2 * I + i], u = gu[r * 2 * I + I + i];
+    const float d = dhu[idx];
+    const float dh = scale[r] * d;
+    hact[idx] = silu_f32(g) * u;
+    dgdu[r * 2 * I + i] = __float2bfloat16_rn(dh * u * silu_grad_f(g));
+    dgdu[r * 2 * I + I + i] = __float2bfloat16_rn(dh * silu_f32(g));
+  }
+}
+
+struct BwLayout16 {
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, parts, x32, gw32, g32,
+      koff, ranges, xperm, doutperm, wguT, wdT, gu, dhu, hact, dgdu, dxr, extra, xT, dyT, hT, dgduT, gus, dhus, hacts,
+      dgdus, wsguT, wsdT, xTs, dyTs, hTs, dgdusT, gamma, dz, total;
+  int64_t Ppad, Tpad;
+};
+
+BwLayout16 bw_layout16(const moe_problem& p) {
+  BwLayout16 b;
+  const int64_t P = p.T * p.k;
+  b.Ppad = round_up(P + 63 * p.E, 64);
+  b.Tpad = round_up(p.T, 64);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = a256(off + bytes);
+    return at;
+  };
+  const size_t f = 4, h2 = 2;
+  b.header = take(sizeof(WsHeader));
+  b.local = take((size_t)dispatch_num_blocks(p.T, p.k) * p.E * 4);
+  b.counts = take((size_t)p.E * 4);
+  b.offsets = take((size_t)(p.E + 1) * 4);
+  b.sorted_pairs = take((size_t)P * 4);
+  b.pair_pos = take((size_t)P * 4);
+  b.tok = take((size_t)P * 4);
+  b.scale = take((size_t)P * f);
+  b.w = take((size_t)P * f);
+  b.dw = take((size_t)P * f);
+  b.L = take((size_t)p.T * p.E * f);
+  b.S = take((size_t)p.T * p.E * f);
+  b.dL = take((size_t)p.T * p.E * f);
+  const int S = router_chunks(p);
+  b.parts = take(S > 1 ? (size_t)S * p.E * p.H * f : 0);
+  b.x32 = take((size_t)p.T * p.H * f);
+  b.gw32 = take((size_t)p.E * p.H * f);
+  b.g32 = take((size_t)p.H * f);
+  b.koff = take((size_t)(p.E + 1) * 4);
+  b.ranges = take(4 * 4);
+  b.xperm = take((size_t)P * p.H * h2);
+  b.doutperm = take((size_t)P * p.H * h2);
+  b.wguT = take((size_t)p.E * p.H * 2 * p.I * h2);
+  b.wdT = take((size_t)p.E * p.I * p.H * h2);
+  b.gu = take((size_t)P * 2 * p.I * f);
+  b.dhu = take((size_t)P * p.I * f);
+  b.hact = take((size_t)P * p.I * f);
+  b.dgdu = take((size_t)P * 2 * p.I * h2);
+  b.dxr = take((size_t)P * p.H * f);
+  b.extra = take((size_t)p.T * p.H * f);
+  b.xT = take((size_t)p.H * b.Ppad * h2);
+  b.dyT = take((size_t)p.H * b.Ppad * h2);
+  b.hT = take((size_t)p.I * b.Ppad * h2);
+  b.dgduT = take((size_t)2 * p.I * b.Ppad * h2);
+  const bool sh = p.shared != MOE_SHARED_NONE;
+  const size_t Is = sh ? (size_t)p.I_shared : 0;
+  const size_t Tp = sh ? (size_t)b.Tpad : 0;
+  b.gus = take((size_t)p.T * 2 * Is * f);
+  b.dhus = take((size_t)p.T * Is * f);
+  b.hacts = take((size_t)p.T * Is * f);
+  b.dgdus = take((size_t)p.T * 2 * Is * h2);
+  b.wsguT = take((size_t)p.H * 2 * Is * h2);
+  b.wsdT = take(Is * p.H * h2);
+  b.xTs = take((size_t)p.H * Tp * h2);
+  b.dyTs = take((size_t)p.H * Tp * h2);
+  b.hTs = take(Is * Tp * h2);
+  b.dgdusT = take(2 * Is * Tp * h2);
+  b.gamma = take(sh ? (size_t)p.T * f : 0);
+  b.dz = take(sh ? (size_t)p.T * f : 0);
+  b.total = off;
+  return b;
+}
+
+template <typename Tin>
+cudaError_t transpose_pad(const Tin* in, int64_t ld_in, const int32_t* rowmap, const float* scale, const int32_t* off,
+                          const int32_t* koff, int E, int X, __nv_bfloat16* out, int64_t ld, cudaStream_t s) {
+  const dim3 grid((unsigned)ceil_div(X, 64), (unsigned)(ld / 64));
+  bw16_transpose_pad<Tin><<<grid, BT, 0, s>>>(in, ld_in, rowmap, scale, off, koff, E, X, out, ld);
+  return cudaGetLastError();
+}
+
+cudaError_t transpose_slabs(const void* in, int64_t B, int64_t R, int64_t C, void* out, cudaStream_t s) {
+  const dim3 grid((unsigned)ceil_div(C, 64), (unsigned)ceil_div(R, 64), (unsigned)B);
+  bw16_transpose<<<grid, BT, 0, s>>>(static_cast<const __nv_bfloat16*>(in), (int)R, (int)C,
+                                     static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+#define BW16_CUDA(...)                                     \
+  do {                                                     \
+    if ((__VA_ARGS__) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void* x_, const void* dout_,
+                         const int64_t* selected, moe_grads* g, void* ws, cudaStream_t s) {
+  const BwLayout16 b = bw_layout16(*p);
+  const bool sh = p->shared != MOE_SHARED_NONE, gated = p->shared == MOE_SHARED_SIGMOID_GATED;
+  const int T = (int)p->T, H = (int)p->H, E = (int)p->E, k = (int)p->k, I = (int)p->I, Is = (int)p->I_shared;
+  const int64_t P = p->T * p->k;
+  using bf = __nv_bfloat16;
+  const bf* x = static_cast<const bf*>(x_);
+  const bf* dout = static_cast<const bf*>(dout_);
+  WsHeader* hdr = at<WsHeader>(ws, b.header);
+  int32_t* err = &hdr->error_bits;
+  int32_t* offsets = at<int32_t>(ws, b.offsets);
+  int32_t* sorted_pairs = at<int32_t>(ws, b.sorted_pairs);
+  int32_t* pair_pos = at<int32_t>(ws, b.pair_pos);
+  int32_t* tok = at<int32_t>(ws, b.tok);
+  float* scale = at<float>(ws, b.scale);
+  float* wts = at<float>(ws, b.w);
+  float* dw = at<float>(ws, b.dw);
+  float* L = at<float>(ws, b.L);
+  float* S = at<float>(ws, b.S);
+  float* dL = at<float>(ws, b.dL);
+  float* x32 = at<float>(ws, b.x32);
+  float* gw32 = at<float>(ws, b.gw32);
+  float* g32 = gated ? at<float>(ws, b.g32) : nullptr;
+  int32_t* koff = at<int32_t>(ws, b.koff);
+  int32_t* ranges = at<int32_t>(ws, b.ranges);
+  bf* xperm = at<bf>(ws, b.xperm);
+  bf* doutperm = at<bf>(ws, b.doutperm);
+  bf* wguT = at<bf>(ws, b.wguT);
+  bf* wdT = at<bf>(ws, b.wdT);
+  float* gu = at<float>(ws, b.gu);
+  float* dhu = at<float>(ws, b.dhu);
+  float* hact = at<float>(ws, b.hact);
+  bf* dgdu = at<bf>(ws, b.dgdu);
+  float* dxr = at<float>(ws, b.dxr);
+  float* extra = at<float>(ws, b.extra);
+  bf* xT = at<bf>(ws, b.xT);
+  bf* dyT = at<bf>(ws, b.dyT);
+  bf* hT = at<bf>(ws, b.hT);
+  bf* dgduT = at<bf>(ws, b.dgduT);
+
+  // fp32 copies for the SIMT router and gate vector
+  bw16_to_f32<<<grid_for((int64_t)T * H), BT, 0, s>>>(x, (int64_t)T * H, x32);
+  bw16_to_f32<<<grid_for((int64_t)E * H), BT, 0, s>>>(static_cast<const bf*>(w->gate_w), (int64_t)E * H, gw32);
+  if (gated) bw16_to_f32<<<grid_for(H), BT, 0, s>>>(static_cast<const bf*>(w->shared_gate), H, g32);
+  // Router: logits, scores and the routing weights of the given choice.
+  BW16_CUDA(run_rows<true, EPI_STORE>(
+      [&] {
+        RowGemm a = row_gemm(x32, nullptr, H, gw32, 0, E, H, nullptr, 1, T, T, err);
+        a.C = L;
+        a.ldc = E;
+        return a;
+      }(),
+      s));
+  bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
+  // Sorted segments of the choice with x_perm; the same permutation of dout.
+  BW16_CUDA(launch_dispatch(MOE_DTYPE_BF16, selected, x, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
+                            at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, xperm, err,
+                            &hdr->dispatch_ticket, s));
+  BW16_CUDA(launch_dispatch(MOE_DTYPE_BF16, selected, dout, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
+                            at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, doutperm, nullptr,
+                            &hdr->dispatch_ticket, s));
+  bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, wts, E, k, tok, scale);
+  bw16_koff<<<1, 32, 0, s>>>(offsets, E, T, koff, ranges);
+  // Transposed weight copies (K-major operands of the data-gradient GEMMs).
+  BW16_CUDA(transpose_slabs(w->gate_up, E, 2 * I, H, wguT, s));  // [E][2I][H] -> [E][H][2I]
+  BW16_CUDA(transpose_slabs(w->down, E, H, I, wdT, s));          // [E][H][I] -> [E][I][H]
+  // Routed experts on the tensor cores.
+  const Segments sg{offsets, (int32_t)E, 0, P};
+  BW16_CUDA(launch_tc_down(sg, xperm, w->gate_up, E, gu, nullptr, nullptr, 2 * I, H, err, s));  // [g | u]
+  BW16_CUDA(launch_tc_down(sg, doutperm, wdT, E, dhu, nullptr, nullptr, I, H, err, s));         // dhu
+  bw16_swiglu<<<grid_for(P * I), BT, 0, s>>>(gu, dhu, scale, offsets + E, P, I, hact, dgdu);
+  BW16_CUDA(launch_tc_down(sg, dgdu, wguT, E, dxr, nullptr, nullptr, H, 2 * I, err, s));       // dx rows
+  bw_rowdot<<<grid_for(P * 32), BT, 0, s>>>(hact, dhu, I, pair_pos, P, nullptr, dw);
+  // Routed weight gradients from padded transposes: dWd = (w dout)^T h, dWgu = [dg du]^T x.
+  BW16_CUDA(transpose_pad<bf>(dout, H, tok, scale, offsets, koff, E, H, dyT, b.Ppad, s));
+  BW16_CUDA(transpose_pad<float>(hact, I, nullptr, nullptr, offsets, koff, E, I, hT, b.Ppad, s));
+  BW16_CUDA(transpose_pad<bf>(dgdu, 2 * I, nullptr, nullptr, offsets, koff, E, 2 * I, dgduT, b.Ppad, s));
+  BW16_CUDA(transpose_pad<bf>(x, H, tok, nullptr, offsets, koff, E, H, xT, b.Ppad, s));
+  BW16_CUDA(launch_wgrad(dyT, hT, b.Ppad, koff, E, H, I, g->d_down, err, s));
+  BW16_CUDA(launch_wgrad(dgduT, xT, b.Ppad, koff, E, 2 * I, H, g->d_gate_up, err, s));
+  // Router backward: dL, dgate_w = dL^T x (in row chunks summed in order), d_bias = sum_t dL.
+  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL);
+  const int nchunk = router_chunks(*p);
+  if (nchunk == 1) {
+    BW16_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x32, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1,
+                        s));
+  } else {
+    float* parts = at<float>(ws, b.parts);
+    const int chunk = (int)ceil_div(T, nchunk);
+    BW16_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x32, nullptr, H, H, nullptr, T, T, parts, err, chunk),
+                        nchunk, s));
+    bw_sum_parts<<<grid_for((int64_t)E * H), BT, 0, s>>>(parts, nchunk, (int64_t)E * H, g->d_gate_w);
+  }
+  if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
+  // Shared expert over all tokens (one segment), scaled by gamma; its dx goes to `extra`.
+  float* dz = nullptr;
+  if (sh) {
+    float* gus = at<float>(ws, b.gus);
+    float* dhus = at<float>(ws, b.dhus);
+    float* hacts = at<float>(ws, b.hacts);
+    bf* dgdus = at<bf>(ws, b.dgdus);
+    bf* wsguT = at<bf>(ws, b.wsguT);
+    bf* wsdT = at<bf>(ws, b.wsdT);
+    float* gamma = at<float>(ws, b.gamma);
+    dz = at<float>(ws, b.dz);
+    const Segments one{nullptr, 1, (int32_t)T, p->T};
+    bw_gamma<<<grid_for((int64_t)T * 32), BT, 0, s>>>(x32, g32, T, H, gamma);
+    BW16_CUDA(transpose_slabs(w->shared_gate_up, 1, 2 * Is, H, wsguT, s));  // [2Is][H] -> [H][2Is]
+    BW16_CUDA(transpose_slabs(w->shared_down, 1, H, Is, wsdT, s));          // [H][Is] -> [Is][H]
+    BW16_CUDA(launch_tc_down(one, x, w->shared_gate_up, 1, gus, nullptr, nullptr, 2 * Is, H, err, s));
+    BW16_CUDA(launch_tc_down(one, dout, wsdT, 1, dhus, nullptr, nullptr, Is, H, err, s));
+    bw16_swiglu<<<grid_for((int64_t)T * Is), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, hacts, dgdus);
+    BW16_CUDA(launch_tc_down(one, dgdus, wsguT, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
+    if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(hacts, dhus, Is, nullptr, T, gamma, dz);
+    bf* xTs = at<bf>(ws, b.xTs);
+    bf* dyTs = at<bf>(ws, b.dyTs);
+    bf* hTs = at<bf>(ws, b.hTs);
+    bf* dgdusT = at<bf>(ws, b.dgdusT);
+    // one segment: ranges = {off: 0, T; koff: 0, Tpad}
+    BW16_CUDA(transpose_pad<bf>(dout, H, nullptr, gamma, ranges, ranges + 2, 1, H, dyTs, b.Tpad, s));
+    BW16_CUDA(transpose_pad<float>(hacts, Is, nullptr, nullptr, ranges, ranges + 2, 1, Is, hTs, b.Tpad, s));
+    BW16_CUDA(transpose_pad<bf>(dgdus, 2 * Is, nullptr, nullptr, ranges, ranges + 2, 1, 2 * Is, dgdusT, b.Tpad, s));
+    BW16_CUDA(transpose_pad<bf>(x, H, nullptr, nullptr, ranges, ranges + 2, 1, H, xTs, b.Tpad, s));
+    BW16_CUDA(launch_wgrad(dyTs, hTs, b.Tpad, ranges + 2, 1, H, Is, g->d_shared_down, err, s));
+    BW16_CUDA(launch_wgrad(dgdusT, xTs, b.Tpad, ranges + 2, 1, 2 * Is, H, g->d_shared_gate_up, err, s));
+    if (gated) bw_dgvec<<<grid_for(H), BT, 0, s>>>(dz, x32, T, H, g->d_shared_gate);
+  }
+  // Router (and shared gate) dx into `extra`, then dx = sum of each token's rows + extra.
+  RowGemm rd = row_gemm(dL, nullptr, E, gw32, 0, H, E, nullptr, 1, T, T, err);
+  rd.C = extra;
+  rd.ldc = H;
+  rd.dz = gated ? dz : nullptr;
+  rd.gvec = gated ? g32 : nullptr;
+  if (sh) BW16_CUDA(run_rows<false, EPI_ADD>(rd, s));
+  else BW16_CUDA(run_rows<false, EPI_STORE>(rd, s));
+  BW16_CUDA(launch_combine(MOE_DTYPE_F32, dxr, pair_pos, extra, g->dx, p->T, p->H, p->k, s));
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace stm
 
@@ -625,7 +1011,7 @@ MOE_API moe_status moe_backward_workspace_size(const moe_problem* p, size_t* byt
   const moe_status st = moe_workspace_size(p, &fwd);  // validates the problem
   if (st != MOE_OK) return st;
   if (bytes == nullptr) return MOE_ERR_INVALID_ARGUMENT;
-  *bytes = bw_layout(*p).total;
+  *bytes = p->dtype == MOE_DTYPE_BF16 ? bw_layout16(*p).total : bw_layout(*p).total;
   return MOE_OK;
 }
 
@@ -640,7 +1026,6 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   size_t need = 0;
   const moe_status st = moe_backward_workspace_size(p, &need);
   if (st != MOE_OK) return st;
-  if (p->dtype != MOE_DTYPE_F32) return MOE_ERR_UNSUPPORTED;
   if (w == nullptr || g == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   const bool sh = p->shared != MOE_SHARED_NONE, gated = p->shared == MOE_SHARED_SIGMOID_GATED;
   const bool has_tokens = p->T > 0;  // per-token arrays and the workspace may be NULL without tokens
@@ -671,6 +1056,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
     return MOE_OK;
   }
   NvtxRange range("moe_backward");
+  if (p->dtype == MOE_DTYPE_BF16) return backward_bf16(p, w, x_, dout_, selected, g, ws, s);
   const BwLayout b = bw_layout(*p);
   const int T = (int)p->T, H = (int)p->H, E = (int)p->E, k = (int)p->k, I = (int)p->I, Is = (int)p->I_shared;
   const int64_t P = p->T * p->k;

@@ -154,10 +154,14 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
                                                                   int32_t* __restrict__ pair_pos,
                                                                   const T* __restrict__ x, T* __restrict__ x_perm,
                                                                   int64_t Tn, int H, int vec_per_slice) {
-  __shared__ int wcnt[DTHREADS / 32][kMaxExperts];
+  // Per-warp counts of each expert (at most 32, so 16 bits) and the slot of
+  // every pair: 5 KB of shared memory, small enough to sit beside a
+  // persistent GEMM CTA on the same SM.
+  __shared__ uint16_t wcnt[DTHREADS / 32][kMaxExperts];
   __shared__ int s_pos[DTHREADS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < (DTHREADS / 32) * kMaxExperts; i += DTHREADS) (&wcnt[0][0])[i] = 0;
+  for (int i = tid; i < (DTHREADS / 32) * kMaxExperts / 2; i += DTHREADS)
+    reinterpret_cast<uint32_t*>(&wcnt[0][0])[i] = 0u;
   __syncthreads();
 
   const int64_t q0 = (int64_t)blockIdx.x * tok_per_blk * k;
@@ -171,20 +175,14 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
   }
   const unsigned peers = __match_any_sync(0xffffffffu, e);
   const int rank = __popc(peers & ((1u << lane) - 1u));
-  if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(peers);
+  if (e >= 0 && rank == 0) wcnt[warp][e] = (uint16_t)__popc(peers);
   __syncthreads();
-  if (tid < E) {
-    int run = bases[(int64_t)blockIdx.x * E + tid];
-#pragma unroll
-    for (int w = 0; w < DTHREADS / 32; ++w) {
-      const int c = wcnt[w][tid];
-      wcnt[w][tid] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
+  // slot = this block's base for the expert + pairs of earlier warps + rank
   int pos = -1;
-  if (e >= 0) pos = wcnt[warp][e] + rank;
+  if (e >= 0) {
+    pos = bases[(int64_t)blockIdx.x * E + e] + rank;
+    for (int w = 0; w < warp; ++w) pos += wcnt[w][e];
+  }
   s_pos[tid] = pos;
   if (blockIdx.y == 0) {
     if (e >= 0) sorted_pairs[pos] = (int32_t)q;
@@ -213,31 +211,37 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
 }
 
 // out[t] = sum_j y_perm[pair_pos[t*k+j]] + shared_out[t]: fp32 rows, summed in
-// slot order in fp32, rounded once to the output type. Four columns per
-// thread (16-byte fp32 loads).
+// slot order in fp32, rounded once to the output type. Work units are the
+// 16-byte column vectors of all tokens, flattened and strided over a grid of
+// a few CTAs per SM, so every SM gets the same share (no partial last wave);
+// consecutive threads take consecutive vectors of one row.
+constexpr int CTHREADS = 256;
+
 template <typename T>
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ y_perm,
-                                                      const int32_t* __restrict__ pair_pos,
-                                                      const float* __restrict__ shared_out, T* __restrict__ out,
-                                                      int H, int k) {
-  __shared__ int pp[kMaxExperts];
-  const int64_t t = blockIdx.x;
-  for (int j = threadIdx.x; j < k; j += blockDim.x) pp[j] = pair_pos[t * k + j];
-  __syncthreads();
+__global__ void __launch_bounds__(CTHREADS) combine_kernel(const float* __restrict__ y_perm,
+                                                           const int32_t* __restrict__ pair_pos,
+                                                           const float* __restrict__ shared_out,
+                                                           T* __restrict__ out, int64_t Tn, int H, int k) {
   const int nvec = H / 4;
-  for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nvec; v += gridDim.y * blockDim.x) {
+  const int64_t units = Tn * nvec;
+  const int64_t stride = (int64_t)gridDim.x * CTHREADS;
+  for (int64_t u = (int64_t)blockIdx.x * CTHREADS + threadIdx.x; u < units; u += stride) {
+    const int64_t t = u / nvec;
+    const int v = (int)(u - t * nvec);
+    const int32_t* pp = pair_pos + t * k;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
     for (int j = 0; j < k; ++j) {
-      const int p = pp[j];
+      const int p = __ldg(pp + j);
       if (p < 0) continue;
-      const float4 y = reinterpret_cast<const float4*>(y_perm + (int64_t)p * H)[v];
+      const float4 y = __ldcs(reinterpret_cast<const float4*>(y_perm + (int64_t)p * H) + v);
       acc.x += y.x;
       acc.y += y.y;
       acc.z += y.z;
       acc.w += y.w;
     }
     if (shared_out != nullptr) {
-      const float4 y = reinterpret_cast<const float4*>(shared_out + t * H)[v];
+      const float4 y = __ldcs(reinterpret_cast<const float4*>(shared_out + t * H) + v);
       acc.x += y.x;
       acc.y += y.y;
       acc.z += y.z;
@@ -292,14 +296,13 @@ cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, i
 
 cudaError_t launch_combine(int dtype, const float* y_perm, const int32_t* pair_pos, const float* shared_out,
                            void* out, int64_t T, int64_t H, int64_t k, cudaStream_t s) {
-  const int64_t nvec = H / 4;
-  const unsigned gy = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ceil_div(nvec, 128), T < 148 ? 16 : 1));
-  dim3 grid((unsigned)T, gy);
+  const int64_t units = T * (H / 4);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, CTHREADS), 148 * 8));
   if (dtype == 0)
-    combine_kernel<float><<<grid, 128, 0, s>>>(y_perm, pair_pos, shared_out, (float*)out, (int)H, (int)k);
+    combine_kernel<float><<<grid, CTHREADS, 0, s>>>(y_perm, pair_pos, shared_out, (float*)out, T, (int)H, (int)k);
   else
-    combine_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(y_perm, pair_pos, shared_out, (__nv_bfloat16*)out, (int)H,
-                                                       (int)k);
+    combine_kernel<__nv_bfloat16><<<grid, CTHREADS, 0, s>>>(y_perm, pair_pos, shared_out, (__nv_bfloat16*)out, T,
+                                                           (int)H, (int)k);
   return cudaGetLastError();
 }
 

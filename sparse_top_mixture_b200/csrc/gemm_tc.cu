@@ -60,7 +60,7 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * UMMA_N;
 constexpr int NTHREADS = 192;
 
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2 };
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2, MODE_WGRAD = 3 };
 
 struct Args {
   const int32_t* offsets;
@@ -77,6 +77,8 @@ struct Args {
   const int32_t* scale_idx;
   int32_t* err;
   int64_t rows_total;
+  int32_t M;        // WGRAD: output rows per expert
+  int32_t m_tiles;  // WGRAD: 128-row tiles of M
 };
 
 struct __align__(8) Ctl {
@@ -105,8 +107,25 @@ struct TileCoord {
 };
 
 // Tile index -> (row tile, column tile, k split); the split varies fastest.
+// WGRAD: tile index -> (expert, row tile of M, column tile of N); the K range
+// is the expert's padded segment [off[e], off[e+1]) (multiples of BK).
+template <int MODE>
 __device__ __forceinline__ TileCoord decode_tile(const Ctl* ctl, int Eseg, const Args& a, int tile) {
   TileCoord c;
+  if constexpr (MODE == MODE_WGRAD) {
+    const int per_e = a.m_tiles * a.n_tiles;
+    c.e = tile / per_e;
+    const int rest = tile - c.e * per_e;
+    const int mt = rest / a.n_tiles;
+    c.n_idx = rest - mt * a.n_tiles;
+    c.split = 0;
+    c.kt0 = ctl->off[c.e] / BK;
+    c.kt1 = ctl->off[c.e + 1] / BK;
+    c.row0 = mt * BM;
+    c.row_end = a.M;
+    c.m64 = c.row_end - c.row0 <= 64;
+    return c;
+  }
   c.split = tile % a.k_splits;
   const int rest = tile / a.k_splits;
   const int mt = rest / a.n_tiles;
@@ -118,6 +137,26 @@ __device__ __forceinline__ TileCoord decode_tile(const Ctl* ctl, int Eseg, const
   c.row_end = ctl->off[c.e + 1];
   c.m64 = c.row_end - c.row0 <= 64;
   return c;
+}
+
+// WGRAD: the padded K offsets [E+1] into shared memory (one warp). They must
+// be non-decreasing multiples of BK inside [0, rows_total] (the operands' K
+// extent); otherwise every expert gets an empty range and MOE_DEVERR_BAD_EXPERT_ID
+// is raised.
+__device__ __forceinline__ void warp_load_k_ranges(const int32_t* __restrict__ offsets, int E, int64_t k_extent,
+                                                   int* off, int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+  for (int e = lane; e <= E; e += 32) {
+    const int v = offsets[e];
+    off[e] = v;
+    bad |= v < 0 || (v % BK) != 0 || (int64_t)v > k_extent || (e > 0 && offsets[e - 1] > v);
+  }
+  if (__any_sync(0xffffffffu, bad)) {
+    __syncwarp();
+    if (lane == 0) raise_error(err, 1);
+    for (int e = lane; e <= E; e += 32) off[e] = 0;
+  }
 }
 
 template <int MODE>
@@ -145,14 +184,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 2)
-    warp_build_tile_table(args.offsets, args.E, args.single_rows, BM, ctl->off, ctl->pre, args.rows_total, args.err);
+  if (warp == 2) {
+    if constexpr (MODE == MODE_WGRAD)
+      warp_load_k_ranges(args.offsets, args.E, args.rows_total, ctl->off, args.err);
+    else
+      warp_build_tile_table(args.offsets, args.E, args.single_rows, BM, ctl->off, ctl->pre, args.rows_total,
+                            args.err);
+  }
   if (warp == 1) tmem_alloc(&ctl->tmem_base, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  const int total_tiles = ctl->pre[Eseg] * args.n_tiles * args.k_splits;
+  const int total_tiles = MODE == MODE_WGRAD ? args.E * args.m_tiles * args.n_tiles
+                                             : ctl->pre[Eseg] * args.n_tiles * args.k_splits;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -162,7 +207,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t issued = 0, last_parity = 0;  // per stage: ever issued, parity of the last issue
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
+        const TileCoord tc = decode_tile<MODE>(ctl, Eseg, args, tile);
         for (int kt = tc.kt0; kt < tc.kt1; ++kt) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, args.err, 1)) { ok = false; break; }
           uint8_t* sa = base + stage * STAGE_BYTES;
@@ -175,7 +220,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_4d(sb, &tmB, &ctl->full[stage], k0, n0, 0, tc.e);
             tma_load_4d(sb + B_BYTES / 2, &tmB, &ctl->full[stage], k0, n0, 1, tc.e);
           } else {
-            tma_load_3d(sb, &tmB, &ctl->full[stage], k0, tc.n_idx * UMMA_N, tc.e);
+            tma_load_3d(sb, &tmB, &ctl->full[stage], k0, tc.n_idx * UMMA_N, MODE == MODE_WGRAD ? 0 : tc.e);
           }
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -195,7 +240,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
+        const TileCoord tc = decode_tile<MODE>(ctl, Eseg, args, tile);
         if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
@@ -230,7 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord tc = decode_tile(ctl, Eseg, args, tile);
+      const TileCoord tc = decode_tile<MODE>(ctl, Eseg, args, tile);
       if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, args.err, 4)) break;
       tc_fence_after();
       // this warp's rows: 32 consecutive (16 for an M=64 tile), lane = row
@@ -244,6 +289,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (MODE == MODE_GATE_UP) {
         epilogue_swiglu(tbase, 0, 128, 4, reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row_w0 * args.ldo,
                         args.ldo, nrows, tc.n_idx * 128, args.N, lane);
+      } else if (MODE == MODE_WGRAD) {
+        // dW[e] rows row_w0.. of M, fp32, row pitch N; an expert without rows
+        // (empty K range, no MMA issued) gets zeros, not the stale accumulator
+        float* orow0 = reinterpret_cast<float*>(args.out) + (int64_t)tc.e * args.M * args.ldo +
+                       (int64_t)row_w0 * args.ldo;
+        if (tc.kt1 > tc.kt0) {
+          epilogue_scale_f32(tbase, UMMA_N / 32, 1.f, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N, args.N,
+                             lane);
+        } else {
+          float z[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) z[q] = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < UMMA_N / 32; ++c) {
+            const int cb = tc.n_idx * UMMA_N + c * 32;
+            if (cb >= args.N || nrows <= 0) break;  // warp-uniform
+            store_block_f32(z, stage, orow0 + cb, args.ldo, nrows, args.N - cb, lane);
+          }
+        }
       } else if (MODE == MODE_DOWN) {
         float sc = 1.f;
         if (valid && args.row_scale != nullptr) sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
@@ -319,6 +383,8 @@ cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensor
   a.scale_idx = scale_idx;
   a.err = err;
   a.rows_total = sg.rows_total;
+  a.M = 0;
+  a.m_tiles = 0;
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM + nseg) * a.n_tiles * a.k_splits;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
@@ -327,6 +393,48 @@ cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensor
 }
 
 }  // namespace
+
+// Weight gradients: out[e][m][n] = sum over k in [koff[e], koff[e+1])
+// of AT[m][k] * BT[n][k], AT [M][ld] and BT [N][ld] bf16 (K-major, each
+// expert's rows a zero-padded run of columns), out fp32 [E][M][N].
+cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32_t* koff, int E, int64_t M, int64_t N,
+                         float* out, int32_t* err, cudaStream_t s) {
+  static std::once_flag attr_once[kSmemAttrDevices];
+  static cudaError_t attr_status[kSmemAttrDevices];
+  const void* kernel = reinterpret_cast<const void*>(tc_grouped_gemm_kernel<MODE_WGRAD>);
+  const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)kSmemBytes, attr_once, attr_status);
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[2] = {(uint64_t)ld, (uint64_t)M};
+    const uint64_t strides[1] = {(uint64_t)ld * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!make_tensor_map_bf16(&tmA, AT, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)ld, (uint64_t)N, 1};
+    const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)ld * N * 2};
+    const uint32_t box[3] = {BK, UMMA_N, 1};
+    if (!make_tensor_map_bf16(&tmB, BT, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  Args a{};
+  a.offsets = koff;
+  a.E = E;
+  a.N = (int32_t)N;
+  a.n_tiles = (int32_t)ceil_div(N, UMMA_N);
+  a.k_splits = 1;
+  a.ldo = N;
+  a.out = out;
+  a.err = err;
+  a.rows_total = ld;  // K extent of the operands
+  a.M = (int32_t)M;
+  a.m_tiles = (int32_t)ceil_div(M, BM);
+  const int64_t tiles = (int64_t)E * a.m_tiles * a.n_tiles;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles));
+  tc_grouped_gemm_kernel<MODE_WGRAD><<<grid, NTHREADS, kSmemBytes, s>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
 
 // ---- host side -----------------------------------------------------------
 
@@ -378,6 +486,7 @@ int tc_gemm_variant(const Segments& sg, bool) {
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                               int64_t I, int64_t H, int32_t* err, cudaStream_t s) {
   if (!get_encode()) return cudaErrorNotSupported;
+  if (tc_gemm_variant(sg, false) == 2) return launch_tc2_gate_up(sg, A, w_gate_up, E_w, h, I, H, err, num_sms(), s);
   CUtensorMap tmA, tmB;
   {
     const uint64_t dims[2] = {(uint64_t)H, (uint64_t)sg.rows_total};
@@ -385,7 +494,6 @@ cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_g
     const uint32_t box[2] = {BK, BM};
     if (!make_tensor_map_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  if (tc_gemm_variant(sg, false) == 2) return launch_tc2_gate_up(sg, tmA, w_gate_up, E_w, h, I, H, err, num_sms(), s);
   {
     // gate_up [E][2][I][H]: dim0 = H, dim1 = I (row within a half), dim2 = half, dim3 = expert
     const uint64_t dims[4] = {(uint64_t)H, (uint64_t)I, 2, (uint64_t)E_w};
@@ -400,6 +508,8 @@ cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down
                            const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                            cudaStream_t s) {
   if (!get_encode()) return cudaErrorNotSupported;
+  if (tc_gemm_variant(sg, true) == 2)
+    return launch_tc2_down(sg, h, w_down, E_w, y, row_scale, scale_idx, H, I, err, num_sms(), s);
   CUtensorMap tmA, tmB;
   {
     const uint64_t dims[2] = {(uint64_t)I, (uint64_t)sg.rows_total};
@@ -407,8 +517,6 @@ cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down
     const uint32_t box[2] = {BK, BM};
     if (!make_tensor_map_bf16(&tmA, h, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  if (tc_gemm_variant(sg, true) == 2)
-    return launch_tc2_down(sg, tmA, w_down, E_w, y, row_scale, scale_idx, H, I, err, num_sms(), s);
   {
     // down [E][H][I]: dim0 = I, dim1 = H, dim2 = expert
     const uint64_t dims[3] = {(uint64_t)I, (uint64_t)H, (uint64_t)E_w};

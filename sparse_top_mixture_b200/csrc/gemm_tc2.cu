@@ -16,6 +16,10 @@
 //   - each CTA's epilogue drains its own TMEM rows and arrives on the
 //     leader's accumulator-empty barrier.
 // No TMA multicast is used: every CTA fetches its own tiles.
+// When K is a multiple of 64, a stage holds two 64-element K atoms of A and
+// of B (a 3-D tensor-map view [K/64][rows][64] whose box spans both atoms),
+// so each TMA operation moves 32 KB, a stage carries eight MMAs and the ring
+// is 3 stages of 64 KB per CTA; otherwise one atom per stage, 6 stages.
 //
 // Used when segments average at least 192 rows. A row tile is 256 rows of one
 // segment. A tile with at most 128 rows left (a segment's tail) runs as an
@@ -48,17 +52,26 @@ using namespace tc;
 
 constexpr int BM2 = 256;         // rows per pair tile
 constexpr int HALF = 128;        // rows of A (and of B) per CTA
-constexpr int BK = 64;
+constexpr int BK = 64;           // K elements per atom (128 bytes: one swizzle row)
+constexpr int ATOM_BYTES = HALF * BK * 2;  // one 128-row x 64-element K atom
 constexpr int UMMA_N = 256;
 constexpr int UMMA_K = 16;
-constexpr int STAGES = 6;
-constexpr int A_BYTES = HALF * BK * 2;
-constexpr int B_BYTES = HALF * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int RING_BYTES = 6 * 2 * ATOM_BYTES;  // 192 KB of stages per CTA
+constexpr int MAX_STAGES = 6;
 constexpr int TMEM_COLS = 2 * UMMA_N;
 constexpr int NTHREADS = 192;
 constexpr uint32_t kIdesc256 = make_idesc(256, UMMA_N);
 constexpr uint32_t kIdesc128 = make_idesc(128, UMMA_N);  // pair tile tails: 64 rows per CTA
+
+// KA K atoms per stage: stage = KA atoms of A then KA atoms of B.
+template <int KA>
+struct Ring {
+  static constexpr int A_BYTES = KA * ATOM_BYTES;
+  static constexpr int B_BYTES = KA * ATOM_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;
+  static_assert(STAGES >= 2 && STAGES <= MAX_STAGES, "ring depth");
+};
 
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 
@@ -68,7 +81,7 @@ struct Args2 {
   int32_t single_rows;
   int32_t N;
   int32_t n_tiles;
-  int32_t k_tiles;
+  int32_t k_tiles;  // stages (KA atoms each) over the whole K
   int64_t ldo;
   void* out;
   const float* row_scale;
@@ -78,11 +91,11 @@ struct Args2 {
 };
 
 struct __align__(8) Ctl2 {
-  uint64_t full[STAGES];   // leader only: both CTAs' bytes of a stage landed
-  uint64_t empty[STAGES];  // both: the pair MMA finished reading a stage
-  uint64_t tfull[2];       // both: accumulator ready
-  uint64_t tempty[2];      // leader only: both CTAs' epilogues drained it
-  uint64_t drain;          // both: every pair MMA complete
+  uint64_t full[MAX_STAGES];   // leader only: both CTAs' bytes of a stage landed
+  uint64_t empty[MAX_STAGES];  // both: the pair MMA finished reading a stage
+  uint64_t tfull[2];           // both: accumulator ready
+  uint64_t tempty[2];          // leader only: both CTAs' epilogues drained it
+  uint64_t drain;              // both: every pair MMA complete
   uint32_t tmem_base;
   int abort;
   int off[kMaxExperts + 1];
@@ -91,14 +104,19 @@ struct __align__(8) Ctl2 {
 
 // Shared memory: the stage ring (its base 1024-byte aligned: the 128-byte
 // swizzle repeats every 1024 bytes), the epilogue staging blocks (one per
-// epilogue warp; used by down), then Ctl2. down declares the dynamic shared
-// memory 1024-byte aligned and checks it (doing nothing if it is not);
-// gate_up requests 1 KB more and rounds its base up. Each variant measured
-// 3-9% faster for its GEMM than the other layout (the same code otherwise).
-constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;
+// epilogue warp; down only: gate_up stores its bf16 rows directly), then
+// Ctl2. down declares the dynamic shared memory 1024-byte aligned and checks
+// it (doing nothing if it is not); gate_up requests 1 KB more and rounds its
+// base up. Each variant measured 3-9% faster for its GEMM than the other
+// layout (the same code otherwise). gate_up's ~200 KB leave room on the SM
+// for the dispatch kernels that run beside a shared expert's GEMM.
+template <int MODE>
+constexpr int epi_bytes2() {
+  return MODE == MODE_DOWN ? 4 * kStageFloatsPerWarp * 4 : 0;
+}
 template <int MODE>
 constexpr size_t smem_bytes2() {
-  return (MODE == MODE_GATE_UP ? 1024 : 0) + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl2);
+  return (MODE == MODE_GATE_UP ? 1024 : 0) + (size_t)RING_BYTES + epi_bytes2<MODE>() + sizeof(Ctl2);
 }
 static_assert(smem_bytes2<MODE_GATE_UP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 static_assert(smem_bytes2<MODE_DOWN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
@@ -123,10 +141,14 @@ __device__ __forceinline__ Tile2 decode_tile2(const Ctl2* ctl, int Eseg, int n_t
   return t;
 }
 
-template <int MODE>
+template <int MODE, int KA>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc2_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmB64, const Args2 args) {
+  constexpr int STAGES = Ring<KA>::STAGES;
+  constexpr int A_BYTES = Ring<KA>::A_BYTES;
+  constexpr int B_BYTES = Ring<KA>::B_BYTES;
+  constexpr int STAGE_BYTES = Ring<KA>::STAGE_BYTES;
   uint8_t* base;
   if constexpr (MODE == MODE_GATE_UP) {
     extern __shared__ uint8_t smem_gu[];
@@ -141,8 +163,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     base = smem_dn;
   }
-  float* epi_stage = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
-  Ctl2* ctl = reinterpret_cast<Ctl2*>(base + STAGES * STAGE_BYTES + EPI_BYTES);
+  float* epi_stage = reinterpret_cast<float*>(base + RING_BYTES);
+  Ctl2* ctl = reinterpret_cast<Ctl2*>(base + RING_BYTES + epi_bytes2<MODE>());
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -192,20 +214,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           if (leader)
             mbar_arrive_expect_tx(&ctl->full[stage],
                                   (uint32_t)(2 * B_BYTES + A_BYTES + (tc.peer_rows ? A_BYTES : 0)));
-          const int k0 = kt * BK;
-          if (leader || tc.peer_rows) tma2_load_2d(sa, &tmA, full_leader, k0, tc.row0 + (int)rank * tc.rows_cta);
+          // K coordinates: with two atoms per stage the views are [atoms][rows][64]
+          // and the stage starts at atom kt*2; with one, K is the innermost
+          // dimension and the stage starts at element kt*64.
+          const int ka = kt * KA;
+          const int cx = KA == 2 ? 0 : ka * BK;
+          const int cz = KA == 2 ? ka : 0;
+          if (leader || tc.peer_rows) tma2_load_3d(sa, &tmA, full_leader, cx, tc.row0 + (int)rank * tc.rows_cta, cz);
           if (MODE == MODE_GATE_UP) {
             if (!tc.tail) {
               // leader: gate rows n0..n0+127; peer: the matching up rows
-              tma2_load_4d(sb, &tmB, full_leader, k0, tc.n_idx * 128, (int)rank, tc.e);
+              tma2_load_5d(sb, &tmB, full_leader, cx, tc.n_idx * 128, cz, (int)rank, tc.e);
             } else {
-              // each CTA: 64 gate rows then the matching 64 up rows
+              // each CTA, per atom: 64 gate rows then the matching 64 up rows
               const int n0 = tc.n_idx * 128 + (int)rank * 64;
-              tma2_load_4d(sb, &tmB64, full_leader, k0, n0, 0, tc.e);
-              tma2_load_4d(sb + B_BYTES / 2, &tmB64, full_leader, k0, n0, 1, tc.e);
+#pragma unroll
+              for (int a = 0; a < KA; ++a) {
+                tma2_load_5d(sb + a * ATOM_BYTES, &tmB64, full_leader, cx, n0, cz + a, 0, tc.e);
+                tma2_load_5d(sb + a * ATOM_BYTES + ATOM_BYTES / 2, &tmB64, full_leader, cx, n0, cz + a, 1, tc.e);
+              }
             }
           } else {
-            tma2_load_3d(sb, &tmB, full_leader, k0, tc.n_idx * UMMA_N + (int)rank * HALF, tc.e);
+            tma2_load_4d(sb, &tmB, full_leader, cx, tc.n_idx * UMMA_N + (int)rank * HALF, cz, tc.e);
           }
           if (leader) {
             issued |= 1u << stage;
@@ -238,12 +268,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, args.err, 13)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(base + stage * STAGE_BYTES);
-          const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
-                       (kt > 0 || kk > 0) ? 1u : 0u);
+          for (int a = 0; a < KA; ++a) {
+            const uint64_t adesc = sw128_desc(sa + a * ATOM_BYTES);
+            const uint64_t bdesc = sw128_desc(sa + A_BYTES + a * ATOM_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / UMMA_K; ++kk)
+              umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+                         (kt > 0 || a > 0 || kk > 0) ? 1u : 0u);
+          }
           umma2_commit_mc(&ctl->empty[stage], 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -317,14 +350,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int MODE>
+template <int MODE, int KA>
 cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmB64,
-                       int64_t N, int64_t K,
-                       void* out, int64_t ldo, const float* row_scale, const int32_t* scale_idx, int32_t* err,
-                       int num_sms, cudaStream_t s) {
-  static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance (MODE)
+                       int64_t N, int64_t K, void* out, int64_t ldo, const float* row_scale,
+                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s) {
+  static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance
   static cudaError_t attr_status[kSmemAttrDevices];
-  const void* kernel = reinterpret_cast<const void*>(tc2_grouped_gemm_kernel<MODE>);
+  const void* kernel = reinterpret_cast<const void*>(tc2_grouped_gemm_kernel<MODE, KA>);
   const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)smem_bytes2<MODE>(), attr_once, attr_status);
   if (attr_err != cudaSuccess) return attr_err;
   Args2 a;
@@ -333,7 +365,7 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   a.single_rows = sg.single_rows;
   a.N = (int32_t)N;
   a.n_tiles = (int32_t)ceil_div(N, MODE == MODE_GATE_UP ? 128 : UMMA_N);
-  a.k_tiles = (int32_t)ceil_div(K, BK);
+  a.k_tiles = (int32_t)ceil_div(K, BK * KA);
   a.ldo = ldo;
   a.out = out;
   a.row_scale = row_scale;
@@ -343,36 +375,80 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM2 + nseg) * a.n_tiles;
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms / 2, max_tiles));
-  tc2_grouped_gemm_kernel<MODE><<<2 * pairs, NTHREADS, smem_bytes2<MODE>(), s>>>(tmA, tmB, tmB64, a);
+  tc2_grouped_gemm_kernel<MODE, KA><<<2 * pairs, NTHREADS, smem_bytes2<MODE>(), s>>>(tmA, tmB, tmB64, a);
   return cudaGetLastError();
+}
+
+// K atoms per stage: two when K splits into whole 64-element atoms (the view
+// [K/64][rows][64] then addresses only elements of each row), else one.
+int katoms(int64_t K) { return K % BK == 0 ? 2 : 1; }
+
+// Tensor maps over a K-major operand of `rows` rows (row pitch K elements,
+// consecutive operand slabs `slab` bytes apart, `nslab` of them, with the
+// gate_up halves as a further dimension when `halves` is 2). Two atoms per
+// stage: dims {64, rows, K/64, (halves,) slabs}, the atom dimension 128 bytes
+// apart, box {64, box_rows, 2, 1, 1}. One atom: dims {K, rows, 1, ...}, box
+// {64, box_rows, 1, ...}, reading zeros past K.
+bool map_kmajor(CUtensorMap* m, const void* ptr, int KA, int64_t K, int64_t rows, int64_t row_pitch_bytes,
+                int halves, int64_t half_bytes, int64_t nslab, int64_t slab_bytes, uint32_t box_rows) {
+  uint64_t dims[5], strides[4];
+  uint32_t box[5];
+  int r = 0;
+  dims[0] = KA == 2 ? (uint64_t)BK : (uint64_t)K;
+  box[0] = BK;
+  dims[1] = (uint64_t)rows;
+  strides[0] = (uint64_t)row_pitch_bytes;
+  box[1] = box_rows;
+  dims[2] = KA == 2 ? (uint64_t)(K / BK) : 1;
+  strides[1] = KA == 2 ? (uint64_t)BK * 2 : (uint64_t)row_pitch_bytes * rows;
+  box[2] = (uint32_t)(KA == 2 && box_rows == HALF ? 2 : 1);
+  r = 3;
+  if (halves == 2) {
+    dims[r] = 2;
+    strides[r - 1] = (uint64_t)half_bytes;
+    box[r] = 1;
+    ++r;
+  }
+  dims[r] = (uint64_t)nslab;
+  strides[r - 1] = (uint64_t)slab_bytes;
+  box[r] = 1;
+  ++r;
+  return make_tensor_map_bf16(m, ptr, r, dims, strides, box);
 }
 
 }  // namespace
 
-cudaError_t launch_tc2_gate_up(const Segments& sg, const CUtensorMap& tmA, const void* w_gate_up, int64_t E_w,
-                               void* h, int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s) {
-  CUtensorMap tmB, tmB64;
-  // gate_up [E][2][I][H]: 128 rows of gate or of up per CTA (full tiles), or
-  // 64 gate + 64 up rows per CTA (tail tiles)
-  const uint64_t dims[4] = {(uint64_t)H, (uint64_t)I, 2, (uint64_t)E_w};
-  const uint64_t strides[3] = {(uint64_t)H * 2, (uint64_t)I * H * 2, (uint64_t)2 * I * H * 2};
-  const uint32_t box[4] = {BK, HALF, 1, 1};
-  const uint32_t box64[4] = {BK, HALF / 2, 1, 1};
-  if (!make_tensor_map_bf16(&tmB, w_gate_up, 4, dims, strides, box)) return cudaErrorInvalidValue;
-  if (!make_tensor_map_bf16(&tmB64, w_gate_up, 4, dims, strides, box64)) return cudaErrorInvalidValue;
-  return launch_tc2<MODE_GATE_UP>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
+int tc2_katoms(int64_t K) { return katoms(K); }
+
+cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
+                               int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s) {
+  const int KA = katoms(H);
+  CUtensorMap tmA, tmB, tmB64;
+  // A: x_perm [rows, H]; gate_up [E][2][I][H]: 128 rows of gate or of up per
+  // CTA (full tiles), or 64 gate + 64 up rows per CTA and atom (tail tiles)
+  if (!map_kmajor(&tmA, A, KA, H, sg.rows_total, H * 2, 1, 0, 1, sg.rows_total * H * 2, HALF))
+    return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF))
+    return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB64, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF / 2))
+    return cudaErrorInvalidValue;
+  if (KA == 2)
+    return launch_tc2<MODE_GATE_UP, 2>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
+  return launch_tc2<MODE_GATE_UP, 1>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
 }
 
-cudaError_t launch_tc2_down(const Segments& sg, const CUtensorMap& tmA, const void* w_down, int64_t E_w, void* y,
+cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_down, int64_t E_w, void* y,
                             const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                             int num_sms, cudaStream_t s) {
-  CUtensorMap tmB;
-  // down [E][H][I], 128 of the tile's 256 output rows per CTA
-  const uint64_t dims[3] = {(uint64_t)I, (uint64_t)H, (uint64_t)E_w};
-  const uint64_t strides[2] = {(uint64_t)I * 2, (uint64_t)H * I * 2};
-  const uint32_t box[3] = {BK, HALF, 1};
-  if (!make_tensor_map_bf16(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
-  return launch_tc2<MODE_DOWN>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+  const int KA = katoms(I);
+  CUtensorMap tmA, tmB;
+  // A: h [rows, I]; down [E][H][I], 128 of the tile's 256 output rows per CTA
+  if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 1, sg.rows_total * I * 2, HALF))
+    return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF)) return cudaErrorInvalidValue;
+  if (KA == 2)
+    return launch_tc2<MODE_DOWN, 2>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+  return launch_tc2<MODE_DOWN, 1>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
 }
 
 }  // namespace stm

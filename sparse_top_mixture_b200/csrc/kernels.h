@@ -119,9 +119,12 @@ bool get_encode();
 bool make_tensor_map_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
                           const uint64_t* strides_bytes, const uint32_t* box);
 int num_sms();
-cudaError_t launch_tc2_gate_up(const Segments& sg, const CUtensorMap& tmA, const void* w_gate_up, int64_t E_w,
-                               void* h, int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s);
-cudaError_t launch_tc2_down(const Segments& sg, const CUtensorMap& tmA, const void* w_down, int64_t E_w, void* y,
+// CTA-pair GEMMs; A is the row-major operand (x_perm or h), the tensor maps
+// are built inside. K atoms per stage: tc2_katoms(K) (2 when K % 64 == 0).
+int tc2_katoms(int64_t K);
+cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
+                               int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s);
+cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_down, int64_t E_w, void* y,
                             const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                             int num_sms, cudaStream_t s);
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
@@ -129,6 +132,12 @@ cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_g
 int tc_router_splits(int64_t T, int64_t H, int64_t E);
 cudaError_t launch_tc_logits(const void* x, const void* gate_w, int64_t T, int64_t H, int64_t E, float* partial,
                              int64_t ldo, int splits, int32_t* err, cudaStream_t s);
+// Weight-gradient GEMM: out[e][m][n] = sum_{k in [koff[e], koff[e+1])}
+// AT[m][k] * BT[n][k]; AT [M][ld], BT [N][ld] bf16, koff [E+1] on the device
+// (non-decreasing multiples of 64, at most ld), out fp32 [E][M][N]; an expert
+// with an empty range gets zeros.
+cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32_t* koff, int E, int64_t M, int64_t N,
+                         float* out, int32_t* err, cudaStream_t s);
 cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down, int64_t E_w, void* y,
                            const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                            cudaStream_t s);

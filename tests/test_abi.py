@@ -129,9 +129,12 @@ def test_backward_validates_before_launching(L):
     p32 = _p(dtype="f32").c()
     assert L.moe_backward_workspace_size(ctypes.byref(p32), ctypes.byref(n)) == 0
     assert n.value >= 256
-    # bf16 problems are not supported
+    # bf16 problems have their own (larger) workspace: the fp32 size is too small for them
     pb = _p(dtype="bf16").c()
-    assert L.moe_backward(ctypes.byref(pb), ctypes.byref(w), 16, 16, 16, ctypes.byref(g), 16, n.value, None) == 2
+    nb = ctypes.c_size_t(0)
+    assert L.moe_backward_workspace_size(ctypes.byref(pb), ctypes.byref(nb)) == 0
+    assert nb.value > n.value
+    assert L.moe_backward(ctypes.byref(pb), ctypes.byref(w), 16, 16, 16, ctypes.byref(g), 16, n.value, None) == 3
     # misaligned dout
     assert L.moe_backward(ctypes.byref(p32), ctypes.byref(w), 16, 8, 16, ctypes.byref(g), 16, n.value, None) == 1
     # logit bias without a d_bias output
