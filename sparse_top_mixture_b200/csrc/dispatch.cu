@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
   // Per-warp counts of each expert (at most 32, so 16 bits) and the slot of
   // every pair: 5 KB of shared memory, small enough to sit beside a
   // persistent GEMM CTA on the same SM.
-  __shared__ uint16_t wcnt[DTHREADS / 32][kMaxExperts];
+  __shared__ __align__(16) uint16_t wcnt[DTHREADS / 32][kMaxExperts];
   __shared__ int s_pos[DTHREADS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < (DTHREADS / 32) * kMaxExperts / 2; i += DTHREADS)

@@ -383,17 +383,21 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
 // [K/64][rows][64] then addresses only elements of each row), else one.
 int katoms(int64_t K) { return K % BK == 0 ? 2 : 1; }
 
-// Tensor maps over a K-major operand of `rows` rows (row pitch K elements,
-// consecutive operand slabs `slab` bytes apart, `nslab` of them, with the
-// gate_up halves as a further dimension when `halves` is 2). Two atoms per
-// stage: dims {64, rows, K/64, (halves,) slabs}, the atom dimension 128 bytes
-// apart, box {64, box_rows, 2, 1, 1}. One atom: dims {K, rows, 1, ...}, box
-// {64, box_rows, 1, ...}, reading zeros past K.
+// Tensor maps over a K-major operand of `rows` rows (row pitch K elements),
+// with the gate_up halves as a further dimension when `halves` is 2 and
+// `nslab` consecutive operand slabs `slab_bytes` apart as the last one when
+// nslab > 0 (none for the activations). Two atoms per stage: dims {64, rows,
+// K/64, (halves,) (slabs)}, the atom dimension 128 bytes apart, box {64,
+// box_rows, 2 or 1, 1, 1}. One atom: dims {K, rows, 1, ...}, box {64,
+// box_rows, 1, ...}, reading zeros past K. The map's rank must equal the
+// rank of the TMA instruction the kernel issues on it (3 for the
+// activations, 5 for gate_up, 4 for down): a mismatch is rejected here, on
+// the host, before any launch.
 bool map_kmajor(CUtensorMap* m, const void* ptr, int KA, int64_t K, int64_t rows, int64_t row_pitch_bytes,
-                int halves, int64_t half_bytes, int64_t nslab, int64_t slab_bytes, uint32_t box_rows) {
+                int halves, int64_t half_bytes, int64_t nslab, int64_t slab_bytes, uint32_t box_rows,
+                int expect_rank) {
   uint64_t dims[5], strides[4];
   uint32_t box[5];
-  int r = 0;
   dims[0] = KA == 2 ? (uint64_t)BK : (uint64_t)K;
   box[0] = BK;
   dims[1] = (uint64_t)rows;
@@ -402,17 +406,20 @@ bool map_kmajor(CUtensorMap* m, const void* ptr, int KA, int64_t K, int64_t rows
   dims[2] = KA == 2 ? (uint64_t)(K / BK) : 1;
   strides[1] = KA == 2 ? (uint64_t)BK * 2 : (uint64_t)row_pitch_bytes * rows;
   box[2] = (uint32_t)(KA == 2 && box_rows == HALF ? 2 : 1);
-  r = 3;
+  int r = 3;
   if (halves == 2) {
     dims[r] = 2;
     strides[r - 1] = (uint64_t)half_bytes;
     box[r] = 1;
     ++r;
   }
-  dims[r] = (uint64_t)nslab;
-  strides[r - 1] = (uint64_t)slab_bytes;
-  box[r] = 1;
-  ++r;
+  if (nslab > 0) {
+    dims[r] = (uint64_t)nslab;
+    strides[r - 1] = (uint64_t)slab_bytes;
+    box[r] = 1;
+    ++r;
+  }
+  if (r != expect_rank) return false;
   return make_tensor_map_bf16(m, ptr, r, dims, strides, box);
 }
 
@@ -424,13 +431,13 @@ cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_
                                int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s) {
   const int KA = katoms(H);
   CUtensorMap tmA, tmB, tmB64;
-  // A: x_perm [rows, H]; gate_up [E][2][I][H]: 128 rows of gate or of up per
-  // CTA (full tiles), or 64 gate + 64 up rows per CTA and atom (tail tiles)
-  if (!map_kmajor(&tmA, A, KA, H, sg.rows_total, H * 2, 1, 0, 1, sg.rows_total * H * 2, HALF))
+  // A: x_perm [rows, H] (3-D loads); gate_up [E][2][I][H] (5-D loads): 128
+  // rows of gate or of up per CTA (full tiles), or 64 gate + 64 up rows per
+  // CTA and atom (tail tiles)
+  if (!map_kmajor(&tmA, A, KA, H, sg.rows_total, H * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF, 5))
     return cudaErrorInvalidValue;
-  if (!map_kmajor(&tmB, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF))
-    return cudaErrorInvalidValue;
-  if (!map_kmajor(&tmB64, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF / 2))
+  if (!map_kmajor(&tmB64, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF / 2, 5))
     return cudaErrorInvalidValue;
   if (KA == 2)
     return launch_tc2<MODE_GATE_UP, 2>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
@@ -442,10 +449,10 @@ cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_dow
                             int num_sms, cudaStream_t s) {
   const int KA = katoms(I);
   CUtensorMap tmA, tmB;
-  // A: h [rows, I]; down [E][H][I], 128 of the tile's 256 output rows per CTA
-  if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 1, sg.rows_total * I * 2, HALF))
-    return cudaErrorInvalidValue;
-  if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF)) return cudaErrorInvalidValue;
+  // A: h [rows, I] (3-D loads); down [E][H][I] (4-D loads), 128 of the
+  // tile's 256 output rows per CTA
+  if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
   if (KA == 2)
     return launch_tc2<MODE_DOWN, 2>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
   return launch_tc2<MODE_DOWN, 1>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);

@@ -1,5 +1,5 @@
 """Expert parallelism: the routed experts split over the ranks of a process
-group, token rows exchanged with all-to-all.
+group, token rows exchanged between the ranks.
 
 The pages describe the experts of one MoE layer as segments of one fused
 weight ("mstar.model.components.moe", SparseMoeBlock fused gate_up/down
@@ -13,23 +13,29 @@ identical to the one-GPU forward is taken here:
 * each rank routes and dispatches its own T tokens over all E experts with
   the library's kernels; because the dispatch sorts rows by expert, the rows
   bound for each rank form one contiguous run of x_perm, in rank order;
-* the per-expert counts go to their owners (all-to-all of E/G counts per
-  peer; one device-to-host read of the counts sizes the row exchange), then
-  the rows and their routing weights (all-to-all with those split sizes);
-* the receiver's rows arrive grouped by source rank, each source's rows
-  sorted by expert. A k = 1 dispatch keyed by the local expert id regroups
-  them into one segment per local expert (stable, so arrival order is kept
-  inside a segment), the grouped SwiGLU scales each row by its weight, and a
-  k = 1 fp32 combine puts the rows back in arrival order;
-* the reverse all-to-all returns every row to its sender, in the sender's
-  x_perm order: exactly the y_perm of the one-GPU forward (fp32 rows), so
-  the shared expert and the combine on the sender finish the layer as there.
+* the per-expert counts go to their owners (an all-to-all of E/G counts per
+  peer). Before the host reads them, everything that needs no remote count
+  is enqueued: this rank's own run of x_perm through its own experts (the
+  grouped SwiGLU over the local experts' segments of the one-GPU segment
+  table, writing those rows of y_perm in place) and the shared expert;
+* one device-to-host read of the counts then sizes the remote exchange:
+  point-to-point sends and receives, one group per exchange (rows, their
+  routing weights and their local expert ids to each other rank; the
+  weighted fp32 rows back);
+* a receiver's remote rows arrive grouped by source rank, each source's rows
+  sorted by expert, each with its local expert id. A k = 1 dispatch keyed by
+  that id regroups them into one segment per local expert (stable, so
+  arrival order is kept inside a segment), the grouped SwiGLU scales each row
+  by its weight, and a k = 1 fp32 combine puts the rows back in arrival
+  order;
+* the rows come back to their senders in the sender's x_perm order: with the
+  local rows, exactly the y_perm of the one-GPU forward (fp32 rows), so the
+  combine finishes the layer as there.
 
 Every per-row result is the same arithmetic as on one GPU; only where a row
-sits in a GEMM tile changes. The collectives are torch.distributed
-all_to_all_single calls (NCCL over NVLink on GPUs). This module holds the
-host orchestration only: every step of the layer's arithmetic runs in the
-library's CUDA kernels.
+sits in a GEMM tile changes. The collectives are torch.distributed calls
+(NCCL over NVLink on GPUs). This module holds the host orchestration only:
+every step of the layer's arithmetic runs in the library's CUDA kernels.
 """
 
 from __future__ import annotations
@@ -52,15 +58,39 @@ def send_splits(counts: Sequence[int], world: int) -> List[int]:
     return [int(v) for v in c.reshape(world, -1).sum(axis=1)]
 
 
-def receive_layout(recv_counts: np.ndarray) -> Tuple[List[int], np.ndarray]:
-    """From the counts received [G, E/G] (row s: source rank s's rows per
-    local expert), the rows received from each source and the local expert
-    id of every received row in arrival order (source-major, then expert)."""
+def local_expert_ids(global_ids: torch.Tensor, owner: int, experts_per_rank: int) -> torch.Tensor:
+    """The owner's local expert id of each row sent to it (int64)."""
+    return global_ids - owner * experts_per_rank
+
+
+@dataclasses.dataclass
+class ExchangePlan:
+    """Where each peer's rows sit: send_off[s] .. send_off[s+1] in this rank's
+    x_perm (and y_perm) go to rank s; recv_off[s] .. recv_off[s] + recvs[s] of
+    the receive buffers come from rank s (remote peers only, in rank order)."""
+    send_off: List[int]
+    recvs: List[int]
+    recv_off: Dict[int, int]
+    remote: List[int]
+    n_recv: int
+
+
+def exchange_plan(counts: Sequence[int], recv_counts: np.ndarray, rank: int) -> ExchangePlan:
+    """From this rank's per-expert counts [E] and the counts its peers send it
+    [G, E/G] (row s: rank s's rows per local expert)."""
     rc = np.asarray(recv_counts, dtype=np.int64)
-    splits = [int(v) for v in rc.sum(axis=1)]
-    local = np.arange(rc.shape[1], dtype=np.int64)
-    ids = np.concatenate([np.repeat(local, row) for row in rc]) if rc.size else np.zeros(0, np.int64)
-    return splits, ids.astype(np.int64)
+    G = rc.shape[0]
+    sends = send_splits(counts, G)
+    send_off = [0]
+    for v in sends:
+        send_off.append(send_off[-1] + v)
+    recvs = [int(v) for v in rc.sum(axis=1)]
+    remote = [s for s in range(G) if s != rank]
+    recv_off, acc = {}, 0
+    for s in remote:
+        recv_off[s] = acc
+        acc += recvs[s]
+    return ExchangePlan(send_off, recvs, recv_off, remote, acc)
 
 
 class WorkspacePool:
@@ -112,43 +142,93 @@ class ExpertParallelMoE:
 
         dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
+    def _exchange(self, sends, recvs) -> None:
+        """One group of point-to-point transfers: ``sends`` and ``recvs`` are
+        lists of (peer, tensor); nothing is sent to or received from this
+        rank itself."""
+        import torch.distributed as dist
+
+        ops = [dist.P2POp(dist.isend, t, dist.get_global_rank(self.group, peer) if self.group else peer, self.group)
+               for peer, t in sends if t.numel()]
+        ops += [dist.P2POp(dist.irecv, t, dist.get_global_rank(self.group, peer) if self.group else peer, self.group)
+                for peer, t in recvs if t.numel()]
+        if ops:
+            for req in dist.batch_isend_irecv(ops):
+                req.wait()
+
+    def _host_counts(self, counts: torch.Tensor, recv_counts: torch.Tensor):
+        """The one device-to-host read of the layer: this rank's counts and the
+        counts its peers send it (synchronises the stream)."""
+        self.trace.append("host_counts")
+        return counts.cpu().numpy(), recv_counts.cpu().numpy().reshape(self.world, self.E_local)
+
     def forward(self, x: torch.Tensor):
         """out [T,H], routing_weights [T,k] fp32, selected_experts [T,k] int64."""
         p, w = self.p, self.w
+        r, G, El = self.rank, self.world, self.E_local
         dev = x.device
+        self.trace = []
         gate = w.get("shared_gate") if p.shared == "sigmoid_gated" else None
         ws = self.pool.get(p)
         rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate, ws=ws)
         d = dispatch(p, sel, x, ws=ws)
 
-        # counts to the experts' owners; one host read sizes the row exchange
+        # counts to the experts' owners
         counts = d["counts"].to(torch.int64)
         recv_counts = torch.empty_like(counts)
         self._a2a(recv_counts, counts, None, None)
-        sends = send_splits(counts.cpu().numpy(), self.world)
-        recvs, local_ids = receive_layout(recv_counts.cpu().numpy().reshape(self.world, self.E_local))
-        n_send, n_recv = sum(sends), sum(recvs)
 
-        # rows (x_perm order) and their routing weights to the owners
-        x_recv = torch.empty(n_recv, p.H, dtype=x.dtype, device=dev)
-        self._a2a(x_recv, d["x_perm"][:n_send], recvs, sends)
-        w_sorted = rw.reshape(-1)[d["sorted_pairs"][:n_send].long()]
-        w_recv = torch.empty(n_recv, dtype=torch.float32, device=dev)
-        self._a2a(w_recv, w_sorted, recvs, sends)
-
-        y_recv = self._local_experts(x_recv, w_recv, local_ids)
-
-        # weighted fp32 rows back to their senders, in x_perm order
-        y_perm = torch.zeros(p.T * p.k, p.H, dtype=torch.float32, device=dev)
-        self._a2a(y_perm[:n_send], y_recv, sends, recvs)
+        # Work that needs no remote count, enqueued before the host read: this
+        # rank's own rows through its own experts (rows of y_perm in place) ...
+        # (as a problem of T*k one-slot rows over the E/G local experts: the same
+        # x_perm rows, routing weights and sorted pair indices)
+        pl = dataclasses.replace(p, T=p.T * p.k, k=1, E=El, I_shared=0, shared="none", bias_mode="none")
+        own_offsets = d["offsets"][r * El:(r + 1) * El + 1]
+        y_perm = grouped_swiglu(pl, d["x_perm"], own_offsets, w["gate_up"], w["down"], rw.view(-1, 1),
+                                d["sorted_pairs"], ws=self.pool.get(pl))
+        self.trace.append("local_experts")
+        if x.is_cuda:  # marks the local GEMM's place in the stream (tests check it ran before the host read)
+            self.local_done = torch.cuda.Event()
+            self.local_done.record()
+        # ... and the shared expert
         shared = None
         if p.shared != "none":
             shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma, ws=ws)
+            self.trace.append("shared_expert")
+
+        # the host read sizes the remote exchange
+        plan = exchange_plan(*self._host_counts(counts, recv_counts), r)
+        send_off, recvs, recv_off, remote, n_recv = plan.send_off, plan.recvs, plan.recv_off, plan.remote, plan.n_recv
+
+        # rows (x_perm order), their routing weights and local expert ids to the owners
+        q_sorted = d["sorted_pairs"][:send_off[-1]].long()
+        w_sorted = rw.reshape(-1)[q_sorted]
+        e_sorted = sel.reshape(-1)[q_sorted]
+        x_recv = torch.empty(n_recv, p.H, dtype=x.dtype, device=dev)
+        w_recv = torch.empty(n_recv, dtype=torch.float32, device=dev)
+        id_recv = torch.empty(n_recv, dtype=torch.int64, device=dev)
+        out_rows, out_w, out_id, in_rows, in_w, in_id = [], [], [], [], [], []
+        for s in remote:
+            a, b = send_off[s], send_off[s + 1]
+            out_rows.append((s, d["x_perm"][a:b]))
+            out_w.append((s, w_sorted[a:b].contiguous()))
+            out_id.append((s, local_expert_ids(e_sorted[a:b], s, El).contiguous()))
+            c, n = recv_off[s], recvs[s]
+            in_rows.append((s, x_recv[c:c + n]))
+            in_w.append((s, w_recv[c:c + n]))
+            in_id.append((s, id_recv[c:c + n]))
+        self._exchange(out_rows + out_w + out_id, in_rows + in_w + in_id)
+
+        y_recv = self._local_experts(x_recv, w_recv, id_recv)
+
+        # weighted fp32 rows back to their senders, into y_perm in x_perm order
+        self._exchange([(s, y_recv[recv_off[s]:recv_off[s] + recvs[s]]) for s in remote],
+                       [(s, y_perm[send_off[s]:send_off[s + 1]]) for s in remote])
         return combine(p, y_perm, d["pair_pos"], shared), rw, sel
 
     __call__ = forward
 
-    def _local_experts(self, x_recv: torch.Tensor, w_recv: torch.Tensor, local_ids: np.ndarray) -> torch.Tensor:
+    def _local_experts(self, x_recv: torch.Tensor, w_recv: torch.Tensor, id_recv: torch.Tensor) -> torch.Tensor:
         """The received rows through this rank's experts, weighted, fp32 [n, H]
         in arrival order."""
         p = self.p
@@ -156,9 +236,8 @@ class ExpertParallelMoE:
         if n == 0:
             return torch.zeros(0, p.H, dtype=torch.float32, device=x_recv.device)
         pr = dataclasses.replace(p, T=n, E=self.E_local, k=1, I_shared=0, bias_mode="none", shared="none")
-        ids = torch.from_numpy(local_ids).to(x_recv.device).view(n, 1)
         ws = self.pool.get(pr)
-        d = dispatch(pr, ids, x_recv, ws=ws)
+        d = dispatch(pr, id_recv.view(n, 1), x_recv, ws=ws)
         y = grouped_swiglu(pr, d["x_perm"], d["offsets"], self.w["gate_up"], self.w["down"], w_recv.view(n, 1),
                            d["sorted_pairs"], ws=ws)
         return combine(dataclasses.replace(pr, dtype="f32"), y, d["pair_pos"], None)

@@ -1,13 +1,15 @@
 """Expert parallelism's host orchestration (sparse_top_mixture_b200/expert_parallel.py)
 with gloo ranks on the CPU.
 
-The split arithmetic is checked by brute force. The whole exchange (counts,
-rows and weights out, the receiver's regrouping by local expert, rows back,
-the combine) runs on 1, 2 and 4 gloo ranks with the library's stage calls
-replaced, inside each test process only, by CPU stand-ins with the same
-contracts built from the oracle; each rank's output must equal the oracle's
-one-process forward of its own tokens with all experts. A planted mistake in
-the receiver's layout must break that equality."""
+The exchange plan (which rows go to and come from which rank) is checked by
+brute force. The whole exchange (counts; this rank's own rows through its
+experts before the host read; rows, weights and local expert ids to the other
+ranks, the receiver's regrouping by local expert, rows back; the combine)
+runs on 1, 2 and 4 gloo ranks with the library's stage calls replaced,
+inside each test process only, by CPU stand-ins with the same contracts built
+from the oracle; each rank's output must equal the oracle's one-process
+forward of its own tokens with all experts. A planted mistake in the local
+expert ids sent with the rows must break that equality."""
 
 import os
 import socket
@@ -38,15 +40,30 @@ def test_send_splits_sum_each_ranks_experts():
         ep.send_splits(counts, 3)
 
 
-def test_receive_layout_brute_force():
+def test_exchange_plan_brute_force():
     rng = np.random.default_rng(0)
     for _ in range(50):
-        G, El = rng.integers(1, 5), rng.integers(1, 5)
+        G, El = int(rng.integers(1, 5)), int(rng.integers(1, 5))
+        rank = int(rng.integers(0, G))
+        counts = rng.integers(0, 4, size=G * El)
         rc = rng.integers(0, 4, size=(G, El))
-        splits, ids = ep.receive_layout(rc)
-        want = [e for s in range(G) for e in range(El) for _ in range(rc[s, e])]
-        assert ids.tolist() == want
-        assert splits == [int(v) for v in rc.sum(axis=1)]
+        plan = ep.exchange_plan(counts, rc, rank)
+        # rank s's rows in x_perm: the rows of experts [s El, (s+1) El), after those of lower ranks
+        for s in range(G):
+            assert plan.send_off[s] == int(counts[:s * El].sum())
+            assert plan.send_off[s + 1] - plan.send_off[s] == int(counts[s * El:(s + 1) * El].sum())
+        assert plan.remote == [s for s in range(G) if s != rank]
+        # receive buffers: remote sources in rank order, each source's rows contiguous
+        at = 0
+        for s in plan.remote:
+            assert plan.recv_off[s] == at and plan.recvs[s] == int(rc[s].sum())
+            at += int(rc[s].sum())
+        assert plan.n_recv == at
+
+
+def test_local_expert_ids():
+    g = torch.tensor([8, 9, 11, 15])
+    assert ep.local_expert_ids(g, 2, 4).tolist() == [0, 1, 3, 7]
 
 
 CASES = {
@@ -71,13 +88,8 @@ def _worker(rank, world, port, case, planted, q, skew=False):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         stage_standins.install(ep)
-        if planted:  # receiver layout in expert-major order instead of arrival order
-            right = ep.receive_layout
-
-            def wrong(rc):
-                splits, ids = right(rc)
-                return splits, np.sort(ids, kind="stable")
-            ep.receive_layout = wrong
+        if planted:  # rows sent with their owner's local expert ids in reverse order
+            ep.local_expert_ids = lambda g, owner, El: (owner + 1) * El - 1 - g
         cfg = workloads.CONFIGS["tiny_fp32"].replace(name="ep", **CASES[case])
         full = workloads.generate(cfg, "cpu")
         if skew:  # a selection bias that sends every pair to rank 0's experts
@@ -129,7 +141,7 @@ def test_expert_parallel_matches_one_process_oracle(world, case):
         assert rel <= 1e-6, f"rank {rank}: rel L2 {rel:.3e}"
 
 
-def test_planted_receive_layout_mistake_is_caught():
+def test_planted_local_id_mistake_is_caught():
     res = _run(2, "sigmoid_gated", planted=True)
     assert max(rel for _, rel, _, _ in res) > 1e-3
 
