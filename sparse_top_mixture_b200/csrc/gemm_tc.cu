@@ -79,6 +79,7 @@ struct Args {
   int64_t rows_total;
   int32_t M;        // WGRAD: output rows per expert
   int32_t m_tiles;  // WGRAD: 128-row tiles of M
+  int32_t n_mma;    // LOGITS: MMA N (the expert count rounded up to 16); else UMMA_N
 };
 
 struct __align__(8) Ctl {
@@ -212,7 +213,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, args.err, 1)) { ok = false; break; }
           uint8_t* sa = base + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(&ctl->full[stage], STAGE_BYTES);
+          // the router's B box has only n_mma rows (its N is the expert count)
+          mbar_arrive_expect_tx(&ctl->full[stage],
+                                MODE == MODE_LOGITS ? (uint32_t)(A_BYTES + args.n_mma * BK * 2) : STAGE_BYTES);
           const int k0 = kt * BK;
           tma_load_2d(sa, &tmA, &ctl->full[stage], k0, tc.row0);
           if (MODE == MODE_GATE_UP) {
@@ -244,7 +247,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
-        const uint32_t idesc = tc.m64 ? kIdesc64 : kIdesc128;
+        const uint32_t idesc = MODE == MODE_LOGITS ? make_idesc(tc.m64 ? 64 : 128, args.n_mma)
+                                                   : (tc.m64 ? kIdesc64 : kIdesc128);
         for (int kt = tc.kt0; kt < tc.kt1; ++kt) {
           if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, args.err, 3)) { ok = false; break; }
           tc_fence_after();
@@ -385,6 +389,7 @@ cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensor
   a.rows_total = sg.rows_total;
   a.M = 0;
   a.m_tiles = 0;
+  a.n_mma = MODE == MODE_LOGITS ? (int32_t)std::min<int64_t>(UMMA_N, round_up(N, 16)) : UMMA_N;
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM + nseg) * a.n_tiles * a.k_splits;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
@@ -429,6 +434,7 @@ cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32
   a.rows_total = ld;  // K extent of the operands
   a.M = (int32_t)M;
   a.m_tiles = (int32_t)ceil_div(M, BM);
+  a.n_mma = UMMA_N;
   const int64_t tiles = (int64_t)E * a.m_tiles * a.n_tiles;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles));
   tc_grouped_gemm_kernel<MODE_WGRAD><<<grid, NTHREADS, kSmemBytes, s>>>(tmA, tmB, a);
@@ -547,9 +553,11 @@ cudaError_t launch_tc_logits(const void* x, const void* gate_w, int64_t T, int64
     if (!make_tensor_map_bf16(&tmA, x, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
+    // N of the router's MMA: the expert count rounded up to 16 (at most 256);
+    // the B box has that many rows (zero fill past E)
     const uint64_t dims[3] = {(uint64_t)H, (uint64_t)E, 1};
     const uint64_t strides[2] = {(uint64_t)H * 2, (uint64_t)E * H * 2};
-    const uint32_t box[3] = {BK, UMMA_N, 1};
+    const uint32_t box[3] = {BK, (uint32_t)std::min<int64_t>(UMMA_N, round_up(E, 16)), 1};
     if (!make_tensor_map_bf16(&tmB, gate_w, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   Segments sg{nullptr, 1, (int32_t)T, T};
