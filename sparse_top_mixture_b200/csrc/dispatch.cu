@@ -211,10 +211,12 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
 }
 
 // out[t] = sum_j y_perm[pair_pos[t*k+j]] + shared_out[t]: fp32 rows, summed in
-// slot order in fp32, rounded once to the output type. Work units are the
-// 16-byte column vectors of all tokens, flattened and strided over a grid of
-// a few CTAs per SM, so every SM gets the same share (no partial last wave);
-// consecutive threads take consecutive vectors of one row.
+// slot order in fp32, rounded once to the output type. A work unit is one
+// token's 4 KB column chunk (256 threads x one 16-byte vector of each of its
+// k rows), so each y row is read as 4 KB contiguous runs; units are strided
+// over a grid of a few CTAs per SM, so every SM gets the same share. A
+// thread loads up to eight slots' pair positions and then issues those rows'
+// loads together, before adding them in slot order.
 constexpr int CTHREADS = 256;
 
 template <typename T>
@@ -223,22 +225,31 @@ __global__ void __launch_bounds__(CTHREADS) combine_kernel(const float* __restri
                                                            const float* __restrict__ shared_out,
                                                            T* __restrict__ out, int64_t Tn, int H, int k) {
   const int nvec = H / 4;
-  const int64_t units = Tn * nvec;
-  const int64_t stride = (int64_t)gridDim.x * CTHREADS;
-  for (int64_t u = (int64_t)blockIdx.x * CTHREADS + threadIdx.x; u < units; u += stride) {
-    const int64_t t = u / nvec;
-    const int v = (int)(u - t * nvec);
+  const int chunks = (nvec + CTHREADS - 1) / CTHREADS;
+  const int64_t units = Tn * chunks;
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int64_t t = u / chunks;
+    const int v = (int)(u - t * chunks) * CTHREADS + threadIdx.x;
+    if (v >= nvec) continue;
     const int32_t* pp = pair_pos + t * k;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-      const int p = __ldg(pp + j);
-      if (p < 0) continue;
-      const float4 y = __ldcs(reinterpret_cast<const float4*>(y_perm + (int64_t)p * H) + v);
-      acc.x += y.x;
-      acc.y += y.y;
-      acc.z += y.z;
-      acc.w += y.w;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int p[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) p[j] = j0 + j < k ? __ldg(pp + j0 + j) : -1;
+      float4 y[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        y[j] = p[j] >= 0 ? __ldcs(reinterpret_cast<const float4*>(y_perm + (int64_t)p[j] * H) + v)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (p[j] < 0) continue;  // skipped pairs and slots past k add nothing
+        acc.x += y[j].x;
+        acc.y += y[j].y;
+        acc.z += y[j].z;
+        acc.w += y[j].w;
+      }
     }
     if (shared_out != nullptr) {
       const float4 y = __ldcs(reinterpret_cast<const float4*>(shared_out + t * H) + v);
@@ -296,8 +307,8 @@ cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, i
 
 cudaError_t launch_combine(int dtype, const float* y_perm, const int32_t* pair_pos, const float* shared_out,
                            void* out, int64_t T, int64_t H, int64_t k, cudaStream_t s) {
-  const int64_t units = T * (H / 4);
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, CTHREADS), 148 * 8));
+  const int64_t units = T * ceil_div(H / 4, CTHREADS);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, 148 * 8));
   if (dtype == 0)
     combine_kernel<float><<<grid, CTHREADS, 0, s>>>(y_perm, pair_pos, shared_out, (float*)out, T, (int)H, (int)k);
   else

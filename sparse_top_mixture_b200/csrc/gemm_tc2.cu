@@ -16,10 +16,9 @@
 //   - each CTA's epilogue drains its own TMEM rows and arrives on the
 //     leader's accumulator-empty barrier.
 // No TMA multicast is used: every CTA fetches its own tiles.
-// When K is a multiple of 64, a stage holds two 64-element K atoms of A and
-// of B (a 3-D tensor-map view [K/64][rows][64] whose box spans both atoms),
-// so each TMA operation moves 32 KB, a stage carries eight MMAs and the ring
-// is 3 stages of 64 KB per CTA; otherwise one atom per stage, 6 stages.
+// The kernel takes the number of 64-element K atoms per stage as a template
+// parameter (two atoms: a 3-D tensor-map view [K/64][rows][64] whose box
+// spans both); it is launched with one (see kAtomsPerStage).
 //
 // Used when segments average at least 192 rows. A row tile is 256 rows of one
 // segment. A tile with at most 128 rows left (a segment's tail) runs as an
@@ -73,7 +72,9 @@ struct Ring {
   static_assert(STAGES >= 2 && STAGES <= MAX_STAGES, "ring depth");
 };
 
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
+// MODE_DOWN_COMBINE: down of a one-segment (shared expert) problem whose
+// epilogue adds each token's routed rows and writes the bf16 output.
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_DOWN_COMBINE = 2 };
 
 struct Args2 {
   const int32_t* offsets;
@@ -88,6 +89,9 @@ struct Args2 {
   const int32_t* scale_idx;
   int32_t* err;
   int64_t rows_total;
+  const float* y_rows;      // DOWN_COMBINE: routed fp32 rows [*, N]
+  const int32_t* pair_pos;  // DOWN_COMBINE: [rows * k], -1 for a skipped pair
+  int32_t k;                // DOWN_COMBINE: slots per token
 };
 
 struct __align__(8) Ctl2 {
@@ -112,7 +116,7 @@ struct __align__(8) Ctl2 {
 // for the dispatch kernels that run beside a shared expert's GEMM.
 template <int MODE>
 constexpr int epi_bytes2() {
-  return MODE == MODE_DOWN ? 4 * kStageFloatsPerWarp * 4 : 0;
+  return MODE != MODE_GATE_UP ? 4 * kStageFloatsPerWarp * 4 : 0;
 }
 template <int MODE>
 constexpr size_t smem_bytes2() {
@@ -120,6 +124,7 @@ constexpr size_t smem_bytes2() {
 }
 static_assert(smem_bytes2<MODE_GATE_UP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 static_assert(smem_bytes2<MODE_DOWN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
+static_assert(smem_bytes2<MODE_DOWN_COMBINE>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
@@ -315,6 +320,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           epilogue_swiglu(tbase, 0, 128, 4, orow0, args.ldo, nrows, tc.n_idx * 128, args.N, lane);
         else
           epilogue_swiglu(tbase, 0, 64, 2, orow0, args.ldo, nrows, tc.n_idx * 128 + half * 64, args.N, lane);
+      } else if (MODE == MODE_DOWN_COMBINE) {
+        float sc = 1.f;
+        if (lane < nrows && args.row_scale != nullptr) sc = args.row_scale[row];
+        __nv_bfloat16* orow0 = reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row_w0 * args.ldo;
+        const int32_t* pp0 = args.pair_pos + (int64_t)row_w0 * args.k;
+        if (!tc.tail)
+          epilogue_scale_combine_bf16(tbase, 8, sc, stage, orow0, args.y_rows, pp0, args.k, args.ldo, nrows,
+                                      tc.n_idx * UMMA_N, args.N, lane);
+        else
+          epilogue_scale_combine_bf16(tbase, 4, sc, stage, orow0, args.y_rows, pp0, args.k, args.ldo, nrows,
+                                      tc.n_idx * UMMA_N + half * 128, args.N, lane);
       } else {
         float sc = 1.f;
         if (lane < nrows && args.row_scale != nullptr)
@@ -332,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       // visible to the leader first); gate_up measured faster with a
       // cluster-scope release after its direct bf16 stores.
       if (lane == 0) {
-        if (MODE == MODE_DOWN) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+        if (MODE != MODE_GATE_UP) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
         else mbar_arrive_remote_release(acc ? tempty_leader1 : tempty_leader0);
       }
       acc ^= 1;
@@ -353,7 +369,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 template <int MODE, int KA>
 cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmB64,
                        int64_t N, int64_t K, void* out, int64_t ldo, const float* row_scale,
-                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s) {
+                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s,
+                       const float* y_rows = nullptr, const int32_t* pair_pos = nullptr, int k = 0) {
   static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance
   static cudaError_t attr_status[kSmemAttrDevices];
   const void* kernel = reinterpret_cast<const void*>(tc2_grouped_gemm_kernel<MODE, KA>);
@@ -372,6 +389,9 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   a.scale_idx = scale_idx;
   a.err = err;
   a.rows_total = sg.rows_total;
+  a.y_rows = y_rows;
+  a.pair_pos = pair_pos;
+  a.k = k;
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM2 + nseg) * a.n_tiles;
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms / 2, max_tiles));
@@ -379,9 +399,14 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   return cudaGetLastError();
 }
 
-// K atoms per stage: two when K splits into whole 64-element atoms (the view
-// [K/64][rows][64] then addresses only elements of each row), else one.
-int katoms(int64_t K) { return K % BK == 0 ? 2 : 1; }
+// K atoms per stage. Two atoms per stage (3 stages of 64 KB: half the TMA
+// operations and barrier round trips for the same bytes in flight; the view
+// [K/64][rows][64], for K a multiple of 64) were measured against one atom
+// per stage (6 stages of 32 KB): no gain on the DSV4- and Zipf-shaped
+// problems and 3-5% slower on the Qwen3-shaped one (its 12-32-step K loops),
+// so the kernels are launched with one atom per stage; the kernel and the map
+// builder keep the atom count as a parameter.
+constexpr int kAtomsPerStage = 1;
 
 // Tensor maps over a K-major operand of `rows` rows (row pitch K elements),
 // with the gate_up halves as a further dimension when `halves` is 2 and
@@ -425,11 +450,10 @@ bool map_kmajor(CUtensorMap* m, const void* ptr, int KA, int64_t K, int64_t rows
 
 }  // namespace
 
-int tc2_katoms(int64_t K) { return katoms(K); }
 
 cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                                int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s) {
-  const int KA = katoms(H);
+  constexpr int KA = kAtomsPerStage;
   CUtensorMap tmA, tmB, tmB64;
   // A: x_perm [rows, H] (3-D loads); gate_up [E][2][I][H] (5-D loads): 128
   // rows of gate or of up per CTA (full tiles), or 64 gate + 64 up rows per
@@ -439,23 +463,31 @@ cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_
     return cudaErrorInvalidValue;
   if (!map_kmajor(&tmB64, w_gate_up, KA, H, I, H * 2, 2, I * H * 2, E_w, 2 * I * H * 2, HALF / 2, 5))
     return cudaErrorInvalidValue;
-  if (KA == 2)
-    return launch_tc2<MODE_GATE_UP, 2>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
-  return launch_tc2<MODE_GATE_UP, 1>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
+  return launch_tc2<MODE_GATE_UP, KA>(sg, tmA, tmB, tmB64, I, H, h, I, nullptr, nullptr, err, num_sms, s);
 }
 
 cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_down, int64_t E_w, void* y,
                             const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                             int num_sms, cudaStream_t s) {
-  const int KA = katoms(I);
+  constexpr int KA = kAtomsPerStage;
   CUtensorMap tmA, tmB;
   // A: h [rows, I] (3-D loads); down [E][H][I] (4-D loads), 128 of the
   // tile's 256 output rows per CTA
   if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
   if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
-  if (KA == 2)
-    return launch_tc2<MODE_DOWN, 2>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
-  return launch_tc2<MODE_DOWN, 1>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+  return launch_tc2<MODE_DOWN, KA>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+}
+
+cudaError_t launch_tc2_down_combine(const Segments& sg, const void* A, const void* w_down, const float* gamma,
+                                    const float* y_rows, const int32_t* pair_pos, int64_t k, void* out, int64_t H,
+                                    int64_t I, int32_t* err, int num_sms, cudaStream_t s) {
+  if (sg.offsets != nullptr) return cudaErrorInvalidValue;  // one segment: row = token
+  constexpr int KA = kAtomsPerStage;
+  CUtensorMap tmA, tmB;
+  if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, 1, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
+  return launch_tc2<MODE_DOWN_COMBINE, KA>(sg, tmA, tmB, tmB, H, I, out, H, gamma, nullptr, err, num_sms, s, y_rows,
+                                           pair_pos, (int)k);
 }
 
 }  // namespace stm

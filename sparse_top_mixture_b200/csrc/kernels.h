@@ -120,13 +120,19 @@ bool make_tensor_map_bf16(CUtensorMap* m, const void* ptr, int rank, const uint6
                           const uint64_t* strides_bytes, const uint32_t* box);
 int num_sms();
 // CTA-pair GEMMs; A is the row-major operand (x_perm or h), the tensor maps
-// are built inside. K atoms per stage: tc2_katoms(K) (2 when K % 64 == 0).
-int tc2_katoms(int64_t K);
+// are built inside.
 cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                                int64_t I, int64_t H, int32_t* err, int num_sms, cudaStream_t s);
 cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_down, int64_t E_w, void* y,
                             const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                             int num_sms, cudaStream_t s);
+// Down GEMM of a one-segment problem (the shared expert, row = token) whose
+// epilogue does the combine: out[t] (bf16) = sum over slots s of
+// y_rows[pair_pos[t*k+s]] (fp32, slot order) + gamma[t] * (h[t] . w_down^T),
+// rounded once; gamma may be NULL (1). CTA pairs only (T >= 192 rows).
+cudaError_t launch_tc2_down_combine(const Segments& sg, const void* A, const void* w_down, const float* gamma,
+                                    const float* y_rows, const int32_t* pair_pos, int64_t k, void* out, int64_t H,
+                                    int64_t I, int32_t* err, int num_sms, cudaStream_t s);
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                               int64_t I, int64_t H, int32_t* err, cudaStream_t s);
 int tc_router_splits(int64_t T, int64_t H, int64_t E);

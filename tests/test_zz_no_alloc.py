@@ -60,9 +60,13 @@ def test_no_alloc_dispatch_skips_bad_ids_without_a_flag():
     assert stm.read_device_error(ws) == stm.DEVERR_BAD_EXPERT_ID  # the workspace call flags it
     pp = got["pair_pos"].cpu().numpy()
     assert pp[7 * p.k + 1] == -1 and pp[20 * p.k] == -1
-    assert int(got["offsets"][-1]) == p.T * p.k - 2
-    for key in KEYS:
+    used = int(got["offsets"][-1])
+    assert used == p.T * p.k - 2
+    # positions past the dispatched pairs are not written by either call
+    for key in ("counts", "offsets", "pair_pos"):
         assert torch.equal(got[key], ref[key]), key
+    assert torch.equal(got["sorted_pairs"][:used], ref["sorted_pairs"][:used])
+    assert torch.equal(got["x_perm"][:used], ref["x_perm"][:used])
 
 
 def test_no_alloc_dispatch_empty_batch():
