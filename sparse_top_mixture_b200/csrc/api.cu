@@ -154,24 +154,6 @@ moe_status do_shared(const moe_problem& p, const Layout& L, const void* x, const
   return MOE_OK;
 }
 
-// The shared expert's gate_up alone (its h rows in the workspace).
-moe_status do_shared_gate_up(const moe_problem& p, const Layout& L, const void* x, const void* sgu, void* ws,
-                             cudaStream_t s) {
-  Segments sg{nullptr, 1, (int32_t)p.T, p.T};
-  MOE_CUDA(launch_tc_gate_up(sg, x, sgu, 1, at<void>(ws, L.h_shared), p.I_shared, p.H, at<int32_t>(ws, L.header), s));
-  return MOE_OK;
-}
-
-// The shared expert's down GEMM with the combine in its epilogue: out =
-// round(sum of each token's routed fp32 rows + gamma * shared row).
-moe_status do_shared_down_combine(const moe_problem& p, const Layout& L, const void* sdn, const float* gamma,
-                                  const float* y_perm, const int32_t* pair_pos, void* out, void* ws, cudaStream_t s) {
-  Segments sg{nullptr, 1, (int32_t)p.T, p.T};
-  MOE_CUDA(launch_tc2_down_combine(sg, at<void>(ws, L.h_shared), sdn, gamma, y_perm, pair_pos, p.k, out, p.H,
-                                   p.I_shared, at<int32_t>(ws, L.header), num_sms(), s));
-  return MOE_OK;
-}
-
 moe_status validate_weights(const moe_problem& p, const moe_weights* w) {
   if (w == nullptr) return MOE_ERR_INVALID_ARGUMENT;
   if (!ok_ptr(w->gate_w) || !ok_ptr(w->gate_up) || !ok_ptr(w->down)) return MOE_ERR_INVALID_ARGUMENT;
@@ -190,17 +172,6 @@ bool shared_overlaps(const moe_problem& p) {
   if (p.shared == MOE_SHARED_NONE) return false;
   const int64_t tiles = ceil_div(p.T, 128) * ceil_div(p.I_shared, 128);
   return tiles <= 74;
-}
-
-// Whether the forward does the combine in the shared expert's down GEMM: a
-// bf16 shared expert too large to overlap the routed GEMMs (see
-// shared_overlaps) whose down GEMM runs on CTA pairs. Its gate_up then runs
-// beside the dispatch (or, on one stream, after the routed down), and its
-// down runs last, reading the routed rows.
-bool fused_combine(const moe_problem& p) {
-  if (p.shared == MOE_SHARED_NONE || p.dtype != MOE_DTYPE_BF16 || shared_overlaps(p)) return false;
-  Segments sh{nullptr, 1, (int32_t)p.T, p.T};
-  return tc_gemm_variant(sh, true) == 2;
 }
 
 // RAII pair of fork / join events for the two-stream forward.
@@ -247,14 +218,9 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   //    routed GEMMs; it runs on `aux` after the route (whose top-k kernel
   //    already computed the gate) beside the dispatch kernels, which fit next
   //    to its persistent CTAs, and `s` waits for it before the routed gate_up.
-  //    When its down GEMM runs on CTA pairs it does the combine in its
-  //    epilogue (fused_combine): then only its gate_up runs on `aux`, and the
-  //    down runs on `s` after the routed down. On one stream the fused
-  //    forward runs the shared gate_up after the routed down.
   const bool use_aux = has_shared && aux != nullptr && aux != s;
   const bool small_shared = use_aux && shared_overlaps(*p);
   const bool large_shared = use_aux && !small_shared;
-  const bool fused = fused_combine(*p);
   float* gamma = at<float>(ws, L.gamma);
   int32_t* counts = at<int32_t>(ws, L.counts);
   int32_t* offsets = at<int32_t>(ws, L.offsets);
@@ -286,12 +252,12 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   if (large_shared) {
     MOE_CUDA(cudaEventRecord(evp.fork, s));
     MOE_CUDA(cudaStreamWaitEvent(aux, evp.fork, 0));
-    if (fused) MOE_TRY(do_shared_gate_up(*p, L, x, w->shared_gate_up, ws, aux));
-    else MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, shared_gamma, shared_out, ws, aux));
+    MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, shared_gamma, shared_out, ws, aux));
     MOE_CUDA(cudaEventRecord(evp.join, aux));
   }
   // With a large shared expert on `aux`, the dispatch stage's interval ends
-  // when both the dispatch and the shared expert's work there are done.
+  // when both the dispatch and the shared expert are done, and the shared
+  // stage is empty.
   MOE_TRY(mark(MOE_STAGE_DISPATCH));
   MOE_TRY(do_dispatch(*p, L, selected, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws, s));
   if (large_shared) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
@@ -300,17 +266,12 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   MOE_TRY(mark(MOE_STAGE_DOWN));
   MOE_TRY(do_grouped_down(*p, L, offsets, w->down, weights, sorted_pairs, y_perm, ws, s));
   MOE_TRY(mark(MOE_STAGE_SHARED));
-  if (has_shared && !use_aux) {
-    if (fused) MOE_TRY(do_shared_gate_up(*p, L, x, w->shared_gate_up, ws, s));
-    else MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, shared_gamma, shared_out, ws, s));
-  }
+  if (has_shared && !use_aux)
+    MOE_TRY(do_shared(*p, L, x, w->shared_gate_up, w->shared_down, shared_gamma, shared_out, ws, s));
   if (small_shared) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
   MOE_TRY(mark(MOE_STAGE_COMBINE));
-  if (fused)
-    MOE_TRY(do_shared_down_combine(*p, L, w->shared_down, shared_gamma, (const float*)y_perm, pair_pos, out, ws, s));
-  else
-    MOE_CUDA(launch_combine(p->dtype, (const float*)y_perm, pair_pos, (const float*)shared_out, out, p->T, p->H,
-                            p->k, s));
+  MOE_CUDA(launch_combine(p->dtype, (const float*)y_perm, pair_pos, (const float*)shared_out, out, p->T, p->H,
+                          p->k, s));
   MOE_TRY(mark(MOE_NUM_STAGES));
   return MOE_OK;
 }
@@ -452,9 +413,7 @@ MOE_API moe_status moe_launches_per_forward(const moe_problem* p, int32_t two_st
     *n = 0;
     return MOE_OK;
   }
-  // router logits + top-k; histogram + scan, permute + gather; combine (done
-  // by the shared expert's down GEMM when fused)
-  int count = 2 + 2 + (fused_combine(*p) ? 0 : 1);
+  int count = 2 + 2 + 1;  // router logits + top-k; histogram + scan, permute + gather; combine
   if (p->dtype == MOE_DTYPE_BF16) {
     Segments routed{reinterpret_cast<const int32_t*>(16), (int32_t)p->E, 0, p->T * p->k};
     count += 2 * tc_gemm_launches(routed);

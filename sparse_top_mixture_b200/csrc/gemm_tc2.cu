@@ -72,9 +72,7 @@ struct Ring {
   static_assert(STAGES >= 2 && STAGES <= MAX_STAGES, "ring depth");
 };
 
-// MODE_DOWN_COMBINE: down of a one-segment (shared expert) problem whose
-// epilogue adds each token's routed rows and writes the bf16 output.
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_DOWN_COMBINE = 2 };
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 
 struct Args2 {
   const int32_t* offsets;
@@ -89,9 +87,6 @@ struct Args2 {
   const int32_t* scale_idx;
   int32_t* err;
   int64_t rows_total;
-  const float* y_rows;      // DOWN_COMBINE: routed fp32 rows [*, N]
-  const int32_t* pair_pos;  // DOWN_COMBINE: [rows * k], -1 for a skipped pair
-  int32_t k;                // DOWN_COMBINE: slots per token
 };
 
 struct __align__(8) Ctl2 {
@@ -124,7 +119,6 @@ constexpr size_t smem_bytes2() {
 }
 static_assert(smem_bytes2<MODE_GATE_UP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 static_assert(smem_bytes2<MODE_DOWN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
-static_assert(smem_bytes2<MODE_DOWN_COMBINE>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
@@ -320,17 +314,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
           epilogue_swiglu(tbase, 0, 128, 4, orow0, args.ldo, nrows, tc.n_idx * 128, args.N, lane);
         else
           epilogue_swiglu(tbase, 0, 64, 2, orow0, args.ldo, nrows, tc.n_idx * 128 + half * 64, args.N, lane);
-      } else if (MODE == MODE_DOWN_COMBINE) {
-        float sc = 1.f;
-        if (lane < nrows && args.row_scale != nullptr) sc = args.row_scale[row];
-        __nv_bfloat16* orow0 = reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)row_w0 * args.ldo;
-        const int32_t* pp0 = args.pair_pos + (int64_t)row_w0 * args.k;
-        if (!tc.tail)
-          epilogue_scale_combine_bf16(tbase, 8, sc, stage, orow0, args.y_rows, pp0, args.k, args.ldo, nrows,
-                                      tc.n_idx * UMMA_N, args.N, lane);
-        else
-          epilogue_scale_combine_bf16(tbase, 4, sc, stage, orow0, args.y_rows, pp0, args.k, args.ldo, nrows,
-                                      tc.n_idx * UMMA_N + half * 128, args.N, lane);
       } else {
         float sc = 1.f;
         if (lane < nrows && args.row_scale != nullptr)
@@ -369,8 +352,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 template <int MODE, int KA>
 cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmB64,
                        int64_t N, int64_t K, void* out, int64_t ldo, const float* row_scale,
-                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s,
-                       const float* y_rows = nullptr, const int32_t* pair_pos = nullptr, int k = 0) {
+                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s) {
   static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance
   static cudaError_t attr_status[kSmemAttrDevices];
   const void* kernel = reinterpret_cast<const void*>(tc2_grouped_gemm_kernel<MODE, KA>);
@@ -389,9 +371,6 @@ cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtenso
   a.scale_idx = scale_idx;
   a.err = err;
   a.rows_total = sg.rows_total;
-  a.y_rows = y_rows;
-  a.pair_pos = pair_pos;
-  a.k = k;
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM2 + nseg) * a.n_tiles;
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms / 2, max_tiles));
@@ -476,18 +455,6 @@ cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_dow
   if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
   if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
   return launch_tc2<MODE_DOWN, KA>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
-}
-
-cudaError_t launch_tc2_down_combine(const Segments& sg, const void* A, const void* w_down, const float* gamma,
-                                    const float* y_rows, const int32_t* pair_pos, int64_t k, void* out, int64_t H,
-                                    int64_t I, int32_t* err, int num_sms, cudaStream_t s) {
-  if (sg.offsets != nullptr) return cudaErrorInvalidValue;  // one segment: row = token
-  constexpr int KA = kAtomsPerStage;
-  CUtensorMap tmA, tmB;
-  if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
-  if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, 1, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
-  return launch_tc2<MODE_DOWN_COMBINE, KA>(sg, tmA, tmB, tmB, H, I, out, H, gamma, nullptr, err, num_sms, s, y_rows,
-                                           pair_pos, (int)k);
 }
 
 }  // namespace stm

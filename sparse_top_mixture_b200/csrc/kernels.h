@@ -126,13 +126,6 @@ cudaError_t launch_tc2_gate_up(const Segments& sg, const void* A, const void* w_
 cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_down, int64_t E_w, void* y,
                             const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                             int num_sms, cudaStream_t s);
-// Down GEMM of a one-segment problem (the shared expert, row = token) whose
-// epilogue does the combine: out[t] (bf16) = sum over slots s of
-// y_rows[pair_pos[t*k+s]] (fp32, slot order) + gamma[t] * (h[t] . w_down^T),
-// rounded once; gamma may be NULL (1). CTA pairs only (T >= 192 rows).
-cudaError_t launch_tc2_down_combine(const Segments& sg, const void* A, const void* w_down, const float* gamma,
-                                    const float* y_rows, const int32_t* pair_pos, int64_t k, void* out, int64_t H,
-                                    int64_t I, int32_t* err, int num_sms, cudaStream_t s);
 cudaError_t launch_tc_gate_up(const Segments& sg, const void* A, const void* w_gate_up, int64_t E_w, void* h,
                               int64_t I, int64_t H, int32_t* err, cudaStream_t s);
 int tc_router_splits(int64_t T, int64_t H, int64_t E);

@@ -92,72 +92,5 @@ __device__ __forceinline__ void epilogue_scale_f32(uint32_t tbase, int nchunks, 
   }
 }
 
-// down of the shared expert with the combine: for token rows of the warp
-// block, out[r][col0 + j] = bf16( sum over slots s < k, in slot order, of
-// y[pair_pos[r*k + s]][col0 + j] + sc * acc[r][j] ) -- the routed rows'
-// fp32 sum, then the gated shared value, rounded once (the same additions in
-// the same order as the separate combine kernel). `nchunks` chunks of 32
-// columns from TMEM column 0 and output column col0; y and out share the
-// row pitch ldo; pp_row0 = pair_pos of the warp block's first row. The scaled
-// accumulator goes through the staging block so that each routed row is
-// read as whole 128-byte segments (8 lanes per row, 4 rows per instruction).
-__device__ __forceinline__ void epilogue_scale_combine_bf16(uint32_t tbase, int nchunks, float sc, float* stage,
-                                                            __nv_bfloat16* out_row0, const float* __restrict__ y,
-                                                            const int32_t* __restrict__ pp_row0, int k, int64_t ldo,
-                                                            int nrows, int col0, int N, int lane) {
-  const int c4 = lane & 7;
-#pragma unroll 1
-  for (int c = 0; c < nchunks; ++c) {
-    uint32_t d[32];
-    tmem_ld32(tbase + c * 32, d);
-    tmem_ld_wait();
-    const int cb = col0 + c * 32;
-    if (cb >= N || nrows <= 0) continue;  // warp-uniform
-    float4* srow = reinterpret_cast<float4*>(stage + lane * kStageStride);
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      srow[q] = make_float4(sc * __uint_as_float(d[4 * q]), sc * __uint_as_float(d[4 * q + 1]),
-                            sc * __uint_as_float(d[4 * q + 2]), sc * __uint_as_float(d[4 * q + 3]));
-    __syncwarp();
-    const int col = cb + c4 * 4;
-#pragma unroll 1
-    for (int it = 0; it < 8; ++it) {
-      const int r = it * 4 + (lane >> 3);
-      if (r < nrows && col < N) {
-        // up to eight slots' rows loaded together, then added in slot order
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < k; s0 += 8) {
-          int p[8];
-#pragma unroll
-          for (int s = 0; s < 8; ++s) p[s] = s0 + s < k ? pp_row0[(int64_t)r * k + s0 + s] : -1;
-          float4 v[8];
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            v[s] = p[s] >= 0 ? __ldcs(reinterpret_cast<const float4*>(y + (int64_t)p[s] * ldo + col))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            if (p[s] < 0) continue;
-            a.x += v[s].x;
-            a.y += v[s].y;
-            a.z += v[s].z;
-            a.w += v[s].w;
-          }
-        }
-        const float4 sv = reinterpret_cast<const float4*>(stage + r * kStageStride)[c4];
-        a.x += sv.x;
-        a.y += sv.y;
-        a.z += sv.z;
-        a.w += sv.w;
-        uint2 o;
-        o.x = pack_bf16x2(a.x, a.y);
-        o.y = pack_bf16x2(a.z, a.w);
-        *reinterpret_cast<uint2*>(out_row0 + (int64_t)r * ldo + col) = o;
-      }
-    }
-    __syncwarp();
-  }
-}
-
 }  // namespace tc
 }  // namespace stm

@@ -83,8 +83,7 @@ def test_launch_counts(L):
     # route 2 (logits, top-k), dispatch 2 (histogram + scan, permute + gather), combine 1, plus the expert GEMMs
     assert stm.launches_per_forward(_p()) == 5 + 2
     assert stm.launches_per_forward(_p(T=8192, E=64, k=6)) == 5 + 2
-    # a shared expert too large to overlap the routed GEMMs does the combine in its down GEMM
-    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256)) == 4 + 2 + 2
+    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256)) == 5 + 2 + 2
     assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256, dtype="f32")) == 5 + 4
     assert stm.launches_per_forward(_p(dtype="f32", shared="plain", I_shared=256)) == 5 + 4
     assert stm.launches_per_forward(_p(T=0)) == 0

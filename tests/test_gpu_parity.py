@@ -102,9 +102,9 @@ def test_both_tensor_core_variants_are_exercised():
 @pytest.mark.parametrize("name", list(SMALL) + ["pairs_shared_skew", "large_shared_gated"])
 def test_staged_calls_match_forward(name):
     """route -> dispatch -> grouped_swiglu -> shared_expert -> combine through
-    the separate entry points equals moe_forward bit for bit (also where the
-    forward does the combine in the shared expert's down GEMM: the same
-    additions in the same order), and each stage matches the oracle."""
+    the separate entry points equals moe_forward bit for bit (also with a
+    shared expert large enough to run beside the dispatch), and each stage
+    matches the oracle."""
     cfg = EDGE.get(name) or SMALL[name]
     cpu, dev = _inputs(cfg)
     p = stm.Problem.from_config(cfg)
