@@ -644,6 +644,8 @@ def main():
     ap.add_argument("--no-backward", action="store_true", help="skip the fp32 backward measurement")
     ap.add_argument("--no-per-config", action="store_true", help="skip the per_config block (the other workloads)")
     ap.add_argument("--per-config-steps", type=int, default=50)
+    ap.add_argument("--backward-only", action="store_true",
+                    help="profiling only: run just the bf16 backward measurement on --config and print it")
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling only: override T (the line then names a reduced workload, not a bench line)")
     ap.add_argument("--experts", type=int, default=None,
@@ -671,6 +673,9 @@ def main():
         from sparse_top_mixture_b200 import build
         build.build()
     pk = peaks()
+    if args.backward_only:  # not a bench line: the backward block alone, for profiling captures
+        print(json.dumps({"backward_only": measure_backward(cfg, local, steps=args.steps, dtype="bf16")}), flush=True)
+        return
 
     run = ForwardRun(cfg, rank, graph=not args.no_graph)
     run.warm(args.warmup)
