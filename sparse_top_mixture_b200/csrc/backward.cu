@@ -639,21 +639,50 @@ __global__ void __launch_bounds__(BT) bw16_to_f32(const __nv_bfloat16* __restric
     out[i] = __bfloat162float(in[i]);
 }
 
-// out[b][c][r] = in[b][r][c] for R x C slabs, 64 x 64 tiles through shared memory.
+// out[b][c][r] = in[b][r][c] for R x C slabs (R, C multiples of 8), 64 x 64
+// tiles through shared memory: each row of a tile is read as eight 16-byte
+// vectors, and each output row of a tile written as eight.
 __global__ void __launch_bounds__(BT) bw16_transpose(const __nv_bfloat16* __restrict__ in, int R, int C,
                                                    __nv_bfloat16* __restrict__ out) {
-  __shared__ __nv_bfloat16 tile[64][66];
+  __shared__ __align__(16) uint16_t tile[64][72];  // 144-byte rows: 16-byte aligned, banks staggered
   const int64_t slab = (int64_t)blockIdx.z * R * C;
   const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
-  for (int i = ty; i < 64; i += 4) {
-    const int r = r0 + i, c = c0 + tx;
-    tile[i][tx] = (r < R && c < C) ? in[slab + (int64_t)r * C + c] : __float2bfloat16_rn(0.f);
+  const uint16_t* src = reinterpret_cast<const uint16_t*>(in) + slab;
+  uint16_t* dst = reinterpret_cast<uint16_t*>(out) + slab;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int idx = threadIdx.x + i * BT;  // 512 vectors: 64 rows x 8
+    const int rr = idx >> 3, v = idx & 7;
+    const int r = r0 + rr, c = c0 + v * 8;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r < R && c < C) val = *reinterpret_cast<const uint4*>(src + (int64_t)r * C + c);
+    *reinterpret_cast<uint4*>(&tile[rr][v * 8]) = val;
   }
   __syncthreads();
-  for (int i = ty; i < 64; i += 4) {
-    const int c = c0 + i, r = r0 + tx;
-    if (c < C && r < R) out[slab + (int64_t)c * R + r] = tile[tx][i];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int idx = threadIdx.x + i * BT;  // 512 vectors: 64 output rows x 8
+    const int cc = idx >> 3, v = idx & 7;
+    const int c = c0 + cc, r = r0 + v * 8;
+    if (c >= C || r >= R) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w[q] = (uint32_t)tile[v * 8 + 2 * q][cc] | ((uint32_t)tile[v * 8 + 2 * q + 1][cc] << 16);
+    *reinterpret_cast<uint4*>(dst + (int64_t)c * R + r) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// L[t][e] = sum over splits s (in order) of part[s][t][e], row pitch ldo.
+__global__ void __launch_bounds__(BT) bw16_sum_logits(const float* __restrict__ part, int splits, int64_t ldo,
+                                                    int T, int E, float* __restrict__ L) {
+  const int64_t n = (int64_t)T * E;
+  for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
+    const int64_t t = i / E;
+    const int e = (int)(i - t * E);
+    float acc = 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += part[((int64_t)sp * T + t) * ldo + e];
+    L[i] = acc;
   }
 }
 
@@ -770,7 +799,8 @@ __global__ void __launch_bounds__(BT) bw16_swiglu(const float* __restrict__ gu, 
 }
 
 struct BwLayout16 {
-  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, parts, x32, gw32, g32,
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, parts, lpart, x32, gw32,
+      g32,
       koff, ranges, xperm, doutperm, wguT, wdT, gu, dhu, hact, dgdu, dxr, extra, xT, dyT, hT, dgduT, gus, dhus, hacts,
       dgdus, wsguT, wsdT, xTs, dyTs, hTs, dgdusT, gamma, dz, total;
   int64_t Ppad, Tpad;
@@ -803,6 +833,7 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.dL = take((size_t)p.T * p.E * f);
   const int S = router_chunks(p);
   b.parts = take(S > 1 ? (size_t)S * p.E * p.H * f : 0);
+  b.lpart = take(router_partial_bytes(MOE_DTYPE_BF16, p.T, p.H, p.E));
   b.x32 = take((size_t)p.T * p.H * f);
   b.gw32 = take((size_t)p.E * p.H * f);
   b.g32 = take((size_t)p.H * f);
@@ -906,15 +937,15 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   bw16_to_f32<<<grid_for((int64_t)T * H), BT, 0, s>>>(x, (int64_t)T * H, x32);
   bw16_to_f32<<<grid_for((int64_t)E * H), BT, 0, s>>>(static_cast<const bf*>(w->gate_w), (int64_t)E * H, gw32);
   if (gated) bw16_to_f32<<<grid_for(H), BT, 0, s>>>(static_cast<const bf*>(w->shared_gate), H, g32);
-  // Router: logits, scores and the routing weights of the given choice.
-  BW16_CUDA(run_rows<true, EPI_STORE>(
-      [&] {
-        RowGemm a = row_gemm(x32, nullptr, H, gw32, 0, E, H, nullptr, 1, T, T, err);
-        a.C = L;
-        a.ldc = E;
-        return a;
-      }(),
-      s));
+  // Router: logits on the tensor cores (the forward's split-K GEMM, its
+  // partials summed in split order), then scores and the routing weights of
+  // the given choice.
+  {
+    const RouterPlan rp = router_plan(MOE_DTYPE_BF16, T, H, E);
+    float* lpart = at<float>(ws, b.lpart);
+    BW16_CUDA(launch_tc_logits(x, w->gate_w, T, H, E, lpart, rp.ldo, rp.splits, err, s));
+    bw16_sum_logits<<<grid_for((int64_t)T * E), BT, 0, s>>>(lpart, rp.splits, rp.ldo, T, E, L);
+  }
   bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
   // Sorted segments of the choice with x_perm; the same permutation of dout.
   BW16_CUDA(launch_dispatch(MOE_DTYPE_BF16, selected, x, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
