@@ -639,37 +639,41 @@ __global__ void __launch_bounds__(BT) bw16_to_f32(const __nv_bfloat16* __restric
     out[i] = __bfloat162float(in[i]);
 }
 
-// out[b][c][r] = in[b][r][c] for R x C slabs (R, C multiples of 8), 64 x 64
-// tiles through shared memory: each row of a tile is read as eight 16-byte
-// vectors, and each output row of a tile written as eight.
+// out[b][c][r] = in[b][r][c] for R x C slabs (R, C multiples of 8). Each
+// thread transposes an 8 x 8 block in registers: eight 16-byte row loads,
+// byte permutes, eight 16-byte column stores. A warp covers 32 rows x 64
+// columns: lanes 0-7 read one 128-byte row segment each step, and the four
+// lanes sharing an 8-column group write 64 consecutive bytes of each output
+// row.
 __global__ void __launch_bounds__(BT) bw16_transpose(const __nv_bfloat16* __restrict__ in, int R, int C,
                                                    __nv_bfloat16* __restrict__ out) {
-  __shared__ __align__(16) uint16_t tile[64][72];  // 144-byte rows: 16-byte aligned, banks staggered
   const int64_t slab = (int64_t)blockIdx.z * R * C;
-  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
   const uint16_t* src = reinterpret_cast<const uint16_t*>(in) + slab;
   uint16_t* dst = reinterpret_cast<uint16_t*>(out) + slab;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // block tile: 8 warps stacked along the rows, 256 rows x 64 columns
+  const int r = blockIdx.y * 256 + warp * 32 + (lane >> 3) * 8;
+  const int c = blockIdx.x * 64 + (lane & 7) * 8;
+  if (r >= R || c >= C) return;
+  uint32_t w[8][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int idx = threadIdx.x + i * BT;  // 512 vectors: 64 rows x 8
-    const int rr = idx >> 3, v = idx & 7;
-    const int r = r0 + rr, c = c0 + v * 8;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r < R && c < C) val = *reinterpret_cast<const uint4*>(src + (int64_t)r * C + c);
-    *reinterpret_cast<uint4*>(&tile[rr][v * 8]) = val;
+  for (int i = 0; i < 8; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src + (int64_t)(r + i) * C + c);
+    w[i][0] = v.x;
+    w[i][1] = v.y;
+    w[i][2] = v.z;
+    w[i][3] = v.w;
   }
-  __syncthreads();
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int idx = threadIdx.x + i * BT;  // 512 vectors: 64 output rows x 8
-    const int cc = idx >> 3, v = idx & 7;
-    const int c = c0 + cc, r = r0 + v * 8;
-    if (c >= C || r >= R) continue;
-    uint32_t w[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      w[q] = (uint32_t)tile[v * 8 + 2 * q][cc] | ((uint32_t)tile[v * 8 + 2 * q + 1][cc] << 16);
-    *reinterpret_cast<uint4*>(dst + (int64_t)c * R + r) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int j = 0; j < 8; ++j) {
+    // output row c + j: element i of it is element j of input row r + i
+    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+    uint4 o;
+    o.x = __byte_perm(w[0][j >> 1], w[1][j >> 1], sel);
+    o.y = __byte_perm(w[2][j >> 1], w[3][j >> 1], sel);
+    o.z = __byte_perm(w[4][j >> 1], w[5][j >> 1], sel);
+    o.w = __byte_perm(w[6][j >> 1], w[7][j >> 1], sel);
+    *reinterpret_cast<uint4*>(dst + (int64_t)(c + j) * R + r) = o;
   }
 }
 
@@ -752,17 +756,30 @@ __global__ void __launch_bounds__(BT) bw16_transpose_pad(const Tin* __restrict__
   {
     const int src = s_src[rr];
     const float sc = s_sc[rr];
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const int c = c0 + q * 16 + i;
-      float v = 0.f;
-      if (src >= 0 && c < X) {
-        if constexpr (sizeof(Tin) == 2) v = __bfloat162float(in[(int64_t)src * ld_in + c]);
-        else v = in[(int64_t)src * ld_in + c];
-        v *= sc;
+    const int cq = c0 + q * 16;  // X is a multiple of 8: a 16-column run is whole, half, or absent
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    if (src >= 0) {
+      const Tin* row = in + (int64_t)src * ld_in + cq;
+      if constexpr (sizeof(Tin) == 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (cq + 8 * h < X) unpack16_bf16(reinterpret_cast<const uint4*>(row)[h], v + 8 * h);
+      } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          if (cq + 4 * h < X) {
+            const float4 f = reinterpret_cast<const float4*>(row)[h];
+            v[4 * h] = f.x;
+            v[4 * h + 1] = f.y;
+            v[4 * h + 2] = f.z;
+            v[4 * h + 3] = f.w;
+          }
       }
-      tile[q * 16 + i][rr] = v;
     }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tile[q * 16 + i][rr] = v[i] * sc;
   }
   __syncthreads();
   const int c = c0 + rr;
@@ -779,22 +796,35 @@ __global__ void __launch_bounds__(BT) bw16_transpose_pad(const Tin* __restrict__
 // SwiGLU backward of one routed row block: for rows r < rows (rows = *nrows
 // when nrows is given) and i < I, with g, u from gu [*, 2I], dhu [*, I] and
 // the row's weight scale[r]: hact = silu(g) u (fp32); dgdu = bf16([dh u
-// silu'(g) | dh silu(g)]), dh = scale dhu.
+// silu'(g) | dh silu(g)]), dh = scale dhu. Four columns per thread (I is a
+// multiple of 8): 16-byte loads of g, u and dhu, 16-byte and 8-byte stores.
 __global__ void __launch_bounds__(BT) bw16_swiglu(const float* __restrict__ gu, const float* __restrict__ dhu,
                                                 const float* __restrict__ scale, const int32_t* __restrict__ nrows,
                                                 int64_t rows, int I, float* __restrict__ hact,
                                                 __nv_bfloat16* __restrict__ dgdu) {
   const int64_t R = nrows ? (int64_t)*nrows : rows;
-  const int64_t n = R * I;
+  const int I4 = I / 4;
+  const int64_t n = R * I4;
   for (int64_t idx = blockIdx.x * (int64_t)BT + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * BT) {
-    const int64_t r = idx / I;
-    const int i = (int)(idx - r * I);
-    const float g = gu[r * 2 * I + i], u = gu[r * 2 * I + I + i];
-    const float d = dhu[idx];
-    const float dh = scale[r] * d;
-    hact[idx] = silu_f32(g) * u;
-    dgdu[r * 2 * I + i] = __float2bfloat16_rn(dh * u * silu_grad_f(g));
-    dgdu[r * 2 * I + I + i] = __float2bfloat16_rn(dh * silu_f32(g));
+    const int64_t r = idx / I4;
+    const int i = (int)(idx - r * I4) * 4;
+    const float4 g4 = *reinterpret_cast<const float4*>(gu + r * 2 * I + i);
+    const float4 u4 = *reinterpret_cast<const float4*>(gu + r * 2 * I + I + i);
+    const float4 d4 = *reinterpret_cast<const float4*>(dhu + r * I + i);
+    const float sc = scale[r];
+    const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w}, d[4] = {d4.x, d4.y, d4.z, d4.w};
+    float h[4], dg[4], du[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float dh = sc * d[q];
+      h[q] = silu_f32(g[q]) * u[q];
+      dg[q] = dh * u[q] * silu_grad_f(g[q]);
+      du[q] = dh * silu_f32(g[q]);
+    }
+    *reinterpret_cast<float4*>(hact + r * I + i) = make_float4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint2*>(dgdu + r * 2 * I + i) = make_uint2(pack_bf16x2(dg[0], dg[1]), pack_bf16x2(dg[2], dg[3]));
+    *reinterpret_cast<uint2*>(dgdu + r * 2 * I + I + i) =
+        make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
   }
 }
 
@@ -881,7 +911,7 @@ cudaError_t transpose_pad(const Tin* in, int64_t ld_in, const int32_t* rowmap, c
 }
 
 cudaError_t transpose_slabs(const void* in, int64_t B, int64_t R, int64_t C, void* out, cudaStream_t s) {
-  const dim3 grid((unsigned)ceil_div(C, 64), (unsigned)ceil_div(R, 64), (unsigned)B);
+  const dim3 grid((unsigned)ceil_div(C, 64), (unsigned)ceil_div(R, 256), (unsigned)B);
   bw16_transpose<<<grid, BT, 0, s>>>(static_cast<const __nv_bfloat16*>(in), (int)R, (int)C,
                                      static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
@@ -963,7 +993,7 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   const Segments sg{offsets, (int32_t)E, 0, P};
   BW16_CUDA(launch_tc_down(sg, xperm, w->gate_up, E, gu, nullptr, nullptr, 2 * I, H, err, s));  // [g | u]
   BW16_CUDA(launch_tc_down(sg, doutperm, wdT, E, dhu, nullptr, nullptr, I, H, err, s));         // dhu
-  bw16_swiglu<<<grid_for(P * I), BT, 0, s>>>(gu, dhu, scale, offsets + E, P, I, hact, dgdu);
+  bw16_swiglu<<<grid_for(P * I / 4), BT, 0, s>>>(gu, dhu, scale, offsets + E, P, I, hact, dgdu);
   BW16_CUDA(launch_tc_down(sg, dgdu, wguT, E, dxr, nullptr, nullptr, H, 2 * I, err, s));       // dx rows
   bw_rowdot<<<grid_for(P * 32), BT, 0, s>>>(hact, dhu, I, pair_pos, P, nullptr, dw);
   // Routed weight gradients from padded transposes: dWd = (w dout)^T h, dWgu = [dg du]^T x.
@@ -1004,7 +1034,7 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     BW16_CUDA(transpose_slabs(w->shared_down, 1, H, Is, wsdT, s));          // [H][Is] -> [Is][H]
     BW16_CUDA(launch_tc_down(one, x, w->shared_gate_up, 1, gus, nullptr, nullptr, 2 * Is, H, err, s));
     BW16_CUDA(launch_tc_down(one, dout, wsdT, 1, dhus, nullptr, nullptr, Is, H, err, s));
-    bw16_swiglu<<<grid_for((int64_t)T * Is), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, hacts, dgdus);
+    bw16_swiglu<<<grid_for((int64_t)T * Is / 4), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, hacts, dgdus);
     BW16_CUDA(launch_tc_down(one, dgdus, wsguT, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
     if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(hacts, dhus, Is, nullptr, T, gamma, dz);
     bf* xTs = at<bf>(ws, b.xTs);

@@ -40,6 +40,11 @@ constexpr int SCAN_THREADS = DTHREADS * HIST_SUB;
 // threads of one warp (tpe = 4..32), which read their ranges with independent
 // loads, combine through a segmented warp scan, and write the running bases.
 // The counts were written by other CTAs of the same grid: read through L2.
+// A range of up to kScanRegs entries is read once, in one round of loads,
+// and kept in registers for the second pass; longer ranges (more than
+// kScanRegs x tpe blocks) are read twice, in rounds of kScanRegs.
+constexpr int kScanRegs = 16;
+
 __device__ void block_scan_counts(int32_t* __restrict__ local, int nblk, int E, int tpe,
                                   int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* tot) {
   const int tid = threadIdx.x;
@@ -47,21 +52,22 @@ __device__ void block_scan_counts(int32_t* __restrict__ local, int nblk, int E, 
   const bool active = e < E;
   const int chunk = (nblk + tpe - 1) / tpe;
   const int b0 = min(nblk, part * chunk), b1 = min(nblk, b0 + chunk);
+  const bool in_regs = b1 - b0 <= kScanRegs;
+  int v[kScanRegs];
   int sum = 0;
   if (active) {
-    for (int b = b0; b < b1; b += 8) {
-      int v[8];
+    for (int b = b0; b < b1; b += kScanRegs) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
+      for (int i = 0; i < kScanRegs; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum += v[i];
+      for (int i = 0; i < kScanRegs; ++i) sum += v[i];
     }
   }
   // segmented inclusive scan over the tpe parts of one expert (same warp)
   int incl = sum;
   for (int o = 1; o < tpe; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (part >= o) incl += v;
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (part >= o) incl += x;
   }
   if (active && part == tpe - 1) tot[e] = incl;
   __syncthreads();
@@ -76,8 +82,8 @@ __device__ void block_scan_counts(int32_t* __restrict__ local, int nblk, int E, 
     int inc = loc;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, inc, o);
-      if (tid >= o) inc += v;
+      const int x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (tid >= o) inc += x;
     }
     int run = inc - loc;
 #pragma unroll
@@ -95,12 +101,13 @@ __device__ void block_scan_counts(int32_t* __restrict__ local, int nblk, int E, 
   __syncthreads();
   if (!active) return;
   int run = tot[e] + incl - sum;
-  for (int b = b0; b < b1; b += 8) {
-    int v[8];
+  for (int b = b0; b < b1; b += kScanRegs) {
+    if (!in_regs) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
+      for (int i = 0; i < kScanRegs; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
+    }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kScanRegs; ++i) {
       if (b + i < b1) local[(int64_t)(b + i) * E + e] = run;
       run += v[i];
     }
