@@ -339,9 +339,10 @@ typedef struct moe_grads {
  *   is needed besides the choice.
  *   fp32 problems run on SIMT kernels in fp32 throughout. bf16 problems
  *   (x, dout and the weights bf16) run the expert GEMMs on the tensor cores
- *   (bf16 operands, fp32 accumulation; [dg du], w*dout and h are rounded to
- *   bf16 where they become operands) and the router in fp32; the gradients
- *   are fp32 for both. Every gradient element is an fp32 sum in a fixed
+ *   and the router's logits and weight gradient on the tensor cores (bf16
+ *   operands, fp32 accumulation; [dg du], w*dout, h and dlogits are rounded
+ *   to bf16 where they become operands), the rest in fp32; the gradients are
+ *   fp32 for both. Every gradient element is an fp32 sum in a fixed
  *   order (no atomics; the router weight gradient adds row-chunk partial sums
  *   in chunk order): results are deterministic. A pair with an expert id outside [0, E) contributes
  *   nothing and sets MOE_DEVERR_BAD_EXPERT_ID in the workspace header.

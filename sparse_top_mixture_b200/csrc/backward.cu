@@ -720,7 +720,7 @@ __global__ void __launch_bounds__(BT) bw16_transpose_pad(const Tin* __restrict__
                                                        const float* __restrict__ scale,
                                                        const int32_t* __restrict__ off,
                                                        const int32_t* __restrict__ koff, int E, int X,
-                                                       __nv_bfloat16* __restrict__ out, int64_t ld) {
+                                                       __nv_bfloat16* __restrict__ out, int64_t ld, int vec) {
   __shared__ float tile[64][65];
   __shared__ int s_off[kMaxExperts + 1], s_koff[kMaxExperts + 1];
   __shared__ int s_src[64];
@@ -760,7 +760,15 @@ __global__ void __launch_bounds__(BT) bw16_transpose_pad(const Tin* __restrict__
     float v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = 0.f;
-    if (src >= 0) {
+    if (src >= 0 && !vec) {  // rows not 16-byte aligned (ld_in or X not a multiple of 8): scalar loads
+      const Tin* row = in + (int64_t)src * ld_in + cq;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (cq + i >= X) break;
+        if constexpr (sizeof(Tin) == 2) v[i] = __bfloat162float(row[i]);
+        else v[i] = row[i];
+      }
+    } else if (src >= 0) {
       const Tin* row = in + (int64_t)src * ld_in + cq;
       if constexpr (sizeof(Tin) == 2) {
 #pragma unroll
@@ -829,9 +837,8 @@ __global__ void __launch_bounds__(BT) bw16_swiglu(const float* __restrict__ gu, 
 }
 
 struct BwLayout16 {
-  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, parts, lpart, x32, gw32,
-      g32,
-      koff, ranges, xperm, doutperm, wguT, wdT, gu, dhu, hact, dgdu, dxr, extra, xT, dyT, hT, dgduT, gus, dhus, hacts,
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, lpart, x32, gw32, g32,
+      koff, ranges, xperm, doutperm, wguT, wdT, gu, dhu, hact, dgdu, dxr, extra, xT, dyT, hT, dgduT, dLT, gus, dhus, hacts,
       dgdus, wsguT, wsdT, xTs, dyTs, hTs, dgdusT, gamma, dz, total;
   int64_t Ppad, Tpad;
 };
@@ -861,8 +868,6 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.L = take((size_t)p.T * p.E * f);
   b.S = take((size_t)p.T * p.E * f);
   b.dL = take((size_t)p.T * p.E * f);
-  const int S = router_chunks(p);
-  b.parts = take(S > 1 ? (size_t)S * p.E * p.H * f : 0);
   b.lpart = take(router_partial_bytes(MOE_DTYPE_BF16, p.T, p.H, p.E));
   b.x32 = take((size_t)p.T * p.H * f);
   b.gw32 = take((size_t)p.E * p.H * f);
@@ -883,6 +888,7 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.dyT = take((size_t)p.H * b.Ppad * h2);
   b.hT = take((size_t)p.I * b.Ppad * h2);
   b.dgduT = take((size_t)2 * p.I * b.Ppad * h2);
+  b.dLT = take((size_t)p.E * b.Tpad * h2);
   const bool sh = p.shared != MOE_SHARED_NONE;
   const size_t Is = sh ? (size_t)p.I_shared : 0;
   const size_t Tp = sh ? (size_t)b.Tpad : 0;
@@ -892,7 +898,7 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.dgdus = take((size_t)p.T * 2 * Is * h2);
   b.wsguT = take((size_t)p.H * 2 * Is * h2);
   b.wsdT = take(Is * p.H * h2);
-  b.xTs = take((size_t)p.H * Tp * h2);
+  b.xTs = take((size_t)p.H * b.Tpad * h2);  // x transposed [H][T_pad]: the router's dgate_w and the shared expert
   b.dyTs = take((size_t)p.H * Tp * h2);
   b.hTs = take(Is * Tp * h2);
   b.dgdusT = take(2 * Is * Tp * h2);
@@ -906,7 +912,8 @@ template <typename Tin>
 cudaError_t transpose_pad(const Tin* in, int64_t ld_in, const int32_t* rowmap, const float* scale, const int32_t* off,
                           const int32_t* koff, int E, int X, __nv_bfloat16* out, int64_t ld, cudaStream_t s) {
   const dim3 grid((unsigned)ceil_div(X, 64), (unsigned)(ld / 64));
-  bw16_transpose_pad<Tin><<<grid, BT, 0, s>>>(in, ld_in, rowmap, scale, off, koff, E, X, out, ld);
+  const int vec = (X % 8 == 0 && ld_in % 8 == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) ? 1 : 0;
+  bw16_transpose_pad<Tin><<<grid, BT, 0, s>>>(in, ld_in, rowmap, scale, off, koff, E, X, out, ld, vec);
   return cudaGetLastError();
 }
 
@@ -1003,19 +1010,14 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   BW16_CUDA(transpose_pad<bf>(x, H, tok, nullptr, offsets, koff, E, H, xT, b.Ppad, s));
   BW16_CUDA(launch_wgrad(dyT, hT, b.Ppad, koff, E, H, I, g->d_down, err, s));
   BW16_CUDA(launch_wgrad(dgduT, xT, b.Ppad, koff, E, 2 * I, H, g->d_gate_up, err, s));
-  // Router backward: dL, dgate_w = dL^T x (in row chunks summed in order), d_bias = sum_t dL.
+  // Router backward: dL (fp32); dgate_w = dL^T x on the tensor cores from K-major transposes
+  // [E][T_pad] (dL rounded to bf16) and [H][T_pad]; d_bias = sum_t dL in fp32.
   bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL);
-  const int nchunk = router_chunks(*p);
-  if (nchunk == 1) {
-    BW16_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x32, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1,
-                        s));
-  } else {
-    float* parts = at<float>(ws, b.parts);
-    const int chunk = (int)ceil_div(T, nchunk);
-    BW16_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x32, nullptr, H, H, nullptr, T, T, parts, err, chunk),
-                        nchunk, s));
-    bw_sum_parts<<<grid_for((int64_t)E * H), BT, 0, s>>>(parts, nchunk, (int64_t)E * H, g->d_gate_w);
-  }
+  bf* dLT = at<bf>(ws, b.dLT);
+  bf* xTs = at<bf>(ws, b.xTs);
+  BW16_CUDA(transpose_pad<float>(dL, E, nullptr, nullptr, ranges, ranges + 2, 1, E, dLT, b.Tpad, s));
+  BW16_CUDA(transpose_pad<bf>(x, H, nullptr, nullptr, ranges, ranges + 2, 1, H, xTs, b.Tpad, s));
+  BW16_CUDA(launch_wgrad(dLT, xTs, b.Tpad, ranges + 2, 1, E, H, g->d_gate_w, err, s));
   if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
   // Shared expert over all tokens (one segment), scaled by gamma; its dx goes to `extra`.
   float* dz = nullptr;
@@ -1037,7 +1039,6 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     bw16_swiglu<<<grid_for((int64_t)T * Is / 4), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, hacts, dgdus);
     BW16_CUDA(launch_tc_down(one, dgdus, wsguT, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
     if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(hacts, dhus, Is, nullptr, T, gamma, dz);
-    bf* xTs = at<bf>(ws, b.xTs);
     bf* dyTs = at<bf>(ws, b.dyTs);
     bf* hTs = at<bf>(ws, b.hTs);
     bf* dgdusT = at<bf>(ws, b.dgdusT);
@@ -1045,7 +1046,6 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     BW16_CUDA(transpose_pad<bf>(dout, H, nullptr, gamma, ranges, ranges + 2, 1, H, dyTs, b.Tpad, s));
     BW16_CUDA(transpose_pad<float>(hacts, Is, nullptr, nullptr, ranges, ranges + 2, 1, Is, hTs, b.Tpad, s));
     BW16_CUDA(transpose_pad<bf>(dgdus, 2 * Is, nullptr, nullptr, ranges, ranges + 2, 1, 2 * Is, dgdusT, b.Tpad, s));
-    BW16_CUDA(transpose_pad<bf>(x, H, nullptr, nullptr, ranges, ranges + 2, 1, H, xTs, b.Tpad, s));
     BW16_CUDA(launch_wgrad(dyTs, hTs, b.Tpad, ranges + 2, 1, H, Is, g->d_shared_down, err, s));
     BW16_CUDA(launch_wgrad(dgdusT, xTs, b.Tpad, ranges + 2, 1, 2 * Is, H, g->d_shared_gate_up, err, s));
     if (gated) bw_dgvec<<<grid_for(H), BT, 0, s>>>(dz, x32, T, H, g->d_shared_gate);

@@ -2,12 +2,13 @@
 the C ABI) against the fp64 backward oracle (oracle/backward.py), on the same
 seeded bf16 inputs (converted exactly) and the oracle's own expert choice.
 
-Tolerance. The GPU rounds three intermediates to bf16 where they become GEMM
-operands: [dg du] (dx and dW_gate_up), w*dout and h (dW_down); each rounding
+Tolerance. The GPU rounds four intermediates to bf16 where they become GEMM
+operands: [dg du] (dx and dW_gate_up), w*dout and h (dW_down), and dlogits
+(the router's dgate_w); each rounding
 moves a value by at most 2^-9 of itself, products and sums are fp32. A
 gradient element therefore carries a relative error of about one or two
 bf16 roundings of the terms it sums (~1e-3 in L2 over a tensor, as for the
-forward), and the router's gradients, computed from fp32 h . dhu, much less.
+forward); the logit bias and the router's dx come from fp32 dlogits.
 The bar: relative L2 <= 5e-3 per tensor (the problem's bf16 output bar) and
 no element off by more than 1e-2 of the tensor's largest magnitude.
 """
