@@ -297,6 +297,18 @@ def backward_flops(cfg) -> float:
     return 16.0 * P * cfg.H * cfg.I + 6.0 * cfg.T * cfg.E * cfg.H + 16.0 * cfg.T * cfg.H * cfg.I_shared
 
 
+def backward_bytes(cfg, active: int, es: int) -> float:
+    """Algorithmic bytes of one backward: the active experts' weights, the
+    router's and the shared expert's read once (``es`` bytes an element), x
+    and dout read once, every weight gradient (all E experts: an expert
+    without rows gets zeros) and dx written once in fp32."""
+    w_routed = 3.0 * cfg.H * cfg.I
+    w_other = cfg.E * cfg.H + 3.0 * cfg.H * cfg.I_shared + (cfg.H if cfg.shared == "sigmoid_gated" else 0)
+    reads = (active * w_routed + w_other) * es + 2.0 * cfg.T * cfg.H * es
+    writes = (cfg.E * w_routed + w_other + (cfg.E if cfg.bias_mode == "logit" else 0)) * 4 + cfg.T * cfg.H * 4
+    return reads + writes
+
+
 def host_memory_available() -> float:
     """Bytes this process may still allocate: the smaller of the host's
     available memory and what its cgroup (v2 or v1) limit leaves."""
@@ -377,33 +389,41 @@ def measure_backward(cfg, local: int, steps: int = 5, cpu: bool = False, dtype: 
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # eager: one C-ABI call per step (its ~25 launches issued from the host)
+    a.record(stream)
+    for _ in range(steps):
+        stm.backward(p, inp, inp["x"], dout, sel, ws=ws, out=grads)
+    b.record(stream)
+    torch.cuda.synchronize()
+    eager_ms = a.elapsed_time(b) / steps
+    # the same call captured once as a CUDA graph and replayed, as the forward is timed
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        stm.backward(p, inp, inp["x"], dout, sel, ws=ws, out=grads)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         a.record(stream)
         for _ in range(steps):
-            stm.backward(p, inp, inp["x"], dout, sel, ws=ws, out=grads)
+            graph.replay()
         b.record(stream)
         torch.cuda.synchronize()
+    del graph
     if stm.read_device_error(ws) != 0:
         raise RuntimeError("device error flag set during the backward")
     ms = a.elapsed_time(b) / steps
     fl = backward_flops(c)
     ck = clk.summary()
     mhz = ck["sm_mhz"] or ck["sm_max_mhz"] or 1965
-    if dtype == "f32":
-        peak = ffma_peak_tflops(mhz)
-        src = f"148 SMs x 128 FFMA lanes x 2 flop x {mhz} MHz (median sampled SM clock)"
-        bound = "alu"
-    else:
-        pk = peaks()
-        peak = pk["bf16_tflops"]
-        src = pk["source"] + " bf16 (burst)"
-        bound = "tensor"
-    achieved = fl / (ms / 1e3) / 1e12
+    active = int(torch.unique(sel[(sel >= 0) & (sel < c.E)]).numel())
+    nbytes = backward_bytes(c, active, 4 if dtype == "f32" else 2)
+    roof = roofline_entry(fl, nbytes, ms, peaks(), dtype, mhz)
     res = {"workload": f"{cfg.name} shapes in {dtype} (T={c.T}, H={c.H}, E={c.E}, k={c.k}, I={c.I}, "
                        f"I_shared={c.I_shared})",
-           "dtype": dtype, "ms": ms, "tokens_per_s": c.T / (ms / 1e3), "steps": steps, "flops": fl, "bound": bound,
-           "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-           "peak_source": src, "clocks": ck}
+           "dtype": dtype, "ms": ms, "launch": "cuda_graph", "eager_ms": eager_ms,
+           "tokens_per_s": c.T / (ms / 1e3), "steps": steps, "flops": fl,
+           "active_experts": active, "tflops": fl / (ms / 1e3) / 1e12, **roof, "traffic": None, "clocks": ck}
     if cpu:
         try:
             res["cpu_baseline"] = backward_cpu_baseline(cfg.replace(dtype="f32"), inp, dout.float())

@@ -1,6 +1,7 @@
 /*
  * moe.h -- C ABI of the B200 (sm_100a) sparse top-k MoE FFN: the forward
- * pass, the aux-loss-free balancer's bias update, and an fp32 backward pass.
+ * pass, the aux-loss-free balancer's bias update, and the backward pass (fp32
+ * problems on SIMT kernels, bf16 problems on the tensor cores).
  *
  * The forward pass, step by step:
  *   route    : logits = x . gate_w^T, scores (softmax / sigmoid / sqrtsoftplus),
@@ -341,8 +342,10 @@ typedef struct moe_grads {
  *   (x, dout and the weights bf16) run the expert GEMMs on the tensor cores
  *   and the router's logits and weight gradient on the tensor cores (bf16
  *   operands, fp32 accumulation; [dg du], w*dout, h and dlogits are rounded
- *   to bf16 where they become operands), the rest in fp32; the gradients are
- *   fp32 for both. Every gradient element is an fp32 sum in a fixed
+ *   to bf16 where they become operands; the weights are read as stored, no
+ *   transposed copy is made), the rest in fp32; the gradients are fp32 for
+ *   both. Nothing in the call allocates or waits on the host: it can be
+ *   captured in a CUDA graph. Every gradient element is an fp32 sum in a fixed
  *   order (no atomics; the router weight gradient adds row-chunk partial sums
  *   in chunk order): results are deterministic. A pair with an expert id outside [0, E) contributes
  *   nothing and sets MOE_DEVERR_BAD_EXPERT_ID in the workspace header.

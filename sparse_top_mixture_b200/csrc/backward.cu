@@ -27,7 +27,7 @@
 // double-buffered in shared memory, 8x8 fp32 outputs per thread; every output
 // element is one thread's fixed-order sum (dgate_w: row-chunk partials added
 // in chunk order), with no atomics, so results are deterministic. bf16
-// problems are not supported.
+// problems take the tensor-core variant at the end of this file.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -399,11 +399,13 @@ __global__ void __launch_bounds__(BT) bw_rowdot(const float* __restrict__ Hact, 
   }
 }
 
-// Router backward, one token per block: dS from dw (renormalisation), dL from dS.
+// Router backward, one token per block: dS from dw (renormalisation), dL from
+// dS; also dL rounded to bf16 into dL16 (row pitch ld16) when given.
 __global__ void __launch_bounds__(BT) bw_router_bwd(const float* __restrict__ L, const float* __restrict__ S,
                                                   const float* __restrict__ w, const float* __restrict__ dw,
                                                   const int64_t* __restrict__ sel, int score, int renorm, int E,
-                                                  int k, float* __restrict__ dL) {
+                                                  int k, float* __restrict__ dL, __nv_bfloat16* __restrict__ dL16,
+                                                  int ld16) {
   __shared__ float dS[kMaxExperts];
   __shared__ float red[BT];
   const int t = blockIdx.x, e = threadIdx.x;
@@ -440,7 +442,10 @@ __global__ void __launch_bounds__(BT) bw_router_bwd(const float* __restrict__ L,
   } else {
     dl = (e < E && s > 0.f) ? ds * sig_f(L[(int64_t)t * E + e]) / (2.f * s) : 0.f;
   }
-  if (e < E) dL[(int64_t)t * E + e] = dl;
+  if (e < E) {
+    dL[(int64_t)t * E + e] = dl;
+    if (dL16) dL16[(int64_t)t * ld16 + e] = __float2bfloat16_rn(dl);
+  }
 }
 
 // out[i] = sum_{s < S} part[s * n + i], in order of s
@@ -619,62 +624,26 @@ WGemm wgrad(const float* A, const int32_t* amap, const float* ascale, int64_t ld
 // ---- bf16 problems: tensor-core backward ------------------------------------------
 // The same chain rule on the 5th-generation tensor cores. bf16 inputs (x,
 // dout, weights) stay bf16 as GEMM operands, products accumulate in fp32:
-//   [g | u] = x_perm Wgu^T (fp32), dhu = dout_perm Wd (fp32, via a transposed
-//   copy Wd^T [E,I,H]), then elementwise h = silu(g) u (fp32) and
-//   [dg | du] rounded to bf16 (the next GEMMs' operand), dx rows =
-//   [dg du] Wgu (fp32, via Wgu^T [E,H,2I]) -- all four on the forward's
-//   grouped kernels over the dispatch's segments; weight gradients on the
-//   weight-gradient mode of the one-CTA kernel, whose K loop walks an
-//   expert's rows: dWd = (w dout)^T h and dWgu = [dg du]^T x from K-major
-//   transposed copies [features][rows] in which every expert's rows are a
-//   run of columns zero-padded to a multiple of 64 (w dout and h rounded to
-//   bf16 there). The router (E logits per token) and the gate vector keep
-//   the fp32 SIMT code above, on fp32 copies of x and gate_w. Gradients are
-//   fp32. Still no atomics: results are deterministic.
+//   [g | u] = x_perm Wgu^T and dhu = dout_perm Wd (fp32), then per row h =
+//   silu(g) u and dw = h . dhu (fp32) and [dg | du] rounded to bf16 (the next
+//   GEMM's operand), dx rows = [dg du] Wgu (fp32) -- on the forward's grouped
+//   kernels over the dispatch's segments, with Wd [E][H][I] and Wgu
+//   [E][2I][H] read as stored (MN-major B operands: no transposed copies);
+//   weight gradients on the weight-gradient mode of the one-CTA kernel, whose
+//   K loop walks an expert's rows and reads both operands MN-major from row
+//   buffers: dWd = (w dout)^T h and dWgu = [dg du]^T x, from copies in which
+//   every expert's rows start at a multiple of 64 and are zero-padded up to
+//   the next (w dout and h rounded to bf16 there), and dgate_w = dlogits^T x
+//   over one segment of all tokens (dlogits rounded to bf16, x as given). The
+//   router's scores and dx and the gate vector keep the fp32 SIMT code above,
+//   on fp32 copies of x and gate_w. Gradients are fp32. Still no atomics:
+//   results are deterministic.
 
 // out[i] = float(in[i])
 __global__ void __launch_bounds__(BT) bw16_to_f32(const __nv_bfloat16* __restrict__ in, int64_t n,
                                                 float* __restrict__ out) {
   for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT)
     out[i] = __bfloat162float(in[i]);
-}
-
-// out[b][c][r] = in[b][r][c] for R x C slabs (R, C multiples of 8). Each
-// thread transposes an 8 x 8 block in registers: eight 16-byte row loads,
-// byte permutes, eight 16-byte column stores. A warp covers 32 rows x 64
-// columns: lanes 0-7 read one 128-byte row segment each step, and the four
-// lanes sharing an 8-column group write 64 consecutive bytes of each output
-// row.
-__global__ void __launch_bounds__(BT) bw16_transpose(const __nv_bfloat16* __restrict__ in, int R, int C,
-                                                   __nv_bfloat16* __restrict__ out) {
-  const int64_t slab = (int64_t)blockIdx.z * R * C;
-  const uint16_t* src = reinterpret_cast<const uint16_t*>(in) + slab;
-  uint16_t* dst = reinterpret_cast<uint16_t*>(out) + slab;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // block tile: 8 warps stacked along the rows, 256 rows x 64 columns
-  const int r = blockIdx.y * 256 + warp * 32 + (lane >> 3) * 8;
-  const int c = blockIdx.x * 64 + (lane & 7) * 8;
-  if (r >= R || c >= C) return;
-  uint32_t w[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 v = *reinterpret_cast<const uint4*>(src + (int64_t)(r + i) * C + c);
-    w[i][0] = v.x;
-    w[i][1] = v.y;
-    w[i][2] = v.z;
-    w[i][3] = v.w;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    // output row c + j: element i of it is element j of input row r + i
-    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-    uint4 o;
-    o.x = __byte_perm(w[0][j >> 1], w[1][j >> 1], sel);
-    o.y = __byte_perm(w[2][j >> 1], w[3][j >> 1], sel);
-    o.z = __byte_perm(w[4][j >> 1], w[5][j >> 1], sel);
-    o.w = __byte_perm(w[6][j >> 1], w[7][j >> 1], sel);
-    *reinterpret_cast<uint4*>(dst + (int64_t)(c + j) * R + r) = o;
-  }
 }
 
 // L[t][e] = sum over splits s (in order) of part[s][t][e], row pitch ldo.
@@ -690,8 +659,8 @@ __global__ void __launch_bounds__(BT) bw16_sum_logits(const float* __restrict__ 
   }
 }
 
-// Padded K offsets of the weight-gradient GEMMs: koff[e] = sum over e' < e of
-// round_up(count[e'], 64); also the one-segment ranges of the shared expert:
+// Padded row offsets of the weight-gradient GEMMs: koff[e] = sum over e' < e
+// of round_up(count[e'], 64); also the one-segment range of all tokens:
 // ranges = {0, T, 0, round_up(T, 64)}.
 __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int32_t* __restrict__ koff,
                           int32_t* __restrict__ ranges) {
@@ -708,139 +677,178 @@ __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int
   ranges[3] = (T + 63) / 64 * 64;
 }
 
-// Transpose of row-major activations into the padded K-major layout:
-// out[c * ld + kk] for kk in [0, ld): inside expert e's run [koff[e],
-// koff[e] + count_e) it holds bf16(scale[r] * in[src(r) * ld_in + c]) with r =
-// off[e] + (kk - koff[e]) and src(r) = rowmap[r] (or r); everywhere else 0.
-// 64 x 64 tiles: a quarter-warp reads 64 consecutive columns of one source
-// row, a quarter-warp writes 64 consecutive kk of one output row.
-template <typename Tin>
-__global__ void __launch_bounds__(BT) bw16_transpose_pad(const Tin* __restrict__ in, int64_t ld_in,
-                                                       const int32_t* __restrict__ rowmap,
-                                                       const float* __restrict__ scale,
-                                                       const int32_t* __restrict__ off,
-                                                       const int32_t* __restrict__ koff, int E, int X,
-                                                       __nv_bfloat16* __restrict__ out, int64_t ld, int vec) {
-  __shared__ float tile[64][65];
-  __shared__ int s_off[kMaxExperts + 1], s_koff[kMaxExperts + 1];
+// Padded row buffers, one block per 64-row group (an expert's run starts at a
+// multiple of 64, so a group lies in one expert e). Row q = koff[e] + j holds,
+// for j < count_e and r = off[e] + j: x_pad[q] = x[tok[r]] and dy_pad[q] =
+// bf16(scale[r] * dout[tok[r]]); rows with j >= count_e are zero in x_pad,
+// dy_pad, h_pad [*, I] and dgdu_pad [*, 2I] (the SwiGLU backward writes the
+// others). 16-byte vectors (H and I are multiples of 8).
+__global__ void __launch_bounds__(BT) bw16_pad_rows(const __nv_bfloat16* __restrict__ x,
+                                                  const __nv_bfloat16* __restrict__ dout,
+                                                  const int32_t* __restrict__ tok, const float* __restrict__ scale,
+                                                  const int32_t* __restrict__ off, const int32_t* __restrict__ koff,
+                                                  int E, int H, int I, __nv_bfloat16* __restrict__ x_pad,
+                                                  __nv_bfloat16* __restrict__ dy_pad,
+                                                  __nv_bfloat16* __restrict__ h_pad,
+                                                  __nv_bfloat16* __restrict__ dgdu_pad) {
   __shared__ int s_src[64];
   __shared__ float s_sc[64];
-  for (int e = threadIdx.x; e <= E; e += BT) {
-    s_off[e] = off[e];
-    s_koff[e] = koff[e];
-  }
-  __syncthreads();
-  const int64_t kk0 = (int64_t)blockIdx.y * 64;
-  const int c0 = blockIdx.x * 64;
-  if (threadIdx.x < 64) {
-    const int kk = (int)(kk0 + threadIdx.x);
-    int lo = 0, hi = E;  // expert with koff[lo] <= kk < koff[lo + 1]
+  __shared__ int s_e;
+  const int q0 = blockIdx.x * 64;
+  if (q0 >= koff[E]) return;  // past the last expert's run (the same for the whole block)
+  if (threadIdx.x == 0) {
+    int lo = 0, hi = E;  // koff[lo] <= q0 < koff[lo + 1]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (s_koff[mid] <= kk) lo = mid;
+      if (koff[mid] <= q0) lo = mid;
       else hi = mid;
     }
-    const int j = kk - s_koff[lo];
+    s_e = lo;
+  }
+  __syncthreads();
+  const int e = s_e;
+  const int j0 = q0 - koff[e];
+  const int cnt = off[e + 1] - off[e];
+  if (threadIdx.x < 64) {
+    const int j = j0 + (int)threadIdx.x;
     int src = -1;
     float sc = 0.f;
-    if (kk < s_koff[E] && j < s_off[lo + 1] - s_off[lo]) {
-      const int r = s_off[lo] + j;
-      src = rowmap ? rowmap[r] : r;
-      sc = scale ? scale[r] : 1.f;
+    if (j < cnt) {
+      const int r = off[e] + j;
+      src = tok[r];
+      sc = scale[r];
     }
     s_src[threadIdx.x] = src;
     s_sc[threadIdx.x] = sc;
   }
   __syncthreads();
-  const int q = threadIdx.x & 3, rr = threadIdx.x >> 2;  // 4 threads per row, 16 columns each
-  {
-    const int src = s_src[rr];
-    const float sc = s_sc[rr];
-    const int cq = c0 + q * 16;  // X is a multiple of 8: a 16-column run is whole, half, or absent
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-    if (src >= 0 && !vec) {  // rows not 16-byte aligned (ld_in or X not a multiple of 8): scalar loads
-      const Tin* row = in + (int64_t)src * ld_in + cq;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (cq + i >= X) break;
-        if constexpr (sizeof(Tin) == 2) v[i] = __bfloat162float(row[i]);
-        else v[i] = row[i];
-      }
-    } else if (src >= 0) {
-      const Tin* row = in + (int64_t)src * ld_in + cq;
-      if constexpr (sizeof(Tin) == 2) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          if (cq + 8 * h < X) unpack16_bf16(reinterpret_cast<const uint4*>(row)[h], v + 8 * h);
-      } else {
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-          if (cq + 4 * h < X) {
-            const float4 f = reinterpret_cast<const float4*>(row)[h];
-            v[4 * h] = f.x;
-            v[4 * h + 1] = f.y;
-            v[4 * h + 2] = f.z;
-            v[4 * h + 3] = f.w;
-          }
-      }
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  const int hv = H / 8;
+  for (int idx = threadIdx.x; idx < 64 * hv; idx += BT) {
+    const int i = idx / hv, v = idx - i * hv;
+    const int64_t q = q0 + i;
+    const int src = s_src[i];
+    uint4 xo = zero, yo = zero;
+    if (src >= 0) {
+      xo = reinterpret_cast<const uint4*>(x + (int64_t)src * H)[v];
+      float f[8];
+      unpack16_bf16(reinterpret_cast<const uint4*>(dout + (int64_t)src * H)[v], f);
+      const float sc = s_sc[i];
+      yo = make_uint4(pack_bf16x2(sc * f[0], sc * f[1]), pack_bf16x2(sc * f[2], sc * f[3]),
+                      pack_bf16x2(sc * f[4], sc * f[5]), pack_bf16x2(sc * f[6], sc * f[7]));
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) tile[q * 16 + i][rr] = v[i] * sc;
+    reinterpret_cast<uint4*>(x_pad + q * H)[v] = xo;
+    reinterpret_cast<uint4*>(dy_pad + q * H)[v] = yo;
   }
-  __syncthreads();
-  const int c = c0 + rr;
-  if (c < X) {
-    __nv_bfloat16* orow = out + (int64_t)c * ld + kk0 + q * 16;
-    uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(tile[rr][q * 16 + 2 * i], tile[rr][q * 16 + 2 * i + 1]);
-    reinterpret_cast<uint4*>(orow)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    reinterpret_cast<uint4*>(orow)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  const int nvalid = max(0, min(64, cnt - j0));
+  const int iv = I / 8, rv = 3 * iv;  // one row: I/8 vectors of h, 2I/8 of [dg | du]
+  for (int idx = threadIdx.x; idx < (64 - nvalid) * rv; idx += BT) {
+    const int i = nvalid + idx / rv, v = idx % rv;
+    const int64_t q = q0 + i;
+    if (v < iv) reinterpret_cast<uint4*>(h_pad + q * I)[v] = zero;
+    else reinterpret_cast<uint4*>(dgdu_pad + q * 2 * I)[v - iv] = zero;
   }
 }
 
-// SwiGLU backward of one routed row block: for rows r < rows (rows = *nrows
-// when nrows is given) and i < I, with g, u from gu [*, 2I], dhu [*, I] and
-// the row's weight scale[r]: hact = silu(g) u (fp32); dgdu = bf16([dh u
-// silu'(g) | dh silu(g)]), dh = scale dhu. Four columns per thread (I is a
-// multiple of 8): 16-byte loads of g, u and dhu, 16-byte and 8-byte stores.
-__global__ void __launch_bounds__(BT) bw16_swiglu(const float* __restrict__ gu, const float* __restrict__ dhu,
-                                                const float* __restrict__ scale, const int32_t* __restrict__ nrows,
-                                                int64_t rows, int I, float* __restrict__ hact,
-                                                __nv_bfloat16* __restrict__ dgdu) {
-  const int64_t R = nrows ? (int64_t)*nrows : rows;
-  const int I4 = I / 4;
-  const int64_t n = R * I4;
-  for (int64_t idx = blockIdx.x * (int64_t)BT + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * BT) {
-    const int64_t r = idx / I4;
-    const int i = (int)(idx - r * I4) * 4;
-    const float4 g4 = *reinterpret_cast<const float4*>(gu + r * 2 * I + i);
-    const float4 u4 = *reinterpret_cast<const float4*>(gu + r * 2 * I + I + i);
-    const float4 d4 = *reinterpret_cast<const float4*>(dhu + r * I + i);
-    const float sc = scale[r];
-    const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w}, d[4] = {d4.x, d4.y, d4.z, d4.w};
-    float h[4], dg[4], du[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float dh = sc * d[q];
-      h[q] = silu_f32(g[q]) * u[q];
-      dg[q] = dh * u[q] * silu_grad_f(g[q]);
-      du[q] = dh * silu_f32(g[q]);
+// SwiGLU backward, one warp per row p < R (R = *nrows when given, else rows),
+// with g, u from gu [*, 2I], dhu [*, I] and the row's weight scale[p]: h =
+// silu(g) u and dh = scale dhu in fp32; [dg | du] = [dh u silu'(g) | dh silu(g)]
+// rounded to bf16 into dgdu [*, 2I]; h rounded to bf16 into h_rows [*, I] and
+// [dg | du] into dgdu_rows (when given) at row q = koff[e] + p - off[e] of p's
+// segment e (q = p without off); dot = sum_i h dhu (fp32, h unrounded) into
+// dot_out[dot_idx[p]] (or [p]; nothing without dot_out), times gamma (1 -
+// gamma) with dot_gamma = gamma. Lanes take 4 columns at a time (I is a
+// multiple of 8): 16-byte loads, 8-byte stores.
+__global__ void __launch_bounds__(BT) bw16_swiglu_rows(const float* __restrict__ gu, const float* __restrict__ dhu,
+                                                     const float* __restrict__ scale, const int32_t* __restrict__ nrows,
+                                                     int64_t rows, int I, const int32_t* __restrict__ off,
+                                                     const int32_t* __restrict__ koff, int E,
+                                                     const int32_t* __restrict__ dot_idx,
+                                                     const float* __restrict__ dot_gamma, float* __restrict__ dot_out,
+                                                     __nv_bfloat16* __restrict__ dgdu,
+                                                     __nv_bfloat16* __restrict__ h_rows,
+                                                     __nv_bfloat16* __restrict__ dgdu_rows) {
+  __shared__ int s_off[kMaxExperts + 1], s_koff[kMaxExperts + 1];
+  if (off) {
+    for (int e = threadIdx.x; e <= E; e += BT) {
+      s_off[e] = off[e];
+      s_koff[e] = koff[e];
     }
-    *reinterpret_cast<float4*>(hact + r * I + i) = make_float4(h[0], h[1], h[2], h[3]);
-    *reinterpret_cast<uint2*>(dgdu + r * 2 * I + i) = make_uint2(pack_bf16x2(dg[0], dg[1]), pack_bf16x2(dg[2], dg[3]));
-    *reinterpret_cast<uint2*>(dgdu + r * 2 * I + I + i) =
-        make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
+  }
+  __syncthreads();
+  const int64_t R = nrows ? (int64_t)*nrows : rows;
+  const int lane = threadIdx.x & 31;
+  for (int64_t p = (blockIdx.x * (int64_t)BT + threadIdx.x) >> 5; p < R; p += ((int64_t)gridDim.x * BT) >> 5) {
+    int64_t q = p;
+    if (off) {
+      int lo = 0, hi = E;  // s_off[lo] <= p < s_off[lo + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_off[mid] <= p) lo = mid;
+        else hi = mid;
+      }
+      q = s_koff[lo] + (p - s_off[lo]);
+    }
+    const float sc = scale[p];
+    const float* grow = gu + p * 2 * I;
+    const float* drow = dhu + p * I;
+    float dot = 0.f;
+    for (int i = lane * 4; i < I; i += 128) {
+      const float4 g4 = *reinterpret_cast<const float4*>(grow + i);
+      const float4 u4 = *reinterpret_cast<const float4*>(grow + I + i);
+      const float4 d4 = *reinterpret_cast<const float4*>(drow + i);
+      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w}, d[4] = {d4.x, d4.y, d4.z, d4.w};
+      float h[4], dg[4], du[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float sg = silu_f32(g[c]);
+        const float dh = sc * d[c];
+        h[c] = sg * u[c];
+        dg[c] = dh * u[c] * silu_grad_f(g[c]);
+        du[c] = dh * sg;
+        dot = fmaf(h[c], d[c], dot);
+      }
+      const uint2 dg2 = make_uint2(pack_bf16x2(dg[0], dg[1]), pack_bf16x2(dg[2], dg[3]));
+      const uint2 du2 = make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
+      *reinterpret_cast<uint2*>(dgdu + p * 2 * I + i) = dg2;
+      *reinterpret_cast<uint2*>(dgdu + p * 2 * I + I + i) = du2;
+      *reinterpret_cast<uint2*>(h_rows + q * I + i) = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+      if (dgdu_rows) {
+        *reinterpret_cast<uint2*>(dgdu_rows + q * 2 * I + i) = dg2;
+        *reinterpret_cast<uint2*>(dgdu_rows + q * 2 * I + I + i) = du2;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane == 0 && dot_out) {
+      if (dot_gamma) dot *= dot_gamma[p] * (1.f - dot_gamma[p]);
+      dot_out[dot_idx ? dot_idx[p] : p] = dot;
+    }
+  }
+}
+
+// out[t][h] = bf16(gamma[t] * in[t][h]), eight columns per thread (H a multiple of 8).
+__global__ void __launch_bounds__(BT) bw16_scale_rows(const __nv_bfloat16* __restrict__ in,
+                                                    const float* __restrict__ gamma, int T, int H,
+                                                    __nv_bfloat16* __restrict__ out) {
+  const int hv = H / 8;
+  const int64_t n = (int64_t)T * hv;
+  for (int64_t idx = blockIdx.x * (int64_t)BT + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * BT) {
+    const int64_t t = idx / hv;
+    float f[8];
+    unpack16_bf16(reinterpret_cast<const uint4*>(in)[idx], f);
+    const float sc = gamma[t];
+    reinterpret_cast<uint4*>(out)[idx] =
+        make_uint4(pack_bf16x2(sc * f[0], sc * f[1]), pack_bf16x2(sc * f[2], sc * f[3]),
+                   pack_bf16x2(sc * f[4], sc * f[5]), pack_bf16x2(sc * f[6], sc * f[7]));
   }
 }
 
 struct BwLayout16 {
-  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, lpart, x32, gw32, g32,
-      koff, ranges, xperm, doutperm, wguT, wdT, gu, dhu, hact, dgdu, dxr, extra, xT, dyT, hT, dgduT, dLT, gus, dhus, hacts,
-      dgdus, wsguT, wsdT, xTs, dyTs, hTs, dgdusT, gamma, dz, total;
-  int64_t Ppad, Tpad;
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, dL16, lpart, x32, gw32,
+      g32, koff, ranges, xperm, doutperm, gu, dhu, dgdu, dxr, extra, xpad, dypad, hpad, dgdupad, gus, dhus, hs, dgdus,
+      dys, gamma, dz, total;
+  int64_t Ppad, Tpad, Epad;
 };
 
 BwLayout16 bw_layout16(const moe_problem& p) {
@@ -848,6 +856,7 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   const int64_t P = p.T * p.k;
   b.Ppad = round_up(P + 63 * p.E, 64);
   b.Tpad = round_up(p.T, 64);
+  b.Epad = round_up(p.E, 8);  // 16-byte rows of the bf16 dlogits
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -868,6 +877,7 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.L = take((size_t)p.T * p.E * f);
   b.S = take((size_t)p.T * p.E * f);
   b.dL = take((size_t)p.T * p.E * f);
+  b.dL16 = take((size_t)p.T * b.Epad * h2);
   b.lpart = take(router_partial_bytes(MOE_DTYPE_BF16, p.T, p.H, p.E));
   b.x32 = take((size_t)p.T * p.H * f);
   b.gw32 = take((size_t)p.E * p.H * f);
@@ -876,52 +886,26 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.ranges = take(4 * 4);
   b.xperm = take((size_t)P * p.H * h2);
   b.doutperm = take((size_t)P * p.H * h2);
-  b.wguT = take((size_t)p.E * p.H * 2 * p.I * h2);
-  b.wdT = take((size_t)p.E * p.I * p.H * h2);
   b.gu = take((size_t)P * 2 * p.I * f);
   b.dhu = take((size_t)P * p.I * f);
-  b.hact = take((size_t)P * p.I * f);
   b.dgdu = take((size_t)P * 2 * p.I * h2);
   b.dxr = take((size_t)P * p.H * f);
   b.extra = take((size_t)p.T * p.H * f);
-  b.xT = take((size_t)p.H * b.Ppad * h2);
-  b.dyT = take((size_t)p.H * b.Ppad * h2);
-  b.hT = take((size_t)p.I * b.Ppad * h2);
-  b.dgduT = take((size_t)2 * p.I * b.Ppad * h2);
-  b.dLT = take((size_t)p.E * b.Tpad * h2);
-  const bool sh = p.shared != MOE_SHARED_NONE;
+  b.xpad = take((size_t)b.Ppad * p.H * h2);
+  b.dypad = take((size_t)b.Ppad * p.H * h2);
+  b.hpad = take((size_t)b.Ppad * p.I * h2);
+  b.dgdupad = take((size_t)b.Ppad * 2 * p.I * h2);
+  const bool sh = p.shared != MOE_SHARED_NONE, gated = p.shared == MOE_SHARED_SIGMOID_GATED;
   const size_t Is = sh ? (size_t)p.I_shared : 0;
-  const size_t Tp = sh ? (size_t)b.Tpad : 0;
   b.gus = take((size_t)p.T * 2 * Is * f);
   b.dhus = take((size_t)p.T * Is * f);
-  b.hacts = take((size_t)p.T * Is * f);
+  b.hs = take((size_t)p.T * Is * h2);
   b.dgdus = take((size_t)p.T * 2 * Is * h2);
-  b.wsguT = take((size_t)p.H * 2 * Is * h2);
-  b.wsdT = take(Is * p.H * h2);
-  b.xTs = take((size_t)p.H * b.Tpad * h2);  // x transposed [H][T_pad]: the router's dgate_w and the shared expert
-  b.dyTs = take((size_t)p.H * Tp * h2);
-  b.hTs = take(Is * Tp * h2);
-  b.dgdusT = take(2 * Is * Tp * h2);
+  b.dys = take(gated ? (size_t)p.T * p.H * h2 : 0);
   b.gamma = take(sh ? (size_t)p.T * f : 0);
   b.dz = take(sh ? (size_t)p.T * f : 0);
   b.total = off;
   return b;
-}
-
-template <typename Tin>
-cudaError_t transpose_pad(const Tin* in, int64_t ld_in, const int32_t* rowmap, const float* scale, const int32_t* off,
-                          const int32_t* koff, int E, int X, __nv_bfloat16* out, int64_t ld, cudaStream_t s) {
-  const dim3 grid((unsigned)ceil_div(X, 64), (unsigned)(ld / 64));
-  const int vec = (X % 8 == 0 && ld_in % 8 == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0) ? 1 : 0;
-  bw16_transpose_pad<Tin><<<grid, BT, 0, s>>>(in, ld_in, rowmap, scale, off, koff, E, X, out, ld, vec);
-  return cudaGetLastError();
-}
-
-cudaError_t transpose_slabs(const void* in, int64_t B, int64_t R, int64_t C, void* out, cudaStream_t s) {
-  const dim3 grid((unsigned)ceil_div(C, 64), (unsigned)ceil_div(R, 256), (unsigned)B);
-  bw16_transpose<<<grid, BT, 0, s>>>(static_cast<const __nv_bfloat16*>(in), (int)R, (int)C,
-                                     static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
 }
 
 #define BW16_CUDA(...)                                     \
@@ -950,6 +934,7 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   float* L = at<float>(ws, b.L);
   float* S = at<float>(ws, b.S);
   float* dL = at<float>(ws, b.dL);
+  bf* dL16 = at<bf>(ws, b.dL16);
   float* x32 = at<float>(ws, b.x32);
   float* gw32 = at<float>(ws, b.gw32);
   float* g32 = gated ? at<float>(ws, b.g32) : nullptr;
@@ -957,18 +942,15 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   int32_t* ranges = at<int32_t>(ws, b.ranges);
   bf* xperm = at<bf>(ws, b.xperm);
   bf* doutperm = at<bf>(ws, b.doutperm);
-  bf* wguT = at<bf>(ws, b.wguT);
-  bf* wdT = at<bf>(ws, b.wdT);
   float* gu = at<float>(ws, b.gu);
   float* dhu = at<float>(ws, b.dhu);
-  float* hact = at<float>(ws, b.hact);
   bf* dgdu = at<bf>(ws, b.dgdu);
   float* dxr = at<float>(ws, b.dxr);
   float* extra = at<float>(ws, b.extra);
-  bf* xT = at<bf>(ws, b.xT);
-  bf* dyT = at<bf>(ws, b.dyT);
-  bf* hT = at<bf>(ws, b.hT);
-  bf* dgduT = at<bf>(ws, b.dgduT);
+  bf* xpad = at<bf>(ws, b.xpad);
+  bf* dypad = at<bf>(ws, b.dypad);
+  bf* hpad = at<bf>(ws, b.hpad);
+  bf* dgdupad = at<bf>(ws, b.dgdupad);
 
   // fp32 copies for the SIMT router and gate vector
   bw16_to_f32<<<grid_for((int64_t)T * H), BT, 0, s>>>(x, (int64_t)T * H, x32);
@@ -993,61 +975,53 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
                             &hdr->dispatch_ticket, s));
   bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, wts, E, k, tok, scale);
   bw16_koff<<<1, 32, 0, s>>>(offsets, E, T, koff, ranges);
-  // Transposed weight copies (K-major operands of the data-gradient GEMMs).
-  BW16_CUDA(transpose_slabs(w->gate_up, E, 2 * I, H, wguT, s));  // [E][2I][H] -> [E][H][2I]
-  BW16_CUDA(transpose_slabs(w->down, E, H, I, wdT, s));          // [E][H][I] -> [E][I][H]
-  // Routed experts on the tensor cores.
+  // Padded rows of x and w dout for the weight gradients.
+  bw16_pad_rows<<<(unsigned)(b.Ppad / 64), BT, 0, s>>>(x, dout, tok, scale, offsets, koff, E, H, I, xpad, dypad, hpad,
+                                                       dgdupad);
+  // Routed experts on the tensor cores; the weights are read as stored.
   const Segments sg{offsets, (int32_t)E, 0, P};
   BW16_CUDA(launch_tc_down(sg, xperm, w->gate_up, E, gu, nullptr, nullptr, 2 * I, H, err, s));  // [g | u]
-  BW16_CUDA(launch_tc_down(sg, doutperm, wdT, E, dhu, nullptr, nullptr, I, H, err, s));         // dhu
-  bw16_swiglu<<<grid_for(P * I / 4), BT, 0, s>>>(gu, dhu, scale, offsets + E, P, I, hact, dgdu);
-  BW16_CUDA(launch_tc_down(sg, dgdu, wguT, E, dxr, nullptr, nullptr, H, 2 * I, err, s));       // dx rows
-  bw_rowdot<<<grid_for(P * 32), BT, 0, s>>>(hact, dhu, I, pair_pos, P, nullptr, dw);
-  // Routed weight gradients from padded transposes: dWd = (w dout)^T h, dWgu = [dg du]^T x.
-  BW16_CUDA(transpose_pad<bf>(dout, H, tok, scale, offsets, koff, E, H, dyT, b.Ppad, s));
-  BW16_CUDA(transpose_pad<float>(hact, I, nullptr, nullptr, offsets, koff, E, I, hT, b.Ppad, s));
-  BW16_CUDA(transpose_pad<bf>(dgdu, 2 * I, nullptr, nullptr, offsets, koff, E, 2 * I, dgduT, b.Ppad, s));
-  BW16_CUDA(transpose_pad<bf>(x, H, tok, nullptr, offsets, koff, E, H, xT, b.Ppad, s));
-  BW16_CUDA(launch_wgrad(dyT, hT, b.Ppad, koff, E, H, I, g->d_down, err, s));
-  BW16_CUDA(launch_wgrad(dgduT, xT, b.Ppad, koff, E, 2 * I, H, g->d_gate_up, err, s));
-  // Router backward: dL (fp32); dgate_w = dL^T x on the tensor cores from K-major transposes
-  // [E][T_pad] (dL rounded to bf16) and [H][T_pad]; d_bias = sum_t dL in fp32.
-  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL);
-  bf* dLT = at<bf>(ws, b.dLT);
-  bf* xTs = at<bf>(ws, b.xTs);
-  BW16_CUDA(transpose_pad<float>(dL, E, nullptr, nullptr, ranges, ranges + 2, 1, E, dLT, b.Tpad, s));
-  BW16_CUDA(transpose_pad<bf>(x, H, nullptr, nullptr, ranges, ranges + 2, 1, H, xTs, b.Tpad, s));
-  BW16_CUDA(launch_wgrad(dLT, xTs, b.Tpad, ranges + 2, 1, E, H, g->d_gate_w, err, s));
+  BW16_CUDA(launch_tc_down_kn(sg, doutperm, w->down, E, dhu, nullptr, nullptr, I, H, err, s));  // dhu
+  // dw of pairs the dispatch dropped (bad expert ids) stays 0
+  BW16_CUDA(cudaMemsetAsync(dw, 0, (size_t)P * sizeof(float), s));
+  bw16_swiglu_rows<<<grid_for(P * 32), BT, 0, s>>>(gu, dhu, scale, offsets + E, P, I, offsets, koff, E, sorted_pairs,
+                                                    nullptr, dw, dgdu, hpad, dgdupad);
+  BW16_CUDA(launch_tc_down_kn(sg, dgdu, w->gate_up, E, dxr, nullptr, nullptr, H, 2 * I, err, s));  // dx rows
+  // Routed weight gradients: dWd = (w dout)^T h, dWgu = [dg du]^T x.
+  BW16_CUDA(launch_wgrad(dypad, H, hpad, I, b.Ppad, koff, b.Ppad, E, H, I, g->d_down, err, s));
+  BW16_CUDA(launch_wgrad(dgdupad, 2 * I, xpad, H, b.Ppad, koff, b.Ppad, E, 2 * I, H, g->d_gate_up, err, s));
+  // Router backward: dL (fp32, and rounded to bf16 for dgate_w = dL^T x over
+  // all tokens on the tensor cores); d_bias = sum_t dL in fp32.
+  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL, dL16,
+                                 (int)b.Epad);
+  BW16_CUDA(launch_wgrad(dL16, b.Epad, x, H, T, ranges + 2, b.Tpad, 1, E, H, g->d_gate_w, err, s));
   if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
   // Shared expert over all tokens (one segment), scaled by gamma; its dx goes to `extra`.
   float* dz = nullptr;
   if (sh) {
     float* gus = at<float>(ws, b.gus);
     float* dhus = at<float>(ws, b.dhus);
-    float* hacts = at<float>(ws, b.hacts);
+    bf* hs = at<bf>(ws, b.hs);
     bf* dgdus = at<bf>(ws, b.dgdus);
-    bf* wsguT = at<bf>(ws, b.wsguT);
-    bf* wsdT = at<bf>(ws, b.wsdT);
     float* gamma = at<float>(ws, b.gamma);
     dz = at<float>(ws, b.dz);
     const Segments one{nullptr, 1, (int32_t)T, p->T};
     bw_gamma<<<grid_for((int64_t)T * 32), BT, 0, s>>>(x32, g32, T, H, gamma);
-    BW16_CUDA(transpose_slabs(w->shared_gate_up, 1, 2 * Is, H, wsguT, s));  // [2Is][H] -> [H][2Is]
-    BW16_CUDA(transpose_slabs(w->shared_down, 1, H, Is, wsdT, s));          // [H][Is] -> [Is][H]
     BW16_CUDA(launch_tc_down(one, x, w->shared_gate_up, 1, gus, nullptr, nullptr, 2 * Is, H, err, s));
-    BW16_CUDA(launch_tc_down(one, dout, wsdT, 1, dhus, nullptr, nullptr, Is, H, err, s));
-    bw16_swiglu<<<grid_for((int64_t)T * Is / 4), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, hacts, dgdus);
-    BW16_CUDA(launch_tc_down(one, dgdus, wsguT, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
-    if (gated) bw_rowdot<<<grid_for((int64_t)T * 32), BT, 0, s>>>(hacts, dhus, Is, nullptr, T, gamma, dz);
-    bf* dyTs = at<bf>(ws, b.dyTs);
-    bf* hTs = at<bf>(ws, b.hTs);
-    bf* dgdusT = at<bf>(ws, b.dgdusT);
-    // one segment: ranges = {off: 0, T; koff: 0, Tpad}
-    BW16_CUDA(transpose_pad<bf>(dout, H, nullptr, gamma, ranges, ranges + 2, 1, H, dyTs, b.Tpad, s));
-    BW16_CUDA(transpose_pad<float>(hacts, Is, nullptr, nullptr, ranges, ranges + 2, 1, Is, hTs, b.Tpad, s));
-    BW16_CUDA(transpose_pad<bf>(dgdus, 2 * Is, nullptr, nullptr, ranges, ranges + 2, 1, 2 * Is, dgdusT, b.Tpad, s));
-    BW16_CUDA(launch_wgrad(dyTs, hTs, b.Tpad, ranges + 2, 1, H, Is, g->d_shared_down, err, s));
-    BW16_CUDA(launch_wgrad(dgdusT, xTs, b.Tpad, ranges + 2, 1, 2 * Is, H, g->d_shared_gate_up, err, s));
+    BW16_CUDA(launch_tc_down_kn(one, dout, w->shared_down, 1, dhus, nullptr, nullptr, Is, H, err, s));
+    bw16_swiglu_rows<<<grid_for((int64_t)T * 32), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, nullptr, nullptr, 0,
+                                                               nullptr, gamma, gated ? dz : nullptr, dgdus, hs,
+                                                               nullptr);
+    BW16_CUDA(launch_tc_down_kn(one, dgdus, w->shared_gate_up, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
+    // w dout for the shared expert is gamma dout (dout itself when ungated)
+    const bf* dys = dout;
+    if (gated) {
+      bf* dyg = at<bf>(ws, b.dys);
+      bw16_scale_rows<<<grid_for((int64_t)T * H / 8), BT, 0, s>>>(dout, gamma, T, H, dyg);
+      dys = dyg;
+    }
+    BW16_CUDA(launch_wgrad(dys, H, hs, Is, T, ranges + 2, b.Tpad, 1, H, Is, g->d_shared_down, err, s));
+    BW16_CUDA(launch_wgrad(dgdus, 2 * Is, x, H, T, ranges + 2, b.Tpad, 1, 2 * Is, H, g->d_shared_gate_up, err, s));
     if (gated) bw_dgvec<<<grid_for(H), BT, 0, s>>>(dz, x32, T, H, g->d_shared_gate);
   }
   // Router (and shared gate) dx into `extra`, then dx = sum of each token's rows + extra.
@@ -1193,7 +1167,7 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   BW_CUDA(run_wgrad(wgrad(dgu, nullptr, nullptr, 2 * I, 2 * I, x, tok, H, H, offsets, 0, P, g->d_gate_up, err), E,
                     s));
   // Router backward: dL, dgate_w = dL^T x (in row chunks summed in order), d_bias = sum_t dL.
-  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL);
+  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL, nullptr, 0);
   const int nchunk = router_chunks(*p);
   if (nchunk == 1) {
     BW_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1, s));

@@ -60,7 +60,11 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * UMMA_N;
 constexpr int NTHREADS = 192;
 
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2, MODE_WGRAD = 3 };
+// MODE_DOWN_KN: the down epilogue over B stored [E][K][N] (N innermost, read
+// MN-major). MODE_WGRAD: both operands stored [K rows][M] and [K rows][N]
+// (read MN-major), K running over each expert's row range.
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2, MODE_WGRAD = 3, MODE_DOWN_KN = 4 };
+constexpr int MN_CHUNK_BYTES = BK * 64 * 2;  // 64 MN elements x 64 K rows of an MN-major operand
 
 struct Args {
   const int32_t* offsets;
@@ -97,10 +101,9 @@ struct __align__(8) Ctl {
 constexpr int EPI_BYTES = 4 * kStageFloatsPerWarp * 4;  // epilogue staging, one block per warp
 constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(Ctl);
 
-constexpr uint32_t kIdesc128 = make_idesc(128, UMMA_N);
-// M=64 tail tiles: the accumulator then occupies TMEM lanes 0-15 of each
-// 32-lane sub-partition (tile row r -> lane (r % 16) + 32 * (r / 16)).
-constexpr uint32_t kIdesc64 = make_idesc(64, UMMA_N);
+// Tiles of M=128, or M=64 for a segment's last 64 rows or fewer: the
+// accumulator then occupies TMEM lanes 0-15 of each 32-lane sub-partition
+// (tile row r -> lane (r % 16) + 32 * (r / 16)).
 
 struct TileCoord {
   int e, row0, row_end, n_idx, kt0, kt1, split;
@@ -217,13 +220,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_arrive_expect_tx(&ctl->full[stage],
                                 MODE == MODE_LOGITS ? (uint32_t)(A_BYTES + args.n_mma * BK * 2) : STAGE_BYTES);
           const int k0 = kt * BK;
-          tma_load_2d(sa, &tmA, &ctl->full[stage], k0, tc.row0);
-          if (MODE == MODE_GATE_UP) {
-            const int n0 = tc.n_idx * 128;  // gate rows, then the matching up rows
-            tma_load_4d(sb, &tmB, &ctl->full[stage], k0, n0, 0, tc.e);
-            tma_load_4d(sb + B_BYTES / 2, &tmB, &ctl->full[stage], k0, n0, 1, tc.e);
+          if (MODE == MODE_WGRAD) {
+            // 64-column chunks of the [K rows][M] and [K rows][N] operands
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j)
+              tma_load_2d(sa + j * MN_CHUNK_BYTES, &tmA, &ctl->full[stage], tc.row0 + 64 * j, k0);
+#pragma unroll
+            for (int j = 0; j < UMMA_N / 64; ++j)
+              tma_load_2d(sb + j * MN_CHUNK_BYTES, &tmB, &ctl->full[stage], tc.n_idx * UMMA_N + 64 * j, k0);
           } else {
-            tma_load_3d(sb, &tmB, &ctl->full[stage], k0, tc.n_idx * UMMA_N, MODE == MODE_WGRAD ? 0 : tc.e);
+            tma_load_2d(sa, &tmA, &ctl->full[stage], k0, tc.row0);
+            if (MODE == MODE_GATE_UP) {
+              const int n0 = tc.n_idx * 128;  // gate rows, then the matching up rows
+              tma_load_4d(sb, &tmB, &ctl->full[stage], k0, n0, 0, tc.e);
+              tma_load_4d(sb + B_BYTES / 2, &tmB, &ctl->full[stage], k0, n0, 1, tc.e);
+            } else if (MODE == MODE_DOWN_KN) {
+#pragma unroll
+              for (int j = 0; j < UMMA_N / 64; ++j)
+                tma_load_3d(sb + j * MN_CHUNK_BYTES, &tmB, &ctl->full[stage], tc.n_idx * UMMA_N + 64 * j, k0, tc.e);
+            } else {
+              tma_load_3d(sb, &tmB, &ctl->full[stage], k0, tc.n_idx * UMMA_N, MODE == MODE_LOGITS ? 0 : tc.e);
+            }
           }
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -247,20 +264,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
+        constexpr bool a_mn = MODE == MODE_WGRAD;
+        constexpr bool b_mn = MODE == MODE_WGRAD || MODE == MODE_DOWN_KN;
         const uint32_t idesc = MODE == MODE_LOGITS ? make_idesc(tc.m64 ? 64 : 128, args.n_mma)
-                                                   : (tc.m64 ? kIdesc64 : kIdesc128);
+                                                   : make_idesc_mn(tc.m64 ? 64 : 128, UMMA_N, a_mn, b_mn);
         for (int kt = tc.kt0; kt < tc.kt1; ++kt) {
           if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, args.err, 3)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(base + stage * STAGE_BYTES);
-          const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+          const uint64_t adesc = a_mn ? sw128_mn_desc(sa, MN_CHUNK_BYTES) : sw128_desc(sa);
+          const uint64_t bdesc = b_mn ? sw128_mn_desc(sa + A_BYTES, MN_CHUNK_BYTES) : sw128_desc(sa + A_BYTES);
+          // K by 16: 32 bytes along a K-major 128-byte row, or 16 rows (2048
+          // bytes) of an MN-major chunk (descriptor units of 16 bytes)
+          constexpr uint64_t a_step = a_mn ? 128 : 2;
+          constexpr uint64_t b_step = b_mn ? 128 : 2;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            // advance K by 16 bf16 = 32 bytes inside the swizzled 128-byte row
-            umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
-                      (kt > tc.kt0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            umma_bf16(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kt > tc.kt0 || kk > 0) ? 1u : 0u);
           umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -312,7 +332,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             store_block_f32(z, stage, orow0 + cb, args.ldo, nrows, args.N - cb, lane);
           }
         }
-      } else if (MODE == MODE_DOWN) {
+      } else if (MODE == MODE_DOWN || MODE == MODE_DOWN_KN) {
         float sc = 1.f;
         if (valid && args.row_scale != nullptr) sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
         epilogue_scale_f32(tbase, UMMA_N / 32, sc, stage,
@@ -399,11 +419,15 @@ cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensor
 
 }  // namespace
 
-// Weight gradients: out[e][m][n] = sum over k in [koff[e], koff[e+1])
-// of AT[m][k] * BT[n][k], AT [M][ld] and BT [N][ld] bf16 (K-major, each
-// expert's rows a zero-padded run of columns), out fp32 [E][M][N].
-cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32_t* koff, int E, int64_t M, int64_t N,
-                         float* out, int32_t* err, cudaStream_t s) {
+// Weight gradients: out[e][m][n] = sum over rows k in [koff[e], koff[e+1])
+// of A[k][m] * B[k][n]. A [rows][lda] and B [rows][ldb] are bf16 row-major
+// (M and N used columns, read MN-major); rows at or past `rows` read as zero,
+// so a K range may run past the last row. koff: E+1 non-decreasing multiples
+// of 64 within [0, k_extent]. out fp32 [E][M][N]; an expert with an empty
+// range gets zeros.
+cudaError_t launch_wgrad(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t rows, const int32_t* koff,
+                         int64_t k_extent, int E, int64_t M, int64_t N, float* out, int32_t* err, cudaStream_t s) {
+  if (!get_encode()) return cudaErrorNotSupported;
   static std::once_flag attr_once[kSmemAttrDevices];
   static cudaError_t attr_status[kSmemAttrDevices];
   const void* kernel = reinterpret_cast<const void*>(tc_grouped_gemm_kernel<MODE_WGRAD>);
@@ -411,16 +435,16 @@ cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap tmA, tmB;
   {
-    const uint64_t dims[2] = {(uint64_t)ld, (uint64_t)M};
-    const uint64_t strides[1] = {(uint64_t)ld * 2};
-    const uint32_t box[2] = {BK, BM};
-    if (!make_tensor_map_bf16(&tmA, AT, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    const uint64_t dims[2] = {(uint64_t)M, (uint64_t)rows};
+    const uint64_t strides[1] = {(uint64_t)lda * 2};
+    const uint32_t box[2] = {64, BK};
+    if (!make_tensor_map_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[3] = {(uint64_t)ld, (uint64_t)N, 1};
-    const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)ld * N * 2};
-    const uint32_t box[3] = {BK, UMMA_N, 1};
-    if (!make_tensor_map_bf16(&tmB, BT, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)rows};
+    const uint64_t strides[1] = {(uint64_t)ldb * 2};
+    const uint32_t box[2] = {64, BK};
+    if (!make_tensor_map_bf16(&tmB, B, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   Args a{};
   a.offsets = koff;
@@ -431,7 +455,7 @@ cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32
   a.ldo = N;
   a.out = out;
   a.err = err;
-  a.rows_total = ld;  // K extent of the operands
+  a.rows_total = k_extent;  // bound of the K ranges
   a.M = (int32_t)M;
   a.m_tiles = (int32_t)ceil_div(M, BM);
   a.n_mma = UMMA_N;
@@ -531,6 +555,29 @@ cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down
     if (!make_tensor_map_bf16(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   return launch_tc<MODE_DOWN>(sg, tmA, tmB, H, I, y, H, row_scale, scale_idx, err, s);
+}
+
+cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+                              const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
+                              cudaStream_t s) {
+  if (!get_encode()) return cudaErrorNotSupported;
+  if (tc_gemm_variant(sg, true) == 2)
+    return launch_tc2_down_kn(sg, A, w_kn, E_w, y, row_scale, scale_idx, N, K, err, num_sms(), s);
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)sg.rows_total};
+    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!make_tensor_map_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    // B [E][K][N]: dim0 = N, dim1 = K, dim2 = expert; 64-column chunks of BK rows
+    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E_w};
+    const uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)K * N * 2};
+    const uint32_t box[3] = {64, BK, 1};
+    if (!make_tensor_map_bf16(&tmB, w_kn, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  return launch_tc<MODE_DOWN_KN>(sg, tmA, tmB, N, K, y, N, row_scale, scale_idx, err, s);
 }
 
 int tc_router_splits(int64_t T, int64_t H, int64_t E) {

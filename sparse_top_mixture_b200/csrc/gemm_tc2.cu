@@ -72,7 +72,11 @@ struct Ring {
   static_assert(STAGES >= 2 && STAGES <= MAX_STAGES, "ring depth");
 };
 
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
+// MODE_DOWN_KN: the down epilogue over B stored [E][K][N] (N innermost),
+// read MN-major: each CTA's 128 B columns are two 64-column chunks of 64 K
+// rows (one K atom per stage only).
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_DOWN_KN = 2 };
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;
 
 struct Args2 {
   const int32_t* offsets;
@@ -119,6 +123,7 @@ constexpr size_t smem_bytes2() {
 }
 static_assert(smem_bytes2<MODE_GATE_UP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 static_assert(smem_bytes2<MODE_DOWN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
+static_assert(smem_bytes2<MODE_DOWN_KN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
@@ -148,6 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   constexpr int A_BYTES = Ring<KA>::A_BYTES;
   constexpr int B_BYTES = Ring<KA>::B_BYTES;
   constexpr int STAGE_BYTES = Ring<KA>::STAGE_BYTES;
+  static_assert(MODE != MODE_DOWN_KN || KA == 1, "MN-major B takes one K atom per stage");
   uint8_t* base;
   if constexpr (MODE == MODE_GATE_UP) {
     extern __shared__ uint8_t smem_gu[];
@@ -233,6 +239,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 tma2_load_5d(sb + a * ATOM_BYTES + ATOM_BYTES / 2, &tmB64, full_leader, cx, n0, cz + a, 1, tc.e);
               }
             }
+          } else if (MODE == MODE_DOWN_KN) {
+            const int n0 = tc.n_idx * UMMA_N + (int)rank * HALF;
+            tma2_load_3d(sb, &tmB, full_leader, n0, ka * BK, tc.e);
+            tma2_load_3d(sb + MN_CHUNK_BYTES, &tmB, full_leader, n0 + 64, ka * BK, tc.e);
           } else {
             tma2_load_4d(sb, &tmB, full_leader, cx, tc.n_idx * UMMA_N + (int)rank * HALF, cz, tc.e);
           }
@@ -259,7 +269,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const Tile2 tc = decode_tile2(ctl, Eseg, args.n_tiles, tile);
-        const uint32_t idesc = tc.tail ? kIdesc128 : kIdesc256;
+        constexpr uint32_t b_mn = MODE == MODE_DOWN_KN ? 1u << 16 : 0u;  // B MN-major
+        const uint32_t idesc = (tc.tail ? kIdesc128 : kIdesc256) | b_mn;
         if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, args.err, 12)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * UMMA_N);
@@ -270,10 +281,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int a = 0; a < KA; ++a) {
             const uint64_t adesc = sw128_desc(sa + a * ATOM_BYTES);
-            const uint64_t bdesc = sw128_desc(sa + A_BYTES + a * ATOM_BYTES);
+            const uint64_t bdesc = MODE == MODE_DOWN_KN ? sw128_mn_desc(sa + A_BYTES, MN_CHUNK_BYTES)
+                                                        : sw128_desc(sa + A_BYTES + a * ATOM_BYTES);
+            // K by 16: 32 bytes along a K-major row; 16 rows (2048 bytes) of an
+            // MN-major chunk (descriptor units of 16 bytes)
+            constexpr uint64_t b_step = MODE == MODE_DOWN_KN ? 128 : 2;
 #pragma unroll
             for (int kk = 0; kk < BK / UMMA_K; ++kk)
-              umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+              umma2_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + b_step * kk, idesc,
                          (kt > 0 || a > 0 || kk > 0) ? 1u : 0u);
           }
           umma2_commit_mc(&ctl->empty[stage], 0x3);
@@ -455,6 +470,19 @@ cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_dow
   if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
   if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
   return launch_tc2<MODE_DOWN, KA>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+}
+
+cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+                               const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
+                               int num_sms, cudaStream_t s) {
+  CUtensorMap tmA, tmB;
+  // A: [rows, K] (3-D loads); B [E][K][N] (3-D loads of 64 columns x 64 K rows)
+  if (!map_kmajor(&tmA, A, 1, K, sg.rows_total, K * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
+  const uint64_t dims[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E_w};
+  const uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)K * N * 2};
+  const uint32_t box[3] = {64, BK, 1};
+  if (!make_tensor_map_bf16(&tmB, w_kn, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  return launch_tc2<MODE_DOWN_KN, 1>(sg, tmA, tmB, tmB, N, K, y, N, row_scale, scale_idx, err, num_sms, s);
 }
 
 }  // namespace stm

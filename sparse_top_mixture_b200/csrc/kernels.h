@@ -132,11 +132,21 @@ int tc_router_splits(int64_t T, int64_t H, int64_t E);
 cudaError_t launch_tc_logits(const void* x, const void* gate_w, int64_t T, int64_t H, int64_t E, float* partial,
                              int64_t ldo, int splits, int32_t* err, cudaStream_t s);
 // Weight-gradient GEMM: out[e][m][n] = sum_{k in [koff[e], koff[e+1])}
-// AT[m][k] * BT[n][k]; AT [M][ld], BT [N][ld] bf16, koff [E+1] on the device
-// (non-decreasing multiples of 64, at most ld), out fp32 [E][M][N]; an expert
-// with an empty range gets zeros.
-cudaError_t launch_wgrad(const void* AT, const void* BT, int64_t ld, const int32_t* koff, int E, int64_t M, int64_t N,
-                         float* out, int32_t* err, cudaStream_t s);
+// A[k][m] * B[k][n]; A [rows][lda] and B [rows][ldb] bf16 row-major (read
+// MN-major; rows at or past `rows` read as zero), koff [E+1] on the device
+// (non-decreasing multiples of 64, at most k_extent), out fp32 [E][M][N]; an
+// expert with an empty range gets zeros.
+cudaError_t launch_wgrad(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t rows, const int32_t* koff,
+                         int64_t k_extent, int E, int64_t M, int64_t N, float* out, int32_t* err, cudaStream_t s);
+// y[p][n] = scale(p) * sum_k A[p][k] * W[e][k][n] over the segments, with W
+// stored [E_w][K][N] (N innermost, read MN-major: no transposed copy); A
+// [rows][K] bf16, y fp32 [rows][N]. The one-CTA or pair kernel as for down.
+cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+                              const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
+                              cudaStream_t s);
+cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+                               const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
+                               int num_sms, cudaStream_t s);
 cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down, int64_t E_w, void* y,
                            const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, int32_t* err,
                            cudaStream_t s);

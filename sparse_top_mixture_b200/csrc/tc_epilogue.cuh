@@ -74,21 +74,35 @@ __device__ __forceinline__ void epilogue_swiglu(uint32_t tbase, int gcol, int uc
 }
 
 // down: y = sc * accumulator in fp32 for `nchunks` chunks of 32 columns
-// starting at TMEM column 0 and output column col0. sc is this lane's row scale.
+// starting at TMEM column 0 and output column col0. sc is this lane's row
+// scale. Two register buffers: the next chunk's TMEM load is in flight while
+// this one is staged and stored (the loads' latency, not the stores, bounded
+// the epilogue when the K loop is short).
 __device__ __forceinline__ void epilogue_scale_f32(uint32_t tbase, int nchunks, float sc, float* stage,
                                                    float* out_row0, int64_t ldo, int nrows, int col0, int N,
                                                    int lane) {
-#pragma unroll 1
-  for (int c = 0; c < nchunks; ++c) {
-    uint32_t d[32];
-    tmem_ld32(tbase + c * 32, d);
-    tmem_ld_wait();
+  auto store = [&](const uint32_t(&d)[32], int c) {
     const int cb = col0 + c * 32;
-    if (cb >= N || nrows <= 0) continue;  // warp-uniform
+    if (cb >= N || nrows <= 0) return;  // warp-uniform
     float v[32];
 #pragma unroll
     for (int q = 0; q < 32; ++q) v[q] = sc * __uint_as_float(d[q]);
     store_block_f32(v, stage, out_row0 + cb, ldo, nrows, N - cb, lane);
+  };
+  uint32_t a[32], b[32];
+  tmem_ld32(tbase, a);
+  tmem_ld_wait_regs(a);
+#pragma unroll 1
+  for (int c = 0; c < nchunks; c += 2) {  // a holds chunk c
+    const bool two = c + 1 < nchunks;
+    if (two) tmem_ld32(tbase + (c + 1) * 32, b);
+    store(a, c);
+    if (!two) break;
+    tmem_ld_wait_regs(b);
+    const bool more = c + 2 < nchunks;
+    if (more) tmem_ld32(tbase + (c + 2) * 32, a);
+    store(b, c + 1);
+    if (more) tmem_ld_wait_regs(a);
   }
 }
 

@@ -145,6 +145,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// The same wait, with the 32 destination registers of an earlier tmem_ld32
+// as operands, so that no use of them can be scheduled before it (needed
+// when other work runs between the load and the wait).
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row core groups 1024 bytes apart (tcgen05 descriptor format:
 // start>>4 in bits 0-13, LBO>>4 in 16-29, SBO>>4 in 32-45, version 1 in
@@ -159,10 +173,30 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle. The
+// operand is stored as chunks of 64 consecutive M (or N) elements: each chunk
+// is a run of K rows of 128 bytes (a TMA box {64, rows} with the MN index
+// innermost), 8-row groups 1024 bytes apart (SBO), consecutive chunks
+// `chunk_bytes` apart (LBO). One K step of 16 rows is 2048 bytes.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t chunk_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((chunk_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9 and 10-12 = 1), both K-major, N>>3 in bits 17-22, M>>4 in 24-28.
 constexpr uint32_t make_idesc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// The same with A (bit 15) and/or B (bit 16) MN-major.
+constexpr uint32_t make_idesc_mn(int M, int N, bool a_mn, bool b_mn) {
+  return make_idesc(M, N) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
 }
 
 

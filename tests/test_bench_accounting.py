@@ -30,6 +30,19 @@ def test_backward_flops_count_every_contraction(name):
 
 
 @pytest.mark.parametrize("name", list(CONFIGS))
+def test_backward_bytes_count_every_tensor(name):
+    c = CONFIGS[name]
+    es = 4 if c.dtype == "f32" else 2
+    active = min(c.E, c.T * c.k) // 2 or 1
+    gu, dn, gw = 2 * c.I * c.H, c.H * c.I, c.E * c.H  # elements of one expert's gate_up, down; the router
+    sh = 3 * c.I_shared * c.H + (c.H if c.shared == "sigmoid_gated" else 0)
+    reads = es * (active * (gu + dn) + gw + sh + 2 * c.T * c.H)              # weights in use, x, dout
+    writes = 4 * (c.E * (gu + dn) + gw + sh + c.T * c.H                      # every gradient, dx
+                  + (c.E if c.bias_mode == "logit" else 0))                  # d_bias
+    assert bench.backward_bytes(c, active, es) == pytest.approx(reads + writes, rel=1e-12)
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
 def test_forward_accounting(name):
     c = CONFIGS[name]
     P = c.T * c.k

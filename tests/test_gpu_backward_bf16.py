@@ -120,3 +120,56 @@ def test_bf16_backward_is_deterministic():
     for key in KEYS:
         if a[key] is not None:
             assert torch.equal(a[key], b[key]), key
+
+
+@pytest.mark.parametrize("name", ["dsv4_flash_ablation", "decode_weight_streaming"])
+def test_bf16_backward_in_a_cuda_graph_matches_eager(name):
+    """The whole backward captured as one CUDA graph (global capture mode:
+    nothing in it may allocate or synchronise) replays to the eager call's
+    gradients bit for bit."""
+    cfg = NAMED[name]
+    cpu = workloads.generate(cfg, "cpu")
+    dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
+    sel = torch.from_numpy(gc.oracle_route(cfg, cpu)["selected_experts"]).cuda()
+    dout = torch.randn(cfg.T, cfg.H, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).cuda()
+    p = stm.Problem.from_config(cfg)
+    ws = torch.zeros(stm.backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    eager = stm.backward(p, dev, dev["x"], dout, sel, ws=ws)
+    eager = {k: (v.clone() if v is not None else None) for k, v in eager.items()}
+    out = {k: torch.full_like(v, float("nan")) for k, v in eager.items() if v is not None}
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="global"):
+        stm.backward(p, dev, dev["x"], dout, sel, ws=ws, out=out)
+    for _ in range(2):
+        graph.replay()
+        torch.cuda.synchronize()
+        for key, v in out.items():
+            assert torch.equal(v, eager[key]), key
+    del graph
+    assert stm.read_device_error(ws) == 0
+
+
+def test_bf16_backward_flags_bad_expert_id():
+    """A pair with an expert id outside [0, E) contributes nothing (its
+    routing-weight gradient is zero) and raises the workspace flag; every
+    other token's dx is unchanged."""
+    cfg = GRID["softmax-none-renorm-none"].replace(name="bad16", T=60, H=48, E=6, k=2, I=32, renormalize=False)
+    cpu = workloads.generate(cfg, "cpu")
+    dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
+    sel = gc.oracle_route(cfg, cpu)["selected_experts"].copy()
+    sel[9, 1] = cfg.E + 2
+    sel[30, 0] = -1
+    p = stm.Problem.from_config(cfg)
+    ws = torch.zeros(stm.backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    dout = torch.randn(cfg.T, cfg.H, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    got = stm.backward(p, dev, dev["x"], dout.cuda(), torch.from_numpy(sel).cuda(), ws=ws)
+    torch.cuda.synchronize()
+    assert stm.read_device_error(ws) == stm.DEVERR_BAD_EXPERT_ID
+    # without renormalisation a slot's weight is its own score: every token
+    # but the two with a dropped pair matches the oracle of the valid choice
+    ref = _oracle_grads(cfg, cpu, gc.np64(dout), np.where((sel < 0) | (sel >= cfg.E), 0, sel))
+    dx = got["dx"].cpu().numpy().astype(np.float64)
+    assert np.isfinite(dx).all()
+    keep = ~np.isin(np.arange(cfg.T), [9, 30])
+    assert gc.rel_l2(dx[keep], ref["dx"][keep]) <= 5e-3
