@@ -340,14 +340,14 @@ typedef struct moe_grads {
  *   is needed besides the choice.
  *   fp32 problems run on SIMT kernels in fp32 throughout. bf16 problems
  *   (x, dout and the weights bf16) run the expert GEMMs on the tensor cores
- *   and the router's logits and weight gradient on the tensor cores (bf16
+ *   and the router's logits, weight gradient and dx on the tensor cores (bf16
  *   operands, fp32 accumulation; [dg du], w*dout, h and dlogits are rounded
  *   to bf16 where they become operands; the weights are read as stored, no
  *   transposed copy is made), the rest in fp32; the gradients are fp32 for
  *   both. Nothing in the call allocates or waits on the host: it can be
  *   captured in a CUDA graph. Every gradient element is an fp32 sum in a fixed
- *   order (no atomics; the router weight gradient adds row-chunk partial sums
- *   in chunk order): results are deterministic. A pair with an expert id outside [0, E) contributes
+ *   order (no atomics; the fp32 router weight gradient adds row-chunk partial
+ *   sums in chunk order): results are deterministic. A pair with an expert id outside [0, E) contributes
  *   nothing and sets MOE_DEVERR_BAD_EXPERT_ID in the workspace header.
  *   Workspace: moe_backward_workspace_size bytes (its header as for
  *   moe_forward, zeroed by moe_workspace_init). Async on `stream`. */

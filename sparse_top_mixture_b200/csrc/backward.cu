@@ -680,14 +680,16 @@ __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int
 // Padded row buffers, one block per 64-row group (an expert's run starts at a
 // multiple of 64, so a group lies in one expert e). Row q = koff[e] + j holds,
 // for j < count_e and r = off[e] + j: x_pad[q] = x[tok[r]] and dy_pad[q] =
-// bf16(scale[r] * dout[tok[r]]); rows with j >= count_e are zero in x_pad,
-// dy_pad, h_pad [*, I] and dgdu_pad [*, 2I] (the SwiGLU backward writes the
-// others). 16-byte vectors (H and I are multiples of 8).
+// bf16(scale[r] * dout[tok[r]]); also dout_perm[r] = dout[tok[r]] (the sorted
+// rows of dout, dense). Rows with j >= count_e are zero in x_pad, dy_pad,
+// h_pad [*, I] and dgdu_pad [*, 2I] (the SwiGLU backward writes the others).
+// 16-byte vectors (H and I are multiples of 8).
 __global__ void __launch_bounds__(BT) bw16_pad_rows(const __nv_bfloat16* __restrict__ x,
                                                   const __nv_bfloat16* __restrict__ dout,
                                                   const int32_t* __restrict__ tok, const float* __restrict__ scale,
                                                   const int32_t* __restrict__ off, const int32_t* __restrict__ koff,
-                                                  int E, int H, int I, __nv_bfloat16* __restrict__ x_pad,
+                                                  int E, int H, int I, __nv_bfloat16* __restrict__ dout_perm,
+                                                  __nv_bfloat16* __restrict__ x_pad,
                                                   __nv_bfloat16* __restrict__ dy_pad,
                                                   __nv_bfloat16* __restrict__ h_pad,
                                                   __nv_bfloat16* __restrict__ dgdu_pad) {
@@ -731,8 +733,10 @@ __global__ void __launch_bounds__(BT) bw16_pad_rows(const __nv_bfloat16* __restr
     uint4 xo = zero, yo = zero;
     if (src >= 0) {
       xo = reinterpret_cast<const uint4*>(x + (int64_t)src * H)[v];
+      const uint4 d = reinterpret_cast<const uint4*>(dout + (int64_t)src * H)[v];
+      reinterpret_cast<uint4*>(dout_perm + (int64_t)(off[e] + j0 + i) * H)[v] = d;
       float f[8];
-      unpack16_bf16(reinterpret_cast<const uint4*>(dout + (int64_t)src * H)[v], f);
+      unpack16_bf16(d, f);
       const float sc = s_sc[i];
       yo = make_uint4(pack_bf16x2(sc * f[0], sc * f[1]), pack_bf16x2(sc * f[2], sc * f[3]),
                       pack_bf16x2(sc * f[4], sc * f[5]), pack_bf16x2(sc * f[6], sc * f[7]));
@@ -827,6 +831,32 @@ __global__ void __launch_bounds__(BT) bw16_swiglu_rows(const float* __restrict__
   }
 }
 
+// out[t][h] += add[t][h] (+ dz[t] * g[h] when dz is given), fp32.
+__global__ void __launch_bounds__(BT) bw16_add_rows(float* __restrict__ out, const float* __restrict__ add,
+                                                  const float* __restrict__ dz, const float* __restrict__ g, int T,
+                                                  int H) {
+  const int hv = H / 4;
+  const int64_t n = (int64_t)T * hv;
+  for (int64_t idx = blockIdx.x * (int64_t)BT + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * BT) {
+    const int64_t t = idx / hv;
+    const int h = (int)(idx - t * hv) * 4;
+    float4 o = reinterpret_cast<float4*>(out)[idx];
+    const float4 a = reinterpret_cast<const float4*>(add)[idx];
+    o.x += a.x;
+    o.y += a.y;
+    o.z += a.z;
+    o.w += a.w;
+    if (dz) {
+      const float z = dz[t];
+      o.x = fmaf(z, g[h], o.x);
+      o.y = fmaf(z, g[h + 1], o.y);
+      o.z = fmaf(z, g[h + 2], o.z);
+      o.w = fmaf(z, g[h + 3], o.w);
+    }
+    reinterpret_cast<float4*>(out)[idx] = o;
+  }
+}
+
 // out[t][h] = bf16(gamma[t] * in[t][h]), eight columns per thread (H a multiple of 8).
 __global__ void __launch_bounds__(BT) bw16_scale_rows(const __nv_bfloat16* __restrict__ in,
                                                     const float* __restrict__ gamma, int T, int H,
@@ -845,9 +875,9 @@ __global__ void __launch_bounds__(BT) bw16_scale_rows(const __nv_bfloat16* __res
 }
 
 struct BwLayout16 {
-  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, dL16, lpart, x32, gw32,
-      g32, koff, ranges, xperm, doutperm, gu, dhu, dgdu, dxr, extra, xpad, dypad, hpad, dgdupad, gus, dhus, hs, dgdus,
-      dys, gamma, dz, total;
+  size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, dL16, lpart, x32, g32,
+      koff, ranges, xperm, doutperm, gu, dhu, dgdu, dxr, extra, xpad, dypad, hpad, dgdupad, gus, dhus, hs, dgdus, dys,
+      rdx, gamma, dz, total;
   int64_t Ppad, Tpad, Epad;
 };
 
@@ -879,9 +909,9 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.dL = take((size_t)p.T * p.E * f);
   b.dL16 = take((size_t)p.T * b.Epad * h2);
   b.lpart = take(router_partial_bytes(MOE_DTYPE_BF16, p.T, p.H, p.E));
-  b.x32 = take((size_t)p.T * p.H * f);
-  b.gw32 = take((size_t)p.E * p.H * f);
-  b.g32 = take((size_t)p.H * f);
+  const bool sh = p.shared != MOE_SHARED_NONE, gated = p.shared == MOE_SHARED_SIGMOID_GATED;
+  b.x32 = take(gated ? (size_t)p.T * p.H * f : 0);  // fp32 x for the shared gate's SIMT kernels
+  b.g32 = take(gated ? (size_t)p.H * f : 0);
   b.koff = take((size_t)(p.E + 1) * 4);
   b.ranges = take(4 * 4);
   b.xperm = take((size_t)P * p.H * h2);
@@ -895,13 +925,13 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.dypad = take((size_t)b.Ppad * p.H * h2);
   b.hpad = take((size_t)b.Ppad * p.I * h2);
   b.dgdupad = take((size_t)b.Ppad * 2 * p.I * h2);
-  const bool sh = p.shared != MOE_SHARED_NONE, gated = p.shared == MOE_SHARED_SIGMOID_GATED;
   const size_t Is = sh ? (size_t)p.I_shared : 0;
   b.gus = take((size_t)p.T * 2 * Is * f);
   b.dhus = take((size_t)p.T * Is * f);
   b.hs = take((size_t)p.T * Is * h2);
   b.dgdus = take((size_t)p.T * 2 * Is * h2);
   b.dys = take(gated ? (size_t)p.T * p.H * h2 : 0);
+  b.rdx = take(sh ? (size_t)p.T * p.H * f : 0);  // the router's dx beside the shared expert's
   b.gamma = take(sh ? (size_t)p.T * f : 0);
   b.dz = take(sh ? (size_t)p.T * f : 0);
   b.total = off;
@@ -935,8 +965,7 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   float* S = at<float>(ws, b.S);
   float* dL = at<float>(ws, b.dL);
   bf* dL16 = at<bf>(ws, b.dL16);
-  float* x32 = at<float>(ws, b.x32);
-  float* gw32 = at<float>(ws, b.gw32);
+  float* x32 = gated ? at<float>(ws, b.x32) : nullptr;
   float* g32 = gated ? at<float>(ws, b.g32) : nullptr;
   int32_t* koff = at<int32_t>(ws, b.koff);
   int32_t* ranges = at<int32_t>(ws, b.ranges);
@@ -952,10 +981,11 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   bf* hpad = at<bf>(ws, b.hpad);
   bf* dgdupad = at<bf>(ws, b.dgdupad);
 
-  // fp32 copies for the SIMT router and gate vector
-  bw16_to_f32<<<grid_for((int64_t)T * H), BT, 0, s>>>(x, (int64_t)T * H, x32);
-  bw16_to_f32<<<grid_for((int64_t)E * H), BT, 0, s>>>(static_cast<const bf*>(w->gate_w), (int64_t)E * H, gw32);
-  if (gated) bw16_to_f32<<<grid_for(H), BT, 0, s>>>(static_cast<const bf*>(w->shared_gate), H, g32);
+  // fp32 copies of x and the gate vector for the shared gate's SIMT kernels
+  if (gated) {
+    bw16_to_f32<<<grid_for((int64_t)T * H), BT, 0, s>>>(x, (int64_t)T * H, x32);
+    bw16_to_f32<<<grid_for(H), BT, 0, s>>>(static_cast<const bf*>(w->shared_gate), H, g32);
+  }
   // Router: logits on the tensor cores (the forward's split-K GEMM, its
   // partials summed in split order), then scores and the routing weights of
   // the given choice.
@@ -966,36 +996,38 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     bw16_sum_logits<<<grid_for((int64_t)T * E), BT, 0, s>>>(lpart, rp.splits, rp.ldo, T, E, L);
   }
   bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
-  // Sorted segments of the choice with x_perm; the same permutation of dout.
+  // Sorted segments of the choice with x_perm.
   BW16_CUDA(launch_dispatch(MOE_DTYPE_BF16, selected, x, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
                             at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, xperm, err,
                             &hdr->dispatch_ticket, s));
-  BW16_CUDA(launch_dispatch(MOE_DTYPE_BF16, selected, dout, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
-                            at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, doutperm, nullptr,
-                            &hdr->dispatch_ticket, s));
   bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, wts, E, k, tok, scale);
   bw16_koff<<<1, 32, 0, s>>>(offsets, E, T, koff, ranges);
-  // Padded rows of x and w dout for the weight gradients.
-  bw16_pad_rows<<<(unsigned)(b.Ppad / 64), BT, 0, s>>>(x, dout, tok, scale, offsets, koff, E, H, I, xpad, dypad, hpad,
-                                                       dgdupad);
+  // The sorted rows of dout; the padded rows of x and w dout for the weight gradients.
+  bw16_pad_rows<<<(unsigned)(b.Ppad / 64), BT, 0, s>>>(x, dout, tok, scale, offsets, koff, E, H, I, doutperm, xpad,
+                                                       dypad, hpad, dgdupad);
   // Routed experts on the tensor cores; the weights are read as stored.
   const Segments sg{offsets, (int32_t)E, 0, P};
   BW16_CUDA(launch_tc_down(sg, xperm, w->gate_up, E, gu, nullptr, nullptr, 2 * I, H, err, s));  // [g | u]
-  BW16_CUDA(launch_tc_down_kn(sg, doutperm, w->down, E, dhu, nullptr, nullptr, I, H, err, s));  // dhu
+  BW16_CUDA(launch_tc_down_kn(sg, doutperm, H, w->down, E, dhu, nullptr, nullptr, I, H, err, s));  // dhu
   // dw of pairs the dispatch dropped (bad expert ids) stays 0
   BW16_CUDA(cudaMemsetAsync(dw, 0, (size_t)P * sizeof(float), s));
   bw16_swiglu_rows<<<grid_for(P * 32), BT, 0, s>>>(gu, dhu, scale, offsets + E, P, I, offsets, koff, E, sorted_pairs,
                                                     nullptr, dw, dgdu, hpad, dgdupad);
-  BW16_CUDA(launch_tc_down_kn(sg, dgdu, w->gate_up, E, dxr, nullptr, nullptr, H, 2 * I, err, s));  // dx rows
+  BW16_CUDA(launch_tc_down_kn(sg, dgdu, 2 * I, w->gate_up, E, dxr, nullptr, nullptr, H, 2 * I, err, s));  // dx rows
   // Routed weight gradients: dWd = (w dout)^T h, dWgu = [dg du]^T x.
   BW16_CUDA(launch_wgrad(dypad, H, hpad, I, b.Ppad, koff, b.Ppad, E, H, I, g->d_down, err, s));
   BW16_CUDA(launch_wgrad(dgdupad, 2 * I, xpad, H, b.Ppad, koff, b.Ppad, E, 2 * I, H, g->d_gate_up, err, s));
-  // Router backward: dL (fp32, and rounded to bf16 for dgate_w = dL^T x over
-  // all tokens on the tensor cores); d_bias = sum_t dL in fp32.
+  // Router backward: dL (fp32, and rounded to bf16 for the tensor cores:
+  // dgate_w = dL^T x over all tokens, the router's dx = dL gate_w with gate_w
+  // [E][H] read as stored); d_bias = sum_t dL in fp32. The router's dx goes
+  // to `extra`, or beside the shared expert's when there is one.
   bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL, dL16,
                                  (int)b.Epad);
   BW16_CUDA(launch_wgrad(dL16, b.Epad, x, H, T, ranges + 2, b.Tpad, 1, E, H, g->d_gate_w, err, s));
   if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
+  const Segments one{nullptr, 1, (int32_t)T, p->T};
+  float* rdx = sh ? at<float>(ws, b.rdx) : extra;
+  BW16_CUDA(launch_tc_down_kn(one, dL16, b.Epad, w->gate_w, 1, rdx, nullptr, nullptr, H, E, err, s));
   // Shared expert over all tokens (one segment), scaled by gamma; its dx goes to `extra`.
   float* dz = nullptr;
   if (sh) {
@@ -1005,14 +1037,13 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     bf* dgdus = at<bf>(ws, b.dgdus);
     float* gamma = at<float>(ws, b.gamma);
     dz = at<float>(ws, b.dz);
-    const Segments one{nullptr, 1, (int32_t)T, p->T};
     bw_gamma<<<grid_for((int64_t)T * 32), BT, 0, s>>>(x32, g32, T, H, gamma);
     BW16_CUDA(launch_tc_down(one, x, w->shared_gate_up, 1, gus, nullptr, nullptr, 2 * Is, H, err, s));
-    BW16_CUDA(launch_tc_down_kn(one, dout, w->shared_down, 1, dhus, nullptr, nullptr, Is, H, err, s));
+    BW16_CUDA(launch_tc_down_kn(one, dout, H, w->shared_down, 1, dhus, nullptr, nullptr, Is, H, err, s));
     bw16_swiglu_rows<<<grid_for((int64_t)T * 32), BT, 0, s>>>(gus, dhus, gamma, nullptr, T, Is, nullptr, nullptr, 0,
                                                                nullptr, gamma, gated ? dz : nullptr, dgdus, hs,
                                                                nullptr);
-    BW16_CUDA(launch_tc_down_kn(one, dgdus, w->shared_gate_up, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
+    BW16_CUDA(launch_tc_down_kn(one, dgdus, 2 * Is, w->shared_gate_up, 1, extra, nullptr, nullptr, H, 2 * Is, err, s));
     // w dout for the shared expert is gamma dout (dout itself when ungated)
     const bf* dys = dout;
     if (gated) {
@@ -1023,15 +1054,10 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     BW16_CUDA(launch_wgrad(dys, H, hs, Is, T, ranges + 2, b.Tpad, 1, H, Is, g->d_shared_down, err, s));
     BW16_CUDA(launch_wgrad(dgdus, 2 * Is, x, H, T, ranges + 2, b.Tpad, 1, 2 * Is, H, g->d_shared_gate_up, err, s));
     if (gated) bw_dgvec<<<grid_for(H), BT, 0, s>>>(dz, x32, T, H, g->d_shared_gate);
+    // extra = the shared expert's dx + the router's (+ the shared gate's dz g)
+    bw16_add_rows<<<grid_for((int64_t)T * H / 4), BT, 0, s>>>(extra, rdx, gated ? dz : nullptr, g32, T, H);
   }
-  // Router (and shared gate) dx into `extra`, then dx = sum of each token's rows + extra.
-  RowGemm rd = row_gemm(dL, nullptr, E, gw32, 0, H, E, nullptr, 1, T, T, err);
-  rd.C = extra;
-  rd.ldc = H;
-  rd.dz = gated ? dz : nullptr;
-  rd.gvec = gated ? g32 : nullptr;
-  if (sh) BW16_CUDA(run_rows<false, EPI_ADD>(rd, s));
-  else BW16_CUDA(run_rows<false, EPI_STORE>(rd, s));
+  // dx = sum of each token's rows + extra.
   BW16_CUDA(launch_combine(MOE_DTYPE_F32, dxr, pair_pos, extra, g->dx, p->T, p->H, p->k, s));
   return MOE_OK;
 }

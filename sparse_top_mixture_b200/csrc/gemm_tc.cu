@@ -557,16 +557,16 @@ cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down
   return launch_tc<MODE_DOWN>(sg, tmA, tmB, H, I, y, H, row_scale, scale_idx, err, s);
 }
 
-cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,
                               const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
                               cudaStream_t s) {
   if (!get_encode()) return cudaErrorNotSupported;
   if (tc_gemm_variant(sg, true) == 2)
-    return launch_tc2_down_kn(sg, A, w_kn, E_w, y, row_scale, scale_idx, N, K, err, num_sms(), s);
+    return launch_tc2_down_kn(sg, A, lda, w_kn, E_w, y, row_scale, scale_idx, N, K, err, num_sms(), s);
   CUtensorMap tmA, tmB;
   {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)sg.rows_total};
-    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint64_t strides[1] = {(uint64_t)lda * 2};
     const uint32_t box[2] = {BK, BM};
     if (!make_tensor_map_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }

@@ -472,12 +472,12 @@ cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_dow
   return launch_tc2<MODE_DOWN, KA>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
 }
 
-cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,
                                const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
                                int num_sms, cudaStream_t s) {
   CUtensorMap tmA, tmB;
-  // A: [rows, K] (3-D loads); B [E][K][N] (3-D loads of 64 columns x 64 K rows)
-  if (!map_kmajor(&tmA, A, 1, K, sg.rows_total, K * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
+  // A: [rows, K] of pitch lda (3-D loads); B [E][K][N] (3-D loads of 64 columns x 64 K rows)
+  if (!map_kmajor(&tmA, A, 1, K, sg.rows_total, lda * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
   const uint64_t dims[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E_w};
   const uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)K * N * 2};
   const uint32_t box[3] = {64, BK, 1};

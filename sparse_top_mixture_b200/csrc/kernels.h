@@ -140,11 +140,12 @@ cudaError_t launch_wgrad(const void* A, int64_t lda, const void* B, int64_t ldb,
                          int64_t k_extent, int E, int64_t M, int64_t N, float* out, int32_t* err, cudaStream_t s);
 // y[p][n] = scale(p) * sum_k A[p][k] * W[e][k][n] over the segments, with W
 // stored [E_w][K][N] (N innermost, read MN-major: no transposed copy); A
-// [rows][K] bf16, y fp32 [rows][N]. The one-CTA or pair kernel as for down.
-cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+// [rows][lda] bf16 (K used columns, lda a multiple of 8), y fp32 [rows][N].
+// The one-CTA or pair kernel as for down.
+cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,
                               const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
                               cudaStream_t s);
-cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, const void* w_kn, int64_t E_w, void* y,
+cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,
                                const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
                                int num_sms, cudaStream_t s);
 cudaError_t launch_tc_down(const Segments& sg, const void* h, const void* w_down, int64_t E_w, void* y,

@@ -4,11 +4,11 @@ seeded bf16 inputs (converted exactly) and the oracle's own expert choice.
 
 Tolerance. The GPU rounds four intermediates to bf16 where they become GEMM
 operands: [dg du] (dx and dW_gate_up), w*dout and h (dW_down), and dlogits
-(the router's dgate_w); each rounding
+(the router's dgate_w and its share of dx); each rounding
 moves a value by at most 2^-9 of itself, products and sums are fp32. A
 gradient element therefore carries a relative error of about one or two
 bf16 roundings of the terms it sums (~1e-3 in L2 over a tensor, as for the
-forward); the logit bias and the router's dx come from fp32 dlogits.
+forward); the logit bias comes from fp32 dlogits.
 The bar: relative L2 <= 5e-3 per tensor (the problem's bf16 output bar) and
 no element off by more than 1e-2 of the tensor's largest magnitude.
 """
