@@ -660,10 +660,12 @@ __global__ void __launch_bounds__(BT) bw16_sum_logits(const float* __restrict__ 
 }
 
 // Padded row offsets of the weight-gradient GEMMs: koff[e] = sum over e' < e
-// of round_up(count[e'], 64); also the one-segment range of all tokens:
-// ranges = {0, T, 0, round_up(T, 64)}.
+// of round_up(count[e'], 64); also the one-segment range of all tokens,
+// ranges = {0, T, 0, round_up(T, 64)}, and its split into `splits` row
+// chunks of `chunk` rows (a multiple of 64) for the router's weight gradient:
+// rsplit[i] = min(i * chunk, round_up(T, 64)), i = 0..splits.
 __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int32_t* __restrict__ koff,
-                          int32_t* __restrict__ ranges) {
+                          int32_t* __restrict__ ranges, int splits, int chunk, int32_t* __restrict__ rsplit) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int run = 0;
   for (int e = 0; e < E; ++e) {
@@ -671,10 +673,12 @@ __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int
     run += (offsets[e + 1] - offsets[e] + 63) / 64 * 64;
   }
   koff[E] = run;
+  const int Tpad = (T + 63) / 64 * 64;
   ranges[0] = 0;
   ranges[1] = T;
   ranges[2] = 0;
-  ranges[3] = (T + 63) / 64 * 64;
+  ranges[3] = Tpad;
+  for (int i = 0; i <= splits; ++i) rsplit[i] = min(i * chunk, Tpad);
 }
 
 // Padded row buffers, one block per 64-row group (an expert's run starts at a
@@ -874,9 +878,24 @@ __global__ void __launch_bounds__(BT) bw16_scale_rows(const __nv_bfloat16* __res
   }
 }
 
+// Row chunks of the bf16 router weight gradient dgate_w = dL^T x: its [E, H]
+// output has few tiles and a T-long reduction, so the reduction is split
+// into at most 16 chunks of whole 64-row steps until about one tile per SM
+// is busy; the partial sums are added in chunk order.
+struct RouterSplit16 {
+  int splits, chunk;
+};
+RouterSplit16 router_split16(const moe_problem& p) {
+  const int64_t tiles = ceil_div(p.E, 128) * ceil_div(p.H, 256);
+  const int64_t steps = ceil_div(p.T, 64);
+  const int64_t want = std::max<int64_t>(1, std::min<int64_t>({ceil_div(148, tiles), steps, 16}));
+  const int64_t chunk = ceil_div(steps, want) * 64;
+  return {(int)ceil_div(round_up(p.T, 64), chunk), (int)chunk};
+}
+
 struct BwLayout16 {
   size_t header, local, counts, offsets, sorted_pairs, pair_pos, tok, scale, w, dw, L, S, dL, dL16, lpart, x32, g32,
-      koff, ranges, xperm, doutperm, gu, dhu, dgdu, dxr, extra, xpad, dypad, hpad, dgdupad, gus, dhus, hs, dgdus, dys,
+      koff, ranges, rsplit, parts, xperm, doutperm, gu, dhu, dgdu, dxr, extra, xpad, dypad, hpad, dgdupad, gus, dhus, hs, dgdus, dys,
       rdx, gamma, dz, total;
   int64_t Ppad, Tpad, Epad;
 };
@@ -914,6 +933,9 @@ BwLayout16 bw_layout16(const moe_problem& p) {
   b.g32 = take(gated ? (size_t)p.H * f : 0);
   b.koff = take((size_t)(p.E + 1) * 4);
   b.ranges = take(4 * 4);
+  const RouterSplit16 rs = router_split16(p);
+  b.rsplit = take((size_t)(rs.splits + 1) * 4);
+  b.parts = take(rs.splits > 1 ? (size_t)rs.splits * p.E * p.H * f : 0);
   b.xperm = take((size_t)P * p.H * h2);
   b.doutperm = take((size_t)P * p.H * h2);
   b.gu = take((size_t)P * 2 * p.I * f);
@@ -1001,7 +1023,9 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
                             at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, xperm, err,
                             &hdr->dispatch_ticket, s));
   bw_rows<<<grid_for(P), BT, 0, s>>>(sorted_pairs, offsets, wts, E, k, tok, scale);
-  bw16_koff<<<1, 32, 0, s>>>(offsets, E, T, koff, ranges);
+  const RouterSplit16 rs = router_split16(*p);
+  int32_t* rsplit = at<int32_t>(ws, b.rsplit);
+  bw16_koff<<<1, 32, 0, s>>>(offsets, E, T, koff, ranges, rs.splits, rs.chunk, rsplit);
   // The sorted rows of dout; the padded rows of x and w dout for the weight gradients.
   bw16_pad_rows<<<(unsigned)(b.Ppad / 64), BT, 0, s>>>(x, dout, tok, scale, offsets, koff, E, H, I, doutperm, xpad,
                                                        dypad, hpad, dgdupad);
@@ -1023,7 +1047,13 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   // to `extra`, or beside the shared expert's when there is one.
   bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL, dL16,
                                  (int)b.Epad);
-  BW16_CUDA(launch_wgrad(dL16, b.Epad, x, H, T, ranges + 2, b.Tpad, 1, E, H, g->d_gate_w, err, s));
+  if (rs.splits > 1) {
+    float* parts = at<float>(ws, b.parts);
+    BW16_CUDA(launch_wgrad(dL16, b.Epad, x, H, T, rsplit, b.Tpad, rs.splits, E, H, parts, err, s));
+    bw_sum_parts<<<grid_for((int64_t)E * H), BT, 0, s>>>(parts, rs.splits, (int64_t)E * H, g->d_gate_w);
+  } else {
+    BW16_CUDA(launch_wgrad(dL16, b.Epad, x, H, T, ranges + 2, b.Tpad, 1, E, H, g->d_gate_w, err, s));
+  }
   if (g->d_bias) bw_colsum<<<grid_for(E), BT, 0, s>>>(dL, E, T, E, g->d_bias);
   const Segments one{nullptr, 1, (int32_t)T, p->T};
   float* rdx = sh ? at<float>(ws, b.rdx) : extra;
