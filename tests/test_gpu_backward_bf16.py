@@ -32,8 +32,13 @@ NAMED = {
     "deepseek_v2_lite_zipf": reduced(CONFIGS["deepseek_v2_lite_zipf"], T=512, H=256, I=136, I_shared=272),
     "dsv4_flash_ablation": reduced(CONFIGS["dsv4_flash_ablation"], T=384, H=512, I=256, I_shared=256),
     "decode_weight_streaming": reduced(CONFIGS["decode_weight_streaming"], T=16, H=1024, I=256, I_shared=256),
-    # about 400 rows per expert: the data-gradient GEMMs run on CTA pairs
+    # about 400 rows per expert: the data-gradient GEMMs run on CTA pairs, the
+    # gate_up GEMM with the SwiGLU backward as its epilogue
     "pairs": CONFIGS["qwen3_30b_a3b"].replace(name="bw_pairs", T=1600, H=384, E=8, k=2, I=192),
+    # the same for a sigmoid-gated shared expert over 1024 tokens (its dz from
+    # the fused epilogue's dot partials), I and I_s not multiples of 128
+    "pairs_gated": CONFIGS["decode_weight_streaming"].replace(name="bw_pairs_gated", T=1024, H=256, E=8, k=2,
+                                                               I=136, I_shared=200),
 }
 
 GRID = {}
