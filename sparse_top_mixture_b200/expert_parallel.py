@@ -14,10 +14,12 @@ identical to the one-GPU forward is taken here:
   the library's kernels; because the dispatch sorts rows by expert, the rows
   bound for each rank form one contiguous run of x_perm, in rank order;
 * the per-expert counts go to their owners (an all-to-all of E/G counts per
-  peer). Before the host reads them, everything that needs no remote count
-  is enqueued: this rank's own run of x_perm through its own experts (the
-  grouped SwiGLU over the local experts' segments of the one-GPU segment
-  table, writing those rows of y_perm in place) and the shared expert;
+  peer). Everything that needs no remote count -- this rank's own run of
+  x_perm through its own experts (the grouped SwiGLU over the local experts'
+  segments of the one-GPU segment table, writing those rows of y_perm in
+  place) and the shared expert -- is enqueued first, on a second stream that
+  starts after the dispatch: the host read below waits only for the dispatch
+  and the count exchange, and the row exchanges overlap the local GEMMs;
 * one device-to-host read of the counts then sizes the remote exchange:
   point-to-point sends and receives, one group per exchange (rows, their
   routing weights and their local expert ids to each other rank; the
@@ -30,7 +32,7 @@ identical to the one-GPU forward is taken here:
   order;
 * the rows come back to their senders in the sender's x_perm order: with the
   local rows, exactly the y_perm of the one-GPU forward (fp32 rows), so the
-  combine finishes the layer as there.
+  combine finishes the layer as there, once the second stream has joined.
 
 Every per-row result is the same arithmetic as on one GPU; only where a row
 sits in a GEMM tile changes. The collectives are torch.distributed calls
@@ -40,6 +42,7 @@ every step of the layer's arithmetic runs in the library's CUDA kernels.
 
 from __future__ import annotations
 
+import contextlib
 import dataclasses
 from typing import Dict, List, Optional, Sequence, Tuple
 
@@ -95,15 +98,16 @@ def exchange_plan(counts: Sequence[int], recv_counts: np.ndarray, rank: int) -> 
 
 class WorkspacePool:
     """Library workspaces kept across calls: one per problem kind (the
-    problem with T set aside), replaced by a larger one only when a call
-    needs more bytes than the kept one has."""
+    problem with T set aside) and user (`slot`: work that may run at the same
+    time on two streams takes two slots), replaced by a larger one only when
+    a call needs more bytes than the kept one has."""
 
     def __init__(self, device):
         self.device = device
-        self._kept: Dict[Problem, Tuple[int, torch.Tensor]] = {}
+        self._kept: Dict[Tuple[Problem, str], Tuple[int, torch.Tensor]] = {}
 
-    def get(self, p: Problem) -> torch.Tensor:
-        key = dataclasses.replace(p, T=0)
+    def get(self, p: Problem, slot: str = "") -> torch.Tensor:
+        key = (dataclasses.replace(p, T=0), slot)
         need = workspace_size(p)
         kept = self._kept.get(key)
         if kept is None or kept[0] < need:
@@ -136,6 +140,7 @@ class ExpertParallelMoE:
         if tuple(gu.shape) != (self.E_local, 2 * p.I, p.H) or tuple(dn.shape) != (self.E_local, p.H, p.I):
             raise ValueError(f"local expert weights must be [{self.E_local}, 2I, H] and [{self.E_local}, H, I]")
         self.pool = WorkspacePool(gu.device)
+        self.side = torch.cuda.Stream(gu.device) if gu.is_cuda else None  # the local GEMMs' stream
 
     def _a2a(self, out: torch.Tensor, inp: torch.Tensor, out_splits, in_splits) -> None:
         import torch.distributed as dist
@@ -173,28 +178,33 @@ class ExpertParallelMoE:
         rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate, ws=ws)
         d = dispatch(p, sel, x, ws=ws)
 
+        # Work that needs no remote count, on the second stream from the end of
+        # the dispatch on: this rank's own rows through its own experts (rows
+        # of y_perm in place; as a problem of T*k one-slot rows over the E/G
+        # local experts: the same x_perm rows, routing weights and sorted pair
+        # indices) and the shared expert.
+        if self.side is not None:
+            main = torch.cuda.current_stream(dev)
+            self.side.wait_stream(main)
+        side_ctx = torch.cuda.stream(self.side) if self.side is not None else contextlib.nullcontext()
+        pl = dataclasses.replace(p, T=p.T * p.k, k=1, E=El, I_shared=0, shared="none", bias_mode="none")
+        own_offsets = d["offsets"][r * El:(r + 1) * El + 1]
+        shared = None
+        with side_ctx:
+            y_perm = grouped_swiglu(pl, d["x_perm"], own_offsets, w["gate_up"], w["down"], rw.view(-1, 1),
+                                    d["sorted_pairs"], ws=self.pool.get(pl, "local"))
+            self.trace.append("local_experts")
+            if self.side is not None:  # marks the local GEMM's place on the second stream (tests check it)
+                self.local_done = torch.cuda.Event()
+                self.local_done.record(self.side)
+            if p.shared != "none":
+                shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma, ws=ws)
+                self.trace.append("shared_expert")
+
         # counts to the experts' owners
         counts = d["counts"].to(torch.int64)
         recv_counts = torch.empty_like(counts)
         self._a2a(recv_counts, counts, None, None)
-
-        # Work that needs no remote count, enqueued before the host read: this
-        # rank's own rows through its own experts (rows of y_perm in place) ...
-        # (as a problem of T*k one-slot rows over the E/G local experts: the same
-        # x_perm rows, routing weights and sorted pair indices)
-        pl = dataclasses.replace(p, T=p.T * p.k, k=1, E=El, I_shared=0, shared="none", bias_mode="none")
-        own_offsets = d["offsets"][r * El:(r + 1) * El + 1]
-        y_perm = grouped_swiglu(pl, d["x_perm"], own_offsets, w["gate_up"], w["down"], rw.view(-1, 1),
-                                d["sorted_pairs"], ws=self.pool.get(pl))
-        self.trace.append("local_experts")
-        if x.is_cuda:  # marks the local GEMM's place in the stream (tests check it ran before the host read)
-            self.local_done = torch.cuda.Event()
-            self.local_done.record()
-        # ... and the shared expert
-        shared = None
-        if p.shared != "none":
-            shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma, ws=ws)
-            self.trace.append("shared_expert")
 
         # the host read sizes the remote exchange
         plan = exchange_plan(*self._host_counts(counts, recv_counts), r)
@@ -224,6 +234,11 @@ class ExpertParallelMoE:
         # weighted fp32 rows back to their senders, into y_perm in x_perm order
         self._exchange([(s, y_recv[recv_off[s]:recv_off[s] + recvs[s]]) for s in remote],
                        [(s, y_perm[send_off[s]:send_off[s + 1]]) for s in remote])
+        if self.side is not None:  # join: the local rows and the shared expert are done
+            main.wait_stream(self.side)
+            y_perm.record_stream(main)
+            if shared is not None:
+                shared.record_stream(main)
         return combine(p, y_perm, d["pair_pos"], shared), rw, sel
 
     __call__ = forward
@@ -236,7 +251,7 @@ class ExpertParallelMoE:
         if n == 0:
             return torch.zeros(0, p.H, dtype=torch.float32, device=x_recv.device)
         pr = dataclasses.replace(p, T=n, E=self.E_local, k=1, I_shared=0, bias_mode="none", shared="none")
-        ws = self.pool.get(pr)
+        ws = self.pool.get(pr, "remote")
         d = dispatch(pr, id_recv.view(n, 1), x_recv, ws=ws)
         y = grouped_swiglu(pr, d["x_perm"], d["offsets"], self.w["gate_up"], self.w["down"], w_recv.view(n, 1),
                            d["sorted_pairs"], ws=ws)

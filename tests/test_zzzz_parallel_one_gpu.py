@@ -51,17 +51,17 @@ def _child(name, port, q):
         res = {}
         ep_layer = ExpertParallelMoE(p, dev)
         # The expert-parallel layer enqueues its own rows' GEMM (and the shared
-        # expert) before its one host read of the counts: when that read is
-        # entered the local GEMM's event has been recorded, and when the read
-        # returns (it synchronises the stream) the GEMM has finished.
+        # expert) before its one host read of the counts, on a second stream:
+        # when that read is entered the local GEMM's event has been recorded,
+        # on a stream other than the one the read synchronises.
         seen = {}
         host_counts = ep_layer._host_counts
 
         def watched(counts, recv_counts):
             seen["recorded_before_read"] = hasattr(ep_layer, "local_done") and "local_experts" in ep_layer.trace
-            out_ = host_counts(counts, recv_counts)
-            seen["done_when_read_returns"] = ep_layer.local_done.query()
-            return out_
+            seen["on_second_stream"] = (ep_layer.side is not None and
+                                        ep_layer.side.cuda_stream != torch.cuda.current_stream().cuda_stream)
+            return host_counts(counts, recv_counts)
         ep_layer._host_counts = watched
         layers = (("ep", ep_layer), ("tp", TensorParallelMoE(p, shard_expert_weights(dev, 0, 1))))
         for label, layer in layers:
@@ -70,7 +70,8 @@ def _child(name, port, q):
             if label == "ep":
                 want = ["local_experts"] + (["shared_expert"] if cfg.shared != "none" else []) + ["host_counts"]
                 assert ep_layer.trace == want, ep_layer.trace
-                assert seen == {"recorded_before_read": True, "done_when_read_returns": True}, seen
+                assert seen == {"recorded_before_read": True, "on_second_stream": True}, seen
+                assert ep_layer.local_done.query()  # joined before the combine
             gsel = sel.cpu().numpy()
             ntie = gc.check_selection(cfg, r, gsel)
             assert ntie == gc.expected_near_ties(cfg.name), f"{name} {label}: {ntie} near-tie tokens"
