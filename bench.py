@@ -371,10 +371,12 @@ def backward_cpu_baseline(cfg32, inp, dout, target_s: float = 8.0) -> dict:
 
 def measure_backward(cfg, local: int, steps: int = 5, cpu: bool = False, dtype: str = "bf16") -> dict:
     """The backward on the given workload's shapes in ``dtype`` (bf16: the
-    tensor-core path, against the measured bf16 peak; f32: the SIMT path,
-    against the FFMA peak at the sampled SM clock), timed with CUDA events on
-    the current stream; with ``cpu``, the backward oracle timed on the host
-    beside it on the same inputs, widened to fp64."""
+    tensor-core path; f32: the SIMT path), timed with CUDA events on the
+    current stream, as eager C-ABI calls (``eager_ms``) and as replays of the
+    same call captured in a CUDA graph (``ms``); its roofline takes the larger
+    of its FLOPs at the bf16 (or FFMA, at the sampled SM clock) peak and its
+    algorithmic bytes at the HBM bandwidth. With ``cpu``, the backward oracle
+    timed on the host beside it on the same inputs, widened to fp64."""
     import sparse_top_mixture_b200 as stm
     c = cfg.replace(dtype=dtype)
     inp = workloads.generate(c, "cuda")
@@ -661,7 +663,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-graph", action="store_true", help="launch each kernel from the host every step")
-    ap.add_argument("--no-backward", action="store_true", help="skip the fp32 backward measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurements (bf16 and fp32)")
     ap.add_argument("--no-per-config", action="store_true", help="skip the per_config block (the other workloads)")
     ap.add_argument("--per-config-steps", type=int, default=50)
     ap.add_argument("--backward-only", action="store_true",
