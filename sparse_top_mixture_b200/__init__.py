@@ -87,6 +87,15 @@ SIGNATURES = {
     "moe_backward": (ctypes.c_int, [_PP, ctypes.POINTER(moe_weights), _VP, _VP, _VP, ctypes.POINTER(moe_grads), _VP,
                                     _SZ, _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_dispatch_slots": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_ep_arena_size": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_ep_arena_offsets": (ctypes.c_int, [_PP, ctypes.c_int32] + [ctypes.POINTER(ctypes.c_size_t)] * 6),
+    "moe_ep_send": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, ctypes.c_uint64, _VP, _VP, _VP, _VP,
+                                   _VP, _VP]),
+    "moe_ep_wait": (ctypes.c_int, [_PP, ctypes.c_int32, _VP, ctypes.c_int32, ctypes.c_uint64, ctypes.c_int64, _VP,
+                                   _VP]),
+    "moe_ep_return": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, ctypes.c_uint64, _VP, _VP, _VP,
+                                     _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -245,6 +254,24 @@ def dispatch(p: Problem, selected, x=None, ws=None) -> Dict[str, torch.Tensor]:
     _check(lib().moe_dispatch(ctypes.byref(p.c()), _ptr(selected), _ptr(x), _ptr(r["counts"]), _ptr(r["offsets"]),
                               _ptr(r["sorted_pairs"]), _ptr(r["pair_pos"]), _ptr(r["x_perm"]), ws.data_ptr(),
                               ws.numel(), _stream(dev)))
+    return r
+
+
+def dispatch_slots(p: Problem, selected, x=None, ws=None) -> Dict[str, torch.Tensor]:
+    """moe_dispatch over slots some of which are empty (ids outside [0, E),
+    e.g. -1): those are skipped (pair_pos -1) without an error flag."""
+    _req(selected, "selected", (p.T, p.k), torch.int64)
+    dev = selected.device
+    P = p.T * p.k
+    ws = new_workspace(p, dev) if ws is None else ws
+    r = {"counts": torch.empty(p.E, dtype=torch.int32, device=dev),
+         "offsets": torch.empty(p.E + 1, dtype=torch.int32, device=dev),
+         "sorted_pairs": torch.empty(P, dtype=torch.int32, device=dev),
+         "pair_pos": torch.empty(P, dtype=torch.int32, device=dev),
+         "x_perm": torch.empty(P, p.H, dtype=p.torch_dtype, device=dev) if x is not None else None}
+    _check(lib().moe_dispatch_slots(ctypes.byref(p.c()), _ptr(selected), _ptr(x), _ptr(r["counts"]),
+                                    _ptr(r["offsets"]), _ptr(r["sorted_pairs"]), _ptr(r["pair_pos"]),
+                                    _ptr(r["x_perm"]), ws.data_ptr(), ws.numel(), _stream(dev)))
     return r
 
 

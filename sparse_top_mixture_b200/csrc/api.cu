@@ -340,6 +340,28 @@ MOE_API moe_status moe_dispatch(const moe_problem* p, const int64_t* selected_ex
                      (cudaStream_t)stream);
 }
 
+MOE_API moe_status moe_dispatch_slots(const moe_problem* p, const int64_t* selected_experts, const void* x,
+                                      int32_t* counts, int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
+                                      void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (!ok_ptr(counts) || !ok_ptr(offsets)) return MOE_ERR_INVALID_ARGUMENT;
+  if (p->T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)p->E * 4, (cudaStream_t)stream));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(p->E + 1) * 4, (cudaStream_t)stream));
+    return MOE_OK;
+  }
+  if (!ok_ptr(selected_experts) || !ok_ptr(sorted_pairs) || !ok_ptr(pair_pos)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((x == nullptr) != (x_perm == nullptr) || !ok_opt(x) || !ok_opt(x_perm)) return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  // ids outside [0, E) are empty slots: skipped, no flag raised
+  MOE_CUDA(launch_dispatch(p->dtype, selected_experts, x, p->T, p->H, p->E, p->k, at<int32_t>(ws, L.local), counts,
+                           offsets, sorted_pairs, pair_pos, x_perm, nullptr, &hdr->dispatch_ticket,
+                           (cudaStream_t)stream));
+  return MOE_OK;
+}
+
 MOE_API moe_status moe_grouped_swiglu(const moe_problem* p, const void* x_perm, const int32_t* offsets,
                                       const void* gate_up, const void* down, const float* routing_weights,
                                       const int32_t* sorted_pairs, void* y_perm, void* ws, size_t ws_bytes,

@@ -149,3 +149,26 @@ def test_backward_validates_before_launching(L):
     wg = stm.moe_weights(16, None, 16, 16, 16, 16, 16)
     gg = stm.moe_grads(16, 16, None, 16, 16, 16, 16, None)
     assert L.moe_backward(ctypes.byref(pg), ctypes.byref(wg), 16, 16, 16, ctypes.byref(gg), 16, 1 << 40, None) == 1
+
+
+def test_ep_arena_layout(L):
+    """The expert-parallel arena's regions: 256-byte aligned, in order, each
+    large enough for what the exchange stores there (host-only calls)."""
+    from sparse_top_mixture_b200.ep_peer import ep_arena_offsets, ep_arena_size
+
+    for kw, G in ((dict(T=64, H=256, E=8, k=2), 2), (dict(T=300, H=328, E=128, k=8), 4),
+                  (dict(T=16, H=7168, E=256, k=8, dtype="f32"), 8), (dict(T=0, H=64, E=4, k=1), 1)):
+        p = _p(**kw)
+        C, es = p.T * p.k, (4 if p.dtype == "f32" else 2)
+        off = ep_arena_offsets(p, G)
+        order = ["rows_flag", "ret_flag", "x", "w", "id", "y"]
+        assert all(off[n] % 256 == 0 for n in order)
+        assert [off[n] for n in order] == sorted(off[n] for n in order)
+        assert off["ret_flag"] - off["rows_flag"] >= 8 * G
+        assert off["w"] - off["x"] >= G * C * p.H * es
+        assert off["id"] - off["w"] >= G * C * 4 and off["y"] - off["id"] >= G * C * 8
+        assert ep_arena_size(p, G) >= off["y"] + C * p.H * 4
+    bad = _p(E=6, k=2)
+    n = ctypes.c_size_t()
+    assert L.moe_ep_arena_size(ctypes.byref(bad.c()), 4, ctypes.byref(n)) == 1  # E not divisible by G
+    assert L.moe_ep_arena_size(ctypes.byref(bad.c()), 0, ctypes.byref(n)) == 1
