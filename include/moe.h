@@ -333,20 +333,22 @@ moe_status moe_forward_counts(const moe_problem *p, const void *ws, size_t ws_by
  * device array of the G arenas' base addresses (this rank's own among them,
  * at index `rank`), `own_arena` this rank's (as a host-side value). Every
  * transfer is a 16-byte store to a peer's arena; nothing is read on the
- * host. Per forward, with an epoch number that grows by one each forward
- * (the first is 1), rank r:
+ * host, and the calls can be captured in a CUDA graph. The arena keeps the
+ * rank's forward count (its epoch): step 2 advances it on the device, and
+ * steps 3, 5 and 6 use it. Per forward, rank r:
  *   1. routes and dispatches its tokens over all E experts (moe_route,
  *      moe_dispatch: sorted rows, offsets [E+1], sorted_pairs);
  *   2. moe_ep_send: stores each sorted row of owner q's experts, with its
  *      routing weight and local expert id, into q's arena (slots
  *      [r*T*k, (r+1)*T*k) belong to source r), marks the rest of those slots
- *      empty (id -1), then publishes epoch into q's rows flag for source r;
+ *      empty (id -1), then publishes the new epoch into q's rows flag for
+ *      source r;
  *   3. moe_ep_wait(which 0): waits for all G sources' rows flags;
  *   4. moe_dispatch_slots over the G*T*k slots of its arena (k 1, E/G
  *      experts, ids and rows from the arena), moe_grouped_swiglu with the
  *      arena's routing weights: y_sorted [G*T*k, H] fp32;
  *   5. moe_ep_return: stores each weighted row back into its source's arena
- *      at the source's sorted position, then publishes epoch into each
+ *      at the source's sorted position, then publishes the epoch into each
  *      source's return flag for owner r;
  *   6. moe_ep_wait(which 1): waits for all G owners' return flags; the
  *      arena's y region [T*k, H] fp32 is then this rank's y_perm, which
@@ -360,24 +362,24 @@ moe_status moe_forward_counts(const moe_problem *p, const void *ws, size_t ws_by
 /* Bytes of one rank's arena for problem p on G ranks. Host only. */
 moe_status moe_ep_arena_size(const moe_problem *p, int32_t G, size_t *bytes);
 /* Byte offsets inside an arena of the rows flags u64[G], return flags u64[G],
- * received rows x [G*T*k, H] (problem dtype), their routing weights
- * fp32 [G*T*k], their local expert ids int64 [G*T*k] and the returned rows
- * y fp32 [T*k, H] (any pointer may be NULL). Host only. */
-moe_status moe_ep_arena_offsets(const moe_problem *p, int32_t G, size_t *rows_flag, size_t *ret_flag, size_t *x,
-                                size_t *w, size_t *id, size_t *y);
+ * the epoch u64, received rows x [G*T*k, H] (problem dtype), their routing
+ * weights fp32 [G*T*k], their local expert ids int64 [G*T*k] and the
+ * returned rows y fp32 [T*k, H] (any pointer may be NULL). Host only. */
+moe_status moe_ep_arena_offsets(const moe_problem *p, int32_t G, size_t *rows_flag, size_t *ret_flag,
+                                size_t *epoch, size_t *x, size_t *w, size_t *id, size_t *y);
 /* Step 2. x_perm [T*k, H], offsets [E+1], sorted_pairs [T*k] from this
  * rank's moe_dispatch; routing_weights [T, k] fp32 and selected_experts
  * [T, k] int64 from its moe_route. Async on `stream`. */
 moe_status moe_ep_send(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
-                       uint64_t epoch, const void *x_perm, const int32_t *offsets, const int32_t *sorted_pairs,
+                       const void *x_perm, const int32_t *offsets, const int32_t *sorted_pairs,
                        const float *routing_weights, const int64_t *selected_experts, moe_stream_t stream);
 /* Steps 3 (which = 0: rows received) and 6 (which = 1: rows returned). */
-moe_status moe_ep_wait(const moe_problem *p, int32_t G, void *own_arena, int32_t which, uint64_t epoch,
-                       int64_t max_polls, int32_t *err, moe_stream_t stream);
+moe_status moe_ep_wait(const moe_problem *p, int32_t G, void *own_arena, int32_t which, int64_t max_polls,
+                       int32_t *err, moe_stream_t stream);
 /* Step 5. y_sorted [G*T*k, H] fp32, offsets1 [E/G + 1] and sorted_pairs1
  * [G*T*k] from step 4. */
 moe_status moe_ep_return(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
-                         uint64_t epoch, const float *y_sorted, const int32_t *offsets1, const int32_t *sorted_pairs1,
+                         const float *y_sorted, const int32_t *offsets1, const int32_t *sorted_pairs1,
                          moe_stream_t stream);
 
 /* Gradient outputs of moe_backward. All fp32, device, caller-owned, 16-byte

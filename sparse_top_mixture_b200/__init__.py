@@ -89,13 +89,10 @@ SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_dispatch_slots": (ctypes.c_int, [_PP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_ep_arena_size": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
-    "moe_ep_arena_offsets": (ctypes.c_int, [_PP, ctypes.c_int32] + [ctypes.POINTER(ctypes.c_size_t)] * 6),
-    "moe_ep_send": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, ctypes.c_uint64, _VP, _VP, _VP, _VP,
-                                   _VP, _VP]),
-    "moe_ep_wait": (ctypes.c_int, [_PP, ctypes.c_int32, _VP, ctypes.c_int32, ctypes.c_uint64, ctypes.c_int64, _VP,
-                                   _VP]),
-    "moe_ep_return": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, ctypes.c_uint64, _VP, _VP, _VP,
-                                     _VP]),
+    "moe_ep_arena_offsets": (ctypes.c_int, [_PP, ctypes.c_int32] + [ctypes.POINTER(ctypes.c_size_t)] * 7),
+    "moe_ep_send": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "moe_ep_wait": (ctypes.c_int, [_PP, ctypes.c_int32, _VP, ctypes.c_int32, ctypes.c_int64, _VP, _VP]),
+    "moe_ep_return": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None

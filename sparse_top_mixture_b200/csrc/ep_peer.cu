@@ -39,13 +39,16 @@ constexpr int EP_THREADS = 256;
 //                     marks and y offset) are in place
 //   ret_flag  u64[G]  epoch at which owner q has returned this rank's rows
 //   done      u32[2]  completed-block counters of this rank's send / return
+//   epoch     u64     this rank's forward count: the send's last block
+//                     advances it and publishes the new value; the waits
+//                     and the return read it on the device
 //   yoff      i32[G]  source s's sorted position of its first row for us
 //   x         [G*C][H] rows received, source s in slots [s*C, (s+1)*C)
 //   w         f32[G*C] their routing weights
 //   id        i64[G*C] their local expert ids, -1 for an empty slot
 //   y         f32[C][H] this rank's own sorted rows, weighted, returned
 struct EpArena {
-  size_t rows_flag, ret_flag, done, yoff, x, w, id, y, total;
+  size_t rows_flag, ret_flag, done, epoch, yoff, x, w, id, y, total;
 };
 
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -61,6 +64,7 @@ EpArena ep_arena(int64_t G, int64_t C, int64_t H, size_t es) {
   a.rows_flag = take((size_t)G * 8);
   a.ret_flag = take((size_t)G * 8);
   a.done = take(8);
+  a.epoch = take(8);
   a.yoff = take((size_t)G * 4);
   a.x = take((size_t)(G * C * H) * es);
   a.w = take((size_t)(G * C) * 4);
@@ -81,11 +85,12 @@ __device__ __forceinline__ uint64_t ld_acquire_sys(const uint64_t* p) {
 }
 
 // Called by every block after its stores: the last block to finish (its
-// stores and every other block's fenced at system scope) publishes `epoch`
-// into flag slot `slot` of every rank's arena (flags at byte offset
-// flag_off), then re-arms the counter.
-__device__ __forceinline__ void publish_when_done(uint32_t* done, uint8_t* const* arenas, int G, size_t flag_off,
-                                                  int slot, uint64_t epoch) {
+// stores and every other block's fenced at system scope) takes this rank's
+// epoch (advanced by one first when `advance`), publishes it into flag slot
+// `slot` of every rank's arena (flags at byte offset flag_off), then re-arms
+// the counter.
+__device__ __forceinline__ void publish_when_done(uint32_t* done, uint64_t* epoch_ctr, bool advance,
+                                                  uint8_t* const* arenas, int G, size_t flag_off, int slot) {
   __shared__ bool last;
   __threadfence_system();
   __syncthreads();
@@ -93,6 +98,9 @@ __device__ __forceinline__ void publish_when_done(uint32_t* done, uint8_t* const
   __syncthreads();
   if (!last) return;
   __threadfence_system();
+  const uint64_t epoch = *epoch_ctr + (advance ? 1u : 0u);
+  __syncthreads();
+  if (advance && threadIdx.x == 0) *epoch_ctr = epoch;
   for (int q = threadIdx.x; q < G; q += blockDim.x)
     st_release_sys(reinterpret_cast<uint64_t*>(arenas[q] + flag_off) + slot, epoch);
   if (threadIdx.x == 0) *done = 0u;
@@ -111,7 +119,7 @@ __global__ void __launch_bounds__(EP_THREADS) ep_send_kernel(uint8_t* const* __r
                                                              const int32_t* __restrict__ sorted_pairs,
                                                              const float* __restrict__ rw,
                                                              const int64_t* __restrict__ sel, uint32_t* done,
-                                                             uint64_t epoch) {
+                                                             uint64_t* epoch_ctr) {
   constexpr int V = Elem<T>::kPerVec;
   const int hv = H / V;
   const int64_t used = offsets[(int64_t)G * El];
@@ -139,7 +147,7 @@ __global__ void __launch_bounds__(EP_THREADS) ep_send_kernel(uint8_t* const* __r
     if (i >= n_q) reinterpret_cast<int64_t*>(arenas[q] + a.id)[(int64_t)rank * C + i] = -1;
     if (i == 0) reinterpret_cast<int32_t*>(arenas[q] + a.yoff)[rank] = offsets[q * El];
   }
-  publish_when_done(done, arenas, G, a.rows_flag, rank, epoch);
+  publish_when_done(done, epoch_ctr, true, arenas, G, a.rows_flag, rank);
 }
 
 // Return: sorted row p1 < offsets1[El] of the receiver's regroup came from
@@ -150,7 +158,7 @@ __global__ void __launch_bounds__(EP_THREADS) ep_return_kernel(uint8_t* const* _
                                                                const float* __restrict__ y_sorted,
                                                                const int32_t* __restrict__ offsets1,
                                                                const int32_t* __restrict__ sorted_pairs1,
-                                                               uint32_t* done, uint64_t epoch) {
+                                                               uint32_t* done, uint64_t* epoch_ctr) {
   const int hv = H / 4;
   const int64_t used = offsets1[El];
   const int32_t* yoff = reinterpret_cast<const int32_t*>(arenas[rank] + a.yoff);
@@ -164,13 +172,15 @@ __global__ void __launch_bounds__(EP_THREADS) ep_return_kernel(uint8_t* const* _
     float* dst = reinterpret_cast<float*>(arenas[s] + a.y) + (yoff[s] + i) * H;
     reinterpret_cast<float4*>(dst)[v] = reinterpret_cast<const float4*>(y_sorted + p1 * H)[v];
   }
-  publish_when_done(done + 1, arenas, G, a.ret_flag, rank, epoch);
+  publish_when_done(done + 1, epoch_ctr, false, arenas, G, a.ret_flag, rank);
 }
 
-// Wait until every one of the G flags at `flags` holds at least `epoch`
-// (acquire), polling each at most max_polls times (about 256 ns apart); on
-// giving up, raise MOE_DEVERR_WAIT_TIMEOUT in *err and return.
-__global__ void ep_wait_kernel(const uint64_t* flags, int G, uint64_t epoch, int64_t max_polls, int32_t* err) {
+// Wait until every one of the G flags at `flags` holds at least this rank's
+// epoch (acquire), polling each at most max_polls times (about 256 ns
+// apart); on giving up, raise MOE_DEVERR_WAIT_TIMEOUT in *err and return.
+__global__ void ep_wait_kernel(const uint64_t* flags, const uint64_t* epoch_ctr, int G, int64_t max_polls,
+                               int32_t* err) {
+  const uint64_t epoch = *epoch_ctr;
   for (int s = threadIdx.x; s < G; s += blockDim.x) {
     int64_t n = 0;
     while (ld_acquire_sys(flags + s) < epoch) {
@@ -212,12 +222,13 @@ MOE_API moe_status moe_ep_arena_size(const moe_problem* p, int32_t G, size_t* by
 }
 
 MOE_API moe_status moe_ep_arena_offsets(const moe_problem* p, int32_t G, size_t* rows_flag, size_t* ret_flag,
-                                        size_t* x, size_t* w, size_t* id, size_t* y) {
+                                        size_t* epoch, size_t* x, size_t* w, size_t* id, size_t* y) {
   const moe_status st = ep_check(p, G, 0);
   if (st != MOE_OK) return st;
   const EpArena a = ep_arena(G, p->T * p->k, p->H, p->dtype == MOE_DTYPE_F32 ? 4 : 2);
   if (rows_flag) *rows_flag = a.rows_flag;
   if (ret_flag) *ret_flag = a.ret_flag;
+  if (epoch) *epoch = a.epoch;
   if (x) *x = a.x;
   if (w) *w = a.w;
   if (id) *id = a.id;
@@ -226,18 +237,19 @@ MOE_API moe_status moe_ep_arena_offsets(const moe_problem* p, int32_t G, size_t*
 }
 
 MOE_API moe_status moe_ep_send(const moe_problem* p, int32_t G, int32_t rank, void* const* arenas, void* own_arena,
-                               uint64_t epoch, const void* x_perm, const int32_t* offsets, const int32_t* sorted_pairs,
+                               const void* x_perm, const int32_t* offsets, const int32_t* sorted_pairs,
                                const float* routing_weights, const int64_t* selected_experts, moe_stream_t stream) {
   moe_status st = ep_check(p, G, rank);
   if (st != MOE_OK) return st;
   const int64_t C = p->T * p->k;
-  if (epoch == 0 || !al16(arenas) || !al16(own_arena) || !al16(offsets)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!al16(arenas) || !al16(own_arena) || !al16(offsets)) return MOE_ERR_INVALID_ARGUMENT;
   if (C > 0 && (!al16(x_perm) || !al16(sorted_pairs) || !al16(routing_weights) || !al16(selected_experts)))
     return MOE_ERR_INVALID_ARGUMENT;
   const EpArena a = ep_arena(G, C, p->H, p->dtype == MOE_DTYPE_F32 ? 4 : 2);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* const* ar = reinterpret_cast<uint8_t* const*>(arenas);
   uint32_t* done = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(own_arena) + a.done);
+  uint64_t* epoch = reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(own_arena) + a.epoch);
   const int E_l = (int)(p->E / G);
   const int grid = ep_grid(std::max<int64_t>((int64_t)G * C, C * (p->H / 4)));
   if (p->dtype == MOE_DTYPE_F32)
@@ -252,30 +264,32 @@ MOE_API moe_status moe_ep_send(const moe_problem* p, int32_t G, int32_t rank, vo
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-MOE_API moe_status moe_ep_wait(const moe_problem* p, int32_t G, void* own_arena, int32_t which, uint64_t epoch,
-                               int64_t max_polls, int32_t* err, moe_stream_t stream) {
+MOE_API moe_status moe_ep_wait(const moe_problem* p, int32_t G, void* own_arena, int32_t which, int64_t max_polls,
+                               int32_t* err, moe_stream_t stream) {
   moe_status st = ep_check(p, G, 0);
   if (st != MOE_OK) return st;
-  if (!al16(own_arena) || (which != 0 && which != 1) || epoch == 0 || max_polls < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (!al16(own_arena) || (which != 0 && which != 1) || max_polls < 1) return MOE_ERR_INVALID_ARGUMENT;
   if (err != nullptr && (reinterpret_cast<uintptr_t>(err) & 3u) != 0) return MOE_ERR_INVALID_ARGUMENT;
   const EpArena a = ep_arena(G, p->T * p->k, p->H, p->dtype == MOE_DTYPE_F32 ? 4 : 2);
   const uint64_t* flags =
       reinterpret_cast<const uint64_t*>(static_cast<uint8_t*>(own_arena) + (which == 0 ? a.rows_flag : a.ret_flag));
-  ep_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flags, G, epoch, max_polls, err);
+  const uint64_t* epoch = reinterpret_cast<const uint64_t*>(static_cast<uint8_t*>(own_arena) + a.epoch);
+  ep_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flags, epoch, G, max_polls, err);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 MOE_API moe_status moe_ep_return(const moe_problem* p, int32_t G, int32_t rank, void* const* arenas, void* own_arena,
-                                 uint64_t epoch, const float* y_sorted, const int32_t* offsets1,
+                                 const float* y_sorted, const int32_t* offsets1,
                                  const int32_t* sorted_pairs1, moe_stream_t stream) {
   moe_status st = ep_check(p, G, rank);
   if (st != MOE_OK) return st;
   const int64_t C = p->T * p->k;
-  if (epoch == 0 || !al16(arenas) || !al16(own_arena) || !al16(offsets1)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!al16(arenas) || !al16(own_arena) || !al16(offsets1)) return MOE_ERR_INVALID_ARGUMENT;
   if (C > 0 && (!al16(y_sorted) || !al16(sorted_pairs1))) return MOE_ERR_INVALID_ARGUMENT;
   const EpArena a = ep_arena(G, C, p->H, p->dtype == MOE_DTYPE_F32 ? 4 : 2);
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* done = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(own_arena) + a.done);
+  uint64_t* epoch = reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(own_arena) + a.epoch);
   const int grid = ep_grid((int64_t)G * C * (p->H / 4));
   ep_return_kernel<<<grid, EP_THREADS, 0, s>>>(reinterpret_cast<uint8_t* const*>(arenas), G, rank, C, (int)p->H,
                                                 (int)(p->E / G), a, y_sorted, offsets1, sorted_pairs1, done, epoch);

@@ -4,8 +4,9 @@ Same layer and layout as ``expert_parallel.ExpertParallelMoE`` (rank r of G
 holds routed experts [r E/G, (r+1) E/G); router and shared expert
 replicated), but the rows move by the library's peer-store kernels
 (``moe_ep_send`` / ``moe_ep_return``) into arenas every rank can address,
-ordered by epoch flags (``moe_ep_wait``), so that nothing is read on the host
-and the whole forward is asynchronous (and can be captured in a CUDA graph).
+ordered by epoch flags (``moe_ep_wait``; each arena keeps its rank's epoch,
+advanced on the device), so that nothing is read on the host and the whole
+forward is asynchronous and can be captured in a CUDA graph.
 The per-row arithmetic is the one-GPU forward's: each rank's output equals
 ``SparseMoE`` on its tokens with all experts.
 
@@ -49,9 +50,9 @@ def ep_arena_size(p: Problem, world: int) -> int:
 
 
 def ep_arena_offsets(p: Problem, world: int) -> Dict[str, int]:
-    v = [ctypes.c_size_t() for _ in range(6)]
+    v = [ctypes.c_size_t() for _ in range(7)]
     _check(lib().moe_ep_arena_offsets(ctypes.byref(p.c()), world, *[ctypes.byref(x) for x in v]))
-    return dict(zip(("rows_flag", "ret_flag", "x", "w", "id", "y"), (x.value for x in v)))
+    return dict(zip(("rows_flag", "ret_flag", "epoch", "x", "w", "id", "y"), (x.value for x in v)))
 
 
 class PeerExpertParallelMoE:
@@ -87,7 +88,6 @@ class PeerExpertParallelMoE:
         self._keep = list(keep)  # peer mappings stay open as long as the layer
         dev = arena.device
         self.side = torch.cuda.Stream(dev)
-        self.epoch = 0
         C = p.T * p.k
         off = ep_arena_offsets(p, world)
         G = world
@@ -97,6 +97,7 @@ class PeerExpertParallelMoE:
         self.recv_w = arena[off["w"]:off["w"] + G * C * 4].view(torch.float32).view(G * C, 1)
         self.recv_id = arena[off["id"]:off["id"] + G * C * 8].view(torch.int64).view(G * C, 1)
         self.y = arena[off["y"]:off["y"] + C * p.H * 4].view(torch.float32).view(C, p.H)
+        self.epoch = arena[off["epoch"]:off["epoch"] + 8].view(torch.int64)  # forwards so far (device)
         self.ws = new_workspace(p, dev)
         self.ws_shared = new_workspace(p, dev) if p.shared != "none" else None  # used on the second stream
         self.pk1 = dataclasses.replace(p, T=G * C, k=1, E=self.E_local, I_shared=0, shared="none", bias_mode="none")
@@ -150,7 +151,6 @@ class PeerExpertParallelMoE:
     def send(self, x: torch.Tensor) -> None:
         p, w = self.p, self.w
         dev = x.device
-        self.epoch += 1
         gate = w.get("shared_gate") if p.shared == "sigmoid_gated" else None
         rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate, ws=self.ws)
         d = dispatch(p, sel, x, ws=self.ws)
@@ -161,7 +161,7 @@ class PeerExpertParallelMoE:
             with torch.cuda.stream(self.side):
                 shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma, ws=self.ws_shared)
         _check(lib().moe_ep_send(ctypes.byref(p.c()), self.world, self.rank, self.ptrs.data_ptr(),
-                                 self.arena.data_ptr(), self.epoch, _ptr(d["x_perm"]), _ptr(d["offsets"]),
+                                 self.arena.data_ptr(), _ptr(d["x_perm"]), _ptr(d["offsets"]),
                                  _ptr(d["sorted_pairs"]), _ptr(rw), _ptr(sel), _stream(dev)))
         self._st = {"rw": rw, "sel": sel, "pair_pos": d["pair_pos"], "shared": shared, "keep": d}
 
@@ -173,7 +173,7 @@ class PeerExpertParallelMoE:
         y_sorted = grouped_swiglu(pk, d1["x_perm"], d1["offsets"], self.w["gate_up"], self.w["down"], self.recv_w,
                                   d1["sorted_pairs"], ws=self.ws1)
         _check(lib().moe_ep_return(ctypes.byref(p.c()), self.world, self.rank, self.ptrs.data_ptr(),
-                                   self.arena.data_ptr(), self.epoch, _ptr(y_sorted), _ptr(d1["offsets"]),
+                                   self.arena.data_ptr(), _ptr(y_sorted), _ptr(d1["offsets"]),
                                    _ptr(d1["sorted_pairs"]), _stream(dev)))
         self._st["keep1"] = (d1, y_sorted)
 
@@ -197,5 +197,5 @@ class PeerExpertParallelMoE:
     __call__ = forward
 
     def _wait(self, which: int) -> None:
-        _check(lib().moe_ep_wait(ctypes.byref(self.p.c()), self.world, self.arena.data_ptr(), which, self.epoch,
-                                 self.max_polls, self.err.data_ptr(), _stream(self.arena.device)))
+        _check(lib().moe_ep_wait(ctypes.byref(self.p.c()), self.world, self.arena.data_ptr(), which, self.max_polls,
+                                 self.err.data_ptr(), _stream(self.arena.device)))

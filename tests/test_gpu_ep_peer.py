@@ -60,9 +60,11 @@ def test_emulated_ranks_match_the_one_gpu_forward(name, G):
 def test_a_wait_for_a_flag_nobody_publishes_gives_up_and_flags_it():
     cfg, p, dev, layers = _setup("qwen3_30b_a3b", 2)
     layer = layers[0]
-    # epoch 5 was never published by anyone: the wait polls 1000 times, raises
-    # the timeout bit and returns; the stream and context stay usable
-    stm.lib().moe_ep_wait(stm.ctypes.byref(p.c()), 2, layer.arena.data_ptr(), 0, 5, 1000, layer.err.data_ptr(),
+    # this rank's epoch moves to 5, which no source has published: the wait
+    # polls 1000 times, raises the timeout bit and returns; the stream and
+    # context stay usable
+    layer.epoch.fill_(5)
+    stm.lib().moe_ep_wait(stm.ctypes.byref(p.c()), 2, layer.arena.data_ptr(), 0, 1000, layer.err.data_ptr(),
                           stm._stream(layer.arena.device))
     torch.cuda.synchronize()
     assert int(layer.err.item()) == stm.DEVERR_WAIT_TIMEOUT
@@ -79,3 +81,37 @@ def test_arena_layout_matches_the_views():
     assert layer.recv_x.data_ptr() == base + off["x"] and layer.recv_x.shape == (4 * C, p.H)
     assert layer.recv_w.data_ptr() == base + off["w"] and layer.recv_id.data_ptr() == base + off["id"]
     assert layer.y.data_ptr() == base + off["y"] and layer.y.shape == (C, p.H)
+
+
+def test_emulated_ranks_replay_as_one_cuda_graph():
+    """All phases of two emulated ranks captured once (global capture mode)
+    and replayed: each replay advances the epochs on the device, and each
+    rank's output matches the one-GPU forward of its tokens."""
+    cfg, p, dev, layers = _setup("qwen3_30b_a3b", 2)
+    ref_layer = stm.SparseMoE(p, dev)
+    xs = [workloads.router_inputs(cfg, rank=r)["x"].cuda() for r in range(2)]
+    outs = [None, None]
+
+    def run():
+        for layer, x in zip(layers, xs):
+            layer.send(x)
+        for layer in layers:
+            layer.experts()
+        for r, layer in enumerate(layers):
+            outs[r] = layer.finish()[0]
+
+    run()  # first run outside the capture: workspaces and streams exist
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="global"):
+        run()
+    for step in range(3):
+        for r, x in enumerate(xs):
+            x.copy_(workloads.router_inputs(cfg, rank=10 + 2 * step + r)["x"].cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        for r, layer in enumerate(layers):
+            assert int(layer.err.item()) == 0
+            assert int(layer.epoch.item()) == 2 + step  # the first run, then one per replay (capture runs nothing)
+            assert torch.equal(outs[r], ref_layer(xs[r])[0]), f"replay {step} rank {r}"
+    del graph
