@@ -20,6 +20,12 @@
 // flag once every block's stores are fenced at system scope (release), and a
 // waiter polls its own flags with acquire loads, up to a caller-given number
 // of polls, after which it raises MOE_DEVERR_WAIT_TIMEOUT and returns.
+// Reuse from one forward to the next needs no further handshake: a sender
+// overwrites an owner's region (forward n+1) only after its own forward n
+// ended, which waited for that owner's returns, published after the owner's
+// GEMM had read the rows; owners store into a sender's y (and sources into
+// an owner's y-offset mailbox) only after the rows of forward n+1 arrived,
+// which the sender sends after its forward-n combine read y.
 #include <cuda_runtime.h>
 
 #include "common.cuh"

@@ -126,6 +126,7 @@ class PeerExpertParallelMoE:
             st = torch.UntypedStorage._new_shared_cuda(*h)
             keep.append(st)
             ptrs.append(st.data_ptr() + off)
+        torch.cuda.synchronize(dev)  # every arena zeroed before any peer stores into it
         dist.barrier(group=group)
         return cls(p, weights, rank, world, arena, ptrs, max_polls, keep)
 
