@@ -382,6 +382,42 @@ moe_status moe_ep_return(const moe_problem *p, int32_t G, int32_t rank, void *co
                          const float *y_sorted, const int32_t *offsets1, const int32_t *sorted_pairs1,
                          moe_stream_t stream);
 
+/* ---- Tensor parallelism over peer memory --------------------------------------
+ * Every expert's I (and I_shared) split over G ranks, the router replicated,
+ * every rank given the same tokens ("mstar.model.components.moe", the
+ * tensor-parallel MoE block); each rank's grouped SwiGLU over its slice gives
+ * partial fp32 rows y_perm [T*k, H] (and a partial shared output [T, H])
+ * whose sums over ranks are the whole ones. The reduction is fused with the
+ * combine and runs on peer memory: arenas as for the expert-parallel exchange
+ * (moe_tp_arena_size bytes each, zeroed once; each keeps its rank's epoch).
+ * H must be a multiple of 8*G. Per forward, rank r:
+ *   1. moe_tp_scatter: for every token, the sum of its k partial rows in slot
+ *      order plus its partial shared row (fp32, the library's combine
+ *      arithmetic), each 1/G column slice stored into that slice's owner's
+ *      arena; then the new epoch published into every owner's part flag;
+ *   2. moe_tp_wait(which 0): waits for all G sources' partial slices;
+ *   3. moe_tp_gather: sums the G slices of its own columns in rank order,
+ *      rounds once to the problem dtype, stores them into every rank's
+ *      output region, publishes the epoch into every rank's out flag;
+ *   4. moe_tp_wait(which 1): the arena's out region [T, H] (problem dtype)
+ *      then holds the layer's output, until this rank's next moe_tp_scatter.
+ * Waits as in the expert-parallel exchange (bounded; timeout flag). */
+moe_status moe_tp_arena_size(const moe_problem *p, int32_t G, size_t *bytes);
+/* Byte offsets of the part flags u64[G], out flags u64[G], the epoch u64,
+ * the partial slices fp32 [G][T][H/G] and the output [T, H]. Host only. */
+moe_status moe_tp_arena_offsets(const moe_problem *p, int32_t G, size_t *part_flag, size_t *out_flag,
+                                size_t *epoch, size_t *part, size_t *out);
+/* Step 1. y_perm [T*k, H] fp32 and pair_pos [T*k] as for moe_combine;
+ * shared_out [T, H] fp32 or NULL. */
+moe_status moe_tp_scatter(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
+                          const float *y_perm, const int32_t *pair_pos, const float *shared_out, moe_stream_t stream);
+/* Step 3. */
+moe_status moe_tp_gather(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
+                         moe_stream_t stream);
+/* Steps 2 (which = 0) and 4 (which = 1). */
+moe_status moe_tp_wait(const moe_problem *p, int32_t G, void *own_arena, int32_t which, int64_t max_polls,
+                       int32_t *err, moe_stream_t stream);
+
 /* Gradient outputs of moe_backward. All fp32, device, caller-owned, 16-byte
  * aligned, fully overwritten (never accumulated into). */
 typedef struct moe_grads {

@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "moe.h"
+#include "peer.cuh"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
 
@@ -78,38 +79,6 @@ EpArena ep_arena(int64_t G, int64_t C, int64_t H, size_t es) {
   a.y = take((size_t)(C * H) * 4);
   a.total = off;
   return a;
-}
-
-__device__ __forceinline__ void st_release_sys(uint64_t* p, uint64_t v) {
-  asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ uint64_t ld_acquire_sys(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Called by every block after its stores: the last block to finish (its
-// stores and every other block's fenced at system scope) takes this rank's
-// epoch (advanced by one first when `advance`), publishes it into flag slot
-// `slot` of every rank's arena (flags at byte offset flag_off), then re-arms
-// the counter.
-__device__ __forceinline__ void publish_when_done(uint32_t* done, uint64_t* epoch_ctr, bool advance,
-                                                  uint8_t* const* arenas, int G, size_t flag_off, int slot) {
-  __shared__ bool last;
-  __threadfence_system();
-  __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(done, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!last) return;
-  __threadfence_system();
-  const uint64_t epoch = *epoch_ctr + (advance ? 1u : 0u);
-  __syncthreads();
-  if (advance && threadIdx.x == 0) *epoch_ctr = epoch;
-  for (int q = threadIdx.x; q < G; q += blockDim.x)
-    st_release_sys(reinterpret_cast<uint64_t*>(arenas[q] + flag_off) + slot, epoch);
-  if (threadIdx.x == 0) *done = 0u;
 }
 
 // Send: sorted row p (< offsets[E], the rows the dispatch kept) of expert e
@@ -179,24 +148,6 @@ __global__ void __launch_bounds__(EP_THREADS) ep_return_kernel(uint8_t* const* _
     reinterpret_cast<float4*>(dst)[v] = reinterpret_cast<const float4*>(y_sorted + p1 * H)[v];
   }
   publish_when_done(done + 1, epoch_ctr, false, arenas, G, a.ret_flag, rank);
-}
-
-// Wait until every one of the G flags at `flags` holds at least this rank's
-// epoch (acquire), polling each at most max_polls times (about 256 ns
-// apart); on giving up, raise MOE_DEVERR_WAIT_TIMEOUT in *err and return.
-__global__ void ep_wait_kernel(const uint64_t* flags, const uint64_t* epoch_ctr, int G, int64_t max_polls,
-                               int32_t* err) {
-  const uint64_t epoch = *epoch_ctr;
-  for (int s = threadIdx.x; s < G; s += blockDim.x) {
-    int64_t n = 0;
-    while (ld_acquire_sys(flags + s) < epoch) {
-      if (++n >= max_polls) {
-        raise_error(err, MOE_DEVERR_WAIT_TIMEOUT);
-        break;
-      }
-      __nanosleep(256);
-    }
-  }
 }
 
 int ep_grid(int64_t units) {
@@ -280,7 +231,7 @@ MOE_API moe_status moe_ep_wait(const moe_problem* p, int32_t G, void* own_arena,
   const uint64_t* flags =
       reinterpret_cast<const uint64_t*>(static_cast<uint8_t*>(own_arena) + (which == 0 ? a.rows_flag : a.ret_flag));
   const uint64_t* epoch = reinterpret_cast<const uint64_t*>(static_cast<uint8_t*>(own_arena) + a.epoch);
-  ep_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flags, epoch, G, max_polls, err);
+  peer_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flags, epoch, G, max_polls, err);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
