@@ -373,6 +373,18 @@ moe_status moe_ep_arena_offsets(const moe_problem *p, int32_t G, size_t *rows_fl
 moe_status moe_ep_send(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
                        const void *x_perm, const int32_t *offsets, const int32_t *sorted_pairs,
                        const float *routing_weights, const int64_t *selected_experts, moe_stream_t stream);
+/* Steps 1 (its dispatch part) and 2 in one: moe_dispatch's histogram and
+ * scan, then the ranking kernel stores each pair's token row straight into
+ * its owner's arena (no x_perm is written), with its routing weight and
+ * local id, marks the owners' empty slots and publishes the new epoch, as
+ * moe_ep_send does. counts, offsets, sorted_pairs and pair_pos as from
+ * moe_dispatch (pair_pos is the combine's); routing_weights [T, k] fp32 from
+ * moe_route; workspace as for moe_dispatch. T = 0 returns
+ * MOE_ERR_UNSUPPORTED (an empty batch sends through moe_ep_send). */
+moe_status moe_ep_dispatch_send(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
+                                const int64_t *selected_experts, const void *x, const float *routing_weights,
+                                int32_t *counts, int32_t *offsets, int32_t *sorted_pairs, int32_t *pair_pos,
+                                void *ws, size_t ws_bytes, moe_stream_t stream);
 /* Steps 3 (which = 0: rows received) and 6 (which = 1: rows returned). */
 moe_status moe_ep_wait(const moe_problem *p, int32_t G, void *own_arena, int32_t which, int64_t max_polls,
                        int32_t *err, moe_stream_t stream);

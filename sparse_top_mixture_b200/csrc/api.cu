@@ -362,6 +362,27 @@ MOE_API moe_status moe_dispatch_slots(const moe_problem* p, const int64_t* selec
   return MOE_OK;
 }
 
+MOE_API moe_status moe_ep_dispatch_send(const moe_problem* p, int32_t G, int32_t rank, void* const* arenas,
+                                        void* own_arena, const int64_t* selected_experts, const void* x,
+                                        const float* routing_weights, int32_t* counts, int32_t* offsets,
+                                        int32_t* sorted_pairs, int32_t* pair_pos, void* ws, size_t ws_bytes,
+                                        moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->T == 0) return MOE_ERR_UNSUPPORTED;  // an empty batch sends through moe_ep_send
+  if (!ok_ptr(counts) || !ok_ptr(offsets) || !ok_ptr(selected_experts) || !ok_ptr(x) || !ok_ptr(sorted_pairs) ||
+      !ok_ptr(pair_pos))
+    return MOE_ERR_INVALID_ARGUMENT;
+  EpDest ep;
+  if (!ep_dest(*p, G, rank, arenas, own_arena, routing_weights, &ep)) return MOE_ERR_INVALID_ARGUMENT;
+  Layout L;
+  MOE_TRY(check_ws(*p, ws, ws_bytes, &L));
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  MOE_CUDA(launch_dispatch_ep(p->dtype, selected_experts, x, p->T, p->H, p->E, p->k, at<int32_t>(ws, L.local),
+                              counts, offsets, sorted_pairs, pair_pos, &hdr->error_bits, &hdr->dispatch_ticket, ep,
+                              (cudaStream_t)stream));
+  return MOE_OK;
+}
+
 MOE_API moe_status moe_grouped_swiglu(const moe_problem* p, const void* x_perm, const int32_t* offsets,
                                       const void* gate_up, const void* down, const float* routing_weights,
                                       const int32_t* sorted_pairs, void* y_perm, void* ws, size_t ws_bytes,

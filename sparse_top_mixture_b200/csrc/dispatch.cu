@@ -25,6 +25,7 @@
 // pure function of the pair order: the result is deterministic.
 #include "common.cuh"
 #include "kernels.h"
+#include "peer.cuh"
 
 namespace stm {
 
@@ -152,20 +153,26 @@ __global__ void __launch_bounds__(SCAN_THREADS) hist_scan_kernel(const int64_t* 
 
 // Rank the block's pairs, write sorted_pairs / pair_pos (column slice 0
 // only), and copy column slice blockIdx.y of each token row to the slots of
-// its k pairs: x_perm[pair_pos[t*k + j]] = x[t].
-template <typename T>
+// its k pairs: x_perm[pair_pos[t*k + j]] = x[t]. With EP (expert
+// parallelism), the row of sorted position p of expert e goes instead to
+// owner q = e / El's arena, slot rank*C + p - offsets[q*El] (plain peer
+// stores), with its routing weight and local id; every CTA then marks its
+// share of the owners' empty slots, and the last one publishes the epoch.
+template <typename T, bool EP>
 __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t* __restrict__ sel, int64_t P, int k,
                                                                   int E, int tok_per_blk,
                                                                   const int32_t* __restrict__ bases,
                                                                   int32_t* __restrict__ sorted_pairs,
                                                                   int32_t* __restrict__ pair_pos,
                                                                   const T* __restrict__ x, T* __restrict__ x_perm,
-                                                                  int64_t Tn, int H, int vec_per_slice) {
+                                                                  int64_t Tn, int H, int vec_per_slice,
+                                                                  const int32_t* __restrict__ offsets, EpDest ep) {
   // Per-warp counts of each expert (at most 32, so 16 bits) and the slot of
   // every pair: 5 KB of shared memory, small enough to sit beside a
   // persistent GEMM CTA on the same SM.
   __shared__ __align__(16) uint16_t wcnt[DTHREADS / 32][kMaxExperts];
   __shared__ int s_pos[DTHREADS];
+  __shared__ int s_dst[EP ? DTHREADS : 1];  // EP: the pair's arena slot, owner in the top bits
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < (DTHREADS / 32) * kMaxExperts / 2; i += DTHREADS)
     reinterpret_cast<uint32_t*>(&wcnt[0][0])[i] = 0u;
@@ -195,7 +202,21 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
     if (e >= 0) sorted_pairs[pos] = (int32_t)q;
     if (active) pair_pos[q] = pos;
   }
-  if (x_perm == nullptr) return;
+  if constexpr (EP) {
+    int owner = -1;
+    int64_t slot = -1;
+    if (e >= 0) {
+      owner = e / ep.El;
+      slot = (int64_t)ep.rank * ep.C + (pos - offsets[owner * ep.El]);
+      if (blockIdx.y == 0) {
+        reinterpret_cast<float*>(ep.arenas[owner] + ep.w_off)[slot] = ep.rw[q];
+        reinterpret_cast<int64_t*>(ep.arenas[owner] + ep.id_off)[slot] = e - owner * ep.El;
+      }
+    }
+    s_dst[tid] = owner;  // the slot follows from pos and the owner's offset below
+  } else {
+    if (x_perm == nullptr) return;
+  }
   __syncthreads();
   // Copy: work items (token of the block, 16-byte vector of this slice),
   // consecutive threads on consecutive vectors of one row.
@@ -203,17 +224,37 @@ __global__ void __launch_bounds__(DTHREADS) permute_gather_kernel(const int64_t*
   const int nvec = H / V;
   const int v0 = blockIdx.y * vec_per_slice;
   const int nv = min(nvec, v0 + vec_per_slice) - v0;
-  if (nv <= 0) return;
+  if (!EP && nv <= 0) return;  // (with EP every CTA must reach the publication below)
   const int64_t t0 = (int64_t)blockIdx.x * tok_per_blk;
   const int ntok = (int)min((int64_t)tok_per_blk, Tn - t0);
-  const int items = ntok * nv;
+  const int items = ntok * max(nv, 0);
   for (int it = tid; it < items; it += DTHREADS) {
     const int i = it / nv, v = v0 + (it - i * nv);
     const uint4 val = reinterpret_cast<const uint4*>(x + (t0 + i) * (int64_t)H)[v];
     for (int j = 0; j < k; ++j) {
       const int p = s_pos[i * k + j];
-      if (p >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)p * H)[v] = val;
+      if (p < 0) continue;
+      if constexpr (EP) {
+        const int owner = s_dst[i * k + j];
+        const int64_t slot = (int64_t)ep.rank * ep.C + (p - offsets[owner * ep.El]);
+        reinterpret_cast<uint4*>(reinterpret_cast<T*>(ep.arenas[owner] + ep.x_off) + slot * H)[v] = val;
+      } else {
+        reinterpret_cast<uint4*>(x_perm + (int64_t)p * H)[v] = val;
+      }
     }
+  }
+  if constexpr (EP) {
+    // the owners' empty slots and where their rows sit in our sorted order
+    const int64_t nb = (int64_t)gridDim.x * gridDim.y;
+    const int64_t b = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+    for (int64_t jj = b * DTHREADS + tid; jj < (int64_t)ep.G * ep.C; jj += nb * DTHREADS) {
+      const int o = (int)(jj / ep.C);
+      const int64_t i = jj - (int64_t)o * ep.C;
+      if (i >= offsets[(o + 1) * ep.El] - offsets[o * ep.El])
+        reinterpret_cast<int64_t*>(ep.arenas[o] + ep.id_off)[(int64_t)ep.rank * ep.C + i] = -1;
+      if (i == 0) reinterpret_cast<int32_t*>(ep.arenas[o] + ep.yoff_off)[ep.rank] = offsets[o * ep.El];
+    }
+    publish_when_done(ep.done, ep.epoch, true, ep.arenas, ep.G, ep.flag_off, ep.rank);
   }
 }
 
@@ -303,12 +344,41 @@ cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, i
   slices = (int)ceil_div(nvec, vps);
   const dim3 grid((unsigned)nblk, (unsigned)slices);
   if (dtype == 0)
-    permute_gather_kernel<float><<<grid, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local, sorted_pairs,
-                                                           pair_pos, (const float*)x, (float*)x_perm, T, (int)H, vps);
+    permute_gather_kernel<float, false><<<grid, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local,
+                                                                  sorted_pairs, pair_pos, (const float*)x,
+                                                                  (float*)x_perm, T, (int)H, vps, nullptr, EpDest{});
   else
-    permute_gather_kernel<__nv_bfloat16><<<grid, DTHREADS, 0, s>>>(
+    permute_gather_kernel<__nv_bfloat16, false><<<grid, DTHREADS, 0, s>>>(
         selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos, (const __nv_bfloat16*)x,
-        (__nv_bfloat16*)x_perm, T, (int)H, vps);
+        (__nv_bfloat16*)x_perm, T, (int)H, vps, nullptr, EpDest{});
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_ep(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
+                               int64_t k, int32_t* local, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
+                               int32_t* pair_pos, int32_t* err, uint32_t* ticket, const EpDest& ep, cudaStream_t s) {
+  const int tpb = (int)dispatch_tokens_per_block(k);
+  const int nblk = (int)dispatch_num_blocks(T, k);
+  const int64_t P = T * k;
+  int ep2 = 1;
+  while (ep2 < E) ep2 <<= 1;
+  const int tpe = std::min(32, SCAN_THREADS / ep2);
+  hist_scan_kernel<<<(unsigned)ceil_div(nblk, HIST_SUB), SCAN_THREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, nblk,
+                                                                             tpe, local, counts, offsets, ticket, err);
+  const int V = dtype == 0 ? 4 : 8;
+  const int64_t nvec = H / V;
+  int slices = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(148 * 8, std::max(nblk, 1)), nvec / 32));
+  const int vps = (int)ceil_div(nvec, slices);
+  slices = (int)ceil_div(nvec, vps);
+  const dim3 grid((unsigned)std::max(nblk, 1), (unsigned)slices);
+  if (dtype == 0)
+    permute_gather_kernel<float, true><<<grid, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local,
+                                                                 sorted_pairs, pair_pos, (const float*)x, nullptr, T,
+                                                                 (int)H, vps, offsets, ep);
+  else
+    permute_gather_kernel<__nv_bfloat16, true><<<grid, DTHREADS, 0, s>>>(
+        selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos, (const __nv_bfloat16*)x, nullptr, T, (int)H,
+        vps, offsets, ep);
   return cudaGetLastError();
 }
 

@@ -166,6 +166,30 @@ moe_status ep_check(const moe_problem* p, int32_t G, int32_t rank) {
 bool al16(const void* q) { return q != nullptr && (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 
 }  // namespace
+
+bool ep_dest(const moe_problem& p, int G, int rank, void* const* arenas, void* own_arena, const float* rw,
+             EpDest* d) {
+  if (ep_check(&p, G, rank) != MOE_OK) return false;
+  if (!al16(arenas) || !al16(own_arena) || (p.T > 0 && !al16(rw))) return false;
+  const int64_t C = p.T * p.k;
+  const EpArena a = ep_arena(G, C, p.H, p.dtype == MOE_DTYPE_F32 ? 4 : 2);
+  uint8_t* own = static_cast<uint8_t*>(own_arena);
+  d->arenas = reinterpret_cast<uint8_t* const*>(arenas);
+  d->G = G;
+  d->rank = rank;
+  d->El = (int)(p.E / G);
+  d->C = C;
+  d->x_off = a.x;
+  d->w_off = a.w;
+  d->id_off = a.id;
+  d->yoff_off = a.yoff;
+  d->flag_off = a.rows_flag;
+  d->rw = rw;
+  d->done = reinterpret_cast<uint32_t*>(own + a.done);
+  d->epoch = reinterpret_cast<uint64_t*>(own + a.epoch);
+  return true;
+}
+
 }  // namespace stm
 
 using namespace stm;

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "moe.h"
+
 #include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
@@ -90,6 +92,28 @@ cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, i
 
 // ---- combine ----------------------------------------------------------
 // y_perm [T*k, H] and shared_out [T, H] are fp32 for every problem dtype.
+// Expert parallelism: where the dispatch stores each pair's row instead of
+// x_perm (the owner's arena, slot rank*C + position inside the owner's
+// run), with its routing weight and local expert id; the empty slots of
+// every owner's region, the y-offset mailbox and the rows flag as for
+// moe_ep_send (ep_peer.cu builds it).
+struct EpDest {
+  uint8_t* const* arenas;  // device array of the G arena base addresses
+  int G, rank, El;
+  int64_t C;               // slots per source: T*k
+  size_t x_off, w_off, id_off, yoff_off, flag_off;
+  const float* rw;         // routing weights [T, k]
+  uint32_t* done;          // this rank's completed-block counter
+  uint64_t* epoch;         // this rank's epoch (advanced and published)
+};
+// moe_ep_dispatch_send's layout helper; false if the problem or G is invalid.
+bool ep_dest(const moe_problem& p, int G, int rank, void* const* arenas, void* own_arena, const float* rw,
+             EpDest* d);
+// The dispatch (histogram, scan, ranking) with each row stored to its
+// owner's arena; x_perm is not written.
+cudaError_t launch_dispatch_ep(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
+                               int64_t k, int32_t* local, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
+                               int32_t* pair_pos, int32_t* err, uint32_t* ticket, const EpDest& ep, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const float* y_perm, const int32_t* pair_pos, const float* shared_out,
                            void* out, int64_t T, int64_t H, int64_t k, cudaStream_t s);
 

@@ -21,7 +21,8 @@ __device__ __forceinline__ uint64_t ld_acquire_sys(const uint64_t* p) {
   return v;
 }
 
-// Called by every block after its stores: the last block to finish (its
+// Called by every block of the grid (1-D or 2-D) after its stores: the last
+// block to finish (its
 // stores and every other block's fenced at system scope) takes this rank's
 // epoch (advanced by one first when `advance`), publishes it into flag slot
 // `slot` of every rank's arena (flags at byte offset flag_off), then re-arms
@@ -31,7 +32,7 @@ __device__ __forceinline__ void publish_when_done(uint32_t* done, uint64_t* epoc
   __shared__ bool last;
   __threadfence_system();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(done, 1u) == gridDim.x - 1;
+  if (threadIdx.x == 0) last = atomicAdd(done, 1u) == gridDim.x * gridDim.y - 1;
   __syncthreads();
   if (!last) return;
   __threadfence_system();

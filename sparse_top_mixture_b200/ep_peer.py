@@ -12,9 +12,12 @@ The per-row arithmetic is the one-GPU forward's: each rank's output equals
 
 A forward is three phases, which ``forward`` runs back to back:
 
-* ``send``: route and dispatch this rank's tokens over all E experts, then
-  store each owner's run of sorted rows (with weights and local ids) into the
-  owner's arena; the shared expert runs on a second stream meanwhile;
+* ``send``: route this rank's tokens, then dispatch them over all E experts
+  with the rows stored straight into their owners' arenas by the dispatch's
+  own ranking kernel (``moe_ep_dispatch_send``: one launch instead of a
+  permutation into x_perm and a copy out of it; ``fused=False`` takes the two
+  steps, ``moe_dispatch`` then ``moe_ep_send``); the shared expert runs on a
+  second stream meanwhile;
 * ``experts``: wait for every source's rows, regroup the received slots by
   local expert (``moe_dispatch_slots``), run the grouped SwiGLU, and store each
   weighted fp32 row back into its source's arena at its sorted position;
@@ -70,10 +73,11 @@ class PeerExpertParallelMoE:
 
     def __init__(self, p: Problem, weights: Dict[str, Optional[torch.Tensor]], rank: int, world: int,
                  arena: torch.Tensor, arena_ptrs: Sequence[int], max_polls: int = DEFAULT_MAX_POLLS,
-                 keep: Sequence[object] = ()):
+                 keep: Sequence[object] = (), fused: bool = True):
         if p.E % world:
             raise ValueError(f"E={p.E} is not divisible by the {world} ranks")
         self.p, self.w, self.rank, self.world = p, weights, rank, world
+        self.fused = fused
         self.E_local = p.E // world
         gu, dn = weights["gate_up"], weights["down"]
         if tuple(gu.shape) != (self.E_local, 2 * p.I, p.H) or tuple(dn.shape) != (self.E_local, p.H, p.I):
@@ -131,7 +135,7 @@ class PeerExpertParallelMoE:
         return cls(p, weights, rank, world, arena, ptrs, max_polls, keep)
 
     @classmethod
-    def emulate(cls, p: Problem, weights: Dict[str, Optional[torch.Tensor]], world: int
+    def emulate(cls, p: Problem, weights: Dict[str, Optional[torch.Tensor]], world: int, fused: bool = True
                 ) -> List["PeerExpertParallelMoE"]:
         """G ranks in this process on one GPU (tests): full-model ``weights``
         split by expert ranges; each wait polls once (run the phases rank by
@@ -145,7 +149,7 @@ class PeerExpertParallelMoE:
             w = dict(weights)
             w["gate_up"] = weights["gate_up"][r * El:(r + 1) * El].contiguous()
             w["down"] = weights["down"][r * El:(r + 1) * El].contiguous()
-            layers.append(cls(p, w, r, world, arenas[r], ptrs, max_polls=1, keep=arenas))
+            layers.append(cls(p, w, r, world, arenas[r], ptrs, max_polls=1, keep=arenas, fused=fused))
         return layers
 
     # -- the three phases ----------------------------------------------------------
@@ -154,16 +158,28 @@ class PeerExpertParallelMoE:
         dev = x.device
         gate = w.get("shared_gate") if p.shared == "sigmoid_gated" else None
         rw, sel, gamma = route(p, x, w["gate_w"], w.get("bias"), gate, ws=self.ws)
-        d = dispatch(p, sel, x, ws=self.ws)
         main = torch.cuda.current_stream(dev)
         shared = None
         if p.shared != "none":  # beside the exchange, on the second stream
             self.side.wait_stream(main)
             with torch.cuda.stream(self.side):
                 shared = shared_expert(p, x, w["shared_gate_up"], w["shared_down"], gamma, ws=self.ws_shared)
-        _check(lib().moe_ep_send(ctypes.byref(p.c()), self.world, self.rank, self.ptrs.data_ptr(),
-                                 self.arena.data_ptr(), _ptr(d["x_perm"]), _ptr(d["offsets"]),
-                                 _ptr(d["sorted_pairs"]), _ptr(rw), _ptr(sel), _stream(dev)))
+        if self.fused and p.T > 0:
+            P = p.T * p.k
+            d = {"counts": torch.empty(p.E, dtype=torch.int32, device=dev),
+                 "offsets": torch.empty(p.E + 1, dtype=torch.int32, device=dev),
+                 "sorted_pairs": torch.empty(P, dtype=torch.int32, device=dev),
+                 "pair_pos": torch.empty(P, dtype=torch.int32, device=dev)}
+            _check(lib().moe_ep_dispatch_send(ctypes.byref(p.c()), self.world, self.rank, self.ptrs.data_ptr(),
+                                              self.arena.data_ptr(), _ptr(sel), _ptr(x), _ptr(rw),
+                                              _ptr(d["counts"]), _ptr(d["offsets"]), _ptr(d["sorted_pairs"]),
+                                              _ptr(d["pair_pos"]), self.ws.data_ptr(), self.ws.numel(),
+                                              _stream(dev)))
+        else:
+            d = dispatch(p, sel, x, ws=self.ws)
+            _check(lib().moe_ep_send(ctypes.byref(p.c()), self.world, self.rank, self.ptrs.data_ptr(),
+                                     self.arena.data_ptr(), _ptr(d["x_perm"]), _ptr(d["offsets"]),
+                                     _ptr(d["sorted_pairs"]), _ptr(rw), _ptr(sel), _stream(dev)))
         self._st = {"rw": rw, "sel": sel, "pair_pos": d["pair_pos"], "shared": shared, "keep": d}
 
     def experts(self) -> None:

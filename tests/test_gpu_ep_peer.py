@@ -1,5 +1,6 @@
-"""Expert parallelism over peer memory (moe_ep_send / moe_ep_wait /
-moe_ep_return / moe_dispatch_slots through the C ABI), on one GPU.
+"""Expert parallelism over peer memory (moe_ep_dispatch_send, or moe_dispatch
+then moe_ep_send; moe_ep_wait, moe_dispatch_slots, moe_ep_return; through
+the C ABI), on one GPU.
 
 G ranks are emulated in this process (``PeerExpertParallelMoE.emulate``):
 their arenas are ordinary device memory, each rank has its own tokens and
@@ -23,21 +24,24 @@ from test_gpu_parity import SMALL
 
 pytestmark = pytest.mark.gpu
 
-CASES = [("qwen3_30b_a3b", 2), ("qwen3_30b_a3b", 4), ("deepseek_v2_lite_zipf", 4), ("dsv4_flash_ablation", 2),
-         ("decode_weight_streaming", 8), ("tiny_fp32", 2), ("qwen3_30b_a3b", 1)]
+# (workload, ranks, send fused into the dispatch)
+CASES = [("qwen3_30b_a3b", 2, True), ("qwen3_30b_a3b", 4, True), ("deepseek_v2_lite_zipf", 4, True),
+         ("dsv4_flash_ablation", 2, True), ("decode_weight_streaming", 8, True), ("tiny_fp32", 2, True),
+         ("qwen3_30b_a3b", 1, True), ("qwen3_30b_a3b", 4, False), ("deepseek_v2_lite_zipf", 4, False),
+         ("tiny_fp32", 2, False)]
 
 
-def _setup(name, G):
+def _setup(name, G, fused=True):
     cfg = SMALL[name]
     p = stm.Problem.from_config(cfg)
     cpu = workloads.generate(cfg, "cpu")
     dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
-    return cfg, p, dev, PeerExpertParallelMoE.emulate(p, dev, G)
+    return cfg, p, dev, PeerExpertParallelMoE.emulate(p, dev, G, fused=fused)
 
 
-@pytest.mark.parametrize("name,G", CASES)
-def test_emulated_ranks_match_the_one_gpu_forward(name, G):
-    cfg, p, dev, layers = _setup(name, G)
+@pytest.mark.parametrize("name,G,fused", CASES)
+def test_emulated_ranks_match_the_one_gpu_forward(name, G, fused):
+    cfg, p, dev, layers = _setup(name, G, fused)
     ref_layer = stm.SparseMoE(p, dev)
     for step in range(3):
         xs = [workloads.router_inputs(cfg, rank=r + G * step)["x"].cuda() for r in range(G)]
