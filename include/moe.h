@@ -385,6 +385,17 @@ moe_status moe_ep_dispatch_send(const moe_problem *p, int32_t G, int32_t rank, v
                                 const int64_t *selected_experts, const void *x, const float *routing_weights,
                                 int32_t *counts, int32_t *offsets, int32_t *sorted_pairs, int32_t *pair_pos,
                                 void *ws, size_t ws_bytes, moe_stream_t stream);
+/* Steps 4 and 5 in one, bf16 problems (the tensor-core GEMMs): the
+ * received slots regrouped by local expert (as moe_dispatch_slots), the
+ * grouped gate_up and SwiGLU, and the down GEMM whose epilogue stores each
+ * weighted fp32 row straight into its source's arena (the return
+ * all-to-all fused with the GEMM: no local y, no separate copy), then the
+ * epoch published into every source's return flag. gate_up [E/G, 2I, H] and
+ * down [E/G, H, I]: this rank's experts. ws: a workspace of
+ * moe_workspace_size bytes for the problem (G*T*k tokens, k 1, E/G experts,
+ * no shared expert, no bias). fp32 problems return MOE_ERR_UNSUPPORTED. */
+moe_status moe_ep_experts(const moe_problem *p, int32_t G, int32_t rank, void *const *arenas, void *own_arena,
+                          const void *gate_up, const void *down, void *ws, size_t ws_bytes, moe_stream_t stream);
 /* Steps 3 (which = 0: rows received) and 6 (which = 1: rows returned). */
 moe_status moe_ep_wait(const moe_problem *p, int32_t G, void *own_arena, int32_t which, int64_t max_polls,
                        int32_t *err, moe_stream_t stream);

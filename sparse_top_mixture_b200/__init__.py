@@ -93,6 +93,7 @@ SIGNATURES = {
     "moe_ep_send": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_ep_wait": (ctypes.c_int, [_PP, ctypes.c_int32, _VP, ctypes.c_int32, ctypes.c_int64, _VP, _VP]),
     "moe_ep_return": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "moe_ep_experts": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_ep_dispatch_send": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                             _VP, _VP, _VP, _SZ, _VP]),
     "moe_tp_arena_size": (ctypes.c_int, [_PP, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),

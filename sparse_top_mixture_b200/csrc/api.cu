@@ -383,6 +383,46 @@ MOE_API moe_status moe_ep_dispatch_send(const moe_problem* p, int32_t G, int32_t
   return MOE_OK;
 }
 
+MOE_API moe_status moe_ep_experts(const moe_problem* p, int32_t G, int32_t rank, void* const* arenas,
+                                  void* own_arena, const void* gate_up, const void* down, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream) {
+  MOE_TRY(validate_problem(p));
+  if (p->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;  // the tensor-core GEMMs only
+  if (G < 1 || rank < 0 || rank >= G || p->E % G != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ok_ptr(arenas) || !ok_ptr(gate_up) || !ok_ptr(down)) return MOE_ERR_INVALID_ARGUMENT;
+  EpViews v;
+  if (!ep_views(*p, G, own_arena, &v)) return MOE_ERR_INVALID_ARGUMENT;
+  // the owner's problem: G*T*k one-slot rows over its E/G experts
+  moe_problem p1 = *p;
+  p1.T = G * v.C;
+  p1.k = 1;
+  p1.E = p->E / G;
+  p1.I_shared = 0;
+  p1.shared = MOE_SHARED_NONE;
+  p1.bias_mode = MOE_BIAS_NONE;
+  MOE_TRY(validate_problem(&p1));
+  Layout L;
+  MOE_TRY(check_ws(p1, ws, ws_bytes, &L));
+  const cudaStream_t s = (cudaStream_t)stream;
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* sorted_pairs = at<int32_t>(ws, L.sorted_pairs);
+  uint8_t* const* ar = reinterpret_cast<uint8_t* const*>(arenas);
+  if (p1.T > 0) {
+    // regroup the occupied slots by local expert (empty slots skipped, no flag)
+    MOE_CUDA(launch_dispatch(p1.dtype, v.id, v.x, p1.T, p1.H, p1.E, 1, at<int32_t>(ws, L.local),
+                             at<int32_t>(ws, L.counts), offsets, sorted_pairs, at<int32_t>(ws, L.pair_pos),
+                             at<void>(ws, L.x_perm), nullptr, &hdr->dispatch_ticket, s));
+    MOE_TRY(do_grouped_gate_up(p1, L, at<void>(ws, L.x_perm), offsets, gate_up, ws, s));
+    // down with each weighted row stored into its source's y (peer stores)
+    const Segments sg{offsets, (int32_t)p1.E, 0, p1.T};
+    MOE_CUDA(launch_tc_down_ep(sg, at<void>(ws, L.h), down, p1.E, v.w, sorted_pairs, p1.H, p1.I,
+                               EpRet{ar, v.C, v.y_off, v.yoff}, &hdr->error_bits, s));
+  }
+  MOE_CUDA(launch_ep_publish(ar, G, rank, v.ret_flag_off, v.epoch, s));
+  return MOE_OK;
+}
+
 MOE_API moe_status moe_grouped_swiglu(const moe_problem* p, const void* x_perm, const int32_t* offsets,
                                       const void* gate_up, const void* down, const float* routing_weights,
                                       const int32_t* sorted_pairs, void* y_perm, void* ws, size_t ws_bytes,

@@ -165,7 +165,36 @@ moe_status ep_check(const moe_problem* p, int32_t G, int32_t rank) {
 
 bool al16(const void* q) { return q != nullptr && (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 
+__global__ void ep_publish_kernel(uint8_t* const* arenas, int G, int rank, size_t flag_off, const uint64_t* epoch) {
+  __threadfence_system();
+  const uint64_t e = *epoch;
+  for (int q = threadIdx.x; q < G; q += blockDim.x)
+    st_release_sys(reinterpret_cast<uint64_t*>(arenas[q] + flag_off) + rank, e);
+}
+
 }  // namespace
+
+bool ep_views(const moe_problem& p, int G, void* own_arena, EpViews* v) {
+  if (ep_check(&p, G, 0) != MOE_OK || !al16(own_arena)) return false;
+  const int64_t C = p.T * p.k;
+  const EpArena a = ep_arena(G, C, p.H, p.dtype == MOE_DTYPE_F32 ? 4 : 2);
+  uint8_t* own = static_cast<uint8_t*>(own_arena);
+  v->x = own + a.x;
+  v->w = reinterpret_cast<float*>(own + a.w);
+  v->id = reinterpret_cast<int64_t*>(own + a.id);
+  v->yoff = reinterpret_cast<int32_t*>(own + a.yoff);
+  v->y_off = a.y;
+  v->ret_flag_off = a.ret_flag;
+  v->epoch = reinterpret_cast<uint64_t*>(own + a.epoch);
+  v->C = C;
+  return true;
+}
+
+cudaError_t launch_ep_publish(uint8_t* const* arenas, int G, int rank, size_t flag_off, const uint64_t* epoch,
+                              cudaStream_t s) {
+  ep_publish_kernel<<<1, 64, 0, s>>>(arenas, G, rank, flag_off, epoch);
+  return cudaGetLastError();
+}
 
 bool ep_dest(const moe_problem& p, int G, int rank, void* const* arenas, void* own_arena, const float* rw,
              EpDest* d) {

@@ -63,7 +63,9 @@ constexpr int NTHREADS = 192;
 // MODE_DOWN_KN: the down epilogue over B stored [E][K][N] (N innermost, read
 // MN-major). MODE_WGRAD: both operands stored [K rows][M] and [K rows][N]
 // (read MN-major), K running over each expert's row range.
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2, MODE_WGRAD = 3, MODE_DOWN_KN = 4 };
+// MODE_DOWN_EP: the down GEMM with each weighted row stored into its
+// source's arena (expert parallelism; EpRet) instead of y.
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_LOGITS = 2, MODE_WGRAD = 3, MODE_DOWN_KN = 4, MODE_DOWN_EP = 5 };
 constexpr int MN_CHUNK_BYTES = BK * 64 * 2;  // 64 MN elements x 64 K rows of an MN-major operand
 
 struct Args {
@@ -84,6 +86,7 @@ struct Args {
   int32_t M;        // WGRAD: output rows per expert
   int32_t m_tiles;  // WGRAD: 128-row tiles of M
   int32_t n_mma;    // LOGITS: MMA N (the expert count rounded up to 16); else UMMA_N
+  EpRet ep;         // DOWN_EP only
 };
 
 struct __align__(8) Ctl {
@@ -338,6 +341,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         epilogue_scale_f32(tbase, UMMA_N / 32, sc, stage,
                            reinterpret_cast<float*>(args.out) + (int64_t)row_w0 * args.ldo, args.ldo, nrows,
                            tc.n_idx * UMMA_N, args.N, lane);
+      } else if (MODE == MODE_DOWN_EP) {
+        // this lane's row came from slot j = s*C + i: to source s's y, row yoff[s] + i
+        float sc = 1.f;
+        float* rp = nullptr;
+        if (valid) {
+          const int64_t j = args.scale_idx[row];
+          sc = args.row_scale[j];
+          const int64_t src = j / args.ep.C;
+          rp = reinterpret_cast<float*>(args.ep.arenas[src] + args.ep.y_off) +
+               (args.ep.yoff[src] + (j - src * args.ep.C)) * args.N;
+        }
+        epilogue_scale_f32_rows(tbase, UMMA_N / 32, sc, stage, rp, nrows, tc.n_idx * UMMA_N, args.N, lane);
       } else {
         // router logits: fp32 partial sum of this k split; the row pitch is a
         // multiple of 4 floats, columns past N are not written.
@@ -372,6 +387,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (MODE == MODE_DOWN_EP) __threadfence_system();  // the rows stored to peers, before any flag
   }
 
   tc_fence_before();
@@ -386,13 +402,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 template <int MODE>
 cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, int64_t N, int64_t K,
                       void* out, int64_t ldo, const float* row_scale, const int32_t* scale_idx, int32_t* err,
-                      cudaStream_t s, int k_splits = 1) {
+                      cudaStream_t s, int k_splits = 1, const EpRet* ep = nullptr) {
   static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance (MODE)
   static cudaError_t attr_status[kSmemAttrDevices];
   const void* kernel = reinterpret_cast<const void*>(tc_grouped_gemm_kernel<MODE>);
   const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)kSmemBytes, attr_once, attr_status);
   if (attr_err != cudaSuccess) return attr_err;
-  Args a;
+  Args a{};
   a.offsets = sg.offsets;
   a.E = sg.E;
   a.single_rows = sg.single_rows;
@@ -410,6 +426,7 @@ cudaError_t launch_tc(const Segments& sg, const CUtensorMap& tmA, const CUtensor
   a.M = 0;
   a.m_tiles = 0;
   a.n_mma = MODE == MODE_LOGITS ? (int32_t)std::min<int64_t>(UMMA_N, round_up(N, 16)) : UMMA_N;
+  if (ep != nullptr) a.ep = *ep;
   const int64_t nseg = sg.offsets ? sg.E : 1;
   const int64_t max_tiles = (sg.rows_total / BM + nseg) * a.n_tiles * a.k_splits;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_tiles));
@@ -578,6 +595,29 @@ cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, int64_t lda, co
     if (!make_tensor_map_bf16(&tmB, w_kn, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   return launch_tc<MODE_DOWN_KN>(sg, tmA, tmB, N, K, y, N, row_scale, scale_idx, err, s);
+}
+
+cudaError_t launch_tc_down_ep(const Segments& sg, const void* h, const void* w_down, int64_t E_w,
+                              const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, const EpRet& ep,
+                              int32_t* err, cudaStream_t s) {
+  if (!get_encode()) return cudaErrorNotSupported;
+  if (row_scale == nullptr || scale_idx == nullptr) return cudaErrorInvalidValue;
+  if (tc_gemm_variant(sg, true) == 2)
+    return launch_tc2_down_ep(sg, h, w_down, E_w, row_scale, scale_idx, H, I, ep, err, num_sms(), s);
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[2] = {(uint64_t)I, (uint64_t)sg.rows_total};
+    const uint64_t strides[1] = {(uint64_t)I * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!make_tensor_map_bf16(&tmA, h, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)I, (uint64_t)H, (uint64_t)E_w};
+    const uint64_t strides[2] = {(uint64_t)I * 2, (uint64_t)H * I * 2};
+    const uint32_t box[3] = {BK, UMMA_N, 1};
+    if (!make_tensor_map_bf16(&tmB, w_down, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  return launch_tc<MODE_DOWN_EP>(sg, tmA, tmB, H, I, nullptr, H, row_scale, scale_idx, err, s, 1, &ep);
 }
 
 int tc_router_splits(int64_t T, int64_t H, int64_t E) {

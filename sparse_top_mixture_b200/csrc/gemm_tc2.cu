@@ -75,7 +75,9 @@ struct Ring {
 // MODE_DOWN_KN: the down epilogue over B stored [E][K][N] (N innermost),
 // read MN-major: each CTA's 128 B columns are two 64-column chunks of 64 K
 // rows (one K atom per stage only).
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_DOWN_KN = 2 };
+// MODE_DOWN_EP: the down GEMM with each weighted row stored into its
+// source's arena (expert parallelism; EpRet) instead of y.
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_DOWN_KN = 2, MODE_DOWN_EP = 3 };
 constexpr int MN_CHUNK_BYTES = 64 * BK * 2;
 
 struct Args2 {
@@ -91,6 +93,7 @@ struct Args2 {
   const int32_t* scale_idx;
   int32_t* err;
   int64_t rows_total;
+  EpRet ep;  // MODE_DOWN_EP only
 };
 
 struct __align__(8) Ctl2 {
@@ -124,6 +127,7 @@ constexpr size_t smem_bytes2() {
 static_assert(smem_bytes2<MODE_GATE_UP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 static_assert(smem_bytes2<MODE_DOWN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 static_assert(smem_bytes2<MODE_DOWN_KN>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
+static_assert(smem_bytes2<MODE_DOWN_EP>() <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 struct Tile2 {
   int e, row0, row_end, n_idx;
@@ -333,12 +337,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         float sc = 1.f;
         if (lane < nrows && args.row_scale != nullptr)
           sc = args.row_scale[args.scale_idx ? args.scale_idx[row] : row];
-        float* orow0 = reinterpret_cast<float*>(args.out) + (int64_t)row_w0 * args.ldo;
-        if (!tc.tail)
-          epilogue_scale_f32(tbase, 8, sc, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N, args.N, lane);
-        else
-          epilogue_scale_f32(tbase, 4, sc, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N + half * 128, args.N,
-                             lane);
+        if constexpr (MODE == MODE_DOWN_EP) {
+          // this lane's row came from slot j = s*C + i: to source s's y, row yoff[s] + i
+          float* rp = nullptr;
+          if (lane < nrows) {
+            const int64_t j = args.scale_idx[row];
+            const int64_t src = j / args.ep.C;
+            rp = reinterpret_cast<float*>(args.ep.arenas[src] + args.ep.y_off) +
+                 (args.ep.yoff[src] + (j - src * args.ep.C)) * args.N;
+          }
+          if (!tc.tail)
+            epilogue_scale_f32_rows(tbase, 8, sc, stage, rp, nrows, tc.n_idx * UMMA_N, args.N, lane);
+          else
+            epilogue_scale_f32_rows(tbase, 4, sc, stage, rp, nrows, tc.n_idx * UMMA_N + half * 128, args.N, lane);
+        } else {
+          float* orow0 = reinterpret_cast<float*>(args.out) + (int64_t)row_w0 * args.ldo;
+          if (!tc.tail)
+            epilogue_scale_f32(tbase, 8, sc, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N, args.N, lane);
+          else
+            epilogue_scale_f32(tbase, 4, sc, stage, orow0, args.ldo, nrows, tc.n_idx * UMMA_N + half * 128, args.N,
+                               lane);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -352,6 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (MODE == MODE_DOWN_EP) __threadfence_system();  // the rows stored to peers, before any flag
   }
 
   tc_fence_before();
@@ -367,13 +387,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 template <int MODE, int KA>
 cudaError_t launch_tc2(const Segments& sg, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmB64,
                        int64_t N, int64_t K, void* out, int64_t ldo, const float* row_scale,
-                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s) {
+                       const int32_t* scale_idx, int32_t* err, int num_sms, cudaStream_t s,
+                       const EpRet* ep = nullptr) {
   static std::once_flag attr_once[kSmemAttrDevices];  // one set per kernel instance
   static cudaError_t attr_status[kSmemAttrDevices];
   const void* kernel = reinterpret_cast<const void*>(tc2_grouped_gemm_kernel<MODE, KA>);
   const cudaError_t attr_err = set_max_dynamic_smem_once(kernel, (int)smem_bytes2<MODE>(), attr_once, attr_status);
   if (attr_err != cudaSuccess) return attr_err;
-  Args2 a;
+  Args2 a{};
+  if (ep != nullptr) a.ep = *ep;
   a.offsets = sg.offsets;
   a.E = sg.E;
   a.single_rows = sg.single_rows;
@@ -470,6 +492,18 @@ cudaError_t launch_tc2_down(const Segments& sg, const void* A, const void* w_dow
   if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
   if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
   return launch_tc2<MODE_DOWN, KA>(sg, tmA, tmB, tmB, H, I, y, H, row_scale, scale_idx, err, num_sms, s);
+}
+
+cudaError_t launch_tc2_down_ep(const Segments& sg, const void* A, const void* w_down, int64_t E_w,
+                               const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I,
+                               const EpRet& ep, int32_t* err, int num_sms, cudaStream_t s) {
+  constexpr int KA = kAtomsPerStage;
+  CUtensorMap tmA, tmB;
+  // as launch_tc2_down: h [rows, I] (3-D loads), down [E][H][I] (4-D loads)
+  if (!map_kmajor(&tmA, A, KA, I, sg.rows_total, I * 2, 1, 0, 0, 0, HALF, 3)) return cudaErrorInvalidValue;
+  if (!map_kmajor(&tmB, w_down, KA, I, H, I * 2, 1, 0, E_w, H * I * 2, HALF, 4)) return cudaErrorInvalidValue;
+  return launch_tc2<MODE_DOWN_EP, KA>(sg, tmA, tmB, tmB, H, I, nullptr, H, row_scale, scale_idx, err, num_sms, s,
+                                      &ep);
 }
 
 cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,

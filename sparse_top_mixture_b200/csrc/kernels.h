@@ -106,6 +106,31 @@ struct EpDest {
   uint32_t* done;          // this rank's completed-block counter
   uint64_t* epoch;         // this rank's epoch (advanced and published)
 };
+// Expert parallelism, the other way: where a down GEMM's weighted rows go
+// instead of y_perm. Sorted row p came from slot j = scale_idx[p] = s*C + i
+// of this rank's arena; its row goes to source s's arena, y region, row
+// yoff[s] + i (yoff: this rank's mailbox).
+struct EpRet {
+  uint8_t* const* arenas;
+  int64_t C;
+  size_t y_off;
+  const int32_t* yoff;
+};
+// This rank's arena regions (expert parallelism), for moe_ep_experts.
+struct EpViews {
+  void* x;          // received rows [G*C][H]
+  float* w;         // their routing weights [G*C]
+  int64_t* id;      // their local expert ids [G*C], -1 for empty slots
+  int32_t* yoff;    // the sources' y offsets [G]
+  size_t y_off, ret_flag_off;
+  uint64_t* epoch;  // this rank's epoch
+  int64_t C;
+};
+bool ep_views(const moe_problem& p, int G, void* own_arena, EpViews* v);
+// Publish this rank's epoch (not advanced) into flag slot `rank` at byte
+// offset flag_off of every arena, after a system-scope fence.
+cudaError_t launch_ep_publish(uint8_t* const* arenas, int G, int rank, size_t flag_off, const uint64_t* epoch,
+                              cudaStream_t s);
 // moe_ep_dispatch_send's layout helper; false if the problem or G is invalid.
 bool ep_dest(const moe_problem& p, int G, int rank, void* const* arenas, void* own_arena, const float* rw,
              EpDest* d);
@@ -169,6 +194,15 @@ cudaError_t launch_wgrad(const void* A, int64_t lda, const void* B, int64_t ldb,
 cudaError_t launch_tc_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,
                               const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
                               cudaStream_t s);
+// The down GEMM with each weighted row stored into its source's arena (EpRet)
+// instead of y; every epilogue warp fences its stores at system scope last.
+// The one-CTA or pair kernel as for down.
+cudaError_t launch_tc_down_ep(const Segments& sg, const void* h, const void* w_down, int64_t E_w,
+                              const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I, const EpRet& ep,
+                              int32_t* err, cudaStream_t s);
+cudaError_t launch_tc2_down_ep(const Segments& sg, const void* A, const void* w_down, int64_t E_w,
+                               const float* row_scale, const int32_t* scale_idx, int64_t H, int64_t I,
+                               const EpRet& ep, int32_t* err, int num_sms, cudaStream_t s);
 cudaError_t launch_tc2_down_kn(const Segments& sg, const void* A, int64_t lda, const void* w_kn, int64_t E_w, void* y,
                                const float* row_scale, const int32_t* scale_idx, int64_t N, int64_t K, int32_t* err,
                                int num_sms, cudaStream_t s);

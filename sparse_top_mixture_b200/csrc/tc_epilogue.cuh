@@ -106,5 +106,55 @@ __device__ __forceinline__ void epilogue_scale_f32(uint32_t tbase, int nchunks, 
   }
 }
 
+// store_block_f32 with a destination per row: row r of the warp block goes
+// to row_ptr of lane r (NULL: not stored) + column offset cb (ncols of the
+// 32 columns, a multiple of 4). The row pointers are exchanged by shuffles.
+__device__ __forceinline__ void store_block_f32_rows(const float (&v)[32], float* stage, float* row_ptr, int cb,
+                                                     int nrows, int ncols, int lane) {
+  float4* srow = reinterpret_cast<float4*>(stage + lane * kStageStride);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) srow[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int c4 = lane & 7;
+  const unsigned long long mine = reinterpret_cast<unsigned long long>(row_ptr);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = it * 4 + (lane >> 3);
+    float* dst = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, mine, r));
+    if (r < nrows && dst != nullptr && c4 * 4 < ncols)
+      *reinterpret_cast<float4*>(dst + cb + c4 * 4) = reinterpret_cast<const float4*>(stage + r * kStageStride)[c4];
+  }
+  __syncwarp();
+}
+
+// epilogue_scale_f32 into per-row destinations (this lane's row at row_ptr,
+// NULL for none), the same pipelined TMEM loads.
+__device__ __forceinline__ void epilogue_scale_f32_rows(uint32_t tbase, int nchunks, float sc, float* stage,
+                                                        float* row_ptr, int nrows, int col0, int N, int lane) {
+  auto store = [&](const uint32_t(&d)[32], int c) {
+    const int cb = col0 + c * 32;
+    if (cb >= N || nrows <= 0) return;  // warp-uniform
+    float v[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) v[q] = sc * __uint_as_float(d[q]);
+    store_block_f32_rows(v, stage, row_ptr, cb, nrows, N - cb, lane);
+  };
+  uint32_t a[32], b[32];
+  tmem_ld32(tbase, a);
+  tmem_ld_wait_regs(a);
+#pragma unroll 1
+  for (int c = 0; c < nchunks; c += 2) {  // a holds chunk c
+    const bool two = c + 1 < nchunks;
+    if (two) tmem_ld32(tbase + (c + 1) * 32, b);
+    store(a, c);
+    if (!two) break;
+    tmem_ld_wait_regs(b);
+    const bool more = c + 2 < nchunks;
+    if (more) tmem_ld32(tbase + (c + 2) * 32, a);
+    store(b, c + 1);
+    if (more) tmem_ld_wait_regs(a);
+  }
+}
+
 }  // namespace tc
 }  // namespace stm

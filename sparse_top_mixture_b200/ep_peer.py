@@ -19,8 +19,11 @@ A forward is three phases, which ``forward`` runs back to back:
   steps, ``moe_dispatch`` then ``moe_ep_send``); the shared expert runs on a
   second stream meanwhile;
 * ``experts``: wait for every source's rows, regroup the received slots by
-  local expert (``moe_dispatch_slots``), run the grouped SwiGLU, and store each
-  weighted fp32 row back into its source's arena at its sorted position;
+  local expert, run the grouped SwiGLU, and store each weighted fp32 row back
+  into its source's arena at its sorted position -- in bf16 one call
+  (``moe_ep_experts``) whose down GEMM epilogue does the stores; otherwise
+  (fp32, or ``fused=False``) ``moe_dispatch_slots``, ``moe_grouped_swiglu``
+  and ``moe_ep_return``;
 * ``finish``: wait for every owner's returns, then combine.
 
 On a node, ``open`` allocates this rank's arena and maps the peers' through
@@ -185,6 +188,13 @@ class PeerExpertParallelMoE:
     def experts(self) -> None:
         p, dev = self.p, self.arena.device
         self._wait(0)
+        if self.fused and p.dtype == "bf16":
+            # regroup, GEMMs, and the down epilogue storing each row into its source's arena
+            _check(lib().moe_ep_experts(ctypes.byref(p.c()), self.world, self.rank, self.ptrs.data_ptr(),
+                                        self.arena.data_ptr(), self.w["gate_up"].data_ptr(),
+                                        self.w["down"].data_ptr(), self.ws1.data_ptr(), self.ws1.numel(),
+                                        _stream(dev)))
+            return
         pk = self.pk1
         d1 = dispatch_slots(pk, self.recv_id, self.recv_x, ws=self.ws1)
         y_sorted = grouped_swiglu(pk, d1["x_perm"], d1["offsets"], self.w["gate_up"], self.w["down"], self.recv_w,
