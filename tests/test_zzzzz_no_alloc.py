@@ -12,9 +12,8 @@ first call would show up in the second. One check runs it inside a CUDA graph
 captured in global mode (any allocation during the capture would fail it),
 after a first call outside the capture has looked up the arrays' addresses.
 
-This file is collected after the parity tests (only the guard-band checks
-come later) so that a run stopping at the first failure has already run
-them.
+This file is collected last (its name sorts after every other test file),
+so that a run stopping at the first failure has already run all the others.
 """
 
 import numpy as np
