@@ -156,5 +156,68 @@ __device__ __forceinline__ void epilogue_scale_f32_rows(uint32_t tbase, int nchu
   }
 }
 
+// Epilogues of swapped tiles (the weights as the MMA's M operand, a segment
+// tail's tokens as its N columns): TMEM lane = output feature, column = row
+// of the tile. `ncols` accumulator columns are read 32 at a time (columns
+// past the tile's rows are read and dropped); `nrows` rows are stored.
+
+// gate_up: lanes 0-15 of this warp hold the gate pre-activations of features
+// f0 .. f0+15 and lanes 16-31 the up pre-activations of the same features.
+// A lane swaps its values with lane ^ 16, so lane L < 16 finishes rows j and
+// lane L + 16 rows j + 16 of feature f0 + L; h = silu(gate) * up rounded to
+// bf16, as in epilogue_swiglu. out_row0: output row of column 0.
+__device__ __forceinline__ void epilogue_swiglu_swapped(uint32_t tbase, int ncols, __nv_bfloat16* out_row0,
+                                                        int64_t ldo, int nrows, int f0, int N, int lane) {
+  const bool lo = lane < 16;
+  const int f = f0 + (lane & 15);
+  __nv_bfloat16* ocol = out_row0 + f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < ncols; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tbase + c0, v);
+    tmem_ld_wait_regs(v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float a = __uint_as_float(v[j]), b = __uint_as_float(v[j + 16]);
+      const float ao = __shfl_xor_sync(0xffffffffu, a, 16);
+      const float bo = __shfl_xor_sync(0xffffffffu, b, 16);
+      const float g = lo ? a : bo, u = lo ? ao : b;
+      const int r = c0 + j + (lo ? 0 : 16);
+      if (r < nrows && f < N) ocol[(int64_t)r * ldo] = __float2bfloat16_rn(silu_f32(g) * u);
+    }
+  }
+}
+
+// down: y = sc * accumulator for feature f0 + lane of rows 0 .. nrows-1,
+// each row's scale read by the lane of the same index and passed round by
+// shuffles. Row r goes to row_ptr(r) + f0 + lane, where row_ptr gives the
+// row's base pointer (NULL: not stored); a warp store writes 128 contiguous
+// bytes of one row.
+template <typename RowScale, typename RowPtr>
+__device__ __forceinline__ void epilogue_scale_f32_swapped(uint32_t tbase, int ncols, int nrows, int f0, int N,
+                                                           int lane, RowScale row_scale, RowPtr row_ptr) {
+  const int f = f0 + lane;
+#pragma unroll 1
+  for (int c0 = 0; c0 < ncols; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tbase + c0, v);
+    const int mine = c0 + lane;
+    float sc = 1.f;
+    float* dst = nullptr;
+    if (mine < nrows) {
+      sc = row_scale(mine);
+      dst = row_ptr(mine);
+    }
+    const unsigned long long dbits = reinterpret_cast<unsigned long long>(dst);
+    tmem_ld_wait_regs(v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float s = __shfl_sync(0xffffffffu, sc, j);
+      float* d = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, dbits, j));
+      if (c0 + j < nrows && d != nullptr && f < N) d[f] = s * __uint_as_float(v[j]);
+    }
+  }
+}
+
 }  // namespace tc
 }  // namespace stm

@@ -149,17 +149,22 @@ def test_staged_calls_match_forward(name):
         gc.assert_within_bound(sh.cpu().double().numpy(), s_ref, s_bnd, "shared")
 
 
+@pytest.mark.parametrize("I", [192, 200])
 @pytest.mark.parametrize("counts", [
     [1, 64, 65, 127, 128, 129, 255, 256, 257, 300, 383, 384, 385, 512, 600, 641],
     [300, 290, 257, 310, 384, 260, 270, 280],
+    [8, 16, 17, 33, 48, 49, 80, 95, 97, 112, 113, 120, 256 + 15, 256 + 16, 256 + 31, 256 + 100, 900, 1000],
 ])
-def test_segment_sizes_around_pair_tile_edges(counts):
+def test_segment_sizes_around_pair_tile_edges(counts, I):
     """Segments whose sizes sit on every edge of the CTA-pair tiling (pieces
-    of at most 128 rows that run as M=128 pair tiles, full and partial
-    256-row tiles): every y row of the grouped SwiGLU matches the fp64
-    per-segment reference within the arithmetic bound. Routing is planted,
+    of at most 128 rows, full and partial 256-row tiles): every y row of the
+    grouped SwiGLU matches the fp64 per-segment reference within the
+    arithmetic bound. Pieces of at most 128 rows run with the operands
+    swapped (their rows as the MMA's N, 16 to 128 in steps of 16, all of
+    which occur here); with I = 200 (not a multiple of 16) gate_up runs them
+    unswapped as M=128 pair MMAs and down still swapped. Routing is planted,
     so the sizes are exact."""
-    E, H, I = len(counts), 256, 192
+    E, H = len(counts), 256
     T = sum(counts)
     g = torch.Generator().manual_seed(len(counts))
     ids = torch.cat([torch.full((c,), e, dtype=torch.int64) for e, c in enumerate(counts)])
