@@ -41,6 +41,8 @@ EDGE = {
     "pairs_tails": CONFIGS["qwen3_30b_a3b"].replace(name="pairs_tails", T=2300, H=320, E=8, k=2, I=200),
     "pairs_shared_skew": CONFIGS["deepseek_v2_lite_zipf"].replace(name="pairs_zipf", T=4200, H=256, I=136,
                                                                   I_shared=272),
+    # k > 8: the forward's top-k does not count (the histogram is a launch of its own)
+    "k_above_8": CONFIGS["qwen3_30b_a3b"].replace(name="k12", T=100, H=128, E=16, k=12, I=64),
     # a sigmoid-gated shared expert too large to overlap the routed GEMMs
     # (8 x 16 row x column tiles): it runs beside the dispatch
     "large_shared_gated": CONFIGS["decode_weight_streaming"].replace(name="large_gated", T=1000, H=512, E=32, k=4,
@@ -99,12 +101,15 @@ def test_both_tensor_core_variants_are_exercised():
     assert paths["qwen3_30b_a3b"] == 1 and paths["decode_weight_streaming"] == 1
 
 
-@pytest.mark.parametrize("name", list(SMALL) + ["pairs_shared_skew", "large_shared_gated"])
+@pytest.mark.parametrize("name", list(SMALL) + ["pairs_shared_skew", "large_shared_gated", "pairs_tails",
+                                                 "k_above_8"])
 def test_staged_calls_match_forward(name):
     """route -> dispatch -> grouped_swiglu -> shared_expert -> combine through
     the separate entry points equals moe_forward bit for bit (also with a
     shared expert large enough to run beside the dispatch), and each stage
-    matches the oracle."""
+    matches the oracle. The forward counts its experts in the top-k launch
+    over blocks of 32 tokens (k <= 8), the staged dispatch over blocks of
+    256/k tokens: the expert counts agree as well."""
     cfg = EDGE.get(name) or SMALL[name]
     cpu, dev = _inputs(cfg)
     p = stm.Problem.from_config(cfg)
@@ -120,6 +125,7 @@ def test_staged_calls_match_forward(name):
     out = stm.combine(p, y, d["pair_pos"], sh)
     torch.cuda.synchronize()
     assert torch.equal(sel, sel_f) and torch.equal(rw, rw_f) and torch.equal(out, out_f)
+    assert torch.equal(moe.forward_counts(), d["counts"])
     # stage-level parity
     gsel = sel.cpu().numpy()
     r = gc.oracle_route(cfg, cpu)
