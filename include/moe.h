@@ -242,11 +242,7 @@ moe_status moe_combine(const moe_problem *p, const void *y_perm, const int32_t *
 
 /* Whole forward: route, dispatch, grouped SwiGLU, shared expert, combine.
  *   x [T,H] -> out [T,H]; routing_weights [T,k] and selected_experts [T,k] are
- *   also written (router contract). All intermediates live in ws. With
- *   k <= 8 the top-k launch also counts each 32-token block's experts and
- *   scans the counts, so the dispatch is one launch (the permutation and
- *   gather); the results equal those of moe_route followed by moe_dispatch
- *   (the same stable order, whatever the block size). */
+ *   also written (router contract). All intermediates live in ws. */
 moe_status moe_forward(const moe_problem *p, const moe_weights *w, const void *x, void *out,
                        float *routing_weights, int64_t *selected_experts, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
@@ -261,7 +257,7 @@ moe_status moe_forward(const moe_problem *p, const moe_weights *w, const void *x
  *       computed by its own small kernel;
  *     - a larger one occupies every SM while it runs, so it starts after the
  *       route (whose top-k kernel computes the gate) and runs beside the
- *       dispatch kernel(s) only; `stream` waits for it before the routed gate_up
+ *       dispatch kernels only; `stream` waits for it before the routed gate_up
  *       GEMM. The dispatch stage's event interval then ends when both are
  *       done and the shared stage's interval is empty.
  *     All work is complete once `stream` has passed the call.

@@ -35,11 +35,7 @@ Layout make_layout(const moe_problem& p) {
   L.header = take(sizeof(WsHeader));
   L.logits = take(router_partial_bytes(p.dtype, p.T, p.H, p.E));
   L.gamma = take((size_t)p.T * 4);
-  // per-block counts of the dispatch's histogram, or of the forward's
-  // counting top-k (its blocks may be smaller)
-  const int64_t tpb_count = route_count_tokens_per_block(p.k);
-  const int64_t nblk = std::max<int64_t>(dispatch_num_blocks(p.T, p.k), tpb_count ? ceil_div(p.T, tpb_count) : 0);
-  L.local = take((size_t)nblk * p.E * 4);
+  L.local = take((size_t)dispatch_num_blocks(p.T, p.k) * p.E * 4);
   L.counts = take((size_t)p.E * 4);
   L.offsets = take((size_t)(p.E + 1) * 4);
   L.sorted_pairs = take((size_t)P * 4);
@@ -103,19 +99,6 @@ moe_status do_route(const moe_problem& p, const Layout& L, const void* x, const 
   MOE_CUDA(launch_route(p.dtype, x, gate_w, shared_gate, bias, p.T, p.H, p.E, p.k, p.score, p.bias_mode,
                         p.renormalize ? 1 : 0, at<float>(ws, L.logits), weights, selected, gamma,
                         at<int32_t>(ws, L.header), s));
-  return MOE_OK;
-}
-
-// The forward's route and the first half of its dispatch in two launches:
-// the router logits, then the top-k, which also counts the experts of each
-// block of tokens and scans the counts (k <= 8; route_count_tokens_per_block).
-moe_status do_route_count(const moe_problem& p, const Layout& L, const void* x, const void* gate_w,
-                          const float* bias, const void* shared_gate, float* weights, int64_t* selected, float* gamma,
-                          int32_t* counts, int32_t* offsets, void* ws, cudaStream_t s) {
-  WsHeader* hdr = at<WsHeader>(ws, L.header);
-  MOE_CUDA(launch_route_count(p.dtype, x, gate_w, shared_gate, bias, p.T, p.H, p.E, p.k, p.score, p.bias_mode,
-                              p.renormalize ? 1 : 0, at<float>(ws, L.logits), weights, selected, gamma,
-                              &hdr->error_bits, at<int32_t>(ws, L.local), counts, offsets, &hdr->dispatch_ticket, s));
   return MOE_OK;
 }
 
@@ -233,9 +216,8 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   //    combine; its sigmoid gate comes from its own small kernel;
   //  - a large one occupies every SM while it runs, so it cannot overlap the
   //    routed GEMMs; it runs on `aux` after the route (whose top-k kernel
-  //    already computed the gate) beside the dispatch's permutation kernel,
-  //    whose CTAs fit next to its persistent CTAs, and `s` waits for it before
-  //    the routed gate_up.
+  //    already computed the gate) beside the dispatch kernels, which fit next
+  //    to its persistent CTAs, and `s` waits for it before the routed gate_up.
   const bool use_aux = has_shared && aux != nullptr && aux != s;
   const bool small_shared = use_aux && shared_overlaps(*p);
   const bool large_shared = use_aux && !small_shared;
@@ -264,16 +246,9 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
     MOE_CUDA(cudaEventRecord(evp.join, aux));
   }
 
-  // With k <= 8 the top-k launch also does the dispatch's histogram and
-  // scan, so the dispatch stage is the permutation alone.
-  const int64_t tpb_count = route_count_tokens_per_block(p->k);
   MOE_TRY(mark(MOE_STAGE_ROUTE));
-  if (tpb_count > 0)
-    MOE_TRY(do_route_count(*p, L, x, w->gate_w, w->bias, (gated && !small_shared) ? w->shared_gate : nullptr,
-                           weights, selected, gamma, counts, offsets, ws, s));
-  else
-    MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, (gated && !small_shared) ? w->shared_gate : nullptr, weights,
-                     selected, gamma, ws, s));
+  MOE_TRY(do_route(*p, L, x, w->gate_w, w->bias, (gated && !small_shared) ? w->shared_gate : nullptr, weights,
+                   selected, gamma, ws, s));
   if (large_shared) {
     MOE_CUDA(cudaEventRecord(evp.fork, s));
     MOE_CUDA(cudaStreamWaitEvent(aux, evp.fork, 0));
@@ -284,11 +259,7 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   // when both the dispatch and the shared expert are done, and the shared
   // stage is empty.
   MOE_TRY(mark(MOE_STAGE_DISPATCH));
-  if (tpb_count > 0)
-    MOE_CUDA(launch_permute(p->dtype, selected, x, p->T, p->H, p->E, p->k, tpb_count, at<int32_t>(ws, L.local),
-                            sorted_pairs, pair_pos, x_perm, s));
-  else
-    MOE_TRY(do_dispatch(*p, L, selected, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws, s));
+  MOE_TRY(do_dispatch(*p, L, selected, x, counts, offsets, sorted_pairs, pair_pos, x_perm, ws, s));
   if (large_shared) MOE_CUDA(cudaStreamWaitEvent(s, evp.join, 0));
   MOE_TRY(mark(MOE_STAGE_GATE_UP));
   MOE_TRY(do_grouped_gate_up(*p, L, x_perm, offsets, w->gate_up, ws, s));
@@ -525,9 +496,7 @@ MOE_API moe_status moe_launches_per_forward(const moe_problem* p, int32_t two_st
     *n = 0;
     return MOE_OK;
   }
-  // router logits, top-k (with the histogram and scan when k <= 8, else a
-  // histogram + scan launch of its own), permute + gather, combine
-  int count = 2 + (route_count_tokens_per_block(p->k) > 0 ? 1 : 2) + 1;
+  int count = 2 + 2 + 1;  // router logits + top-k; histogram + scan, permute + gather; combine
   if (p->dtype == MOE_DTYPE_BF16) {
     Segments routed{reinterpret_cast<const int32_t*>(16), (int32_t)p->E, 0, p->T * p->k};
     count += 2 * tc_gemm_launches(routed);

@@ -26,7 +26,6 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "peer.cuh"
-#include "scan.cuh"
 
 namespace stm {
 
@@ -35,7 +34,86 @@ namespace {
 constexpr int DTHREADS = 256;     // pairs per dispatch block
 constexpr int HIST_SUB = 4;       // dispatch blocks per histogram CTA
 constexpr int SCAN_THREADS = DTHREADS * HIST_SUB;
-static_assert(SCAN_THREADS == kScanThreads, "the scan runs on one CTA of the histogram grid");
+
+// Exclusive scan of the [nblk x E] per-block counts by one CTA of
+// SCAN_THREADS threads: counts, offsets, and (in place) the base position of
+// every (block, expert) run. Each expert's column is split among `tpe`
+// threads of one warp (tpe = 4..32), which read their ranges with independent
+// loads, combine through a segmented warp scan, and write the running bases.
+// The counts were written by other CTAs of the same grid: read through L2.
+// A range of up to kScanRegs entries is read once, in one round of loads,
+// and kept in registers for the second pass; longer ranges (more than
+// kScanRegs x tpe blocks) are read twice, in rounds of kScanRegs.
+constexpr int kScanRegs = 16;
+
+__device__ void block_scan_counts(int32_t* __restrict__ local, int nblk, int E, int tpe,
+                                  int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* tot) {
+  const int tid = threadIdx.x;
+  const int e = tid / tpe, part = tid % tpe;
+  const bool active = e < E;
+  const int chunk = (nblk + tpe - 1) / tpe;
+  const int b0 = min(nblk, part * chunk), b1 = min(nblk, b0 + chunk);
+  const bool in_regs = b1 - b0 <= kScanRegs;
+  int v[kScanRegs];
+  int sum = 0;
+  if (active) {
+    for (int b = b0; b < b1; b += kScanRegs) {
+#pragma unroll
+      for (int i = 0; i < kScanRegs; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
+#pragma unroll
+      for (int i = 0; i < kScanRegs; ++i) sum += v[i];
+    }
+  }
+  // segmented inclusive scan over the tpe parts of one expert (same warp)
+  int incl = sum;
+  for (int o = 1; o < tpe; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (part >= o) incl += x;
+  }
+  if (active && part == tpe - 1) tot[e] = incl;
+  __syncthreads();
+  if (tid < 32) {  // exclusive scan of the expert totals, 8 per lane
+    int c[8], loc = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      c[i] = ee < E ? tot[ee] : 0;
+      loc += c[i];
+    }
+    int inc = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (tid >= o) inc += x;
+    }
+    int run = inc - loc;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      if (ee < E) {
+        counts[ee] = c[i];
+        offsets[ee] = run;
+        tot[ee] = run;
+      }
+      run += c[i];
+    }
+    if (tid == 31) offsets[E] = inc;
+  }
+  __syncthreads();
+  if (!active) return;
+  int run = tot[e] + incl - sum;
+  for (int b = b0; b < b1; b += kScanRegs) {
+    if (!in_regs) {
+#pragma unroll
+      for (int i = 0; i < kScanRegs; ++i) v[i] = (b + i < b1) ? __ldcg(local + (int64_t)(b + i) * E + e) : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < kScanRegs; ++i) {
+      if (b + i < b1) local[(int64_t)(b + i) * E + e] = run;
+      run += v[i];
+    }
+  }
+}
 
 __global__ void __launch_bounds__(SCAN_THREADS) hist_scan_kernel(const int64_t* __restrict__ sel, int64_t P, int k,
                                                                  int E, int tok_per_blk, int nblk, int tpe,
@@ -255,17 +333,6 @@ cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, i
   const int tpe = std::min(32, SCAN_THREADS / ep);
   hist_scan_kernel<<<(unsigned)ceil_div(nblk, HIST_SUB), SCAN_THREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, nblk,
                                                                              tpe, local, counts, offsets, ticket, err);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_permute(dtype, selected, x, T, H, E, k, tpb, local, sorted_pairs, pair_pos, x_perm, s);
-}
-
-cudaError_t launch_permute(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
-                           int64_t k, int64_t tpb, const int32_t* local, int32_t* sorted_pairs, int32_t* pair_pos,
-                           void* x_perm, cudaStream_t s) {
-  if (tpb < 1 || tpb * k > DTHREADS) return cudaErrorInvalidValue;
-  const int nblk = (int)ceil_div(T, tpb);
-  const int64_t P = T * k;
   // Column slices per dispatch block: enough CTAs for about eight per SM,
   // each slice at least 32 vectors (512 bytes) of a row.
   const int V = dtype == 0 ? 4 : 8;
@@ -277,12 +344,12 @@ cudaError_t launch_permute(int dtype, const int64_t* selected, const void* x, in
   slices = (int)ceil_div(nvec, vps);
   const dim3 grid((unsigned)nblk, (unsigned)slices);
   if (dtype == 0)
-    permute_gather_kernel<float, false><<<grid, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, (int)tpb, local,
+    permute_gather_kernel<float, false><<<grid, DTHREADS, 0, s>>>(selected, P, (int)k, (int)E, tpb, local,
                                                                   sorted_pairs, pair_pos, (const float*)x,
                                                                   (float*)x_perm, T, (int)H, vps, nullptr, EpDest{});
   else
     permute_gather_kernel<__nv_bfloat16, false><<<grid, DTHREADS, 0, s>>>(
-        selected, P, (int)k, (int)E, (int)tpb, local, sorted_pairs, pair_pos, (const __nv_bfloat16*)x,
+        selected, P, (int)k, (int)E, tpb, local, sorted_pairs, pair_pos, (const __nv_bfloat16*)x,
         (__nv_bfloat16*)x_perm, T, (int)H, vps, nullptr, EpDest{});
   return cudaGetLastError();
 }

@@ -82,17 +82,6 @@ cudaError_t launch_shared_gate(int dtype, const void* x, const void* g, int64_t 
 cudaError_t launch_topk(const float* partial, int splits, int64_t ldo, int64_t T, int64_t E, int64_t k, int score,
                         int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
                         const void* x, const void* shared_gate, int64_t H, int dtype, float* gamma, cudaStream_t s);
-// The forward's route with the dispatch's histogram and scan folded into the
-// top-k launch: top-k CTAs of route_count_tokens_per_block(k) tokens (0: no
-// such variant for this k) each count their tokens' experts into row
-// blockIdx of local [ceil(T / tokens) x E]; the last CTA to finish scans them
-// into counts, offsets and the per-block bases that launch_permute reads.
-int64_t route_count_tokens_per_block(int64_t k);
-cudaError_t launch_route_count(int dtype, const void* x, const void* gate_w, const void* shared_gate,
-                               const float* bias, int64_t T, int64_t H, int64_t E, int64_t k, int score,
-                               int bias_mode, int renorm, float* partial, float* weights, int64_t* selected,
-                               float* gamma, int32_t* err, int32_t* local, int32_t* counts, int32_t* offsets,
-                               uint32_t* ticket, cudaStream_t s);
 
 // ---- dispatch ---------------------------------------------------------
 int64_t dispatch_tokens_per_block(int64_t k);
@@ -100,12 +89,6 @@ int64_t dispatch_num_blocks(int64_t T, int64_t k);
 cudaError_t launch_dispatch(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
                             int64_t k, int32_t* local, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
                             int32_t* pair_pos, void* x_perm, int32_t* err, uint32_t* ticket, cudaStream_t s);
-// The dispatch's second launch alone: rank each block of `tpb` tokens' pairs
-// from the bases in `local` (written by a histogram and scan over blocks of
-// the same size) and copy the token rows to their slots.
-cudaError_t launch_permute(int dtype, const int64_t* selected, const void* x, int64_t T, int64_t H, int64_t E,
-                           int64_t k, int64_t tpb, const int32_t* local, int32_t* sorted_pairs, int32_t* pair_pos,
-                           void* x_perm, cudaStream_t s);
 
 // ---- combine ----------------------------------------------------------
 // y_perm [T*k, H] and shared_out [T, H] are fp32 for every problem dtype.

@@ -15,7 +15,6 @@
 // partials in a fixed order, so routing is bit-reproducible run to run.
 #include "common.cuh"
 #include "kernels.h"
-#include "scan.cuh"
 
 namespace stm {
 
@@ -120,24 +119,22 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 constexpr int TOPK_WARPS = 8;
 
-// Top-k tokens per CTA of the forward's counting variant, and its largest k.
-constexpr int kHistTokens = kScanThreads / 32;
-constexpr int kHistMaxK = 8;
-
-// Token t's scores, top-k and weights, computed by one warp: lane l owns
-// experts [l*NS, l*NS + NS), NS = 1, 2, 4 or 8 (E up to 32, 64, 128 or 256),
-// so a lane reads its logits of one partial with one or two 16-byte loads
-// when rows are 16-byte aligned. sw / se: this warp's k slots in shared
-// memory. hist (shared memory, or NULL): the lane that owns a selected
-// expert adds 1 to its count.
+// One warp per token; lane l owns experts [l*NS, l*NS + NS), NS = 1, 2, 4 or
+// 8 (E up to 32, 64, 128 or 256), so a lane reads its logits of one partial
+// with one or two 16-byte loads when rows are 16-byte aligned.
 template <typename TX, int NS>
-__device__ __forceinline__ void topk_token(const float* __restrict__ partial, int splits, int64_t ldo, int vec4,
-                                           int Tn, int E, int k, int score, int bias_mode, int renorm,
-                                           const float* __restrict__ bias, float* __restrict__ weights,
-                                           int64_t* __restrict__ selected, const TX* __restrict__ x,
-                                           const TX* __restrict__ shared_gate, int H, float* __restrict__ gamma,
-                                           int t, float* sw, int* se, int* hist) {
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ partial, int splits,
+                                                                int64_t ldo, int vec4, int Tn, int E, int k,
+                                                                int score, int bias_mode, int renorm,
+                                                                const float* __restrict__ bias,
+                                                                float* __restrict__ weights,
+                                                                int64_t* __restrict__ selected,
+                                                                const TX* __restrict__ x,
+                                                                const TX* __restrict__ shared_gate, int H,
+                                                                float* __restrict__ gamma) {
   const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * TOPK_WARPS + (threadIdx.x >> 5);
+  if (t >= Tn) return;
   const int e0 = lane * NS;
 
   float logit[NS], sc[NS];
@@ -208,6 +205,9 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ partial, in
 
   // Slot j's expert and raw weight go to shared memory, written by the lane
   // that owns the expert; the renormalising sum runs in slot order.
+  __shared__ float s_w[TOPK_WARPS][kMaxExperts];
+  __shared__ int s_e[TOPK_WARPS][kMaxExperts];
+  const int wid = threadIdx.x >> 5;
   for (int j = 0; j < k; ++j) {
     // This lane's best live expert: largest key, then lowest index.
     uint32_t bk = 0;
@@ -224,20 +224,19 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ partial, in
       for (int i = 0; i < NS; ++i)
         if (i == bi) w = sc[i];
       live &= ~(1u << bi);
-      sw[j] = w;
-      se[j] = we;
-      if (hist != nullptr) atomicAdd(&hist[we], 1);
+      s_w[wid][j] = w;
+      s_e[wid][j] = we;
     }
   }
   __syncwarp();
   float tot = 0.f;
   if (renorm)
-    for (int j = 0; j < k; ++j) tot += sw[j];
+    for (int j = 0; j < k; ++j) tot += s_w[wid][j];
   for (int j = lane; j < k; j += 32) {
-    float w = sw[j];
+    float w = s_w[wid][j];
     if (renorm) w = tot > 0.f ? w / tot : 0.f;
     weights[(int64_t)t * k + j] = w;
-    selected[(int64_t)t * k + j] = (int64_t)se[j];
+    selected[(int64_t)t * k + j] = (int64_t)s_e[wid][j];
   }
   if (gamma != nullptr) {
     // gamma[t] = sigmoid(x[t] . shared_gate): fp32 dot product, lanes over
@@ -262,64 +261,6 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ partial, in
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) gamma[t] = 1.0f / (1.0f + expf(-acc));
   }
-}
-
-template <typename TX, int NS>
-__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ partial, int splits,
-                                                                int64_t ldo, int vec4, int Tn, int E, int k,
-                                                                int score, int bias_mode, int renorm,
-                                                                const float* __restrict__ bias,
-                                                                float* __restrict__ weights,
-                                                                int64_t* __restrict__ selected,
-                                                                const TX* __restrict__ x,
-                                                                const TX* __restrict__ shared_gate, int H,
-                                                                float* __restrict__ gamma) {
-  __shared__ float s_w[TOPK_WARPS][kMaxExperts];
-  __shared__ int s_e[TOPK_WARPS][kMaxExperts];
-  const int wid = threadIdx.x >> 5;
-  const int t = blockIdx.x * TOPK_WARPS + wid;
-  if (t >= Tn) return;
-  topk_token<TX, NS>(partial, splits, ldo, vec4, Tn, E, k, score, bias_mode, renorm, bias, weights, selected, x,
-                     shared_gate, H, gamma, t, s_w[wid], s_e[wid], nullptr);
-}
-
-// The same top-k, in CTAs of kHistTokens tokens (k <= kHistMaxK, so at most
-// 256 pairs: one block of the dispatch's counting sort), each also counting
-// its tokens' experts (in shared memory; counts do not depend on the order of
-// the additions). Each CTA stores its counts as row blockIdx.x of `local`
-// [nblk x E]; the CTA that finishes last (an atomic ticket, no CTA waits on
-// another) scans them into counts, offsets and the per-block bases, as the
-// dispatch's histogram kernel does, and resets the ticket.
-template <typename TX, int NS>
-__global__ void __launch_bounds__(kScanThreads) topk_count_kernel(
-    const float* __restrict__ partial, int splits, int64_t ldo, int vec4, int Tn, int E, int k, int score,
-    int bias_mode, int renorm, const float* __restrict__ bias, float* __restrict__ weights,
-    int64_t* __restrict__ selected, const TX* __restrict__ x, const TX* __restrict__ shared_gate, int H,
-    float* __restrict__ gamma, int nblk, int tpe, int32_t* __restrict__ local, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, uint32_t* __restrict__ ticket) {
-  __shared__ float s_w[kHistTokens][kHistMaxK];
-  __shared__ int s_e[kHistTokens][kHistMaxK];
-  __shared__ int hist[kMaxExperts];
-  __shared__ int last;
-  for (int e = threadIdx.x; e < E; e += kScanThreads) hist[e] = 0;
-  __syncthreads();
-  const int wid = threadIdx.x >> 5;
-  const int t = blockIdx.x * kHistTokens + wid;
-  if (t < Tn)
-    topk_token<TX, NS>(partial, splits, ldo, vec4, Tn, E, k, score, bias_mode, renorm, bias, weights, selected, x,
-                       shared_gate, H, gamma, t, s_w[wid], s_e[wid], hist);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kScanThreads) local[(int64_t)blockIdx.x * E + e] = hist[e];
-  // Publish this CTA's counts, then take a ticket: the CTA that draws the
-  // last one sees every other CTA's counts and does the scan.
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  block_scan_counts(local, nblk, E, tpe, counts, offsets, hist);
-  if (threadIdx.x == 0) *ticket = 0u;  // ready for the next forward on this workspace
 }
 
 // gamma[t] = sigmoid(x[t] . g), one warp per token.
@@ -421,50 +362,7 @@ void launch_topk_t(dim3 grid, const float* partial, int splits, int64_t ldo, int
                           selected, x, shared_gate, H, gamma, s);
 }
 
-template <typename TX, int NS>
-void launch_topk_count_ns(const float* partial, int splits, int64_t ldo, int vec4, int64_t T, int64_t E, int64_t k,
-                          int score, int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
-                          const void* x, const void* shared_gate, int64_t H, float* gamma, int32_t* local,
-                          int32_t* counts, int32_t* offsets, uint32_t* ticket, cudaStream_t s) {
-  const int nblk = (int)ceil_div(T, kHistTokens);
-  topk_count_kernel<TX, NS><<<(unsigned)nblk, kScanThreads, 0, s>>>(
-      partial, splits, ldo, vec4, (int)T, (int)E, (int)k, score, bias_mode, renorm, bias, weights, selected,
-      (const TX*)x, (const TX*)shared_gate, (int)H, gamma, nblk, scan_threads_per_expert(E), local, counts, offsets,
-      ticket);
-}
-
-template <typename TX>
-void launch_topk_count_t(const float* partial, int splits, int64_t ldo, int vec4, int64_t T, int64_t E, int64_t k,
-                         int score, int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
-                         const void* x, const void* shared_gate, int64_t H, float* gamma, int32_t* local,
-                         int32_t* counts, int32_t* offsets, uint32_t* ticket, cudaStream_t s) {
-  if (E <= 32)
-    launch_topk_count_ns<TX, 1>(partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
-                                selected, x, shared_gate, H, gamma, local, counts, offsets, ticket, s);
-  else if (E <= 64)
-    launch_topk_count_ns<TX, 2>(partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
-                                selected, x, shared_gate, H, gamma, local, counts, offsets, ticket, s);
-  else if (E <= 128)
-    launch_topk_count_ns<TX, 4>(partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
-                                selected, x, shared_gate, H, gamma, local, counts, offsets, ticket, s);
-  else
-    launch_topk_count_ns<TX, 8>(partial, splits, ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
-                                selected, x, shared_gate, H, gamma, local, counts, offsets, ticket, s);
-}
-
-// Router logits into `partial` (tensor cores for bf16, SIMT for fp32).
-cudaError_t launch_logits(int dtype, const void* x, const void* gate_w, int64_t T, int64_t H, int64_t E,
-                          float* partial, int32_t* err, const RouterPlan& plan, cudaStream_t s) {
-  if (plan.tensor_cores) return launch_tc_logits(x, gate_w, T, H, E, partial, plan.ldo, plan.splits, err, s);
-  dim3 grid((unsigned)ceil_div(T, RBM), (unsigned)ceil_div(E, RBN), (unsigned)plan.splits);
-  router_logits_kernel<float><<<grid, RTHREADS, 0, s>>>((const float*)x, (const float*)gate_w, partial, (int)T,
-                                                        (int)H, (int)E, (int)plan.ldo, plan.k_per_split);
-  return cudaGetLastError();
-}
-
 }  // namespace
-
-int64_t route_count_tokens_per_block(int64_t k) { return k <= kHistMaxK ? kHistTokens : 0; }
 
 cudaError_t launch_topk(const float* partial, int splits, int64_t ldo, int64_t T, int64_t E, int64_t k, int score,
                         int bias_mode, int renorm, const float* bias, float* weights, int64_t* selected,
@@ -485,31 +383,18 @@ cudaError_t launch_route(int dtype, const void* x, const void* gate_w, const voi
                          float* partial, float* weights, int64_t* selected, float* gamma, int32_t* err,
                          cudaStream_t s) {
   const RouterPlan plan = router_plan(dtype, T, H, E);
-  const cudaError_t e = launch_logits(dtype, x, gate_w, T, H, E, partial, err, plan, s);
+  cudaError_t e;
+  if (plan.tensor_cores) {
+    e = launch_tc_logits(x, gate_w, T, H, E, partial, plan.ldo, plan.splits, err, s);
+  } else {
+    dim3 grid((unsigned)ceil_div(T, RBM), (unsigned)ceil_div(E, RBN), (unsigned)plan.splits);
+    router_logits_kernel<float><<<grid, RTHREADS, 0, s>>>((const float*)x, (const float*)gate_w, partial, (int)T,
+                                                          (int)H, (int)E, (int)plan.ldo, plan.k_per_split);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   return launch_topk(partial, plan.splits, plan.ldo, T, E, k, score, bias_mode, renorm, bias, weights, selected, x,
                      shared_gate, H, dtype, shared_gate ? gamma : nullptr, s);
-}
-
-cudaError_t launch_route_count(int dtype, const void* x, const void* gate_w, const void* shared_gate,
-                               const float* bias, int64_t T, int64_t H, int64_t E, int64_t k, int score,
-                               int bias_mode, int renorm, float* partial, float* weights, int64_t* selected,
-                               float* gamma, int32_t* err, int32_t* local, int32_t* counts, int32_t* offsets,
-                               uint32_t* ticket, cudaStream_t s) {
-  if (k > kHistMaxK) return cudaErrorInvalidValue;
-  const RouterPlan plan = router_plan(dtype, T, H, E);
-  const cudaError_t e = launch_logits(dtype, x, gate_w, T, H, E, partial, err, plan, s);
-  if (e != cudaSuccess) return e;
-  const int vec4 = (plan.ldo % 4 == 0 && (reinterpret_cast<uintptr_t>(partial) & 15u) == 0) ? 1 : 0;
-  if (dtype == 0)
-    launch_topk_count_t<float>(partial, plan.splits, plan.ldo, vec4, T, E, k, score, bias_mode, renorm, bias, weights,
-                               selected, x, shared_gate, H, shared_gate ? gamma : nullptr, local, counts, offsets,
-                               ticket, s);
-  else
-    launch_topk_count_t<__nv_bfloat16>(partial, plan.splits, plan.ldo, vec4, T, E, k, score, bias_mode, renorm, bias,
-                                       weights, selected, x, shared_gate, H, shared_gate ? gamma : nullptr, local,
-                                       counts, offsets, ticket, s);
-  return cudaGetLastError();
 }
 
 }  // namespace stm

@@ -80,14 +80,12 @@ def test_gemm_path(L):
 
 
 def test_launch_counts(L):
-    # k <= 8: route 2 (logits; top-k with the dispatch's histogram and scan), dispatch 1 (permute + gather),
-    # combine 1, plus the expert GEMMs; k > 8: the histogram + scan is a launch of its own
-    assert stm.launches_per_forward(_p()) == 4 + 2
-    assert stm.launches_per_forward(_p(T=8192, E=64, k=6)) == 4 + 2
-    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256)) == 4 + 2 + 2
-    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256, dtype="f32")) == 4 + 4
-    assert stm.launches_per_forward(_p(dtype="f32", shared="plain", I_shared=256)) == 4 + 4
-    assert stm.launches_per_forward(_p(E=16, k=12)) == 5 + 2
+    # route 2 (logits, top-k), dispatch 2 (histogram + scan, permute + gather), combine 1, plus the expert GEMMs
+    assert stm.launches_per_forward(_p()) == 5 + 2
+    assert stm.launches_per_forward(_p(T=8192, E=64, k=6)) == 5 + 2
+    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256)) == 5 + 2 + 2
+    assert stm.launches_per_forward(_p(T=8192, E=64, k=6, shared="plain", I_shared=256, dtype="f32")) == 5 + 4
+    assert stm.launches_per_forward(_p(dtype="f32", shared="plain", I_shared=256)) == 5 + 4
     assert stm.launches_per_forward(_p(T=0)) == 0
     gated = _p(shared="sigmoid_gated", I_shared=256)  # small shared expert: runs on the aux stream
     assert stm.launches_per_forward(gated, two_streams=True) == stm.launches_per_forward(gated) + 1
