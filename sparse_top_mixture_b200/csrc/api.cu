@@ -216,8 +216,10 @@ moe_status forward_impl(const moe_problem* p, const moe_weights* w, const void* 
   //    combine; its sigmoid gate comes from its own small kernel;
   //  - a large one occupies every SM while it runs, so it cannot overlap the
   //    routed GEMMs; it runs on `aux` after the route (whose top-k kernel
-  //    already computed the gate) beside the dispatch kernels, which fit next
-  //    to its persistent CTAs, and `s` waits for it before the routed gate_up.
+  //    already computed the gate) beside the dispatch (the permutation
+  //    kernel's CTAs fit next to its persistent CTAs; the histogram's
+  //    1024-thread CTAs wait for free SMs), and `s` waits for it before the
+  //    routed gate_up.
   const bool use_aux = has_shared && aux != nullptr && aux != s;
   const bool small_shared = use_aux && shared_overlaps(*p);
   const bool large_shared = use_aux && !small_shared;
