@@ -688,6 +688,8 @@ __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int
 // rows of dout, dense). Rows with j >= count_e are zero in x_pad, dy_pad,
 // h_pad [*, I] and dgdu_pad [*, 2I] (the SwiGLU backward writes the others).
 // 16-byte vectors (H and I are multiples of 8).
+constexpr int kPadBatch = 4;
+
 __global__ void __launch_bounds__(BT) bw16_pad_rows(const __nv_bfloat16* __restrict__ x,
                                                   const __nv_bfloat16* __restrict__ dout,
                                                   const int32_t* __restrict__ tok, const float* __restrict__ scale,
@@ -730,23 +732,43 @@ __global__ void __launch_bounds__(BT) bw16_pad_rows(const __nv_bfloat16* __restr
   __syncthreads();
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
   const int hv = H / 8;
-  for (int idx = threadIdx.x; idx < 64 * hv; idx += BT) {
-    const int i = idx / hv, v = idx - i * hv;
-    const int64_t q = q0 + i;
-    const int src = s_src[i];
-    uint4 xo = zero, yo = zero;
-    if (src >= 0) {
-      xo = reinterpret_cast<const uint4*>(x + (int64_t)src * H)[v];
-      const uint4 d = reinterpret_cast<const uint4*>(dout + (int64_t)src * H)[v];
-      reinterpret_cast<uint4*>(dout_perm + (int64_t)(off[e] + j0 + i) * H)[v] = d;
-      float f[8];
-      unpack16_bf16(d, f);
-      const float sc = s_sc[i];
-      yo = make_uint4(pack_bf16x2(sc * f[0], sc * f[1]), pack_bf16x2(sc * f[2], sc * f[3]),
-                      pack_bf16x2(sc * f[4], sc * f[5]), pack_bf16x2(sc * f[6], sc * f[7]));
+  const int total = 64 * hv;
+  // kPadBatch vectors a thread at a time: their loads are all issued before
+  // the first store, so each thread keeps several rows' loads in flight.
+  for (int base = threadIdx.x; base < total; base += BT * kPadBatch) {
+    uint4 xv[kPadBatch], dv[kPadBatch];
+#pragma unroll
+    for (int u = 0; u < kPadBatch; ++u) {
+      const int idx = base + u * BT;
+      xv[u] = zero;
+      dv[u] = zero;
+      if (idx < total) {
+        const int i = idx / hv, v = idx - i * hv;
+        const int src = s_src[i];
+        if (src >= 0) {
+          xv[u] = reinterpret_cast<const uint4*>(x + (int64_t)src * H)[v];
+          dv[u] = reinterpret_cast<const uint4*>(dout + (int64_t)src * H)[v];
+        }
+      }
     }
-    reinterpret_cast<uint4*>(x_pad + q * H)[v] = xo;
-    reinterpret_cast<uint4*>(dy_pad + q * H)[v] = yo;
+#pragma unroll
+    for (int u = 0; u < kPadBatch; ++u) {
+      const int idx = base + u * BT;
+      if (idx >= total) break;
+      const int i = idx / hv, v = idx - i * hv;
+      const int64_t q = q0 + i;
+      uint4 yo = zero;
+      if (s_src[i] >= 0) {
+        reinterpret_cast<uint4*>(dout_perm + (int64_t)(off[e] + j0 + i) * H)[v] = dv[u];
+        float f[8];
+        unpack16_bf16(dv[u], f);
+        const float sc = s_sc[i];
+        yo = make_uint4(pack_bf16x2(sc * f[0], sc * f[1]), pack_bf16x2(sc * f[2], sc * f[3]),
+                        pack_bf16x2(sc * f[4], sc * f[5]), pack_bf16x2(sc * f[6], sc * f[7]));
+      }
+      reinterpret_cast<uint4*>(x_pad + q * H)[v] = xv[u];
+      reinterpret_cast<uint4*>(dy_pad + q * H)[v] = yo;
+    }
   }
   const int nvalid = max(0, min(64, cnt - j0));
   const int iv = I / 8, rv = 3 * iv;  // one row: I/8 vectors of h, 2I/8 of [dg | du]
