@@ -17,6 +17,7 @@ namespace stm {
 namespace {
 
 constexpr int SBM = 64, SBN = 64, SBK = 16, STHREADS = 256;
+static_assert(SBM == SBN && SBM * SBK % STHREADS == 0, "tile loads: whole elements per thread");
 
 template <bool GATE_UP>
 __global__ void __launch_bounds__(STHREADS) simt_grouped_kernel(const float* __restrict__ A,
@@ -51,21 +52,41 @@ __global__ void __launch_bounds__(STHREADS) simt_grouped_kernel(const float* __r
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[g][i][j] = 0.f;
 
-  for (int k0 = 0; k0 < K; k0 += SBK) {
-    for (int i = tid; i < SBM * SBK; i += STHREADS) {
+  // The next K slice is read into registers while the current one is
+  // multiplied out of shared memory (the same products in the same order).
+  constexpr int G = GATE_UP ? 2 : 1;
+  constexpr int PER = SBM * SBK / STHREADS;  // elements of a tile per thread (SBN == SBM)
+  float ra[PER], rb[G][PER];
+  auto load_slice = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int i = tid + u * STHREADS;
       const int r = i / SBK, c = i % SBK;
       const int row = row0 + r, kk = k0 + c;
-      As[c][r] = (row < row_end && kk < K) ? A[(int64_t)row * K + kk] : 0.f;
-    }
+      ra[u] = (row < row_end && kk < K) ? A[(int64_t)row * K + kk] : 0.f;
 #pragma unroll
-    for (int g = 0; g < (GATE_UP ? 2 : 1); ++g) {
-      for (int i = tid; i < SBN * SBK; i += STHREADS) {
-        const int r = i / SBK, c = i % SBK;
-        const int n = n0 + r, kk = k0 + c;
-        Bs[g][c][r] = (n < N && kk < K) ? We[((int64_t)g * N + n) * K + kk] : 0.f;
+      for (int g = 0; g < G; ++g) {
+        const int n = n0 + r;
+        rb[g][u] = (n < N && kk < K) ? We[((int64_t)g * N + n) * K + kk] : 0.f;
       }
     }
-    __syncthreads();
+  };
+  auto store_slice = [&]() {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int i = tid + u * STHREADS;
+      const int r = i / SBK, c = i % SBK;
+      As[c][r] = ra[u];
+#pragma unroll
+      for (int g = 0; g < G; ++g) Bs[g][c][r] = rb[g][u];
+    }
+  };
+  load_slice(0);
+  store_slice();
+  __syncthreads();
+  for (int k0 = 0; k0 < K; k0 += SBK) {
+    const bool more = k0 + SBK < K;
+    if (more) load_slice(k0 + SBK);
 #pragma unroll
     for (int kk = 0; kk < SBK; ++kk) {
       float a[4];
@@ -83,6 +104,10 @@ __global__ void __launch_bounds__(STHREADS) simt_grouped_kernel(const float* __r
       }
     }
     __syncthreads();
+    if (more) {
+      store_slice();
+      __syncthreads();
+    }
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
