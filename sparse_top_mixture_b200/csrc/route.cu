@@ -44,40 +44,42 @@ __global__ void __launch_bounds__(RTHREADS) router_logits_kernel(const T* __rest
 
   constexpr int VPR = RBK / V;         // vectors per tile row
   constexpr int NV = RBM * VPR;        // vectors per tile
-  for (int k0 = kb; k0 < ke; k0 += RBK) {
-    for (int i = tid; i < NV; i += RTHREADS) {
-      const int r = i / VPR, c = (i % VPR) * V;
-      const int kk = k0 + c;
-      float f[8];
-      // A: token rows
-      {
-        const int row = m0 + r;
-        if (row < Tn && kk < ke) {
-          const uint4 v = *reinterpret_cast<const uint4*>(x + (int64_t)row * H + kk);
-          if constexpr (V == 8) unpack16_bf16(v, f); else unpack16(v, f, nullptr);
-        } else {
+  static_assert(RBM == RBN && NV % RTHREADS == 0, "tile loads: whole vectors per thread");
+  constexpr int PV = NV / RTHREADS;
+  // The next K slice is read into registers while the current one is
+  // multiplied out of shared memory (the same products in the same order).
+  uint4 va[PV], vb[PV];
+  auto load_slice = [&](int k0) {
 #pragma unroll
-          for (int q = 0; q < V; ++q) f[q] = 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < V; ++q) As[c + q][r] = f[q];
-      }
-      // B: expert rows
-      {
-        const int col = n0 + r;
-        if (col < E && kk < ke) {
-          const T* src = gate_w + (int64_t)col * H;
-          const uint4 v = *reinterpret_cast<const uint4*>(src + kk);
-          if constexpr (V == 8) unpack16_bf16(v, f); else unpack16(v, f, nullptr);
-        } else {
-#pragma unroll
-          for (int q = 0; q < V; ++q) f[q] = 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < V; ++q) Bs[c + q][r] = f[q];
-      }
+    for (int u = 0; u < PV; ++u) {
+      const int i = tid + u * RTHREADS;
+      const int r = i / VPR, kk = k0 + (i % VPR) * V;
+      const int row = m0 + r, col = n0 + r;
+      va[u] = (row < Tn && kk < ke) ? *reinterpret_cast<const uint4*>(x + (int64_t)row * H + kk)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+      vb[u] = (col < E && kk < ke) ? *reinterpret_cast<const uint4*>(gate_w + (int64_t)col * H + kk)
+                                   : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+  auto store_slice = [&]() {
+#pragma unroll
+    for (int u = 0; u < PV; ++u) {
+      const int i = tid + u * RTHREADS;
+      const int r = i / VPR, c = (i % VPR) * V;
+      float f[8];
+      if constexpr (V == 8) unpack16_bf16(va[u], f); else unpack16(va[u], f, nullptr);
+#pragma unroll
+      for (int q = 0; q < V; ++q) As[c + q][r] = f[q];
+      if constexpr (V == 8) unpack16_bf16(vb[u], f); else unpack16(vb[u], f, nullptr);
+#pragma unroll
+      for (int q = 0; q < V; ++q) Bs[c + q][r] = f[q];
+    }
+  };
+  if (kb < ke) load_slice(kb);
+  for (int k0 = kb; k0 < ke; k0 += RBK) {
+    store_slice();
     __syncthreads();
+    if (k0 + RBK < ke) load_slice(k0 + RBK);
 #pragma unroll 8
     for (int kk = 0; kk < RBK; ++kk) {
       float a[4], b[4];
