@@ -305,59 +305,80 @@ __global__ void __launch_bounds__(BT, 2) bw_wgrad_gemm(WGemm a) {
 
 // ---- router and small per-row kernels ---------------------------------------------
 
-// One token per block: logits L (+ logit bias, in place), scores S and the
+// Warps per block and experts per lane of the per-token router kernels
+// (one warp per token; lane l owns experts l, l + 32, ...).
+constexpr int kTokWarps = BT / 32;
+constexpr int kExpPerLane = kMaxExperts / 32;
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// One token per warp: logits L (+ logit bias, in place), scores S and the
 // routing weights w of its k chosen experts (slot order), as in the forward.
 __global__ void __launch_bounds__(BT) bw_scores(float* __restrict__ L, const float* __restrict__ bias, int bias_mode,
-                                              int score, int renorm, const int64_t* __restrict__ sel, int E, int k,
-                                              float* __restrict__ S, float* __restrict__ w) {
-  __shared__ float red[BT];
-  __shared__ float s_sc[kMaxExperts];
-  const int t = blockIdx.x, e = threadIdx.x;
-  float l = -INFINITY;
-  if (e < E) {
-    l = L[(int64_t)t * E + e];
-    if (bias_mode == MOE_BIAS_LOGIT) {
-      l += bias[e];
-      L[(int64_t)t * E + e] = l;
+                                              int score, int renorm, const int64_t* __restrict__ sel, int T, int E,
+                                              int k, float* __restrict__ S, float* __restrict__ w) {
+  __shared__ float s_sc[kTokWarps][kMaxExperts];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTokWarps + wid;
+  if (t >= T) return;  // the whole warp; no block-wide barrier follows
+  float l[kExpPerLane], sc[kExpPerLane];
+#pragma unroll
+  for (int i = 0; i < kExpPerLane; ++i) {
+    const int e = i * 32 + lane;
+    l[i] = -INFINITY;
+    if (e < E) {
+      float v = L[(int64_t)t * E + e];
+      if (bias_mode == MOE_BIAS_LOGIT) {
+        v += bias[e];
+        L[(int64_t)t * E + e] = v;
+      }
+      l[i] = v;
     }
   }
-  float sc = 0.f;
   if (score == MOE_SCORE_SOFTMAX) {
-    red[e] = l;
-    __syncthreads();
-    for (int o = BT / 2; o > 0; o >>= 1) {
-      if (e < o) red[e] = fmaxf(red[e], red[e + o]);
-      __syncthreads();
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kExpPerLane; ++i) m = fmaxf(m, l[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float z = 0.f;
+#pragma unroll
+    for (int i = 0; i < kExpPerLane; ++i) {
+      sc[i] = i * 32 + lane < E ? expf(l[i] - m) : 0.f;
+      z += sc[i];
     }
-    const float m = red[0];
-    __syncthreads();
-    const float z = e < E ? expf(l - m) : 0.f;
-    red[e] = z;
-    __syncthreads();
-    for (int o = BT / 2; o > 0; o >>= 1) {
-      if (e < o) red[e] += red[e + o];
-      __syncthreads();
-    }
-    sc = z / red[0];
+    z = warp_sum_f(z);
+#pragma unroll
+    for (int i = 0; i < kExpPerLane; ++i) sc[i] = sc[i] / z;
   } else if (score == MOE_SCORE_SIGMOID) {
-    sc = sig_f(l);
+#pragma unroll
+    for (int i = 0; i < kExpPerLane; ++i) sc[i] = sig_f(l[i]);
   } else {
-    sc = sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
+#pragma unroll
+    for (int i = 0; i < kExpPerLane; ++i) sc[i] = sqrtf(fmaxf(l[i], 0.f) + log1pf(expf(-fabsf(l[i]))));
   }
-  if (e < E) {
-    S[(int64_t)t * E + e] = sc;
-    s_sc[e] = sc;
+#pragma unroll
+  for (int i = 0; i < kExpPerLane; ++i) {
+    const int e = i * 32 + lane;
+    if (e < E) {
+      S[(int64_t)t * E + e] = sc[i];
+      s_sc[wid][e] = sc[i];
+    }
   }
-  __syncthreads();
-  if (e == 0) {
+  __syncwarp();
+  if (lane == 0) {
     float tot = 0.f;
     for (int j = 0; j < k; ++j) {
       const int64_t ej = sel[(int64_t)t * k + j];
-      tot += (ej >= 0 && ej < E) ? s_sc[ej] : 0.f;
+      tot += (ej >= 0 && ej < E) ? s_sc[wid][ej] : 0.f;
     }
     for (int j = 0; j < k; ++j) {
       const int64_t ej = sel[(int64_t)t * k + j];
-      float v = (ej >= 0 && ej < E) ? s_sc[ej] : 0.f;
+      float v = (ej >= 0 && ej < E) ? s_sc[wid][ej] : 0.f;
       if (renorm) v = tot > 0.f ? v / tot : 0.f;
       w[(int64_t)t * k + j] = v;
     }
@@ -399,19 +420,21 @@ __global__ void __launch_bounds__(BT) bw_rowdot(const float* __restrict__ Hact, 
   }
 }
 
-// Router backward, one token per block: dS from dw (renormalisation), dL from
+// Router backward, one token per warp: dS from dw (renormalisation), dL from
 // dS; also dL rounded to bf16 into dL16 (row pitch ld16) when given.
 __global__ void __launch_bounds__(BT) bw_router_bwd(const float* __restrict__ L, const float* __restrict__ S,
                                                   const float* __restrict__ w, const float* __restrict__ dw,
-                                                  const int64_t* __restrict__ sel, int score, int renorm, int E,
-                                                  int k, float* __restrict__ dL, __nv_bfloat16* __restrict__ dL16,
-                                                  int ld16) {
-  __shared__ float dS[kMaxExperts];
-  __shared__ float red[BT];
-  const int t = blockIdx.x, e = threadIdx.x;
-  if (e < E) dS[e] = 0.f;
-  __syncthreads();
-  if (e == 0) {
+                                                  const int64_t* __restrict__ sel, int score, int renorm, int T,
+                                                  int E, int k, float* __restrict__ dL,
+                                                  __nv_bfloat16* __restrict__ dL16, int ld16) {
+  __shared__ float s_dS[kTokWarps][kMaxExperts];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTokWarps + wid;
+  if (t >= T) return;  // the whole warp; no block-wide barrier follows
+  float* dS = s_dS[wid];
+  for (int e = lane; e < E; e += 32) dS[e] = 0.f;
+  __syncwarp();
+  if (lane == 0) {
     float tot = 0.f, dww = 0.f;
     for (int j = 0; j < k; ++j) {
       const int64_t ej = sel[(int64_t)t * k + j];
@@ -425,24 +448,28 @@ __global__ void __launch_bounds__(BT) bw_router_bwd(const float* __restrict__ L,
       dS[ej] += renorm ? (tot > 0.f ? (d - dww) / tot : 0.f) : d;
     }
   }
-  __syncthreads();
-  const float s = e < E ? S[(int64_t)t * E + e] : 0.f;
-  const float ds = e < E ? dS[e] : 0.f;
-  float dl;
-  if (score == MOE_SCORE_SOFTMAX) {
-    red[e] = ds * s;
-    __syncthreads();
-    for (int o = BT / 2; o > 0; o >>= 1) {
-      if (e < o) red[e] += red[e + o];
-      __syncthreads();
-    }
-    dl = s * (ds - red[0]);
-  } else if (score == MOE_SCORE_SIGMOID) {
-    dl = ds * s * (1.f - s);
-  } else {
-    dl = (e < E && s > 0.f) ? ds * sig_f(L[(int64_t)t * E + e]) / (2.f * s) : 0.f;
+  __syncwarp();
+  float sv[kExpPerLane], ds[kExpPerLane];
+#pragma unroll
+  for (int i = 0; i < kExpPerLane; ++i) {
+    const int e = i * 32 + lane;
+    sv[i] = e < E ? S[(int64_t)t * E + e] : 0.f;
+    ds[i] = e < E ? dS[e] : 0.f;
   }
-  if (e < E) {
+  float red = 0.f;
+  if (score == MOE_SCORE_SOFTMAX) {
+#pragma unroll
+    for (int i = 0; i < kExpPerLane; ++i) red += ds[i] * sv[i];
+    red = warp_sum_f(red);
+  }
+#pragma unroll
+  for (int i = 0; i < kExpPerLane; ++i) {
+    const int e = i * 32 + lane;
+    if (e >= E) continue;
+    float dl;
+    if (score == MOE_SCORE_SOFTMAX) dl = sv[i] * (ds[i] - red);
+    else if (score == MOE_SCORE_SIGMOID) dl = ds[i] * sv[i] * (1.f - sv[i]);
+    else dl = sv[i] > 0.f ? ds[i] * sig_f(L[(int64_t)t * E + e]) / (2.f * sv[i]) : 0.f;
     dL[(int64_t)t * E + e] = dl;
     if (dL16) dL16[(int64_t)t * ld16 + e] = __float2bfloat16_rn(dl);
   }
@@ -1039,7 +1066,8 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
     BW16_CUDA(launch_tc_logits(x, w->gate_w, T, H, E, lpart, rp.ldo, rp.splits, err, s));
     bw16_sum_logits<<<grid_for((int64_t)T * E), BT, 0, s>>>(lpart, rp.splits, rp.ldo, T, E, L);
   }
-  bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
+  bw_scores<<<(unsigned)ceil_div(T, kTokWarps), BT, 0, s>>>(L, w->bias, p->bias_mode, p->score,
+                                                              p->renormalize ? 1 : 0, selected, (int)T, E, k, S, wts);
   // Sorted segments of the choice with x_perm.
   BW16_CUDA(launch_dispatch(MOE_DTYPE_BF16, selected, x, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
                             at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, xperm, err,
@@ -1067,8 +1095,9 @@ moe_status backward_bf16(const moe_problem* p, const moe_weights* w, const void*
   // dgate_w = dL^T x over all tokens, the router's dx = dL gate_w with gate_w
   // [E][H] read as stored); d_bias = sum_t dL in fp32. The router's dx goes
   // to `extra`, or beside the shared expert's when there is one.
-  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL, dL16,
-                                 (int)b.Epad);
+  bw_router_bwd<<<(unsigned)ceil_div(T, kTokWarps), BT, 0, s>>>(L, S, wts, dw, selected, p->score,
+                                                                  p->renormalize ? 1 : 0, (int)T, E, k, dL, dL16,
+                                                                  (int)b.Epad);
   if (rs.splits > 1) {
     float* parts = at<float>(ws, b.parts);
     BW16_CUDA(launch_wgrad(dL16, b.Epad, x, H, T, rsplit, b.Tpad, rs.splits, E, H, parts, err, s));
@@ -1205,7 +1234,8 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
         return a;
       }(),
       s));
-  bw_scores<<<T, BT, 0, s>>>(L, w->bias, p->bias_mode, p->score, p->renormalize ? 1 : 0, selected, E, k, S, wts);
+  bw_scores<<<(unsigned)ceil_div(T, kTokWarps), BT, 0, s>>>(L, w->bias, p->bias_mode, p->score,
+                                                              p->renormalize ? 1 : 0, selected, (int)T, E, k, S, wts);
   // Sorted segments of the choice, each row's token and weight.
   BW_CUDA(launch_dispatch(MOE_DTYPE_F32, selected, nullptr, p->T, p->H, p->E, p->k, at<int32_t>(ws, b.local),
                           at<int32_t>(ws, b.counts), offsets, sorted_pairs, pair_pos, nullptr, err,
@@ -1245,7 +1275,8 @@ MOE_API moe_status moe_backward(const moe_problem* p, const moe_weights* w, cons
   BW_CUDA(run_wgrad(wgrad(dgu, nullptr, nullptr, 2 * I, 2 * I, x, tok, H, H, offsets, 0, P, g->d_gate_up, err), E,
                     s));
   // Router backward: dL, dgate_w = dL^T x (in row chunks summed in order), d_bias = sum_t dL.
-  bw_router_bwd<<<T, BT, 0, s>>>(L, S, wts, dw, selected, p->score, p->renormalize ? 1 : 0, E, k, dL, nullptr, 0);
+  bw_router_bwd<<<(unsigned)ceil_div(T, kTokWarps), BT, 0, s>>>(L, S, wts, dw, selected, p->score,
+                                                                  p->renormalize ? 1 : 0, (int)T, E, k, dL, nullptr, 0);
   const int nchunk = router_chunks(*p);
   if (nchunk == 1) {
     BW_CUDA(run_wgrad(wgrad(dL, nullptr, nullptr, E, E, x, nullptr, H, H, nullptr, T, T, g->d_gate_w, err), 1, s));
