@@ -480,7 +480,8 @@ __global__ void __launch_bounds__(BT) bw_sum_parts(const float* __restrict__ par
                                                  float* __restrict__ out) {
   for (int64_t i = blockIdx.x * (int64_t)BT + threadIdx.x; i < n; i += (int64_t)gridDim.x * BT) {
     float acc = 0.f;
-    for (int q = 0; q < S; ++q) acc += part[q * n + i];
+#pragma unroll 4
+    for (int q = 0; q < S; ++q) acc += part[q * n + i];  // in part order; unrolled so loads overlap
     out[i] = acc;
   }
 }
@@ -681,7 +682,8 @@ __global__ void __launch_bounds__(BT) bw16_sum_logits(const float* __restrict__ 
     const int64_t t = i / E;
     const int e = (int)(i - t * E);
     float acc = 0.f;
-    for (int sp = 0; sp < splits; ++sp) acc += part[((int64_t)sp * T + t) * ldo + e];
+#pragma unroll 4
+    for (int sp = 0; sp < splits; ++sp) acc += part[((int64_t)sp * T + t) * ldo + e];  // in split order
     L[i] = acc;
   }
 }
@@ -691,21 +693,44 @@ __global__ void __launch_bounds__(BT) bw16_sum_logits(const float* __restrict__ 
 // ranges = {0, T, 0, round_up(T, 64)}, and its split into `splits` row
 // chunks of `chunk` rows (a multiple of 64) for the router's weight gradient:
 // rsplit[i] = min(i * chunk, round_up(T, 64)), i = 0..splits.
+// One warp: lane l scans experts [l*per, l*per + per), per = ceil(E / 32),
+// then the lanes' totals are scanned with shuffles.
 __global__ void bw16_koff(const int32_t* __restrict__ offsets, int E, int T, int32_t* __restrict__ koff,
                           int32_t* __restrict__ ranges, int splits, int chunk, int32_t* __restrict__ rsplit) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int run = 0;
-  for (int e = 0; e < E; ++e) {
-    koff[e] = run;
-    run += (offsets[e + 1] - offsets[e] + 63) / 64 * 64;
+  const int lane = threadIdx.x;
+  if (lane >= 32 || blockIdx.x != 0) return;
+  constexpr int kPer = kMaxExperts / 32;
+  const int per = (E + 31) / 32;
+  int padded[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane * per + i;
+    padded[i] = (i < per && e < E) ? (offsets[e + 1] - offsets[e] + 63) / 64 * 64 : 0;
+    sum += padded[i];
   }
-  koff[E] = run;
-  const int Tpad = (T + 63) / 64 * 64;
-  ranges[0] = 0;
-  ranges[1] = T;
-  ranges[2] = 0;
-  ranges[3] = Tpad;
-  for (int i = 0; i <= splits; ++i) rsplit[i] = min(i * chunk, Tpad);
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane * per + i;
+    if (i < per && e < E) koff[e] = run;
+    run += padded[i];
+  }
+  if (lane == 31) koff[E] = incl;
+  if (lane == 0) {
+    const int Tpad = (T + 63) / 64 * 64;
+    ranges[0] = 0;
+    ranges[1] = T;
+    ranges[2] = 0;
+    ranges[3] = Tpad;
+    for (int i = 0; i <= splits; ++i) rsplit[i] = min(i * chunk, Tpad);
+  }
 }
 
 // Padded row buffers, one block per 64-row group (an expert's run starts at a
