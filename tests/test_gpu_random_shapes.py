@@ -1,5 +1,6 @@
-"""GPU parity on seeded random problem shapes: the bf16 forward through the C
-ABI against the fp64 oracle, over shapes the named problems do not reach.
+"""GPU parity on seeded random problem shapes: the bf16 forward and backward
+through the C ABI against the fp64 oracles, over shapes the named problems do
+not reach.
 
 Each case draws E, k, rows per expert (mostly enough for the CTA-pair GEMMs,
 so segment tails of every size occur), H, I (with and without I % 16 == 0),
@@ -14,6 +15,10 @@ is off by up to half a unit in the last place, 2^-9 relative. Without it the
 max-abs criterion 3e-2 * rms(ref) cannot hold for outputs whose largest
 elements are about 8x their rms or more (k <= 2 without renormalisation draws
 such outputs): there the rounding of the exact value alone exceeds it.
+
+The backward cases (fewer tokens, for the fp64 backward oracle's sake) use the
+bf16 backward's bar: relative L2 <= 5e-3 per gradient tensor and no element
+off by more than 1e-2 of the tensor's largest magnitude.
 """
 
 import random
@@ -24,18 +29,19 @@ import torch
 
 import gpu_check as gc
 import sparse_top_mixture_b200 as stm
+from test_gpu_backward_bf16 import _check_grads, _run
 import workloads
 from workloads import CONFIGS
 
 pytestmark = pytest.mark.gpu
 
 
-def _case(seed: int):
+def _case(seed: int, max_tokens: int = 3000):
     rng = random.Random(seed)
     E = rng.choice([4, 6, 8, 12, 16])
     k = min(rng.choice([1, 2, 3, 4]), E)
     per_expert = rng.choice([200, 260, 300, 400, 520, 700])
-    T = min(3000, max(8, per_expert * E // k + rng.randint(-37, 37)))
+    T = min(max_tokens, max(8, per_expert * E // k + rng.randint(-37, 37)))
     H = rng.choice([128, 136, 192, 256, 264, 384])
     I = rng.choice([64, 96, 104, 128, 136, 200, 256])
     score = rng.choice(["softmax", "sigmoid", "sqrtsoftplus"])
@@ -69,3 +75,10 @@ def test_random_shape_forward(seed):
     bound = 3e-2 * rms + 2.0 ** -9 * np.abs(ref)
     worst = float((np.abs(got - ref) / bound).max())
     assert worst <= 1.0, f"{cfg}: error x{worst:.3f} of its bound"
+
+
+@pytest.mark.parametrize("seed", list(range(100, 112)))
+def test_random_shape_backward(seed):
+    cfg = _case(seed, max_tokens=1500)
+    got, ref = _run(cfg)
+    _check_grads(got, ref, cfg.name)
