@@ -5,7 +5,8 @@ not reach.
 Each case draws E, k, rows per expert (mostly enough for the CTA-pair GEMMs,
 so segment tails of every size occur), H, I (with and without I % 16 == 0),
 the score function, renormalisation and the shared-expert kind, from a fixed
-seed. The selection is checked as in the other parity tests (bit-exact up to
+seed; further cases draw a logit or a selection-only bias, and a few tokens
+over many experts (decode). The selection is checked as in the other parity tests (bit-exact up to
 near ties), the routing weights to 1e-5, and the output to relative L2
 <= 5e-3 and, per element, |got - ref| <= 3e-2 * rms(ref) + 2^-9 * |ref|.
 
@@ -48,14 +49,32 @@ def _case(seed: int, max_tokens: int = 3000):
     shared = rng.choice(["none", "none", "plain", "sigmoid_gated"])
     I_shared = rng.choice([64, 96, 136, 256]) if shared != "none" else 0
     renorm = rng.choice([True, False])
+    bias_mode = rng.choice(["none", "none", "logit", "select"])
     return CONFIGS["qwen3_30b_a3b"].replace(name=f"random{seed}", T=T, H=H, E=E, k=k, I=I, score=score,
                                             shared=shared, I_shared=I_shared, renormalize=renorm,
-                                            bias_kind="none", bias_mode="none", seed=1000 + seed)
+                                            bias_kind="none" if bias_mode == "none" else "uniform0.1",
+                                            bias_mode=bias_mode, seed=1000 + seed)
 
 
-@pytest.mark.parametrize("seed", list(range(24)))
+def _decode_case(seed: int):
+    """A few tokens over many experts (the one-CTA GEMMs, M=64 tiles, most
+    experts empty), as in weight-streaming decode."""
+    rng = random.Random(seed)
+    E = rng.choice([64, 128, 256])
+    k = rng.choice([4, 6, 8])
+    T = rng.choice([1, 3, 16, 31, 64])
+    H = rng.choice([256, 512, 1024, 1032])
+    I = rng.choice([128, 192, 256, 264])
+    shared = rng.choice(["none", "plain", "sigmoid_gated"])
+    I_shared = rng.choice([128, 256]) if shared != "none" else 0
+    score = rng.choice(["softmax", "sigmoid", "sqrtsoftplus"])
+    return CONFIGS["decode_weight_streaming"].replace(name=f"decode{seed}", T=T, H=H, E=E, k=k, I=I, score=score,
+                                                      shared=shared, I_shared=I_shared, seed=2000 + seed)
+
+
+@pytest.mark.parametrize("seed", list(range(24)) + [f"decode{i}" for i in range(8)])
 def test_random_shape_forward(seed):
-    cfg = _case(seed)
+    cfg = _decode_case(int(seed[6:])) if isinstance(seed, str) else _case(seed)
     cpu = workloads.generate(cfg, "cpu")
     dev = {name: (v.cuda() if v is not None else None) for name, v in cpu.items()}
     moe = stm.SparseMoE(stm.Problem.from_config(cfg), dev)
