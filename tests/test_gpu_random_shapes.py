@@ -17,6 +17,11 @@ max-abs criterion 3e-2 * rms(ref) cannot hold for outputs whose largest
 elements are about 8x their rms or more (k <= 2 without renormalisation draws
 such outputs): there the rounding of the exact value alone exceeds it.
 
+The expert-parallel cases run G ranks over peer memory, emulated on one GPU
+(each phase for every rank in turn), on random shapes: each rank's output,
+routing weights and selection must equal the one-GPU forward of its tokens
+bit for bit, as in the named expert-parallel tests.
+
 The backward cases (fewer tokens, for the fp64 backward oracle's sake) use the
 bf16 backward's bar: relative L2 <= 5e-3 per gradient tensor and no element
 off by more than 1e-2 of the tensor's largest magnitude.
@@ -30,6 +35,7 @@ import torch
 
 import gpu_check as gc
 import sparse_top_mixture_b200 as stm
+from sparse_top_mixture_b200.ep_peer import PeerExpertParallelMoE
 from test_gpu_backward_bf16 import _check_grads, _run
 import workloads
 from workloads import CONFIGS
@@ -101,3 +107,29 @@ def test_random_shape_backward(seed):
     cfg = _case(seed, max_tokens=1500)
     got, ref = _run(cfg)
     _check_grads(got, ref, cfg.name)
+
+
+@pytest.mark.parametrize("seed", list(range(200, 208)))
+def test_random_shape_expert_parallel_matches_one_gpu(seed):
+    cfg = _case(seed, max_tokens=1500)
+    G = 4 if cfg.E % 4 == 0 and seed % 2 == 0 else 2
+    fused = seed % 3 != 0
+    p = stm.Problem.from_config(cfg)
+    cpu = workloads.generate(cfg, "cpu")
+    dev = {name: (v.cuda() if v is not None else None) for name, v in cpu.items()}
+    layers = PeerExpertParallelMoE.emulate(p, dev, G, fused=fused)
+    ref_layer = stm.SparseMoE(p, dev)
+    for step in range(2):
+        xs = [workloads.router_inputs(cfg, rank=r + G * step)["x"].cuda() for r in range(G)]
+        for layer, x in zip(layers, xs):
+            layer.send(x)
+        for layer in layers:
+            layer.experts()
+        got = [layer.finish() for layer in layers]
+        torch.cuda.synchronize()
+        for r, (layer, x, (out, rw, sel)) in enumerate(zip(layers, xs, got)):
+            ref_out, ref_rw, ref_sel = ref_layer(x)
+            torch.cuda.synchronize()
+            assert int(layer.err.item()) == 0, f"rank {r}: a wait gave up"
+            assert torch.equal(sel, ref_sel) and torch.equal(rw, ref_rw), f"{cfg} G={G} rank {r} step {step}"
+            assert torch.equal(out, ref_out), f"{cfg} G={G} fused={fused} rank {r} step {step}: output"
