@@ -22,11 +22,17 @@ The expert-parallel cases run G ranks over peer memory, emulated on one GPU
 routing weights and selection must equal the one-GPU forward of its tokens
 bit for bit, as in the named expert-parallel tests.
 
+The tensor-parallel cases shard every expert's I over G ranks emulated the
+same way: every rank's output must equal, bit for bit, the ranks' fp32
+combines of their partial rows summed in rank order and rounded once, and be
+within the bound above of the oracle.
+
 The backward cases (fewer tokens, for the fp64 backward oracle's sake) use the
 bf16 backward's bar: relative L2 <= 5e-3 per gradient tensor and no element
 off by more than 1e-2 of the tensor's largest magnitude.
 """
 
+import dataclasses
 import random
 
 import numpy as np
@@ -36,6 +42,7 @@ import torch
 import gpu_check as gc
 import sparse_top_mixture_b200 as stm
 from sparse_top_mixture_b200.ep_peer import PeerExpertParallelMoE
+from sparse_top_mixture_b200.tp_peer import PeerTensorParallelMoE
 from test_gpu_backward_bf16 import _check_grads, _run
 import workloads
 from workloads import CONFIGS
@@ -78,6 +85,14 @@ def _decode_case(seed: int):
                                                       shared=shared, I_shared=I_shared, seed=2000 + seed)
 
 
+def _assert_output_close(got, ref, what):
+    assert np.isfinite(got).all()
+    assert gc.rel_l2(got, ref) <= 5e-3, f"{what}: rel L2 {gc.rel_l2(got, ref):.3e}"
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    worst = float((np.abs(got - ref) / (3e-2 * rms + 2.0 ** -9 * np.abs(ref))).max())
+    assert worst <= 1.0, f"{what}: error x{worst:.3f} of its bound"
+
+
 @pytest.mark.parametrize("seed", list(range(24)) + [f"decode{i}" for i in range(8)])
 def test_random_shape_forward(seed):
     cfg = _decode_case(int(seed[6:])) if isinstance(seed, str) else _case(seed)
@@ -93,13 +108,49 @@ def test_random_shape_forward(seed):
     assert ntie == 0, f"{cfg}: {ntie} tokens took the near-tie escape"
     o = gc.oracle_forward(cfg, cpu, selected=gsel)
     assert np.abs(rw.cpu().double().numpy() - o["routing_weights"]).max() <= 1e-5
-    got, ref = out.cpu().double().numpy(), o["out"]
-    assert np.isfinite(got).all()
-    assert gc.rel_l2(got, ref) <= 5e-3, f"{cfg}: rel L2 {gc.rel_l2(got, ref):.3e}"
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    bound = 3e-2 * rms + 2.0 ** -9 * np.abs(ref)
-    worst = float((np.abs(got - ref) / bound).max())
-    assert worst <= 1.0, f"{cfg}: error x{worst:.3f} of its bound"
+    _assert_output_close(out.cpu().double().numpy(), o["out"], str(cfg))
+
+
+def _tp_case(seed: int):
+    """Sizes the tensor-parallel layer takes: H, I and I_s multiples of 8G."""
+    rng = random.Random(seed)
+    G = rng.choice([2, 4])
+    base = _case(seed, max_tokens=1200)
+    m = 8 * G
+    H = rng.choice([4, 6, 8, 12]) * m
+    I = rng.choice([2, 3, 4, 6]) * m
+    I_shared = rng.choice([2, 4]) * m if base.shared != "none" else 0
+    return G, base.replace(name=f"tp{seed}", H=H, I=I, I_shared=I_shared)
+
+
+@pytest.mark.parametrize("seed", list(range(300, 306)))
+def test_random_shape_tensor_parallel_sums_partials_in_rank_order(seed):
+    G, cfg = _tp_case(seed)
+    p = stm.Problem.from_config(cfg)
+    cpu = workloads.generate(cfg, "cpu")
+    dev = {name: (v.cuda() if v is not None else None) for name, v in cpu.items()}
+    layers = PeerTensorParallelMoE.emulate(p, dev, G)
+    for step in range(2):
+        x = workloads.router_inputs(cfg, rank=step)["x"].cuda()
+        for layer in layers:
+            layer.partial(x)
+        for layer in layers:
+            layer.reduce()
+        got = [layer.finish() for layer in layers]
+        acc = None
+        for layer in layers:
+            d, y, shared = layer._st["keep"]
+            part = stm.combine(dataclasses.replace(layer.local, dtype="f32"), y, d["pair_pos"], shared)
+            acc = part.clone() if acc is None else acc + part
+        ref = acc.to(p.torch_dtype)
+        torch.cuda.synchronize()
+        for r, (layer, (out, rw, sel)) in enumerate(zip(layers, got)):
+            assert int(layer.err.item()) == 0, f"rank {r}: a wait gave up"
+            assert torch.equal(out, ref), f"{cfg} G={G} rank {r} step {step}"
+        if step == 0:
+            gsel = got[0][2].cpu().numpy()
+            o = gc.oracle_forward(cfg, {**cpu, "x": x.cpu()}, selected=gsel)
+            _assert_output_close(got[0][0].cpu().double().numpy(), o["out"], f"{cfg} G={G}")
 
 
 @pytest.mark.parametrize("seed", list(range(100, 112)))
