@@ -22,6 +22,10 @@ The expert-parallel cases run G ranks over peer memory, emulated on one GPU
 routing weights and selection must equal the one-GPU forward of its tokens
 bit for bit, as in the named expert-parallel tests.
 
+The fp32 cases (the SIMT kernels: ragged K slices of 16, 64-row tiles) take
+the fp32 bar: relative L2 <= 1e-5 and max-abs <= 1e-5 of the largest
+magnitude.
+
 The tensor-parallel cases shard every expert's I over G ranks emulated the
 same way: every rank's output must equal, bit for bit, the ranks' fp32
 combines of their partial rows summed in rank order and rounded once, and be
@@ -109,6 +113,26 @@ def test_random_shape_forward(seed):
     o = gc.oracle_forward(cfg, cpu, selected=gsel)
     assert np.abs(rw.cpu().double().numpy() - o["routing_weights"]).max() <= 1e-5
     _assert_output_close(out.cpu().double().numpy(), o["out"], str(cfg))
+
+
+@pytest.mark.parametrize("seed", list(range(400, 408)))
+def test_random_shape_fp32_forward(seed):
+    rng = random.Random(seed)
+    base = _case(seed, max_tokens=600)
+    cfg = base.replace(name=f"fp32_{seed}", dtype="f32", H=rng.choice([40, 72, 136, 200]),
+                       I=rng.choice([24, 56, 88, 136]), I_shared=rng.choice([24, 40]) if base.shared != "none" else 0)
+    cpu = workloads.generate(cfg, "cpu")
+    dev = {name: (v.cuda() if v is not None else None) for name, v in cpu.items()}
+    moe = stm.SparseMoE(stm.Problem.from_config(cfg), dev)
+    out, rw, sel = moe(dev["x"])
+    torch.cuda.synchronize()
+    assert moe.read_device_error() == 0
+    r = gc.oracle_route(cfg, cpu)
+    gsel = sel.cpu().numpy()
+    assert gc.check_selection(cfg, r, gsel) == 0
+    o = gc.oracle_forward(cfg, cpu, selected=gsel)
+    assert np.abs(rw.cpu().double().numpy() - o["routing_weights"]).max() <= 1e-5
+    gc.assert_close(out.cpu().double().numpy(), o["out"], "f32", cfg.name)
 
 
 def _tp_case(seed: int):
