@@ -33,7 +33,8 @@ within the bound above of the oracle.
 
 The backward cases (fewer tokens, for the fp64 backward oracle's sake) use the
 bf16 backward's bar: relative L2 <= 5e-3 per gradient tensor and no element
-off by more than 1e-2 of the tensor's largest magnitude.
+off by more than 1e-2 of the tensor's largest magnitude; the fp32 backward
+cases the fp32 backward's bar (1e-5 and 1e-4).
 """
 
 import dataclasses
@@ -48,6 +49,7 @@ import sparse_top_mixture_b200 as stm
 from sparse_top_mixture_b200.ep_peer import PeerExpertParallelMoE
 from sparse_top_mixture_b200.tp_peer import PeerTensorParallelMoE
 from test_gpu_backward_bf16 import _check_grads, _run
+import test_gpu_backward as bw32
 import workloads
 from workloads import CONFIGS
 
@@ -208,3 +210,13 @@ def test_random_shape_expert_parallel_matches_one_gpu(seed):
             assert int(layer.err.item()) == 0, f"rank {r}: a wait gave up"
             assert torch.equal(sel, ref_sel) and torch.equal(rw, ref_rw), f"{cfg} G={G} rank {r} step {step}"
             assert torch.equal(out, ref_out), f"{cfg} G={G} fused={fused} rank {r} step {step}: output"
+
+
+@pytest.mark.parametrize("seed", list(range(500, 506)))
+def test_random_shape_fp32_backward(seed):
+    rng = random.Random(seed)
+    base = _case(seed, max_tokens=400)
+    cfg = base.replace(name=f"bw32_{seed}", dtype="f32", H=rng.choice([40, 72, 136]), I=rng.choice([24, 56, 88]),
+                       I_shared=rng.choice([24, 40]) if base.shared != "none" else 0)
+    got, ref = bw32._run(cfg)
+    bw32._check_grads(got, ref, cfg.name)
