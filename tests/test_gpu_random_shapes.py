@@ -22,6 +22,10 @@ The expert-parallel cases run G ranks over peer memory, emulated on one GPU
 routing weights and selection must equal the one-GPU forward of its tokens
 bit for bit, as in the named expert-parallel tests.
 
+The staged cases call the stages one by one (route, dispatch, grouped
+SwiGLU, shared expert, combine) and must equal the whole forward bit for bit,
+with the dispatch equal to the oracle's stable permutation.
+
 The fp32 cases (the SIMT kernels: ragged K slices of 16, 64-row tiles) take
 the fp32 bar: relative L2 <= 1e-5 and max-abs <= 1e-5 of the largest
 magnitude.
@@ -220,3 +224,24 @@ def test_random_shape_fp32_backward(seed):
                        I_shared=rng.choice([24, 40]) if base.shared != "none" else 0)
     got, ref = bw32._run(cfg)
     bw32._check_grads(got, ref, cfg.name)
+
+
+@pytest.mark.parametrize("seed", list(range(600, 608)))
+def test_random_shape_staged_calls_match_forward(seed):
+    cfg = _case(seed, max_tokens=2000) if seed % 2 == 0 else _decode_case(seed)
+    cpu = workloads.generate(cfg, "cpu")
+    dev = {name: (v.cuda() if v is not None else None) for name, v in cpu.items()}
+    p = stm.Problem.from_config(cfg)
+    out_f, rw_f, sel_f = stm.SparseMoE(p, dev)(dev["x"])
+    ws = stm.new_workspace(p)
+    rw, sel, gam = stm.route(p, dev["x"], dev["gate_w"], dev["bias"], dev["shared_gate"], ws=ws)
+    d = stm.dispatch(p, sel, dev["x"], ws=ws)
+    y = stm.grouped_swiglu(p, d["x_perm"], d["offsets"], dev["gate_up"], dev["down"], rw, d["sorted_pairs"], ws=ws)
+    sh = None
+    if cfg.shared != "none":
+        sh = stm.shared_expert(p, dev["x"], dev["shared_gate_up"], dev["shared_down"], gam, ws=ws)
+    out = stm.combine(p, y, d["pair_pos"], sh)
+    torch.cuda.synchronize()
+    assert stm.read_device_error(ws) == 0
+    assert torch.equal(sel, sel_f) and torch.equal(rw, rw_f) and torch.equal(out, out_f), str(cfg)
+    gc.assert_dispatch_exact(d, sel.cpu().numpy(), cfg.E)
